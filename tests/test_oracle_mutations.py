@@ -1,0 +1,78 @@
+"""Planted mistakes in the oracle (on the CPU): each mutated copy must fail a pin.
+
+A copy of the oracle source gets one plausible slip (a flipped sign, a
+transposed operand, reversed conv taps, a dropped term or clamp, the read
+placed before the write), is compiled to a temporary library, and the pins of
+``test_oracle_pins`` are run against it.  At least one pin has to fail for
+every mutation; otherwise the pins would not be constraining that part.
+"""
+
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+from oracle import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "kda_oracle.c")
+
+MUTATIONS = {
+    "delta_sign": ("dl[j] = (vt[j] - p[j]) * beta", "dl[j] = (p[j] - vt[j]) * beta"),
+    "delta_sign_rec": ("dl[j] = (vt[j] - p[j]) * bt", "dl[j] = (p[j] - vt[j]) * bt"),
+    "predict_transposed": ("acc += kt[i] * S[i * D + j];", "acc += kt[i] * S[j * D + i];"),
+    "read_transposed": ("acc += qt[i] * S[i * D + j];", "acc += qt[i] * S[j * D + i];"),
+    "conv_taps_reversed": ("J->conv_w[c * KCONV + j] *", "J->conv_w[c * KCONV + (KCONV - 1 - j)] *"),
+    "no_lower_bound": ("gt[i] = g < J->lower_bound ? J->lower_bound : g;", "gt[i] = g;"),
+    "no_dt_bias": (" + J->dt_bias[h * D + i];", ";"),
+    "no_silu": ("dst[i] = silu(acc);", "dst[i] = acc;"),
+    "write_without_k": ("S[i * D + j] += kt[i] * dl[j];", "S[i * D + j] += dl[j];"),
+    "decay_exp_of_neg": ("double e = exp(gt[i]);", "double e = exp(-gt[i]);"),
+    "eps_outside_root": ("1.0 / sqrt(sq + J->eps)", "1.0 / (sqrt(sq) + J->eps)"),
+    "conv_history_shift": ("raw_at(J, n, t - (KCONV - 1) + j, c)", "raw_at(J, n, t - KCONV + j, c)"),
+    "beta_not_sigmoid": ("const double beta = sigmoid(J->b[row * H + h]);",
+                         "const double beta = J->b[row * H + h];"),
+}
+
+PIN_TESTS = [
+    lambda: [pins.test_recurrence_matches_unrolled_product(T, D, s)
+             for T, D, s in [(1, 2, 0), (3, 3, 1), (8, 4, 2)]],
+    pins.test_delta_rule_retrieval_identity,
+    pins.test_beta_zero_only_decays,
+    pins.test_prologue_matches_torch_conv1d_and_scipy,
+    pins.test_gate_closed_forms,
+    pins.test_lower_bound_decay_closed_form,
+    pins.test_forward_equals_prologue_then_recurrence,
+    lambda: [pins.test_prefill_then_decode_equals_long_prefill(a, b) for a, b in [(7, 5), (1, 4)]],
+]
+
+
+def _build_mutant(old, new, tmpdir):
+    src = open(SRC).read()
+    assert old in src, "mutation anchor not found: %r" % old
+    path_c = os.path.join(tmpdir, "mut.c")
+    path_so = os.path.join(tmpdir, "libmut.so")
+    open(path_c, "w").write(src.replace(old, new))
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+                           "-o", path_so, path_c, "-lm"])
+    return path_so
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name):
+    old, new = MUTATIONS[name]
+    with tempfile.TemporaryDirectory() as d:
+        so = _build_mutant(old, new, d)
+        prev = oracle.swap_library(so)
+        caught = []
+        try:
+            for pin in PIN_TESTS:
+                try:
+                    pin()
+                except AssertionError:
+                    caught.append(pin)
+        finally:
+            oracle.swap_library(None)
+            oracle._lib = prev
+    assert caught, "no pin failed for planted mistake %r" % name

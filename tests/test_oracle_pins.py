@@ -1,0 +1,262 @@
+"""Pins for the fp64 oracle: every check here is independent of the oracle's code.
+
+The oracle restates the KDA forward pass from the AliceAI-Foundation KDA
+write-up ("二、KDA 线性注意力" section: per-token loop, gate formula, causal conv
+kernel 4 / padding 3 / no bias + SiLU, L2-normalised q/k) and the
+Ling-3.0-flash-VL config table (kda_lower_bound -5.0).  These tests pin it to
+things fixed by the mathematics or by library routines:
+
+* recurrence      -> brute-force unrolled matrix product (dense numpy algebra)
+* delta rule      -> retrieval identity with beta=1, g=0, unit key
+* decay / gate    -> beta=0 closed form, lower-bound e^{-5n} closed form,
+                     a hand-computed scalar gate, the alpha -> -inf limit
+* prologue        -> torch Conv1d (groups=channels, padding 3, truncated),
+                     scipy expit / numpy logaddexp, unit norms
+* state hand-off  -> prefill(T1) + T2 decode steps == prefill(T1 + T2)
+* varlen packing  -> packed run == separate runs (bitwise)
+"""
+
+import numpy as np
+import pytest
+import scipy.special as sp
+import torch
+
+from oracle import oracle
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------- recurrence
+
+def _brute_force(q, k, v, g, beta, S0):
+    """S_t = P(t,0) S0 + sum_s P(t,s) beta_s k_s v_s^T with A_t = (I - beta_t k_t k_t^T) diag(e^{g_t}),
+    P(t,s) = A_t A_{t-1} ... A_{s+1};  o_t = S_t^T q_t."""
+    T, D = q.shape
+    A = [(np.eye(D) - beta[t] * np.outer(k[t], k[t])) @ np.diag(np.exp(g[t])) for t in range(T)]
+
+    def P(t, s):
+        M = np.eye(D)
+        for r in range(s + 1, t + 1):
+            M = A[r] @ M
+        return M
+
+    outs, S = [], None
+    for t in range(T):
+        S = P(t, -1) @ S0 + sum(P(t, s) @ (beta[s] * np.outer(k[s], v[s])) for s in range(t + 1))
+        outs.append(S.T @ q[t])
+    return np.stack(outs), S
+
+
+@pytest.mark.parametrize("T,D,seed", [(1, 2, 0), (3, 3, 1), (8, 4, 2), (7, 4, 3)])
+def test_recurrence_matches_unrolled_product(T, D, seed):
+    r = _rng(seed)
+    q, k, v = r.standard_normal((3, T, 1, D))
+    g = -r.uniform(0.0, 2.0, (T, 1, D))
+    beta = r.uniform(0.05, 0.95, (T, 1))
+    S0 = r.standard_normal((1, 1, D, D))          # non-symmetric: a transposed S fails
+    o, S = oracle.recurrence([0, T], q, k, v, g, beta, S0)
+    o_ref, S_ref = _brute_force(q[:, 0], k[:, 0], v[:, 0], g[:, 0], beta[:, 0], S0[0, 0])
+    np.testing.assert_allclose(o[:, 0], o_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(S[0, 0], S_ref, rtol=0, atol=1e-12)
+
+
+def test_recurrence_scale_multiplies_output_only():
+    r = _rng(5)
+    T, D = 5, 3
+    q, k, v = r.standard_normal((3, T, 1, D))
+    g = -r.uniform(0, 1, (T, 1, D))
+    beta = r.uniform(0, 1, (T, 1))
+    o1, S1 = oracle.recurrence([0, T], q, k, v, g, beta, None, scale=1.0)
+    o2, S2 = oracle.recurrence([0, T], q, k, v, g, beta, None, scale=0.25)
+    np.testing.assert_allclose(o2, 0.25 * o1, rtol=1e-14, atol=0)
+    np.testing.assert_array_equal(S1, S2)
+
+
+def test_delta_rule_retrieval_identity():
+    """beta=1, g=0, unit key: reading with q = k right after the write returns v."""
+    r = _rng(7)
+    T, D = 6, 8
+    k = r.standard_normal((T, 1, D))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = r.standard_normal((T, 1, D))
+    g = np.zeros((T, 1, D))
+    beta = np.ones((T, 1))
+    S0 = r.standard_normal((1, 1, D, D))
+    o, _ = oracle.recurrence([0, T], k.copy(), k, v, g, beta, S0)
+    np.testing.assert_allclose(o, v, rtol=0, atol=1e-12)
+
+
+def test_beta_zero_only_decays():
+    r = _rng(8)
+    T, D = 5, 4
+    q, k, v = r.standard_normal((3, T, 1, D))
+    g = -r.uniform(0, 3, (T, 1, D))
+    S0 = r.standard_normal((1, 1, D, D))
+    o, S = oracle.recurrence([0, T], q, k, v, g, np.zeros((T, 1)), S0)
+    Gam = np.cumsum(g[:, 0], axis=0)                    # [T, D]
+    for t in range(T):
+        St = np.exp(Gam[t])[:, None] * S0[0, 0]
+        np.testing.assert_allclose(o[t, 0], St.T @ q[t, 0], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(S[0, 0], np.exp(Gam[-1])[:, None] * S0[0, 0], rtol=1e-12)
+
+
+# ---------------------------------------------------------------- prologue
+
+def _prologue_inputs(seed, lens, H, D, conv_std=0.5):
+    r = _rng(seed)
+    T = sum(lens)
+    HD = H * D
+    return dict(
+        cu=np.concatenate([[0], np.cumsum(lens)]).astype(np.int64),
+        q=r.standard_normal((T, HD)), k=r.standard_normal((T, HD)), v=r.standard_normal((T, HD)),
+        conv_w=r.standard_normal((3, HD, 4)) * conv_std,
+        alpha=r.standard_normal((T, H, D)), b=r.standard_normal((T, H)),
+        A_log=np.log(r.uniform(1, 16, H)), dt_bias=r.uniform(-1, 1, (H, D)))
+
+
+def _torch_conv_silu(x, w):
+    """nn.Conv1d(C, C, groups=C, kernel_size=4, padding=3, bias=False) on [T, C], output truncated to T, then SiLU."""
+    T, C = x.shape
+    xt = torch.from_numpy(x.T[None].copy())                        # [1, C, T]
+    wt = torch.from_numpy(w[:, None, :].copy())                    # [C, 1, 4]
+    y = torch.nn.functional.conv1d(xt, wt, padding=3, groups=C)[0, :, :T].T.numpy()
+    return y * sp.expit(y)
+
+
+def test_prologue_matches_torch_conv1d_and_scipy():
+    H, D, lens = 2, 8, [11, 5, 2]
+    I = _prologue_inputs(11, lens, H, D)
+    qn, kn, vc, g, beta = oracle.prologue(I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"],
+                                          I["alpha"], I["b"], I["A_log"], I["dt_bias"])
+    eps = 1e-6
+    for n in range(len(lens)):
+        a, z = I["cu"][n], I["cu"][n + 1]
+        for blk, (name, got) in enumerate((("q", qn), ("k", kn), ("v", vc))):
+            y = _torch_conv_silu(I[name][a:z], I["conv_w"][blk])      # [L, H*D]
+            y = y.reshape(z - a, H, D)
+            if name != "v":
+                y = y / np.sqrt((y * y).sum(-1, keepdims=True) + eps)
+            np.testing.assert_allclose(got[a:z], y, rtol=1e-12, atol=1e-14)
+    x = I["alpha"] + I["dt_bias"][None]
+    g_ref = np.maximum(-np.exp(I["A_log"])[None, :, None] * np.logaddexp(0.0, x), -5.0)
+    np.testing.assert_allclose(g, g_ref, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(beta, sp.expit(I["b"]), rtol=1e-14)
+
+
+def test_prologue_unit_norms():
+    H, D = 3, 16
+    I = _prologue_inputs(12, [40], H, D)
+    qn, kn, vc, _, _ = oracle.prologue(I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"],
+                                       I["alpha"], I["b"], I["A_log"], I["dt_bias"])
+    for x in (qn, kn):
+        nrm = np.linalg.norm(x, axis=-1)
+        np.testing.assert_allclose(nrm, 1.0, atol=1e-5)   # eps=1e-6 inside the root
+    assert not np.allclose(np.linalg.norm(vc, axis=-1), 1.0)
+
+
+def test_gate_closed_forms():
+    """A_log = ln 2, alpha + dt_bias = 0 -> g = -2 ln 2; alpha -> +inf -> g = -5 exactly;
+    alpha -> -inf -> g -> 0 from below."""
+    H, D = 1, 4
+    I = _prologue_inputs(13, [3], H, D)
+    I["A_log"] = np.array([np.log(2.0)])
+    I["dt_bias"] = np.array([[0.0, 0.0, 0.5, -0.5]])
+    I["alpha"] = np.array([[[0.0, 1e4, -0.5, 0.5]], [[-1e4, 0.0, 0.0, 0.0]], [[3.0, 3.0, 3.0, 3.0]]])
+    _, _, _, g, _ = oracle.prologue(I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"],
+                                    I["alpha"], I["b"], I["A_log"], I["dt_bias"])
+    assert abs(g[0, 0, 0] - (-2.0 * np.log(2.0))) < 1e-15
+    assert g[0, 0, 1] == -5.0
+    assert abs(g[0, 0, 2] - (-2.0 * np.log(2.0))) < 1e-15
+    assert abs(g[0, 0, 3] - (-2.0 * np.log(2.0))) < 1e-15
+    assert -1e-300 < g[1, 0, 0] <= 0.0
+    # 2 * softplus(3 + 0.5) = 7.06 > 5: clamped; 2 * softplus(2.5) = 5.16: clamped; 2*softplus(3)=6.1: clamped
+    assert np.all(g[2, 0] == -5.0)
+
+
+def test_lower_bound_decay_closed_form():
+    """k = 0 (zero raw inputs) and alpha -> +inf: after n steps S = e^{-5n} S0."""
+    H, D, n = 2, 4, 6
+    I = _prologue_inputs(14, [n], H, D)
+    for name in ("q", "k", "v"):
+        I[name] = np.zeros_like(I[name])
+    I["alpha"] = np.full_like(I["alpha"], 1e4)
+    S0 = _rng(15).standard_normal((1, H, D, D))
+    o, S1, _, _ = oracle.forward(I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"], I["alpha"],
+                                 I["b"], I["A_log"], I["dt_bias"], state0=S0)
+    np.testing.assert_allclose(S1, np.exp(-5.0 * n) * S0, rtol=1e-12)
+    assert np.all(o == 0.0)
+
+
+# ---------------------------------------------------------------- composition
+
+def test_forward_equals_prologue_then_recurrence():
+    H, D, lens = 2, 8, [9, 4]
+    I = _prologue_inputs(16, lens, H, D)
+    S0 = _rng(17).standard_normal((2, H, D, D)) * 0.1
+    o, S1, _, _ = oracle.forward(I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"], I["alpha"],
+                                 I["b"], I["A_log"], I["dt_bias"], state0=S0)
+    qn, kn, vc, g, beta = oracle.prologue(I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"],
+                                          I["alpha"], I["b"], I["A_log"], I["dt_bias"])
+    o2, S2 = oracle.recurrence(I["cu"], qn, kn, vc, g, beta, S0)
+    np.testing.assert_allclose(o, o2, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(S1, S2, rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("T1,T2", [(7, 5), (1, 4), (2, 1), (0, 3)])
+def test_prefill_then_decode_equals_long_prefill(T1, T2):
+    H, D = 2, 8
+    I = _prologue_inputs(18, [T1 + T2], H, D)
+    S0 = _rng(19).standard_normal((1, H, D, D)) * 0.1
+    args = lambda a, z: (I["q"][a:z], I["k"][a:z], I["v"][a:z], I["conv_w"], I["alpha"][a:z],
+                         I["b"][a:z], I["A_log"], I["dt_bias"])
+    o_long, S_long, C_long, _ = oracle.forward([0, T1 + T2], H, D, *args(0, T1 + T2), state0=S0)
+    o1, S, C, _ = oracle.forward([0, T1], H, D, *args(0, T1), state0=S0)
+    outs = [o1]
+    for t in range(T1, T1 + T2):
+        q, k, v, w, al, b, A, dt = args(t, t + 1)
+        o_t, S, C = oracle.decode_step(H, D, S, C, q, k, v, al, b, w, A, dt)
+        outs.append(o_t)
+    np.testing.assert_allclose(np.concatenate(outs), o_long, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(S, S_long, rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(C, C_long)
+
+
+def test_final_conv_state_holds_last_three_raw_tokens():
+    H, D = 2, 4
+    I = _prologue_inputs(20, [6, 2], H, D)
+    _, _, C, _ = oracle.forward(I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"], I["alpha"],
+                                I["b"], I["A_log"], I["dt_bias"])
+    raw = np.concatenate([I["q"], I["k"], I["v"]], axis=1)            # [T, 3*H*D]
+    np.testing.assert_array_equal(C[0], raw[3:6])
+    np.testing.assert_array_equal(C[1, 0], 0.0)                        # history before a 2-token sequence
+    np.testing.assert_array_equal(C[1, 1:], raw[6:8])
+
+
+def test_varlen_equals_separate_sequences():
+    H, D, lens = 2, 8, [5, 1, 12, 3]
+    I = _prologue_inputs(21, lens, H, D)
+    S0 = _rng(22).standard_normal((len(lens), H, D, D)) * 0.1
+    o, S1, C1, _ = oracle.forward(I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"], I["alpha"],
+                                  I["b"], I["A_log"], I["dt_bias"], state0=S0)
+    cu = I["cu"]
+    for n in range(len(lens)):
+        a, z = cu[n], cu[n + 1]
+        o_n, S_n, C_n, _ = oracle.forward([0, z - a], H, D, I["q"][a:z], I["k"][a:z], I["v"][a:z],
+                                          I["conv_w"], I["alpha"][a:z], I["b"][a:z], I["A_log"],
+                                          I["dt_bias"], state0=S0[n:n + 1])
+        np.testing.assert_array_equal(o[a:z], o_n)
+        np.testing.assert_array_equal(S1[n], S_n[0])
+        np.testing.assert_array_equal(C1[n], C_n[0])
+
+
+def test_thread_count_does_not_change_results():
+    H, D, lens = 4, 8, [10, 7]
+    I = _prologue_inputs(23, lens, H, D)
+    a = oracle.forward(I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"], I["alpha"], I["b"],
+                       I["A_log"], I["dt_bias"], nthreads=1)
+    b = oracle.forward(I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"], I["alpha"], I["b"],
+                       I["A_log"], I["dt_bias"], nthreads=5)
+    for x, y in zip(a[:3], b[:3]):
+        np.testing.assert_array_equal(x, y)
