@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""KDA forward benchmark on B200: prefill tokens/s (+ % of bf16 tensor peak) and
+decode-step state GB/s (+ % of HBM), one JSON line on stdout.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workloads (seeded, synthetic; see gated_delta_rule_70_b200/workloads.py):
+  prefill  B=4, T=8192, H=32, d=128, bf16 I/O, fp32 state   (the step that `value` times)
+  decode   256 sequences x 32 heads, d=128, state from a T=1024 prefill, 64 steps
+
+A "step" is one kda prefill over the whole batch: the prologue kernel
+(conv4+SiLU, L2 norm, gate, beta) followed by the recurrence kernel, issued
+through the C ABI with every input already resident in HBM.  The inputs
+(1.3 GB) are larger than L2, so no flush is needed between steps.  Per-kernel
+durations come from CUDA events recorded on the launching stream around each
+C-ABI call inside the timed region.  `e2e` repeats the step through the same
+C ABI with host (pinned) inputs: H2D copies, the prefill and the D2H read of
+o and the final state are all inside its timed region.
+
+Multi-GPU (torchrun, one process per GPU): the (sequence, head) units are
+independent, so every rank runs its own batch with no data-path collective
+(weak scaling); time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the CPU baseline) on a bounded
+sample of the same workload on this host's cores; rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HBM_FALLBACK_GBS = 6650.0
+BF16_FALLBACK_TFLOPS = 1590.0
+C = 64  # chunk length used for the algorithmic flop count
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": HBM_FALLBACK_GBS, "bf16_tflops": BF16_FALLBACK_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def prefill_flops_per_token_head(d: int, c: int = C) -> float:
+    """Algorithmic flops of the chunked form per (token, head): C(3dk + 2dv) + 6 dk dv + C^2/3."""
+    return c * (3 * d + 2 * d) + 6 * d * d + c * c / 3.0
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": float(max(smax)) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from gated_delta_rule_70_b200 import build as kbuild
+    from gated_delta_rule_70_b200 import kda
+    from gated_delta_rule_70_b200 import workloads as W
+
+    if rank == 0:
+        kbuild.build_library()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks = measured_peaks()
+
+    s = W.spec("prefill_4x8k")
+    inp = W.make_inputs(s)
+    N, H, d = s.num_seqs, s.H, s.d
+    T_total = s.total_tokens
+    up = lambda a: W.to_device(a, dev)
+    q, k, v = up(inp["q"]), up(inp["k"]), up(inp["v"])
+    conv_w, alpha, b = up(inp["conv_w"]), up(inp["alpha"]), up(inp["b"])
+    A_log, dt_bias, S0 = up(inp["A_log"]), up(inp["dt_bias"]), up(inp["S0"])
+    bf = torch.bfloat16
+    qn, kn, vc = (torch.empty((T_total, H, d), dtype=bf, device=dev) for _ in range(3))
+    g = torch.empty((T_total, H, d), dtype=torch.float32, device=dev)
+    beta = torch.empty((T_total, H), dtype=torch.float32, device=dev)
+    fc = torch.empty((N, 3, 3 * H * d), dtype=bf, device=dev)
+    o = torch.empty((T_total, H, d), dtype=bf, device=dev)
+    fs = torch.empty((N, H, d, d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        kda.prologue(q, k, v, conv_w, alpha, b, A_log, dt_bias, num_seqs=N,
+                     out=(qn, kn, vc, g, beta, fc))
+        if ev is not None:
+            ev[1].record(stream)
+        kda.recurrence(qn, kn, vc, g, beta, S0, num_seqs=N, out=o, final_state=fs)
+        if ev is not None:
+            ev[2].record(stream)
+
+    launches_per_step = 3  # prologue, conv-state copy, recurrence
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    pro_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    rec_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+
+    # ---- decode workload (state from a T=1024 prefill), timed per step
+    sd = W.spec("decode_256")
+    dinp = W.make_inputs(sd)
+    dup = lambda a: W.to_device(a, dev)
+    d_o, d_state, d_conv = kda.prefill(dup(dinp["q"]), dup(dinp["k"]), dup(dinp["v"]),
+                                       dup(dinp["conv_w"]), dup(dinp["alpha"]), dup(dinp["b"]),
+                                       dup(dinp["A_log"]), dup(dinp["dt_bias"]),
+                                       num_seqs=sd.num_seqs)
+    del dinp, d_o
+    dsteps = [W.make_decode_step(sd, i) for i in range(64)]
+    dsteps = [{kk: dup(vv) for kk, vv in x.items()} for x in dsteps]
+    d_cw, d_A, d_dt = dup(W.make_params(sd)["conv_w"]), dup(W.make_params(sd)["A_log"]), \
+        dup(W.make_params(sd)["dt_bias"])
+    d_out = torch.empty((sd.num_seqs, sd.H, sd.d), dtype=bf, device=dev)
+
+    def dstep(x):
+        kda.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["b"], d_cw, d_A, d_dt, d_state,
+                        d_conv, out=d_out)
+
+    for i in range(3):
+        dstep(dsteps[i])
+    torch.cuda.synchronize(dev)
+    de = [torch.cuda.Event(enable_timing=True) for _ in range(65)]
+    for i in range(64):
+        de[i].record(stream)
+        dstep(dsteps[i])
+    de[64].record(stream)
+    torch.cuda.synchronize(dev)
+    dec_ms = [de[i].elapsed_time(de[i + 1]) for i in range(64)]
+    clock_info = clocks.stop()
+
+    # ---- e2e through the C ABI with host buffers
+    pin = lambda t: t.detach().cpu().pin_memory()
+    hq, hk, hv, ha, hb = pin(q), pin(k), pin(v), pin(alpha), pin(b)
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hs = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+    ws = torch.empty(kda.prefill_workspace_size(
+        kda.make_shape(N, s.seq_len, H, d, bf), False), dtype=torch.uint8, device=dev)
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True); alpha.copy_(ha, non_blocking=True)
+        b.copy_(hb, non_blocking=True)
+        kda.prefill(q, k, v, conv_w, alpha, b, A_log, dt_bias, initial_state=S0, num_seqs=N,
+                    out=o, final_state=fs, workspace=ws, want_conv_state=False, check=False)
+        ho.copy_(o, non_blocking=True)
+        hs.copy_(fs, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, ha, hb))
+    d2h = ho.numel() * ho.element_size() + hs.numel() * hs.element_size()
+
+    # ---- max over ranks
+    stats = torch.tensor([elapsed_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(stats, op=torch.distributed.ReduceOp.MAX)
+    elapsed_ms, e2e_ms = float(stats[0]), float(stats[1])
+    if rank != 0:
+        return None
+
+    ms_per_step = elapsed_ms / args.steps
+    tokens = T_total * world
+    value = tokens / (ms_per_step * 1e-3)
+    flops = prefill_flops_per_token_head(d) * T_total * H
+    tc_tflops = flops / (ms_per_step * 1e-3) / 1e12
+    # algorithmic bytes per launch
+    esz = 2
+    pro_bytes = T_total * H * (4 * d * esz + esz + 3 * d * esz + 4 * d + 4) + N * 9 * H * d * esz
+    rec_bytes = T_total * H * (3 * d * esz + 4 * d + 4 + d * esz) + 2 * N * H * d * d * 4
+    pro_gbs = pro_bytes / (pro_ms * 1e-3) / 1e9
+    rec_gbs = rec_bytes / (rec_ms * 1e-3) / 1e9
+    dominant = ("recurrence", rec_ms, rec_bytes, rec_gbs) if rec_ms >= pro_ms else \
+        ("prologue", pro_ms, pro_bytes, pro_gbs)
+    dec_step_ms = float(np.median(dec_ms))
+    dec_bytes = decode_bytes(sd.num_seqs, sd.H, sd.d)
+    dec_gbs = dec_bytes / (dec_step_ms * 1e-3) / 1e9
+    line = {
+        "metric": "KDA prefill tokens/s and % bf16 TC peak; decode state GB/s vs HBM peak",
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "prefill B=4 T=8192 H=32 d=128 bf16 I/O fp32 state (S0~N(0,0.02))",
+                   "global_batch": 4 * world, "seq_len": 8192, "heads": H, "head_dim": d,
+                   "parallelism": "dp%d (independent sequences per rank)" % world,
+                   "l2": "inputs 1.3 GB > 126 MB L2, no flush"},
+        "tc": {"algorithmic_tflops": tc_tflops, "flop_per_token_head": prefill_flops_per_token_head(d),
+               "frac_of_measured_bf16": tc_tflops / peaks["bf16_tflops"],
+               "frac_of_2250_datasheet": tc_tflops / 2250.0},
+        "kernels_ms": {"prologue": pro_ms, "recurrence": rec_ms},
+        "roofline": {"kernel": dominant[0], "bound": "hbm", "achieved": dominant[3],
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dominant[3] / peaks["hbm_gbs"],
+                     "traffic": None, "algorithmic_bytes": dominant[2],
+                     "peak_source": peaks["source"] + " (burst copy)"},
+        "decode": {"workload": "256 seqs x 32 heads, d=128, fp32 state, 64 steps",
+                   "ms_per_step": dec_step_ms, "algorithmic_bytes": dec_bytes, "GB_s": dec_gbs,
+                   "frac_of_measured_hbm": dec_gbs / peaks["hbm_gbs"],
+                   "frac_of_8000_datasheet": dec_gbs / 8000.0,
+                   "tokens_per_s": sd.num_seqs / (dec_step_ms * 1e-3)},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step * args.steps + 64,
+        "clocks": clock_info,
+        "peaks": peaks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+    return line
+
+
+def decode_bytes(N, H, d, esz=2):
+    """Algorithmic bytes of one decode step: state read+write, conv state r/w, token in, o out."""
+    state = 2 * N * H * d * d * 4
+    conv = 2 * N * 3 * 3 * H * d * esz
+    tok = N * H * (3 * d * esz + d * esz + esz) + N * H * d * esz
+    return state + conv + tok
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+
+def cpu_baseline(seconds: float = 15.0, tokens: int = None):
+    """Time the fp64 oracle on a bounded sample of the prefill workload (first sequence, all 32
+    heads, the first `tokens` tokens; default the whole 8192-token sequence, about 17
+    core-seconds) on all host cores; tokens/s counts every head."""
+    from gated_delta_rule_70_b200 import workloads as W
+    from oracle import oracle
+
+    s = W.spec("prefill_4x8k")
+    cores = os.cpu_count() or 1
+    if tokens is None:
+        tokens = s.seq_len
+    t1 = tokens
+    params = W.make_params(s)
+    tok = W.make_tokens(s, 0, t1)
+    f = {kk: W.as_f64(vv) for kk, vv in {**params, **tok}.items()}
+    S0 = W.make_initial_state(s)[:1].astype(np.float64)
+    t0 = time.perf_counter()
+    _, _, _, used = oracle.forward([0, t1], s.H, s.d, f["q"], f["k"], f["v"], f["conv_w"],
+                                   f["alpha"], f["b"], f["A_log"], f["dt_bias"], state0=S0)
+    dt = time.perf_counter() - t0
+    return {"value": t1 / dt, "unit": "tokens/s", "cores": int(used), "kind": "oracle",
+            "sample": "sequence 0 of prefill B=4 T=8192 H=32 d=128: first %d tokens, all 32 heads, "
+                      "fp64 C oracle, %d threads over heads, %.1f s" % (t1, used, dt)}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return None
+    from oracle import oracle
+    oracle.build()
+    per_step_tokens = args.ref_tokens
+    for _ in range(args.warmup):
+        cpu_baseline(tokens=max(64, per_step_tokens // 4))
+    t0 = time.perf_counter()
+    samples = [cpu_baseline(tokens=per_step_tokens) for _ in range(args.steps)]
+    dt = time.perf_counter() - t0
+    value = per_step_tokens * args.steps / dt
+    cb = dict(samples[-1])
+    cb["value"] = value
+    return {
+        "impl": "reference",
+        "metric": "KDA prefill tokens/s and % bf16 TC peak; decode state GB/s vs HBM peak",
+        "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "prefill B=4 T=8192 H=32 d=128 (oracle sample: sequence 0, "
+                               "first %d tokens, all heads)" % per_step_tokens,
+                   "global_batch": 4, "seq_len": 8192, "parallelism": "host threads over heads"},
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-tokens", type=int, default=1024)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

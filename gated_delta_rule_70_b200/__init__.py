@@ -1,0 +1,9 @@
+"""B200-native (sm_100a) Kimi Delta Attention forward pass.
+
+The compute lives in ``libkda.so`` (CUDA kernels behind the C ABI declared in
+``include/kda.h``); ``gated_delta_rule_70_b200.kda`` is its ctypes binding and
+``gated_delta_rule_70_b200.workloads`` draws the seeded synthetic inputs.
+"""
+
+from .kda import (KdaError, KdaLibraryError, decode_step, load_library, prefill,  # noqa: F401
+                  prefill_workspace_size, prologue, recurrence, status_string)

@@ -1,0 +1,236 @@
+// C ABI of libkda.so (declared in include/kda.h): argument validation,
+// workspace layout and kernel dispatch.  Every step of the forward pass runs
+// in this library's CUDA kernels; there is no host-side compute path.
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "kda_common.cuh"
+#include "kda_internal.h"
+
+namespace {
+
+using namespace kda;
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+kda_status check_shape(const kda_shape *s) {
+  if (s == nullptr) return KDA_ERR_INVALID_ARGUMENT;
+  if (s->num_seqs < 0 || s->seq_len < 0 || s->num_heads < 1 || s->head_dim < 1)
+    return KDA_ERR_INVALID_ARGUMENT;
+  if (s->io_dtype != KDA_BF16 && s->io_dtype != KDA_FP32) return KDA_ERR_INVALID_ARGUMENT;
+  if (!std::isfinite(s->lower_bound) || !std::isfinite(s->l2norm_eps) || s->l2norm_eps < 0.f ||
+      !std::isfinite(s->scale))
+    return KDA_ERR_INVALID_ARGUMENT;
+  if (s->head_dim != 64 && s->head_dim != 128) return KDA_ERR_UNSUPPORTED;
+  if (s->num_heads > 64) return KDA_ERR_UNSUPPORTED;
+  return KDA_OK;
+}
+
+// Total packed tokens: dense N * seq_len, varlen seq_len.
+int64_t total_tokens(const kda_shape *s, const int32_t *cu) {
+  return cu ? (int64_t)s->seq_len : (int64_t)s->num_seqs * s->seq_len;
+}
+
+size_t esize(const kda_shape *s) { return s->io_dtype == KDA_BF16 ? 2 : 4; }
+
+struct WsLayout {
+  size_t err, qn, kn, vc, g, beta, total;
+};
+
+WsLayout ws_layout(const kda_shape *s, int64_t T) {
+  const size_t thd = (size_t)T * s->num_heads * s->head_dim;
+  WsLayout L;
+  size_t off = 0;
+  L.err = off; off += kAlign;
+  L.qn = off; off = align_up(off + thd * esize(s));
+  L.kn = off; off = align_up(off + thd * esize(s));
+  L.vc = off; off = align_up(off + thd * esize(s));
+  L.g = off; off = align_up(off + thd * 4);
+  L.beta = off; off = align_up(off + (size_t)T * s->num_heads * 4);
+  L.total = off;
+  return L;
+}
+
+#define KDA_REQUIRE(p) do { if ((p) == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT; } while (0)
+#define KDA_OPTIONAL(p) do { if ((p) != nullptr && !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT; } while (0)
+
+kda_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+PrologueArgs make_prologue_args(const kda_shape *s, int64_t T, const void *q, const void *k,
+                                const void *v, const void *conv_w, const void *alpha, const void *b,
+                                const float *A_log, const float *dt_bias, const void *conv0,
+                                const int32_t *cu) {
+  PrologueArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.N = s->num_seqs; a.H = s->num_heads; a.D = s->head_dim; a.seq_len = s->seq_len;
+  a.total_tokens = T; a.io_dtype = s->io_dtype; a.cu = cu;
+  a.q = q; a.k = k; a.v = v; a.conv_w = conv_w; a.alpha = alpha; a.b = b;
+  a.A_log = A_log; a.dt_bias = dt_bias; a.conv0 = conv0;
+  a.lower_bound = s->lower_bound; a.eps = s->l2norm_eps;
+  return a;
+}
+
+RecurrenceArgs make_recurrence_args(const kda_shape *s, int64_t T, const void *qn, const void *kn,
+                                    const void *vc, const float *g, const float *beta,
+                                    const float *state0, const int32_t *cu, void *o, float *state1) {
+  RecurrenceArgs ra;
+  std::memset(&ra, 0, sizeof ra);
+  ra.N = s->num_seqs; ra.H = s->num_heads; ra.D = s->head_dim;
+  ra.seq_len = s->seq_len; ra.total_tokens = T; ra.io_dtype = s->io_dtype;
+  ra.cu = cu; ra.qn = qn; ra.kn = kn; ra.vc = vc; ra.g = g; ra.beta = beta;
+  ra.state0 = state0; ra.scale = s->scale; ra.o = o; ra.state1 = state1;
+  return ra;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kda_prefill_workspace_size(const kda_shape *shape, int is_varlen) {
+  if (check_shape(shape) != KDA_OK) return 0;
+  const int64_t T = is_varlen ? (int64_t)shape->seq_len : (int64_t)shape->num_seqs * shape->seq_len;
+  return ws_layout(shape, T).total;
+}
+
+kda_status kda_prefill(const kda_shape *shape, const void *q, const void *k, const void *v,
+                       const void *conv_w, const void *alpha, const void *b, const float *A_log,
+                       const float *dt_bias, const float *initial_state,
+                       const void *initial_conv_state, const int32_t *cu_seqlens, void *o,
+                       float *final_state, void *final_conv_state, void *workspace,
+                       size_t workspace_bytes, void *stream_) {
+  kda_status st = check_shape(shape);
+  if (st != KDA_OK) return st;
+  if (shape->num_seqs == 0) return KDA_OK;
+  const int64_t T = total_tokens(shape, cu_seqlens);
+  if (T > 0) {
+    KDA_REQUIRE(q); KDA_REQUIRE(k); KDA_REQUIRE(v); KDA_REQUIRE(alpha); KDA_REQUIRE(b);
+    KDA_REQUIRE(o);
+  }
+  KDA_REQUIRE(conv_w); KDA_REQUIRE(A_log); KDA_REQUIRE(dt_bias); KDA_REQUIRE(final_state);
+  KDA_OPTIONAL(initial_state); KDA_OPTIONAL(initial_conv_state); KDA_OPTIONAL(final_conv_state);
+  if (cu_seqlens != nullptr && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_INVALID_ARGUMENT;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)))
+    return KDA_ERR_WORKSPACE;
+  const WsLayout L = ws_layout(shape, T);
+  if (workspace_bytes < L.total) return KDA_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  char *ws = static_cast<char *>(workspace);
+  int *err = reinterpret_cast<int *>(ws + L.err);
+
+  cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), stream);
+  if (e != cudaSuccess) return KDA_ERR_CUDA;
+
+  PrologueArgs pa = make_prologue_args(shape, T, q, k, v, conv_w, alpha, b, A_log, dt_bias,
+                                       initial_conv_state, cu_seqlens);
+  pa.qn = ws + L.qn; pa.kn = ws + L.kn; pa.vc = ws + L.vc;
+  pa.g = reinterpret_cast<float *>(ws + L.g);
+  pa.beta = reinterpret_cast<float *>(ws + L.beta);
+  pa.err = err;
+  if ((e = launch_prologue(pa, stream)) != cudaSuccess) return KDA_ERR_CUDA;
+
+  RecurrenceArgs ra = make_recurrence_args(shape, T, pa.qn, pa.kn, pa.vc, pa.g, pa.beta,
+                                           initial_state, cu_seqlens, o, final_state);
+  ra.err = err;
+  if ((e = launch_recurrence(ra, stream)) != cudaSuccess) return KDA_ERR_CUDA;
+
+  if (final_conv_state != nullptr)
+    if ((e = launch_conv_state_out(pa, final_conv_state, stream)) != cudaSuccess) return KDA_ERR_CUDA;
+  return KDA_OK;
+}
+
+kda_status kda_prefill_status(const void *workspace, void *stream_) {
+  if (workspace == nullptr) return KDA_ERR_INVALID_ARGUMENT;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  if (word == ERR_BAD_CU_SEQLENS) return KDA_ERR_INVALID_ARGUMENT;
+  if (word == ERR_TIMEOUT) return KDA_ERR_TIMEOUT;
+  return word == ERR_NONE ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_prologue(const kda_shape *shape, const void *q, const void *k, const void *v,
+                        const void *conv_w, const void *alpha, const void *b, const float *A_log,
+                        const float *dt_bias, const void *initial_conv_state,
+                        const int32_t *cu_seqlens, void *qn, void *kn, void *vc, float *g,
+                        float *beta, void *final_conv_state, void *stream_) {
+  kda_status st = check_shape(shape);
+  if (st != KDA_OK) return st;
+  const int64_t T = total_tokens(shape, cu_seqlens);
+  if (shape->num_seqs == 0) return KDA_OK;
+  if (T > 0) {
+    KDA_REQUIRE(q); KDA_REQUIRE(k); KDA_REQUIRE(v); KDA_REQUIRE(alpha); KDA_REQUIRE(b);
+    KDA_REQUIRE(qn); KDA_REQUIRE(kn); KDA_REQUIRE(vc); KDA_REQUIRE(g); KDA_REQUIRE(beta);
+  }
+  KDA_REQUIRE(conv_w); KDA_REQUIRE(A_log); KDA_REQUIRE(dt_bias);
+  KDA_OPTIONAL(initial_conv_state); KDA_OPTIONAL(final_conv_state);
+  if (cu_seqlens != nullptr && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_INVALID_ARGUMENT;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  PrologueArgs pa = make_prologue_args(shape, T, q, k, v, conv_w, alpha, b, A_log, dt_bias,
+                                       initial_conv_state, cu_seqlens);
+  pa.qn = qn; pa.kn = kn; pa.vc = vc; pa.g = g; pa.beta = beta; pa.err = nullptr;
+  if (launch_prologue(pa, stream) != cudaSuccess) return KDA_ERR_CUDA;
+  if (final_conv_state != nullptr && launch_conv_state_out(pa, final_conv_state, stream) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  return KDA_OK;
+}
+
+kda_status kda_recurrence(const kda_shape *shape, const void *qn, const void *kn, const void *vc,
+                          const float *g, const float *beta, const float *initial_state,
+                          const int32_t *cu_seqlens, void *o, float *final_state, void *stream_) {
+  kda_status st = check_shape(shape);
+  if (st != KDA_OK) return st;
+  if (shape->num_seqs == 0) return KDA_OK;
+  const int64_t T = total_tokens(shape, cu_seqlens);
+  if (T > 0) {
+    KDA_REQUIRE(qn); KDA_REQUIRE(kn); KDA_REQUIRE(vc); KDA_REQUIRE(g); KDA_REQUIRE(beta);
+    KDA_REQUIRE(o);
+  }
+  KDA_REQUIRE(final_state); KDA_OPTIONAL(initial_state);
+  if (cu_seqlens != nullptr && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_INVALID_ARGUMENT;
+  RecurrenceArgs ra = make_recurrence_args(shape, T, qn, kn, vc, g, beta, initial_state, cu_seqlens,
+                                           o, final_state);
+  return cuda_status(launch_recurrence(ra, static_cast<cudaStream_t>(stream_)));
+}
+
+kda_status kda_decode_step(const kda_shape *shape, const void *q, const void *k, const void *v,
+                           const void *alpha, const void *b, const void *conv_w,
+                           const float *A_log, const float *dt_bias, float *state,
+                           void *conv_state, void *o, void *stream_) {
+  kda_status st = check_shape(shape);
+  if (st != KDA_OK) return st;
+  if (shape->num_seqs == 0) return KDA_OK;
+  KDA_REQUIRE(q); KDA_REQUIRE(k); KDA_REQUIRE(v); KDA_REQUIRE(alpha); KDA_REQUIRE(b);
+  KDA_REQUIRE(conv_w); KDA_REQUIRE(A_log); KDA_REQUIRE(dt_bias); KDA_REQUIRE(state);
+  KDA_REQUIRE(conv_state); KDA_REQUIRE(o);
+  DecodeArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.N = shape->num_seqs; a.H = shape->num_heads; a.D = shape->head_dim; a.io_dtype = shape->io_dtype;
+  a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.b = b; a.conv_w = conv_w;
+  a.A_log = A_log; a.dt_bias = dt_bias;
+  a.lower_bound = shape->lower_bound; a.eps = shape->l2norm_eps; a.scale = shape->scale;
+  a.state = state; a.conv_state = conv_state; a.o = o;
+  return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream_)));
+}
+
+const char *kda_status_string(kda_status status) {
+  switch (status) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARGUMENT: return "KDA_ERR_INVALID_ARGUMENT: bad pointer, size or cu_seqlens";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: shape not implemented (head_dim 64/128, heads <= 64)";
+    case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA call or launch failed";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a bounded device wait gave up";
+  }
+  return "KDA: unknown status";
+}
+
+int kda_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,190 @@
+// KDA prologue: depthwise causal conv (kernel 4, no bias) + SiLU on q, k, v;
+// L2 normalisation of q and k per head; gate g = max(-exp(A_log) *
+// softplus(alpha + dt_bias), lower_bound); beta = sigmoid(b).
+//
+// Source of the operation: AliceAI-Foundation KDA write-up, section
+// "二、KDA 线性注意力" (q/k/v_conv1d with kernel 4, padding 3, no bias, SiLU;
+// use_qk_l2norm_in_kernel; the gate formula), and the Ling-3.0-flash-VL config
+// table (kda_lower_bound = -5.0).
+//
+// Streaming design: a group of d/8 threads owns one (head, 16-token tile); each
+// thread owns 8 consecutive channels and walks the tile's tokens in order,
+// keeping the 3-token conv history in registers.  All global traffic is 16-byte
+// vector loads/stores; a warp touches 512 contiguous bytes per row (two heads
+// of d = 128).  The L2 norm is a shuffle reduction inside the group.
+#include "kda_common.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+
+constexpr int PRO_TPT = 16;      // tokens per thread (one tile)
+constexpr int PRO_THREADS = 256;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(PRO_THREADS)
+prologue_kernel(PrologueArgs a) {
+  constexpr int G = D / 8;  // threads per (token, head) row
+  const int H = a.H;
+  const int64_t HD = (int64_t)H * D;
+  const int64_t total = a.total_tokens;
+  const int64_t rg = ((int64_t)blockIdx.x * PRO_THREADS + threadIdx.x) / G;
+  const int lane_in_group = threadIdx.x % G;
+  const int h = (int)(rg % H);
+  const int64_t tile = rg / H;
+  const int64_t t0 = tile * PRO_TPT;
+  if (t0 >= total) return;
+  const int64_t t1 = min(t0 + (int64_t)PRO_TPT, total);
+  const int c0 = h * D + lane_in_group * 8;  // channel within a q/k/v block
+  const T *__restrict__ conv0 = reinterpret_cast<const T *>(a.conv0);
+
+  // Validate cu_seqlens once (block 0, thread 0); bounds are clamped everywhere anyway.
+  if (a.cu != nullptr && blockIdx.x == 0 && threadIdx.x == 0 && a.err != nullptr) {
+    bool ok = a.cu[0] == 0 && (int64_t)a.cu[a.N] == total;
+    for (int n = 0; n < a.N && ok; ++n) ok = a.cu[n + 1] >= a.cu[n];
+    if (!ok) atomicExch(a.err, ERR_BAD_CU_SEQLENS);
+  }
+
+  const int n0 = seq_of_token(a.cu, a.N, a.seq_len, t0);
+  // the G lanes of this row group (all take the same trip counts)
+  const unsigned group_mask = (G == 32 ? 0xffffffffu : ((1u << G) - 1u) << ((threadIdx.x % 32) & ~(G - 1)));
+
+#pragma unroll 1
+  for (int blk = 0; blk < 3; ++blk) {
+    const T *__restrict__ x = reinterpret_cast<const T *>(blk == 0 ? a.q : (blk == 1 ? a.k : a.v));
+    T *__restrict__ y = reinterpret_cast<T *>(blk == 0 ? a.qn : (blk == 1 ? a.kn : a.vc));
+    const T *__restrict__ w = reinterpret_cast<const T *>(a.conv_w) + ((int64_t)blk * HD + c0) * KCONV;
+    float wr[8][KCONV];  // 8 channels x 4 taps = 32 contiguous elements, 2 channels per load
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      float t8[8];
+      load8(w + i * KCONV, t8);
+#pragma unroll
+      for (int j = 0; j < KCONV; ++j) { wr[i][j] = t8[j]; wr[i + 1][j] = t8[KCONV + j]; }
+    }
+    // history hist[m][i]: raw input at token (t - 3 + m), m = 0..2
+    float hist[3][8];
+    int n = n0;
+    int64_t s, e;
+    seq_bounds(a.cu, n, a.seq_len, total, s, e);
+    auto load_history = [&](int64_t t) {
+#pragma unroll
+      for (int m = 0; m < 3; ++m) {
+        const int64_t tm = t - 3 + m;
+        const int64_t slot = tm - s + 3;  // history slot; < 0 only for malformed cu_seqlens
+        if (tm >= s && tm >= 0) {
+          load8(x + tm * HD + c0, hist[m]);
+        } else if (conv0 != nullptr && slot >= 0 && slot < 3) {
+          load8(conv0 + ((int64_t)n * 3 + slot) * 3 * HD + blk * HD + c0, hist[m]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) hist[m][i] = 0.f;
+        }
+      }
+    };
+    load_history(t0);
+#pragma unroll 4
+    for (int64_t t = t0; t < t1; ++t) {
+      if (t >= e) {  // crossed into a later sequence (varlen): restart the history
+        while (n + 1 < a.N && t >= e) { ++n; seq_bounds(a.cu, n, a.seq_len, total, s, e); }
+        load_history(t);
+      }
+      float xt[8], yt[8];
+      load8_stream(x + t * HD + c0, xt);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float acc = wr[i][0] * hist[0][i];
+        acc = fmaf(wr[i][1], hist[1][i], acc);
+        acc = fmaf(wr[i][2], hist[2][i], acc);
+        acc = fmaf(wr[i][3], xt[i], acc);
+        yt[i] = silu_f(acc);
+        hist[0][i] = hist[1][i];
+        hist[1][i] = hist[2][i];
+        hist[2][i] = xt[i];
+      }
+      if (blk < 2) {
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = fmaf(yt[i], yt[i], ss);
+#pragma unroll
+        for (int off = G / 2; off >= 1; off >>= 1) ss += __shfl_xor_sync(group_mask, ss, off);
+        const float r = rsqrtf(ss + a.eps);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) yt[i] *= r;
+      }
+      store8(y + (t * H + h) * D + lane_in_group * 8, yt);
+    }
+  }
+
+  // gate and beta
+  const float negA = -expf(a.A_log[h]);
+  float bias[8];
+  load8(a.dt_bias + h * D + lane_in_group * 8, bias);
+  const T *__restrict__ alpha = reinterpret_cast<const T *>(a.alpha);
+  const T *__restrict__ bb = reinterpret_cast<const T *>(a.b);
+#pragma unroll 4
+  for (int64_t t = t0; t < t1; ++t) {
+    float al[8], gt[8];
+    load8_stream(alpha + (t * H + h) * D + lane_in_group * 8, al);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) gt[i] = gate_f(al[i] + bias[i], negA, a.lower_bound);
+    store8(a.g + (t * H + h) * D + lane_in_group * 8, gt);
+    if (lane_in_group == 0) a.beta[t * H + h] = sigmoid_f(to_f32(bb[t * H + h]));
+  }
+}
+
+// final_conv_state[n][m][c] = raw input of token (end_n - 3 + m), or the
+// incoming history / zero when the sequence is shorter than 3 tokens.
+template <typename T>
+__global__ void conv_state_out_kernel(PrologueArgs a, T *__restrict__ out) {
+  const int64_t HD = (int64_t)a.H * a.D;
+  const int64_t per_seq = 3 * 3 * HD;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= per_seq * a.N) return;
+  const int n = (int)(idx / per_seq);
+  const int m = (int)((idx / (3 * HD)) % 3);
+  const int64_t c = idx % (3 * HD);
+  int64_t s, e;
+  seq_bounds(a.cu, n, a.seq_len, a.total_tokens, s, e);
+  const int64_t t = e - 3 + m;
+  T val;
+  if (t >= s) {
+    const int blk = (int)(c / HD);
+    const T *x = reinterpret_cast<const T *>(blk == 0 ? a.q : (blk == 1 ? a.k : a.v));
+    val = x[t * HD + (c % HD)];
+  } else if (a.conv0 != nullptr) {
+    val = reinterpret_cast<const T *>(a.conv0)[((int64_t)n * 3 + (t - s + 3)) * 3 * HD + c];
+  } else {
+    val = from_f32<T>(0.f);
+  }
+  out[idx] = val;
+}
+
+cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t stream) {
+  if (a.total_tokens == 0) return cudaSuccess;
+  const int64_t tiles = (a.total_tokens + PRO_TPT - 1) / PRO_TPT;
+  const int G = a.D / 8;
+  const int64_t threads = tiles * a.H * G;
+  const int64_t blocks = (threads + PRO_THREADS - 1) / PRO_THREADS;
+  if (a.io_dtype == KDA_BF16) {
+    if (a.D == 128) prologue_kernel<__nv_bfloat16, 128><<<(unsigned)blocks, PRO_THREADS, 0, stream>>>(a);
+    else prologue_kernel<__nv_bfloat16, 64><<<(unsigned)blocks, PRO_THREADS, 0, stream>>>(a);
+  } else {
+    if (a.D == 128) prologue_kernel<float, 128><<<(unsigned)blocks, PRO_THREADS, 0, stream>>>(a);
+    else prologue_kernel<float, 64><<<(unsigned)blocks, PRO_THREADS, 0, stream>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_conv_state_out(const PrologueArgs &a, void *out, cudaStream_t stream) {
+  const int64_t n = (int64_t)a.N * 9 * a.H * a.D;
+  if (n == 0) return cudaSuccess;
+  const int threads = 256;
+  const unsigned blocks = (unsigned)((n + threads - 1) / threads);
+  if (a.io_dtype == KDA_BF16)
+    conv_state_out_kernel<__nv_bfloat16><<<blocks, threads, 0, stream>>>(a, (__nv_bfloat16 *)out);
+  else
+    conv_state_out_kernel<float><<<blocks, threads, 0, stream>>>(a, (float *)out);
+  return cudaGetLastError();
+}
+
+}  // namespace kda

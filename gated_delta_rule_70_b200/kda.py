@@ -1,0 +1,239 @@
+"""Thin Python binding of libkda.so (ctypes).
+
+Argument marshalling only: tensors are passed to the C ABI as device
+pointers, the stream is torch's current stream, and every step of the KDA
+forward pass runs in the library's CUDA kernels.  Nothing here computes on the
+host, and there is no fallback: if ``libkda.so`` is missing or fails to load,
+every call raises ``KdaLibraryError``.
+
+Names follow the C ABI in ``include/kda.h``: ``prefill``, ``prologue``,
+``recurrence``, ``decode_step``, ``prefill_workspace_size``, ``status_string``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
+_lib = None
+
+KDA_OK, KDA_ERR_INVALID_ARGUMENT, KDA_ERR_UNSUPPORTED = 0, 1, 2
+KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = 3, 4, 5
+KDA_BF16, KDA_FP32 = 0, 1
+
+EXPORTED = ["kda_prefill_workspace_size", "kda_prefill", "kda_prefill_status", "kda_prologue",
+            "kda_recurrence", "kda_decode_step", "kda_status_string", "kda_version"]
+
+
+class KdaLibraryError(RuntimeError):
+    """libkda.so is missing or could not be loaded."""
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__("%s failed: %s" % (what, status_string(status)))
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("seq_len", ctypes.c_int32),
+                ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("lower_bound", ctypes.c_float), ("l2norm_eps", ctypes.c_float),
+                ("scale", ctypes.c_float), ("io_dtype", ctypes.c_int32)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libkda.so (build it first with ``gated_delta_rule_70_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise KdaLibraryError("libkda.so not found at %s; run `python -m gated_delta_rule_70_b200.build`"
+                              % _LIB_PATH)
+    try:
+        lib = ctypes.CDLL(_LIB_PATH)
+    except OSError as e:
+        raise KdaLibraryError("cannot load %s: %s" % (_LIB_PATH, e)) from e
+    P, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    SP = ctypes.POINTER(Shape)
+    lib.kda_prefill_workspace_size.argtypes = [SP, i32]
+    lib.kda_prefill_workspace_size.restype = sz
+    lib.kda_prefill.argtypes = [SP] + [P] * 14 + [P, sz, P]
+    lib.kda_prefill.restype = i32
+    lib.kda_prefill_status.argtypes = [P, P]
+    lib.kda_prefill_status.restype = i32
+    lib.kda_prologue.argtypes = [SP] + [P] * 16 + [P]
+    lib.kda_prologue.restype = i32
+    lib.kda_recurrence.argtypes = [SP] + [P] * 9 + [P]
+    lib.kda_recurrence.restype = i32
+    lib.kda_decode_step.argtypes = [SP] + [P] * 11 + [P]
+    lib.kda_decode_step.restype = i32
+    lib.kda_status_string.argtypes = [i32]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_version.argtypes = []
+    lib.kda_version.restype = i32
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().kda_status_string(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("KDA tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("KDA tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return KDA_BF16
+    if dt == torch.float32:
+        return KDA_FP32
+    raise ValueError("io dtype must be bfloat16 or float32, got %s" % dt)
+
+
+def make_shape(num_seqs: int, seq_len: int, num_heads: int, head_dim: int, io_dtype: torch.dtype,
+               lower_bound: float = -5.0, l2norm_eps: float = 1e-6, scale: float = 1.0) -> Shape:
+    return Shape(num_seqs, seq_len, num_heads, head_dim, lower_bound, l2norm_eps, scale,
+                 _dtype_code(io_dtype))
+
+
+def prefill_workspace_size(shape: Shape, varlen: bool) -> int:
+    return int(load_library().kda_prefill_workspace_size(ctypes.byref(shape), int(varlen)))
+
+
+def _check(status: int, what: str):
+    if status != KDA_OK:
+        raise KdaError(status, what)
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, conv_w: torch.Tensor,
+            alpha: torch.Tensor, b: torch.Tensor, A_log: torch.Tensor, dt_bias: torch.Tensor,
+            initial_state: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None,
+            initial_conv_state: Optional[torch.Tensor] = None, *, num_seqs: Optional[int] = None,
+            lower_bound: float = -5.0, l2norm_eps: float = 1e-6,
+            scale: float = 1.0, want_conv_state: bool = True, out: Optional[torch.Tensor] = None,
+            final_state: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+            check: bool = True) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
+    """KDA prefill.  q, k, v: [T_total, H*d] (or [B, T, H*d] dense); alpha: [.., H, d];
+    b: [.., H].  Returns (o [T_total, H, d], final_state [N, H, d, d], final_conv_state
+    [N, 3, 3*H*d] or None).  ``check`` synchronises and raises on device-side errors."""
+    lib = load_library()
+    H, d = alpha.shape[-2], alpha.shape[-1]
+    if cu_seqlens is not None:
+        N = cu_seqlens.numel() - 1
+        T_total = q.numel() // (H * d)
+        shape = make_shape(N, T_total, H, d, q.dtype, lower_bound, l2norm_eps, scale)
+    else:
+        if q.dim() == 3:
+            N, T = q.shape[0], q.shape[1]
+        else:
+            N = 1 if num_seqs is None else num_seqs
+            T = q.numel() // (H * d) // N
+        T_total = N * T
+        shape = make_shape(N, T, H, d, q.dtype, lower_bound, l2norm_eps, scale)
+    dev = q.device
+    o = out if out is not None else torch.empty((T_total, H, d), dtype=q.dtype, device=dev)
+    fs = final_state if final_state is not None else torch.empty((N, H, d, d), dtype=torch.float32,
+                                                                 device=dev)
+    fc = (torch.empty((N, 3, 3 * H * d), dtype=q.dtype, device=dev) if want_conv_state else None)
+    ws_bytes = prefill_workspace_size(shape, cu_seqlens is not None)
+    ws = workspace
+    if ws is None or ws.numel() < ws_bytes:
+        ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    st = lib.kda_prefill(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w), _ptr(alpha),
+                         _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(initial_state),
+                         _ptr(initial_conv_state), _ptr(cu_seqlens), _ptr(o), _ptr(fs), _ptr(fc),
+                         _ptr(ws), ctypes.c_size_t(ws.numel()), _stream(dev))
+    _check(st, "kda_prefill")
+    if check:
+        _check(lib.kda_prefill_status(_ptr(ws), _stream(dev)), "kda_prefill (device)")
+    return o, fs, fc
+
+
+def _prefill_shape(q, alpha, cu_seqlens, num_seqs, lower_bound, l2norm_eps, scale):
+    H, d = alpha.shape[-2], alpha.shape[-1]
+    T_total = q.numel() // (H * d)
+    if cu_seqlens is not None:
+        return make_shape(cu_seqlens.numel() - 1, T_total, H, d, q.dtype, lower_bound, l2norm_eps,
+                          scale), T_total
+    N = (q.shape[0] if q.dim() == 3 else 1) if num_seqs is None else num_seqs
+    return make_shape(N, T_total // max(N, 1), H, d, q.dtype, lower_bound, l2norm_eps, scale), T_total
+
+
+def prologue(q, k, v, conv_w, alpha, b, A_log, dt_bias, cu_seqlens=None, initial_conv_state=None,
+             *, num_seqs: Optional[int] = None, lower_bound: float = -5.0, l2norm_eps: float = 1e-6,
+             want_conv_state: bool = False, out=None):
+    """The prologue alone: returns (qn, kn, vc [T,H,d] io dtype, g [T,H,d] fp32, beta [T,H] fp32,
+    final_conv_state [N,3,3*H*d] or None).  ``out`` may pass those six buffers preallocated."""
+    lib = load_library()
+    shape, T_total = _prefill_shape(q, alpha, cu_seqlens, num_seqs, lower_bound, l2norm_eps, 1.0)
+    H, d, N = shape.num_heads, shape.head_dim, shape.num_seqs
+    dev = q.device
+    if out is None:
+        qn, kn, vc = (torch.empty((T_total, H, d), dtype=q.dtype, device=dev) for _ in range(3))
+        g = torch.empty((T_total, H, d), dtype=torch.float32, device=dev)
+        beta = torch.empty((T_total, H), dtype=torch.float32, device=dev)
+        fc = torch.empty((N, 3, 3 * H * d), dtype=q.dtype, device=dev) if want_conv_state else None
+    else:
+        qn, kn, vc, g, beta, fc = out
+    st = lib.kda_prologue(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w), _ptr(alpha),
+                          _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(initial_conv_state),
+                          _ptr(cu_seqlens), _ptr(qn), _ptr(kn), _ptr(vc), _ptr(g), _ptr(beta),
+                          _ptr(fc), _stream(dev))
+    _check(st, "kda_prologue")
+    return qn, kn, vc, g, beta, fc
+
+
+def recurrence(qn, kn, vc, g, beta, initial_state=None, cu_seqlens=None, *,
+               num_seqs: Optional[int] = None, scale: float = 1.0, out=None, final_state=None):
+    """The recurrence on prepared inputs (what ``prologue`` returns): (o [T,H,d], final_state)."""
+    lib = load_library()
+    T_total, H, d = qn.shape
+    if cu_seqlens is not None:
+        shape = make_shape(cu_seqlens.numel() - 1, T_total, H, d, qn.dtype, scale=scale)
+    else:
+        N = 1 if num_seqs is None else num_seqs
+        shape = make_shape(N, T_total // max(N, 1), H, d, qn.dtype, scale=scale)
+    dev = qn.device
+    o = out if out is not None else torch.empty((T_total, H, d), dtype=qn.dtype, device=dev)
+    fs = final_state if final_state is not None else torch.empty(
+        (shape.num_seqs, H, d, d), dtype=torch.float32, device=dev)
+    st = lib.kda_recurrence(ctypes.byref(shape), _ptr(qn), _ptr(kn), _ptr(vc), _ptr(g), _ptr(beta),
+                            _ptr(initial_state), _ptr(cu_seqlens), _ptr(o), _ptr(fs), _stream(dev))
+    _check(st, "kda_recurrence")
+    return o, fs
+
+
+def decode_step(q, k, v, alpha, b, conv_w, A_log, dt_bias, state: torch.Tensor,
+                conv_state: torch.Tensor, *, lower_bound: float = -5.0, l2norm_eps: float = 1e-6,
+                scale: float = 1.0, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One token per sequence; updates ``state`` [N,H,d,d] and ``conv_state`` [N,3,3*H*d] in
+    place and returns o [N, H, d]."""
+    lib = load_library()
+    N, H, d = state.shape[0], state.shape[1], state.shape[2]
+    shape = make_shape(N, 1, H, d, q.dtype, lower_bound, l2norm_eps, scale)
+    o = out if out is not None else torch.empty((N, H, d), dtype=q.dtype, device=q.device)
+    st = lib.kda_decode_step(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b),
+                             _ptr(conv_w), _ptr(A_log), _ptr(dt_bias), _ptr(state),
+                             _ptr(conv_state), _ptr(o), _stream(q.device))
+    _check(st, "kda_decode_step")
+    return o

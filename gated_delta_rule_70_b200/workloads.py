@@ -205,3 +205,19 @@ def small(name: str, seq_lens: List[int], H: int, d: int, io_dtype: str = "bf16"
     """A reduced workload with the same distributions, for parity tests the oracle finishes quickly."""
     return Spec(name, io_dtype, list(seq_lens), H=H, d=d, seed=seed, s0_std=s0_std,
                 alpha_mu=alpha_mu, varlen=varlen)
+
+
+def to_device(arr: Optional[np.ndarray], device="cuda"):
+    """Upload a stored input (bf16 bits -> torch.bfloat16, fp32 -> float32, int32 as is)."""
+    import torch
+    if arr is None:
+        return None
+    if arr.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(np.ascontiguousarray(arr)).to(device)
+
+
+def from_device(t) -> np.ndarray:
+    """fp64 copy of a device tensor (bf16/fp32)."""
+    import torch
+    return t.detach().to(torch.float64).cpu().numpy()

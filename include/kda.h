@@ -1,0 +1,190 @@
+/*
+ * kda.h -- C ABI of libkda.so: the Kimi Delta Attention (KDA) forward pass on
+ * one NVIDIA B200 (sm_100a).
+ *
+ * What is computed (per sequence n, head h, token t; AliceAI-Foundation KDA
+ * write-up, section "二、KDA 线性注意力": the per-token loop, the gate formula,
+ * the depthwise causal conv with kernel 4 / padding 3 / no bias + SiLU, and
+ * L2-normalised q, k; Ling-3.0-flash-VL config table: kda_safe_gate = true,
+ * kda_lower_bound = -5.0):
+ *
+ *   prologue   x~_t[c] = sum_{j=0..3} conv_w[c][j] * x_{t-3+j}[c]   (x_{<0}: conv history)
+ *              x^_t    = SiLU(x~_t)                                   for q, k and v channels
+ *              q_t     = q^_t / sqrt(|q^_t|^2 + eps),  k_t likewise   (per head, over d)
+ *              g_t[i]  = max(-exp(A_log[h]) * softplus(alpha_t[h][i] + dt_bias[h][i]), lower_bound)
+ *              beta_t  = sigmoid(b_t[h])
+ *   recurrence S  <- diag(exp(g_t)) S                 S: [d_k, d_v] fp32 state
+ *              d_t = beta_t * (v_t - S^T k_t)
+ *              S  <- S + k_t d_t^T
+ *              o_t = scale * S^T q_t
+ *
+ * Prefill and decode share the state interface: the final_state a prefill
+ * returns seeds kda_decode_step with no recomputation (same write-up, section
+ * "五": the prefill/decode kernels share initial_state / final_state), and the
+ * conv history is carried as the raw inputs of the last 3 tokens (section "四":
+ * kernel - 1 = 3 conv states per channel).
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer is a DEVICE pointer unless stated otherwise; the caller
+ *     owns every buffer, including the workspace.  The library allocates no
+ *     memory, keeps no global state and is thread-safe across streams.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  Return codes report argument checks and launch
+ *     errors; device-side conditions are reported by kda_prefill_status().
+ *   - Argument errors are detected before any launch: NULL required pointers,
+ *     pointers not 16-byte aligned, unsupported shapes.  Nothing is launched
+ *     then and the outputs are untouched.
+ *   - Layouts are row-major and tokens are packed: dense batches are N
+ *     sequences of seq_len tokens back to back (token row = n * seq_len + t);
+ *     varlen batches give cu_seqlens [N + 1] (int32, device) with
+ *     cu_seqlens[0] = 0 and cu_seqlens[N] = total tokens.
+ *   - io dtype (kda_shape.io_dtype): bf16 or fp32 for q, k, v, conv_w, alpha,
+ *     b, o and the conv history.  A_log, dt_bias and states are always fp32.
+ *   - Channel blocks of the conv: c in [0, H*d) is q, [H*d, 2*H*d) is k,
+ *     [2*H*d, 3*H*d) is v; conv_w[blk][c][3] multiplies the current token.
+ *
+ * Supported shapes: head_dim 64 or 128; num_heads 1..64; any sequence
+ * length >= 0.  bf16 with head_dim 128 runs the tensor-core chunk kernel;
+ * other combinations run the CUDA-core token kernel (fp32 test mode).
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARGUMENT = 1, /* NULL / misaligned pointer, bad sizes, bad cu_seqlens */
+    KDA_ERR_UNSUPPORTED = 2,      /* valid but not implemented (e.g. head_dim 96) */
+    KDA_ERR_WORKSPACE = 3,        /* workspace NULL or smaller than *_workspace_size() */
+    KDA_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed */
+    KDA_ERR_TIMEOUT = 5           /* a bounded device-side wait gave up */
+} kda_status;
+
+typedef enum { KDA_BF16 = 0, KDA_FP32 = 1 } kda_dtype;
+
+typedef struct {
+    int32_t num_seqs;    /* N: sequences (dense batch size, or number of varlen sequences) */
+    int32_t seq_len;     /* dense: tokens per sequence; varlen: total packed tokens */
+    int32_t num_heads;   /* H (q, k and v heads alike) */
+    int32_t head_dim;    /* d = d_k = d_v: 64 or 128 */
+    float lower_bound;   /* safe-gate lower bound on g: -5.0f */
+    float l2norm_eps;    /* added to |x|^2 inside the square root: 1e-6f */
+    float scale;         /* output scale on S^T q: 1.0f (the pages apply none) */
+    int32_t io_dtype;    /* kda_dtype */
+} kda_shape;
+
+/* Bytes of device workspace kda_prefill() needs for this shape (0 on a bad
+ * shape).  is_varlen != 0: shape->seq_len is the packed token total (the call
+ * will pass cu_seqlens); 0: dense, num_seqs * seq_len tokens. */
+size_t kda_prefill_workspace_size(const kda_shape *shape, int is_varlen);
+
+/*
+ * kda_prefill -- prologue + recurrence over whole sequences.
+ *
+ *   q, k, v            [T_total, H*d] io dtype, raw (pre-conv) projections
+ *   conv_w             [3, H*d, 4]    io dtype
+ *   alpha              [T_total, H, d] io dtype
+ *   b                  [T_total, H]   io dtype
+ *   A_log              [H]            fp32
+ *   dt_bias            [H, d]         fp32
+ *   initial_state      [N, H, d, d]   fp32 or NULL (zeros); S[i][j], i = key, j = value
+ *   initial_conv_state [N, 3, 3*H*d]  io dtype or NULL (zeros): raw inputs of the
+ *                                     3 tokens before each sequence, oldest first
+ *   cu_seqlens         [N + 1]        int32 or NULL (dense: N sequences of seq_len)
+ *   o                  [T_total, H, d] io dtype, written
+ *   final_state        [N, H, d, d]   fp32, written; may equal initial_state
+ *   final_conv_state   [N, 3, 3*H*d]  io dtype or NULL; may not overlap the inputs
+ *   workspace          >= kda_prefill_workspace_size(shape) bytes, 256-byte aligned
+ *
+ * A sequence of length 0 copies its initial state (or zeros) to final_state.
+ * Bad cu_seqlens (not starting at 0, decreasing, or not ending at T_total)
+ * are caught on the device: every access stays clamped in bounds and
+ * kda_prefill_status() then returns KDA_ERR_INVALID_ARGUMENT.
+ */
+kda_status kda_prefill(const kda_shape *shape,
+                       const void *q, const void *k, const void *v,
+                       const void *conv_w, const void *alpha, const void *b,
+                       const float *A_log, const float *dt_bias,
+                       const float *initial_state, const void *initial_conv_state,
+                       const int32_t *cu_seqlens,
+                       void *o, float *final_state, void *final_conv_state,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * kda_prefill_status -- synchronises `stream` and reads the device error word
+ * the last kda_prefill() on this workspace left: KDA_OK, KDA_ERR_INVALID_ARGUMENT
+ * (bad cu_seqlens), KDA_ERR_TIMEOUT (a bounded wait gave up) or KDA_ERR_CUDA.
+ */
+kda_status kda_prefill_status(const void *workspace, void *stream);
+
+/*
+ * kda_prologue -- the prologue alone (conv4 + SiLU, L2 norm, gate, beta).
+ * Same inputs as kda_prefill; outputs
+ *   qn, kn, vc        [T_total, H, d] io dtype (L2-normalised q, k; conv'd v)
+ *   g                 [T_total, H, d] fp32 (after the lower-bound clamp)
+ *   beta              [T_total, H]    fp32
+ *   final_conv_state  [N, 3, 3*H*d]   io dtype or NULL, as in kda_prefill
+ * Bad cu_seqlens are clamped (no out-of-bounds access) but not reported here.
+ */
+kda_status kda_prologue(const kda_shape *shape,
+                        const void *q, const void *k, const void *v,
+                        const void *conv_w, const void *alpha, const void *b,
+                        const float *A_log, const float *dt_bias,
+                        const void *initial_conv_state, const int32_t *cu_seqlens,
+                        void *qn, void *kn, void *vc, float *g, float *beta,
+                        void *final_conv_state, void *stream);
+
+/*
+ * kda_recurrence -- the recurrence alone, on prepared per-token inputs
+ * (what kda_prologue writes):
+ *   qn, kn, vc     [T_total, H, d] io dtype
+ *   g              [T_total, H, d] fp32, gate values (log-decay, <= 0)
+ *   beta           [T_total, H]    fp32
+ *   initial_state  [N, H, d, d]    fp32 or NULL (zeros)
+ *   cu_seqlens     [N + 1] int32 or NULL (dense)
+ *   o              [T_total, H, d] io dtype, written
+ *   final_state    [N, H, d, d]    fp32, written; may equal initial_state
+ * kda_prefill is exactly kda_prologue followed by kda_recurrence.
+ */
+kda_status kda_recurrence(const kda_shape *shape,
+                          const void *qn, const void *kn, const void *vc,
+                          const float *g, const float *beta,
+                          const float *initial_state, const int32_t *cu_seqlens,
+                          void *o, float *final_state, void *stream);
+
+/*
+ * kda_decode_step -- one new token for each of N sequences, in place.
+ *
+ *   q, k, v      [N, H*d]       io dtype, raw projections of the new token
+ *   alpha        [N, H, d]      io dtype
+ *   b            [N, H]         io dtype
+ *   conv_w, A_log, dt_bias      as in kda_prefill
+ *   state        [N, H, d, d]   fp32, read and overwritten (a prefill's final_state)
+ *   conv_state   [N, 3, 3*H*d]  io dtype, read and shifted by one token in place
+ *   o            [N, H, d]      io dtype, written
+ *
+ * shape->seq_len is ignored.  Needs no workspace.
+ */
+kda_status kda_decode_step(const kda_shape *shape,
+                           const void *q, const void *k, const void *v,
+                           const void *alpha, const void *b,
+                           const void *conv_w, const float *A_log, const float *dt_bias,
+                           float *state, void *conv_state, void *o, void *stream);
+
+/* Static description of a status code (never NULL). */
+const char *kda_status_string(kda_status status);
+
+/* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

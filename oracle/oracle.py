@@ -150,3 +150,30 @@ def decode_step(H: int, D: int, state, conv_state, q, k, v, alpha, b, conv_w, A_
                            state0=state, conv0=conv_state, lower_bound=lower_bound,
                            eps=eps, scale=scale, nthreads=nthreads)
     return o, s1, c1
+
+
+def pair_inputs(f64: dict, H: int, D: int, cu, n: int, h: int, t_end: Optional[int] = None):
+    """Slice packed fp64 inputs down to one (sequence n, head h) pair (H = 1), optionally
+    keeping only the first t_end tokens of the sequence."""
+    a = int(cu[n])
+    z = int(cu[n + 1]) if t_end is None else a + t_end
+    sl = lambda x: np.ascontiguousarray(x[a:z, h * D:(h + 1) * D])
+    out = dict(q=sl(f64["q"]), k=sl(f64["k"]), v=sl(f64["v"]),
+               conv_w=np.ascontiguousarray(f64["conv_w"][:, h * D:(h + 1) * D, :]),
+               alpha=np.ascontiguousarray(f64["alpha"][a:z, h:h + 1, :]),
+               b=np.ascontiguousarray(f64["b"][a:z, h:h + 1]),
+               A_log=np.ascontiguousarray(f64["A_log"][h:h + 1]),
+               dt_bias=np.ascontiguousarray(f64["dt_bias"][h:h + 1]))
+    S0 = f64.get("S0")
+    out["state0"] = None if S0 is None else np.ascontiguousarray(S0[n:n + 1, h:h + 1])
+    return out, z - a
+
+
+def forward_pair(f64: dict, H: int, D: int, cu, n: int, h: int, t_end: Optional[int] = None,
+                 lower_bound: float = -5.0, eps: float = 1e-6, scale: float = 1.0):
+    """Oracle prefill of one (sequence, head) pair: (o [L, D], final_state [D, D])."""
+    P, L = pair_inputs(f64, H, D, cu, n, h, t_end)
+    o, s1, _, _ = forward([0, L], 1, D, P["q"], P["k"], P["v"], P["conv_w"], P["alpha"], P["b"],
+                          P["A_log"], P["dt_bias"], state0=P["state0"], lower_bound=lower_bound,
+                          eps=eps, scale=scale, nthreads=1)
+    return o[:, 0], s1[0, 0]

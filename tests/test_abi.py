@@ -1,0 +1,110 @@
+"""The C ABI library loads, exports every entry point include/kda.h declares, and
+rejects bad arguments on the host (no GPU needed: these paths return before any
+CUDA call)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_70_b200 import build, kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    hdr = open(os.path.join(ROOT, "include", "kda.h")).read()
+    hdr = re.sub(r"/\*.*?\*/", "", hdr, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z_0-9]+)\s*\(", hdr)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build_library()
+    return kda.load_library()
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ("kda_prefill", "kda_decode_step", "kda_prefill_workspace_size", "kda_status_string",
+              "kda_prologue", "kda_recurrence", "kda_prefill_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    assert set(kda.EXPORTED) >= set(_declared_functions())
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        s = kda.status_string(code)
+        assert s.startswith("KDA_")
+    assert "unknown" in kda.status_string(99)
+    assert lib.kda_version() >= 100
+
+
+def test_workspace_size_rules(lib):
+    sh = kda.make_shape(4, 8192, 32, 128, __import__("torch").bfloat16)
+    dense = kda.prefill_workspace_size(sh, False)
+    varlen = kda.prefill_workspace_size(sh, True)
+    T = 4 * 8192
+    assert dense >= T * 32 * 128 * (3 * 2 + 4) + T * 32 * 4
+    assert varlen < dense
+    bad = kda.make_shape(4, 8192, 32, 96, __import__("torch").bfloat16)
+    assert kda.prefill_workspace_size(bad, False) == 0
+
+
+def _call_prefill(lib, shape, ptrs=None, ws=None, ws_bytes=0):
+    P = ctypes.c_void_p
+    x = P(256) if ptrs is None else ptrs
+    return lib.kda_prefill(ctypes.byref(shape) if shape is not None else None,
+                           x, x, x, x, x, x, x, x, None, None, None, x, x, None,
+                           ws, ctypes.c_size_t(ws_bytes), None)
+
+
+def test_host_validation_codes(lib):
+    import torch
+    ok = kda.make_shape(1, 16, 2, 64, torch.float32)
+    assert _call_prefill(lib, None) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert _call_prefill(lib, kda.make_shape(1, 16, 2, 96, torch.float32)) == kda.KDA_ERR_UNSUPPORTED
+    assert _call_prefill(lib, kda.make_shape(1, 16, 65, 64, torch.float32)) == kda.KDA_ERR_UNSUPPORTED
+    assert _call_prefill(lib, kda.make_shape(-1, 16, 2, 64, torch.float32)) == kda.KDA_ERR_INVALID_ARGUMENT
+    bad_dtype = kda.make_shape(1, 16, 2, 64, torch.float32)
+    bad_dtype.io_dtype = 7
+    assert _call_prefill(lib, bad_dtype) == kda.KDA_ERR_INVALID_ARGUMENT
+    nan_lb = kda.make_shape(1, 16, 2, 64, torch.float32, lower_bound=float("nan"))
+    assert _call_prefill(lib, nan_lb) == kda.KDA_ERR_INVALID_ARGUMENT
+    # misaligned tensor pointer
+    assert _call_prefill(lib, ok, ptrs=ctypes.c_void_p(258)) == kda.KDA_ERR_INVALID_ARGUMENT
+    # missing / small / misaligned workspace
+    assert _call_prefill(lib, ok) == kda.KDA_ERR_WORKSPACE
+    assert _call_prefill(lib, ok, ws=ctypes.c_void_p(4096), ws_bytes=16) == kda.KDA_ERR_WORKSPACE
+    assert _call_prefill(lib, ok, ws=ctypes.c_void_p(4096 + 16), ws_bytes=1 << 30) == kda.KDA_ERR_WORKSPACE
+    # zero sequences: nothing to do
+    assert _call_prefill(lib, kda.make_shape(0, 16, 2, 64, torch.float32)) == kda.KDA_OK
+
+
+def test_decode_and_prologue_validation(lib):
+    import torch
+    P = ctypes.c_void_p
+    x, nul = P(256), None
+    sh = kda.make_shape(2, 1, 2, 128, torch.bfloat16)
+    assert lib.kda_decode_step(ctypes.byref(sh), x, x, x, x, x, x, x, x, nul, x, x, None) \
+        == kda.KDA_ERR_INVALID_ARGUMENT
+    assert lib.kda_decode_step(ctypes.byref(kda.make_shape(2, 1, 2, 32, torch.bfloat16)),
+                               x, x, x, x, x, x, x, x, x, x, x, None) == kda.KDA_ERR_UNSUPPORTED
+    sh = kda.make_shape(1, 8, 2, 64, torch.float32)
+    assert lib.kda_prologue(ctypes.byref(sh), x, x, x, x, x, x, x, x, None, None,
+                            x, x, P(260), x, x, None, None) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert lib.kda_recurrence(ctypes.byref(sh), x, x, x, x, x, None, None, x, None, None) \
+        == kda.KDA_ERR_INVALID_ARGUMENT
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    t = torch.zeros(16)
+    with pytest.raises(ValueError):
+        kda._ptr(t)

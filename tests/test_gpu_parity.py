@@ -1,0 +1,253 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Metric (per sequence n and head h): ||x_gpu - x_ref||_2 / ||x_ref||_2 over
+(t, d_v) for o and over (d_k, d_v) for the final state; the maximum over all
+(n, h) must stay within 1e-2 for bf16 I/O (fp32 accumulation) and 1e-4 in the
+fp32 test mode.  Small cases span several 64-token chunks and a ragged tail and
+run the oracle on everything; full-size workloads run the GPU in the launch
+configuration the bench times and check sampled (sequence, head) pairs, which
+the oracle computes one by one.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_70_b200 import kda
+from gated_delta_rule_70_b200 import workloads as W
+from oracle import oracle
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"bf16": 1e-2, "fp32": 1e-4}
+
+
+def _dev(arr):
+    return W.to_device(arr)
+
+
+def gpu_prefill(s: W.Spec, inp: dict, conv0=None, want_conv=True):
+    cu = _dev(inp["cu_seqlens"]) if s.varlen else None
+    o, fs, fc = kda.prefill(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["conv_w"]),
+                            _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]),
+                            _dev(inp["dt_bias"]), initial_state=_dev(inp["S0"]), cu_seqlens=cu,
+                            initial_conv_state=_dev(conv0), num_seqs=s.num_seqs,
+                            lower_bound=s.lower_bound, l2norm_eps=s.eps, scale=s.scale,
+                            want_conv_state=want_conv)
+    torch.cuda.synchronize()
+    return o, fs, fc
+
+
+def f64_inputs(inp):
+    return {k: W.as_f64(v) for k, v in inp.items() if k != "cu_seqlens"}
+
+
+def oracle_prefill(s: W.Spec, inp: dict, conv0=None):
+    f = f64_inputs(inp)
+    return oracle.forward(inp["cu_seqlens"], s.H, s.d, f["q"], f["k"], f["v"], f["conv_w"],
+                          f["alpha"], f["b"], f["A_log"], f["dt_bias"], state0=f["S0"],
+                          conv0=W.as_f64(conv0), lower_bound=s.lower_bound, eps=s.eps,
+                          scale=s.scale)
+
+
+def rel_l2(x, ref):
+    den = np.linalg.norm(ref)
+    num = np.linalg.norm(x - ref)
+    if den == 0.0:
+        return num
+    return num / den
+
+
+def max_pair_err(o_gpu, o_ref, cu, H):
+    worst = 0.0
+    for n in range(len(cu) - 1):
+        a, z = int(cu[n]), int(cu[n + 1])
+        if z == a:
+            continue
+        for h in range(H):
+            worst = max(worst, rel_l2(o_gpu[a:z, h], o_ref[a:z, h]))
+    return worst
+
+
+def max_state_err(s_gpu, s_ref):
+    N, H = s_ref.shape[:2]
+    return max(rel_l2(s_gpu[n, h], s_ref[n, h]) for n in range(N) for h in range(H))
+
+
+def check_prefill(s: W.Spec, conv0=None):
+    inp = W.make_inputs(s)
+    o, fs, fc = gpu_prefill(s, inp, conv0)
+    o_ref, s_ref, c_ref, _ = oracle_prefill(s, inp, conv0)
+    tol = TOL[s.io_dtype]
+    eo = max_pair_err(W.from_device(o), o_ref, inp["cu_seqlens"], s.H)
+    es = max_state_err(W.from_device(fs), s_ref)
+    assert eo <= tol, "o rel-L2 %.3g > %.0e" % (eo, tol)
+    assert es <= tol, "final_state rel-L2 %.3g > %.0e" % (es, tol)
+    # conv history is a copy of raw inputs: bit-exact
+    np.testing.assert_array_equal(W.from_device(fc), c_ref)
+    return eo, es
+
+
+# ------------------------------------------------------------------ prologue
+
+@pytest.mark.parametrize("io,d,lens,varlen", [("bf16", 128, [1, 2, 17, 70], True),
+                                              ("fp32", 64, [33, 5], True),
+                                              ("bf16", 128, [40, 40], False),
+                                              ("fp32", 128, [19], False)])
+def test_prologue_parity(io, d, lens, varlen):
+    s = W.small("pro", lens, H=3, d=d, io_dtype=io, seed=7, varlen=varlen)
+    inp = W.make_inputs(s)
+    rng = np.random.default_rng(3)
+    conv0 = W._store(rng.standard_normal((s.num_seqs, 3, 3 * s.H * d)).astype(np.float32), io)
+    cu = _dev(inp["cu_seqlens"]) if varlen else None
+    qn, kn, vc, g, beta, _ = kda.prologue(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]),
+                                       _dev(inp["conv_w"]), _dev(inp["alpha"]), _dev(inp["b"]),
+                                       _dev(inp["A_log"]), _dev(inp["dt_bias"]), cu_seqlens=cu,
+                                       initial_conv_state=_dev(conv0), num_seqs=s.num_seqs)
+    torch.cuda.synchronize()
+    f = f64_inputs(inp)
+    ref = oracle.prologue(inp["cu_seqlens"], s.H, d, f["q"], f["k"], f["v"], f["conv_w"],
+                          f["alpha"], f["b"], f["A_log"], f["dt_bias"], conv0=W.as_f64(conv0))
+    rt = 2.0 ** -8 if io == "bf16" else 2e-6     # bf16 outputs carry one rounding
+    for got, want in zip((qn, kn, vc), ref[:3]):
+        np.testing.assert_allclose(W.from_device(got), want, rtol=rt, atol=rt * 0.05)
+    np.testing.assert_allclose(W.from_device(g), ref[3], rtol=2e-6, atol=1e-6)
+    np.testing.assert_allclose(W.from_device(beta), ref[4], rtol=2e-6, atol=1e-7)
+
+
+# ------------------------------------------------------------------ prefill, small
+
+def test_prefill_tiny_fp32_workload():
+    """The fp32 test-mode workload exactly (B=1, T=256, H=2, d=64): 1e-4."""
+    check_prefill(W.spec("tiny_fp32"))
+
+
+@pytest.mark.parametrize("lens,H,seed", [([200, 200], 4, 11), ([64], 2, 12), ([1], 2, 13),
+                                         ([3, 130], 2, 14)])
+def test_prefill_bf16_dense(lens, H, seed):
+    s = W.small("dense", lens, H=H, d=128, seed=seed, s0_std=0.02)
+    if len(set(lens)) > 1:
+        s.varlen = True
+    check_prefill(s)
+
+
+def test_prefill_bf16_varlen_edges():
+    """Empty, 1-token, exactly-one-chunk, chunk+1 and multi-chunk sequences packed together."""
+    s = W.small("varlen", [1, 3, 64, 65, 0, 130, 17], H=2, d=128, seed=15, s0_std=0.02,
+                varlen=True)
+    check_prefill(s)
+
+
+def test_prefill_bf16_slow_decay():
+    """alpha ~ N(-2, 1): the slow-decay distribution of the long-context workload."""
+    s = W.small("slow", [300], H=2, d=128, seed=16, alpha_mu=-2.0)
+    check_prefill(s)
+
+
+def test_prefill_fp32_varlen_with_conv_history():
+    s = W.small("fp32v", [5, 70, 2], H=2, d=64, io_dtype="fp32", seed=17, s0_std=0.02,
+                varlen=True)
+    conv0 = W._store(np.random.default_rng(4).standard_normal((3, 3, 3 * 2 * 64)).astype(np.float32),
+                     "fp32")
+    check_prefill(s, conv0)
+
+
+def test_prefill_in_place_state():
+    """final_state may be the same buffer as initial_state."""
+    s = W.small("inplace", [100, 100], H=2, d=128, seed=18, s0_std=0.02)
+    inp = W.make_inputs(s)
+    st = _dev(inp["S0"]).clone()
+    o, fs, _ = kda.prefill(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["conv_w"]),
+                           _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]),
+                           _dev(inp["dt_bias"]), initial_state=st, num_seqs=2, final_state=st)
+    o_ref, s_ref, _, _ = oracle_prefill(s, inp)
+    assert max_state_err(W.from_device(st), s_ref) <= TOL["bf16"]
+    assert max_pair_err(W.from_device(o), o_ref, inp["cu_seqlens"], s.H) <= TOL["bf16"]
+
+
+def test_bad_cu_seqlens_is_reported():
+    s = W.small("bad", [10, 10, 10], H=2, d=128, seed=19, varlen=True)
+    inp = W.make_inputs(s)
+    inp["cu_seqlens"] = np.array([0, 12, 5, 30], dtype=np.int32)    # decreasing
+    with pytest.raises(kda.KdaError) as e:
+        gpu_prefill(s, inp)
+    assert e.value.status == kda.KDA_ERR_INVALID_ARGUMENT
+    inp["cu_seqlens"] = np.array([0, 10, 20, 29], dtype=np.int32)   # wrong total
+    with pytest.raises(kda.KdaError):
+        gpu_prefill(s, inp)
+    # the context is still healthy afterwards
+    check_prefill(W.small("after", [20], H=2, d=128, seed=20))
+
+
+# ------------------------------------------------------------------ decode
+
+def _decode_inputs(s: W.Spec, step):
+    return W.make_decode_step(s, step)
+
+
+def test_decode_parity_and_handoff():
+    """prefill(T1) -> decode steps on GPU vs the oracle, and against one long GPU prefill."""
+    H, d, N, T1, steps = 3, 128, 5, 70, 4
+    s = W.small("dec", [T1] * N, H=H, d=d, seed=21, s0_std=0.02)
+    inp = W.make_inputs(s)
+    o, st, cs = gpu_prefill(s, inp)
+    f = f64_inputs(inp)
+    o_ref, s_ref, c_ref, _ = oracle_prefill(s, inp)
+    for step in range(steps):
+        x = _decode_inputs(s, step)
+        o_t = kda.decode_step(_dev(x["q"]), _dev(x["k"]), _dev(x["v"]), _dev(x["alpha"]),
+                              _dev(x["b"]), _dev(inp["conv_w"]), _dev(inp["A_log"]),
+                              _dev(inp["dt_bias"]), st, cs)
+        xf = {k: W.as_f64(v) for k, v in x.items()}
+        o_r, s_ref, c_ref = oracle.decode_step(H, d, s_ref, c_ref, xf["q"], xf["k"], xf["v"],
+                                               xf["alpha"], xf["b"], f["conv_w"], f["A_log"],
+                                               f["dt_bias"])
+        torch.cuda.synchronize()
+        og = W.from_device(o_t)
+        worst = max(rel_l2(og[n, h], o_r[n, h]) for n in range(N) for h in range(H))
+        assert worst <= TOL["bf16"], (step, worst)
+        np.testing.assert_array_equal(W.from_device(cs), c_ref)
+    assert max_state_err(W.from_device(st), s_ref) <= TOL["bf16"]
+
+
+def test_decode_fp32_d64():
+    H, d, N = 2, 64, 3
+    s = W.small("dec32", [9] * N, H=H, d=d, io_dtype="fp32", seed=22, s0_std=0.1)
+    inp = W.make_inputs(s)
+    o, st, cs = gpu_prefill(s, inp)
+    f = f64_inputs(inp)
+    _, s_ref, c_ref, _ = oracle_prefill(s, inp)
+    x = _decode_inputs(s, 0)
+    o_t = kda.decode_step(_dev(x["q"]), _dev(x["k"]), _dev(x["v"]), _dev(x["alpha"]), _dev(x["b"]),
+                          _dev(inp["conv_w"]), _dev(inp["A_log"]), _dev(inp["dt_bias"]), st, cs)
+    xf = {k: W.as_f64(v) for k, v in x.items()}
+    o_r, s_r, c_r = oracle.decode_step(H, d, s_ref, c_ref, xf["q"], xf["k"], xf["v"], xf["alpha"],
+                                       xf["b"], f["conv_w"], f["A_log"], f["dt_bias"])
+    torch.cuda.synchronize()
+    og = W.from_device(o_t)
+    assert max(rel_l2(og[n, h], o_r[n, h]) for n in range(N) for h in range(H)) <= TOL["fp32"]
+    assert max_state_err(W.from_device(st), s_r) <= TOL["fp32"]
+
+
+def test_prefill_plus_decode_equals_long_prefill_gpu():
+    """The state hand-off on the GPU alone: prefill(T1) + T2 decode steps vs prefill(T1 + T2)."""
+    H, d, T1, T2 = 2, 128, 100, 6
+    s = W.small("handoff", [T1 + T2], H=H, d=d, seed=23, s0_std=0.02)
+    inp = W.make_inputs(s)
+    o_long, s_long, _ = gpu_prefill(s, inp)
+    s1 = W.small("handoff", [T1], H=H, d=d, seed=23, s0_std=0.02)
+    cut = {k: (v[:T1] if k in ("q", "k", "v", "alpha", "b") else v) for k, v in inp.items()}
+    cut["cu_seqlens"] = np.array([0, T1], dtype=np.int32)
+    o1, st, cs = gpu_prefill(s1, cut)
+    outs = [W.from_device(o1)]
+    for t in range(T1, T1 + T2):
+        o_t = kda.decode_step(_dev(inp["q"][t:t + 1]), _dev(inp["k"][t:t + 1]), _dev(inp["v"][t:t + 1]),
+                              _dev(inp["alpha"][t:t + 1]), _dev(inp["b"][t:t + 1]),
+                              _dev(inp["conv_w"]), _dev(inp["A_log"]), _dev(inp["dt_bias"]), st, cs)
+        outs.append(W.from_device(o_t))
+    torch.cuda.synchronize()
+    o_cat = np.concatenate(outs)
+    ol = W.from_device(o_long)
+    for h in range(H):
+        assert rel_l2(o_cat[:, h], ol[:, h]) <= TOL["bf16"]
+    assert max_state_err(W.from_device(st), W.from_device(s_long)) <= TOL["bf16"]
