@@ -216,7 +216,7 @@ def run_ours(args, rank, world, local_rank):
     hs = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
     e2e_steps = max(1, min(args.steps, 5))
     ws = torch.empty(kda.prefill_workspace_size(
-        kda.make_shape(N, s.seq_len, H, d, bf), False), dtype=torch.uint8, device=dev)
+        kda.make_shape(N, s.seq_lens[0], H, d, bf), False), dtype=torch.uint8, device=dev)
 
     def e2e_step():
         q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True)
@@ -325,7 +325,7 @@ def cpu_baseline(seconds: float = 15.0, tokens: int = None):
     s = W.spec("prefill_4x8k")
     cores = os.cpu_count() or 1
     if tokens is None:
-        tokens = s.seq_len
+        tokens = s.seq_lens[0]
     t1 = tokens
     params = W.make_params(s)
     tok = W.make_tokens(s, 0, t1)

@@ -87,6 +87,14 @@ RecurrenceArgs make_recurrence_args(const kda_shape *s, int64_t T, const void *q
   return ra;
 }
 
+// bf16 with head_dim 128 runs on the tensor cores; every other shape on CUDA cores.
+cudaError_t run_recurrence(const RecurrenceArgs &ra, cudaStream_t stream) {
+#ifndef KDA_TOKEN_KERNEL_ONLY
+  if (ra.io_dtype == KDA_BF16 && ra.D == 128) return launch_chunk_tc(ra, stream);
+#endif
+  return launch_recurrence(ra, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -136,7 +144,7 @@ kda_status kda_prefill(const kda_shape *shape, const void *q, const void *k, con
   RecurrenceArgs ra = make_recurrence_args(shape, T, pa.qn, pa.kn, pa.vc, pa.g, pa.beta,
                                            initial_state, cu_seqlens, o, final_state);
   ra.err = err;
-  if ((e = launch_recurrence(ra, stream)) != cudaSuccess) return KDA_ERR_CUDA;
+  if ((e = run_recurrence(ra, stream)) != cudaSuccess) return KDA_ERR_CUDA;
 
   if (final_conv_state != nullptr)
     if ((e = launch_conv_state_out(pa, final_conv_state, stream)) != cudaSuccess) return KDA_ERR_CUDA;
@@ -196,7 +204,7 @@ kda_status kda_recurrence(const kda_shape *shape, const void *qn, const void *kn
   if (cu_seqlens != nullptr && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_INVALID_ARGUMENT;
   RecurrenceArgs ra = make_recurrence_args(shape, T, qn, kn, vc, g, beta, initial_state, cu_seqlens,
                                            o, final_state);
-  return cuda_status(launch_recurrence(ra, static_cast<cudaStream_t>(stream_)));
+  return cuda_status(run_recurrence(ra, static_cast<cudaStream_t>(stream_)));
 }
 
 kda_status kda_decode_step(const kda_shape *shape, const void *q, const void *k, const void *v,

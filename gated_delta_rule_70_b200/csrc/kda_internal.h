@@ -59,6 +59,7 @@ struct DecodeArgs {
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t stream);
 cudaError_t launch_conv_state_out(const PrologueArgs &a, void *out, cudaStream_t stream);
 cudaError_t launch_recurrence(const RecurrenceArgs &a, cudaStream_t stream);
+cudaError_t launch_chunk_tc(const RecurrenceArgs &a, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 
 }  // namespace kda

@@ -44,10 +44,15 @@ _TAGS = {"q": 1, "k": 2, "v": 3, "alpha": 4, "b": 5, "conv_w": 6, "A_log": 7,
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round fp32 values to bf16 (nearest, ties to even); return the uint16 bits."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    bias = 0x7FFF + ((u >> 16) & 1)
-    return ((u + bias) >> 16).astype(np.uint16)
+    """Round finite fp32 values to bf16 (nearest, ties to even); return the uint16 bits.
+    In uint32: the largest finite pattern plus 0x8000 stays below 2**32."""
+    u = np.array(x, dtype=np.float32, copy=True).view(np.uint32)
+    lsb = u >> 16
+    lsb &= 1
+    lsb += 0x7FFF
+    u += lsb
+    u >>= 16
+    return u.astype(np.uint16)
 
 
 def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
@@ -124,11 +129,17 @@ def _store(x: np.ndarray, io_dtype: str) -> np.ndarray:
 
 
 def _token_tensor(s: Spec, tag: str, t0: int, t1: int, width: int, mu: float = 0.0,
-                  std: float = 1.0) -> np.ndarray:
-    """Rows [t0, t1) of a [total_tokens, width] N(mu, std) tensor, drawn blockwise."""
-    out = np.empty((t1 - t0, width), dtype=np.float32)
-    b0, b1 = t0 // BLOCK, (t1 - 1) // BLOCK if t1 > t0 else -1
-    for blk in range(b0, b1 + 1):
+                  std: float = 1.0, store: Optional[str] = None) -> np.ndarray:
+    """Rows [t0, t1) of a [total_tokens, width] N(mu, std) tensor, drawn blockwise (blocks in
+    parallel threads; each block has its own generator, so the result does not depend on the
+    thread count).  ``store`` = "bf16" returns bf16 bits, else fp32 values."""
+    import concurrent.futures
+    out = np.empty((t1 - t0, width), dtype=np.uint16 if store == "bf16" else np.float32)
+    if t1 <= t0:
+        return out
+    b0, b1 = t0 // BLOCK, (t1 - 1) // BLOCK
+
+    def one(blk):
         rng = np.random.default_rng([s.seed, _TAGS[tag], blk])
         lo, hi = blk * BLOCK, min((blk + 1) * BLOCK, s.total_tokens)
         block = rng.standard_normal((hi - lo, width), dtype=np.float32)
@@ -137,7 +148,16 @@ def _token_tensor(s: Spec, tag: str, t0: int, t1: int, width: int, mu: float = 0
         if mu != 0.0:
             block += np.float32(mu)
         a, z = max(lo, t0), min(hi, t1)
-        out[a - t0:z - t0] = block[a - lo:z - lo]
+        part = block[a - lo:z - lo]
+        out[a - t0:z - t0] = bf16_bits(part) if store == "bf16" else part
+
+    nblk = b1 - b0 + 1
+    if nblk == 1:
+        one(b0)
+    else:
+        import os
+        with concurrent.futures.ThreadPoolExecutor(max_workers=min(nblk, os.cpu_count() or 1)) as ex:
+            list(ex.map(one, range(b0, b1 + 1)))
     return out
 
 
@@ -157,12 +177,13 @@ def make_tokens(s: Spec, t0: int = 0, t1: Optional[int] = None) -> Dict[str, np.
     """Token-indexed inputs for packed rows [t0, t1): q, k, v [T, H*d], alpha [T, H, d], b [T, H]."""
     t1 = s.total_tokens if t1 is None else t1
     HD = s.H * s.d
+    st = s.io_dtype
     out = {}
     for tag in ("q", "k", "v"):
-        out[tag] = _store(_token_tensor(s, tag, t0, t1, HD), s.io_dtype)
-    out["alpha"] = _store(_token_tensor(s, "alpha", t0, t1, HD, mu=s.alpha_mu),
-                          s.io_dtype).reshape(t1 - t0, s.H, s.d)
-    out["b"] = _store(_token_tensor(s, "b", t0, t1, s.H), s.io_dtype)
+        out[tag] = _token_tensor(s, tag, t0, t1, HD, store=st)
+    out["alpha"] = _token_tensor(s, "alpha", t0, t1, HD, mu=s.alpha_mu,
+                                 store=st).reshape(t1 - t0, s.H, s.d)
+    out["b"] = _token_tensor(s, "b", t0, t1, s.H, store=st)
     return out
 
 
