@@ -125,6 +125,9 @@ def run_ours(args, rank, world, local_rank):
     peaks = measured_peaks()
 
     s = W.spec("prefill_4x8k")
+    if args.batch != 4:   # profiling runs: the same distributions on fewer sequences
+        s = W.Spec("prefill_%dx8k" % args.batch, "bf16", [8192] * args.batch, H=32, d=128, seed=1,
+                   s0_std=0.02)
     inp = W.make_inputs(s)
     N, H, d = s.num_seqs, s.H, s.d
     T_total = s.total_tokens
@@ -178,6 +181,12 @@ def run_ours(args, rank, world, local_rank):
     pro_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     rec_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
 
+    if args.only == "prefill":
+        clock_info = clocks.stop()
+        line = {"metric": "prefill only (profiling run)", "ms_per_step": elapsed_ms / args.steps,
+                "kernels_ms": {"prologue": pro_ms, "recurrence": rec_ms}, "clocks": clock_info}
+        return line if rank == 0 else None
+
     # ---- decode workload (state from a T=1024 prefill), timed per step
     sd = W.spec("decode_256")
     dinp = W.make_inputs(sd)
@@ -214,7 +223,7 @@ def run_ours(args, rank, world, local_rank):
     hq, hk, hv, ha, hb = pin(q), pin(k), pin(v), pin(alpha), pin(b)
     ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     hs = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
-    e2e_steps = max(1, min(args.steps, 5))
+    e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, 5))
     ws = torch.empty(kda.prefill_workspace_size(
         kda.make_shape(N, s.seq_lens[0], H, d, bf), False), dtype=torch.uint8, device=dev)
 
@@ -227,7 +236,8 @@ def run_ours(args, rank, world, local_rank):
         ho.copy_(o, non_blocking=True)
         hs.copy_(fs, non_blocking=True)
 
-    e2e_step()
+    if e2e_steps:
+        e2e_step()
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -236,12 +246,12 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps if e2e_steps else float("nan")
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, ha, hb))
     d2h = ho.numel() * ho.element_size() + hs.numel() * hs.element_size()
 
     # ---- max over ranks
-    stats = torch.tensor([elapsed_ms, e2e_ms], dtype=torch.float64, device=dev)
+    stats = torch.tensor([elapsed_ms, 0.0 if args.no_e2e else e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:
         torch.distributed.all_reduce(stats, op=torch.distributed.ReduceOp.MAX)
     elapsed_ms, e2e_ms = float(stats[0]), float(stats[1])
@@ -294,8 +304,9 @@ def run_ours(args, rank, world, local_rank):
                    "frac_of_measured_hbm": dec_gbs / peaks["hbm_gbs"],
                    "frac_of_8000_datasheet": dec_gbs / 8000.0,
                    "tokens_per_s": sd.num_seqs / (dec_step_ms * 1e-3)},
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "e2e": None if args.no_e2e else {
+            "value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps + 64,
         "clocks": clock_info,
         "peaks": peaks,
@@ -377,6 +388,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-tokens", type=int, default=1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=4,
+                    help="prefill sequences (the measured workload is 4; smaller only for profiling)")
+    ap.add_argument("--only", choices=["all", "prefill"], default="all")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

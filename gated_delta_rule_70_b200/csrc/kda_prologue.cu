@@ -17,11 +17,36 @@
 
 namespace kda {
 
-constexpr int PRO_TPT = 16;      // tokens per thread (one tile)
+constexpr int PRO_TPT = 8;       // tokens per thread (one tile)
 constexpr int PRO_THREADS = 256;
 
+// 8 consecutive elements held undecoded, so a tile's loads can all be issued
+// before any arithmetic (one round trip to HBM per tile, not one per token).
+template <typename T> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+  uint4 u;
+  __device__ __forceinline__ void load(const __nv_bfloat16 *p) { u = __ldcs(reinterpret_cast<const uint4 *>(p)); }
+  __device__ __forceinline__ void zero() { u = make_uint4(0, 0, 0, 0); }
+  __device__ __forceinline__ void get(float (&x)[8]) const {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { float2 f = __bfloat1622float2(h[i]); x[2 * i] = f.x; x[2 * i + 1] = f.y; }
+  }
+};
+template <> struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float *p) {
+    a = __ldcs(reinterpret_cast<const float4 *>(p));
+    b = __ldcs(reinterpret_cast<const float4 *>(p + 4));
+  }
+  __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ void get(float (&x)[8]) const {
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+};
+
 template <typename T, int D>
-__global__ void __launch_bounds__(PRO_THREADS)
+__global__ void __launch_bounds__(PRO_THREADS, 2)
 prologue_kernel(PrologueArgs a) {
   constexpr int G = D / 8;  // threads per (token, head) row
   const int H = a.H;
@@ -82,14 +107,9 @@ prologue_kernel(PrologueArgs a) {
       }
     };
     load_history(t0);
-#pragma unroll 4
-    for (int64_t t = t0; t < t1; ++t) {
-      if (t >= e) {  // crossed into a later sequence (varlen): restart the history
-        while (n + 1 < a.N && t >= e) { ++n; seq_bounds(a.cu, n, a.seq_len, total, s, e); }
-        load_history(t);
-      }
-      float xt[8], yt[8];
-      load8_stream(x + t * HD + c0, xt);
+    // conv + SiLU (+ L2 norm for q, k) of one token whose raw input is xt
+    auto emit = [&](int64_t t, const float (&xt)[8]) {
+      float yt[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float acc = wr[i][0] * hist[0][i];
@@ -112,6 +132,30 @@ prologue_kernel(PrologueArgs a) {
         for (int i = 0; i < 8; ++i) yt[i] *= r;
       }
       store8(y + (t * H + h) * D + lane_in_group * 8, yt);
+    };
+    if (t0 + PRO_TPT <= e && t1 - t0 == PRO_TPT) {
+      // whole tile inside one sequence: issue every load, then compute
+      Raw8<T> raw[PRO_TPT];
+#pragma unroll
+      for (int j = 0; j < PRO_TPT; ++j) raw[j].load(x + (t0 + j) * HD + c0);
+#pragma unroll
+      for (int j = 0; j < PRO_TPT; ++j) {
+        float xt[8];
+        raw[j].get(xt);
+        emit(t0 + j, xt);
+      }
+    } else {
+      // tile crosses a sequence boundary or the end: token by token
+#pragma unroll 1
+      for (int64_t t = t0; t < t1; ++t) {
+        if (t >= e) {
+          while (n + 1 < a.N && t >= e) { ++n; seq_bounds(a.cu, n, a.seq_len, total, s, e); }
+          load_history(t);
+        }
+        float xt[8];
+        load8(x + t * HD + c0, xt);
+        emit(t, xt);
+      }
     }
   }
 
@@ -121,14 +165,28 @@ prologue_kernel(PrologueArgs a) {
   load8(a.dt_bias + h * D + lane_in_group * 8, bias);
   const T *__restrict__ alpha = reinterpret_cast<const T *>(a.alpha);
   const T *__restrict__ bb = reinterpret_cast<const T *>(a.b);
-#pragma unroll 4
-  for (int64_t t = t0; t < t1; ++t) {
+  Raw8<T> araw[PRO_TPT];
+  float bvals[PRO_TPT];
+#pragma unroll
+  for (int j = 0; j < PRO_TPT; ++j) {
+    if (t0 + j < t1) {
+      araw[j].load(alpha + ((t0 + j) * H + h) * D + lane_in_group * 8);
+      bvals[j] = lane_in_group == 0 ? to_f32(bb[(t0 + j) * H + h]) : 0.f;
+    } else {
+      araw[j].zero();
+      bvals[j] = 0.f;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < PRO_TPT; ++j) {
+    const int64_t t = t0 + j;
+    if (t >= t1) break;
     float al[8], gt[8];
-    load8_stream(alpha + (t * H + h) * D + lane_in_group * 8, al);
+    araw[j].get(al);
 #pragma unroll
     for (int i = 0; i < 8; ++i) gt[i] = gate_f(al[i] + bias[i], negA, a.lower_bound);
     store8(a.g + (t * H + h) * D + lane_in_group * 8, gt);
-    if (lane_in_group == 0) a.beta[t * H + h] = sigmoid_f(to_f32(bb[t * H + h]));
+    if (lane_in_group == 0) a.beta[t * H + h] = sigmoid_f(bvals[j]);
   }
 }
 
