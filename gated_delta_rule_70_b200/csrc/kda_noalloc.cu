@@ -1,0 +1,120 @@
+// kda_prefill_noalloc: the prefill for callers that cannot allocate device
+// memory.
+//
+// kda_prefill asks the caller for a workspace: the prologue's outputs (q, k, v
+// after conv / normalisation, the gate and beta) and the error word live
+// there between the prologue and recurrence kernels.  Some callers cannot
+// provide one: code running where cudaMalloc is forbidden or unavailable
+// (inside a host callback, under an allocator that must not grow, or in an
+// embedding that owns all device memory and hands out only input/output
+// buffers).  This entry point takes its scratch from a fixed-size array in
+// device memory that belongs to the library instead.
+//
+// The array below is reserved on every GPU that loads the library, for as long
+// as the library stays loaded.  Host code may not take its address directly:
+// on the host the name `g_prefill_scratch` is only a stand-in, so the device
+// address is obtained once per device with cudaGetSymbolAddress (while that
+// device is current) and then passed to the kernels as a plain pointer.
+#include <mutex>
+
+#include "kda_common.cuh"
+#include "kda_internal.h"
+
+namespace {
+
+using namespace kda;
+
+static __device__ __align__(256) unsigned char g_prefill_scratch[KDA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_setup_mu;
+void *g_scratch_addr[kMaxDevices] = {};
+
+// Device address of this device's copy of the scratch array (set up on first use).
+cudaError_t scratch_address(void **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_prefill_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+constexpr size_t kAlign = 256;
+inline size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+inline bool ok16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" kda_status kda_prefill_noalloc(
+    const kda_shape *s, const void *q, const void *k, const void *v, const void *conv_w,
+    const void *alpha, const void *b, const float *A_log, const float *dt_bias,
+    const float *initial_state, const void *initial_conv_state, const int32_t *cu_seqlens, void *o,
+    float *final_state, void *final_conv_state, void *stream_) {
+  if (s == nullptr || s->num_seqs < 0 || s->seq_len < 0 || s->num_heads < 1 ||
+      (s->io_dtype != KDA_BF16 && s->io_dtype != KDA_FP32))
+    return KDA_ERR_INVALID_ARGUMENT;
+  if (s->head_dim != 64 && s->head_dim != 128) return KDA_ERR_UNSUPPORTED;
+  if (s->num_heads > 64) return KDA_ERR_UNSUPPORTED;
+  if (s->num_seqs == 0) return KDA_OK;
+  const int64_t T = cu_seqlens ? (int64_t)s->seq_len : (int64_t)s->num_seqs * s->seq_len;
+  const size_t es = s->io_dtype == KDA_BF16 ? 2 : 4;
+  const size_t thd = (size_t)T * s->num_heads * s->head_dim;
+  // scratch layout: error word | qn | kn | vc | g | beta
+  const size_t off_qn = kAlign, off_kn = up(off_qn + thd * es), off_vc = up(off_kn + thd * es);
+  const size_t off_g = up(off_vc + thd * es), off_b = up(off_g + thd * 4);
+  const size_t need = up(off_b + (size_t)T * s->num_heads * 4);
+  if (need > KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_WORKSPACE;
+  if (T > 0 && (!q || !k || !v || !alpha || !b || !o || !ok16(q) || !ok16(k) || !ok16(v) ||
+                !ok16(alpha) || !ok16(b) || !ok16(o)))
+    return KDA_ERR_INVALID_ARGUMENT;
+  if (!conv_w || !A_log || !dt_bias || !final_state || !ok16(conv_w) || !ok16(A_log) ||
+      !ok16(dt_bias) || !ok16(final_state) || !ok16(initial_state) || !ok16(initial_conv_state) ||
+      !ok16(final_conv_state))
+    return KDA_ERR_INVALID_ARGUMENT;
+  if (cu_seqlens != nullptr && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return KDA_ERR_INVALID_ARGUMENT;
+
+  void *base = nullptr;
+  if (scratch_address(&base) != cudaSuccess) return KDA_ERR_CUDA;
+  char *ws = static_cast<char *>(base);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  // The array keeps the previous call's contents; only the error word must start at zero.
+  if (cudaMemsetAsync(ws, 0, sizeof(int), stream) != cudaSuccess) return KDA_ERR_CUDA;
+
+  PrologueArgs pa{};
+  pa.N = s->num_seqs; pa.H = s->num_heads; pa.D = s->head_dim; pa.seq_len = s->seq_len;
+  pa.total_tokens = T; pa.io_dtype = s->io_dtype; pa.cu = cu_seqlens;
+  pa.q = q; pa.k = k; pa.v = v; pa.conv_w = conv_w; pa.alpha = alpha; pa.b = b;
+  pa.A_log = A_log; pa.dt_bias = dt_bias; pa.conv0 = initial_conv_state;
+  pa.lower_bound = s->lower_bound; pa.eps = s->l2norm_eps;
+  pa.qn = ws + off_qn; pa.kn = ws + off_kn; pa.vc = ws + off_vc;
+  pa.g = reinterpret_cast<float *>(ws + off_g);
+  pa.beta = reinterpret_cast<float *>(ws + off_b);
+  pa.err = reinterpret_cast<int *>(ws);
+  if (launch_prologue(pa, stream) != cudaSuccess) return KDA_ERR_CUDA;
+
+  RecurrenceArgs ra{};
+  ra.N = s->num_seqs; ra.H = s->num_heads; ra.D = s->head_dim; ra.seq_len = s->seq_len;
+  ra.total_tokens = T; ra.io_dtype = s->io_dtype; ra.cu = cu_seqlens;
+  ra.qn = pa.qn; ra.kn = pa.kn; ra.vc = pa.vc; ra.g = pa.g; ra.beta = pa.beta;
+  ra.state0 = initial_state; ra.scale = s->scale; ra.o = o; ra.state1 = final_state;
+  ra.err = pa.err;
+#ifndef KDA_TOKEN_KERNEL_ONLY
+  const cudaError_t e = (s->io_dtype == KDA_BF16 && s->head_dim == 128) ? launch_chunk_tc(ra, stream)
+                                                                         : launch_recurrence(ra, stream);
+#else
+  const cudaError_t e = launch_recurrence(ra, stream);
+#endif
+  if (e != cudaSuccess) return KDA_ERR_CUDA;
+  if (final_conv_state != nullptr && launch_conv_state_out(pa, final_conv_state, stream) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  return KDA_OK;
+}

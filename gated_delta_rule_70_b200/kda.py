@@ -26,7 +26,8 @@ KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = 3, 4, 5
 KDA_BF16, KDA_FP32 = 0, 1
 
 EXPORTED = ["kda_prefill_workspace_size", "kda_prefill", "kda_prefill_status", "kda_prologue",
-            "kda_recurrence", "kda_decode_step", "kda_status_string", "kda_version"]
+            "kda_recurrence", "kda_decode_step", "kda_status_string", "kda_version",
+            "kda_prefill_noalloc"]
 
 
 class KdaLibraryError(RuntimeError):

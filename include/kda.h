@@ -177,6 +177,40 @@ kda_status kda_decode_step(const kda_shape *shape,
                            const void *conv_w, const float *A_log, const float *dt_bias,
                            float *state, void *conv_state, void *o, void *stream);
 
+/*
+ * kda_prefill_noalloc -- kda_prefill for callers that cannot allocate device
+ * memory.  The pages describe no such variant; it exists for embeddings where
+ * cudaMalloc is not allowed or not possible (a caller that owns all device
+ * memory and lends the library only its inputs and outputs, code running
+ * under an allocator that must not grow, a host callback).
+ *
+ * Same arguments and results as kda_prefill minus the workspace: the
+ * prologue's intermediate tensors live in a library-owned array of
+ * KDA_NOALLOC_SCRATCH_BYTES in device memory, which every GPU that loads the
+ * library holds until the library is unloaded.  The call allocates nothing.
+ *
+ *   - A shape whose intermediates need more than KDA_NOALLOC_SCRATCH_BYTES
+ *     (bf16, d = 128: about 1.25 KiB per token per head, e.g. 800 tokens at
+ *     32 heads) returns KDA_ERR_WORKSPACE and launches nothing.
+ *   - The first call on each device looks up that device's address of the
+ *     array (cudaGetSymbolAddress, with the device current).  Make that first
+ *     call before any stream capture.
+ *   - All calls share the one array and it keeps the previous call's
+ *     contents; calls that overlap on the GPU (other streams, other threads)
+ *     race with each other.  Serialise them.
+ *   - Device-side conditions (bad cu_seqlens, a bounded wait that gave up)
+ *     are not reported by this entry point; use kda_prefill to see them.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (32u << 20)
+kda_status kda_prefill_noalloc(const kda_shape *shape,
+                               const void *q, const void *k, const void *v,
+                               const void *conv_w, const void *alpha, const void *b,
+                               const float *A_log, const float *dt_bias,
+                               const float *initial_state, const void *initial_conv_state,
+                               const int32_t *cu_seqlens,
+                               void *o, float *final_state, void *final_conv_state,
+                               void *stream);
+
 /* Static description of a status code (never NULL). */
 const char *kda_status_string(kda_status status);
 
