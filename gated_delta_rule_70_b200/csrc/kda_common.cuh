@@ -81,12 +81,31 @@ __device__ __forceinline__ void store8(float *p, const float (&x)[8]) {
   *reinterpret_cast<float4 *>(p + 4) = make_float4(x[4], x[5], x[6], x[7]);
 }
 
-// softplus(x) = log(1 + e^x) in the overflow-free form max(x, 0) + log1p(e^{-|x|}).
-__device__ __forceinline__ float softplus_f(float x) {
-  return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));
+// Elementwise math on the special-function unit: 2^x and log2(x) by their
+// hardware approximations (relative error about 2^-22) and an approximate
+// division; every function below is built from its definition on top of them.
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
-__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + expf(-x)); }
-__device__ __forceinline__ float silu_f(float x) { return x / (1.f + expf(-x)); }
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// softplus(x) = log(1 + e^x) in the overflow-free form max(x, 0) + log(1 + e^{-|x|}).
+__device__ __forceinline__ float softplus_f(float x) {
+  return fmaxf(x, 0.f) + kLn2 * lg2_approx(1.f + ex2_approx(-fabsf(x) * kLog2e));
+}
+// sigmoid(x) = 1 / (1 + e^{-x}); for x -> -inf the denominator is +inf and the result 0.
+__device__ __forceinline__ float sigmoid_f(float x) {
+  return __fdividef(1.f, 1.f + ex2_approx(-x * kLog2e));
+}
+// SiLU(x) = x sigmoid(x)
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.f + ex2_approx(-x * kLog2e)); }
 
 // Gate: g = max(-exp(A_log) * softplus(alpha + dt_bias), lower_bound); negA = -exp(A_log).
 __device__ __forceinline__ float gate_f(float alpha_plus_bias, float negA, float lower_bound) {
