@@ -143,6 +143,8 @@ def run_ours(args, rank, world, local_rank):
     o = torch.empty((T_total, H, d), dtype=bf, device=dev)
     fs = torch.empty((N, H, d, d), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    rws = torch.empty(kda.recurrence_workspace_size(kda.make_shape(N, s.seq_lens[0], H, d, bf), False),
+                      dtype=torch.uint8, device=dev)
 
     def step(ev=None):
         if ev is not None:
@@ -151,11 +153,11 @@ def run_ours(args, rank, world, local_rank):
                      out=(qn, kn, vc, g, beta, fc))
         if ev is not None:
             ev[1].record(stream)
-        kda.recurrence(qn, kn, vc, g, beta, S0, num_seqs=N, out=o, final_state=fs)
+        kda.recurrence(qn, kn, vc, g, beta, S0, num_seqs=N, out=o, final_state=fs, workspace=rws)
         if ev is not None:
             ev[2].record(stream)
 
-    launches_per_step = 3  # prologue, conv-state copy, recurrence
+    launches_per_step = 4  # prologue, conv-state copy, chunk_prep, state_pass
 
     for _ in range(args.warmup):
         step()

@@ -6,4 +6,5 @@ The compute lives in ``libkda.so`` (CUDA kernels behind the C ABI declared in
 """
 
 from .kda import (KdaError, KdaLibraryError, decode_step, load_library, prefill,  # noqa: F401
-                  prefill_workspace_size, prologue, recurrence, status_string)
+                  prefill_workspace_size, prologue, recurrence, recurrence_workspace_size,
+                  status_string)

@@ -38,24 +38,6 @@ int64_t total_tokens(const kda_shape *s, const int32_t *cu) {
 
 size_t esize(const kda_shape *s) { return s->io_dtype == KDA_BF16 ? 2 : 4; }
 
-struct WsLayout {
-  size_t err, qn, kn, vc, g, beta, total;
-};
-
-WsLayout ws_layout(const kda_shape *s, int64_t T) {
-  const size_t thd = (size_t)T * s->num_heads * s->head_dim;
-  WsLayout L;
-  size_t off = 0;
-  L.err = off; off += kAlign;
-  L.qn = off; off = align_up(off + thd * esize(s));
-  L.kn = off; off = align_up(off + thd * esize(s));
-  L.vc = off; off = align_up(off + thd * esize(s));
-  L.g = off; off = align_up(off + thd * 4);
-  L.beta = off; off = align_up(off + (size_t)T * s->num_heads * 4);
-  L.total = off;
-  return L;
-}
-
 #define KDA_REQUIRE(p) do { if ((p) == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT; } while (0)
 #define KDA_OPTIONAL(p) do { if ((p) != nullptr && !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT; } while (0)
 
@@ -87,14 +69,6 @@ RecurrenceArgs make_recurrence_args(const kda_shape *s, int64_t T, const void *q
   return ra;
 }
 
-// bf16 with head_dim 128 runs on the tensor cores; every other shape on CUDA cores.
-cudaError_t run_recurrence(const RecurrenceArgs &ra, cudaStream_t stream) {
-#ifndef KDA_TOKEN_KERNEL_ONLY
-  if (ra.io_dtype == KDA_BF16 && ra.D == 128) return launch_chunk_tc(ra, stream);
-#endif
-  return launch_recurrence(ra, stream);
-}
-
 }  // namespace
 
 extern "C" {
@@ -102,7 +76,15 @@ extern "C" {
 size_t kda_prefill_workspace_size(const kda_shape *shape, int is_varlen) {
   if (check_shape(shape) != KDA_OK) return 0;
   const int64_t T = is_varlen ? (int64_t)shape->seq_len : (int64_t)shape->num_seqs * shape->seq_len;
-  return ws_layout(shape, T).total;
+  return workspace_layout(shape->num_seqs, shape->num_heads, shape->head_dim, shape->seq_len, T,
+                          shape->io_dtype, is_varlen != 0, true).total;
+}
+
+size_t kda_recurrence_workspace_size(const kda_shape *shape, int is_varlen) {
+  if (check_shape(shape) != KDA_OK) return 0;
+  const int64_t T = is_varlen ? (int64_t)shape->seq_len : (int64_t)shape->num_seqs * shape->seq_len;
+  return workspace_layout(shape->num_seqs, shape->num_heads, shape->head_dim, shape->seq_len, T,
+                          shape->io_dtype, is_varlen != 0, false).total;
 }
 
 kda_status kda_prefill(const kda_shape *shape, const void *q, const void *k, const void *v,
@@ -124,7 +106,9 @@ kda_status kda_prefill(const kda_shape *shape, const void *q, const void *k, con
   if (cu_seqlens != nullptr && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_INVALID_ARGUMENT;
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)))
     return KDA_ERR_WORKSPACE;
-  const WsLayout L = ws_layout(shape, T);
+  const bool varlen = cu_seqlens != nullptr;
+  const WsLayout L = workspace_layout(shape->num_seqs, shape->num_heads, shape->head_dim,
+                                      shape->seq_len, T, shape->io_dtype, varlen, true);
   if (workspace_bytes < L.total) return KDA_ERR_WORKSPACE;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   char *ws = static_cast<char *>(workspace);
@@ -144,7 +128,7 @@ kda_status kda_prefill(const kda_shape *shape, const void *q, const void *k, con
   RecurrenceArgs ra = make_recurrence_args(shape, T, pa.qn, pa.kn, pa.vc, pa.g, pa.beta,
                                            initial_state, cu_seqlens, o, final_state);
   ra.err = err;
-  if ((e = run_recurrence(ra, stream)) != cudaSuccess) return KDA_ERR_CUDA;
+  if ((e = run_recurrence(ra, varlen, ws, L, stream)) != cudaSuccess) return KDA_ERR_CUDA;
 
   if (final_conv_state != nullptr)
     if ((e = launch_conv_state_out(pa, final_conv_state, stream)) != cudaSuccess) return KDA_ERR_CUDA;
@@ -191,7 +175,8 @@ kda_status kda_prologue(const kda_shape *shape, const void *q, const void *k, co
 
 kda_status kda_recurrence(const kda_shape *shape, const void *qn, const void *kn, const void *vc,
                           const float *g, const float *beta, const float *initial_state,
-                          const int32_t *cu_seqlens, void *o, float *final_state, void *stream_) {
+                          const int32_t *cu_seqlens, void *o, float *final_state, void *workspace,
+                          size_t workspace_bytes, void *stream_) {
   kda_status st = check_shape(shape);
   if (st != KDA_OK) return st;
   if (shape->num_seqs == 0) return KDA_OK;
@@ -202,9 +187,19 @@ kda_status kda_recurrence(const kda_shape *shape, const void *qn, const void *kn
   }
   KDA_REQUIRE(final_state); KDA_OPTIONAL(initial_state);
   if (cu_seqlens != nullptr && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_INVALID_ARGUMENT;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)))
+    return KDA_ERR_WORKSPACE;
+  const bool varlen = cu_seqlens != nullptr;
+  const WsLayout L = workspace_layout(shape->num_seqs, shape->num_heads, shape->head_dim,
+                                      shape->seq_len, T, shape->io_dtype, varlen, false);
+  if (workspace_bytes < L.total) return KDA_ERR_WORKSPACE;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  char *ws = static_cast<char *>(workspace);
+  if (cudaMemsetAsync(ws + L.err, 0, sizeof(int), stream) != cudaSuccess) return KDA_ERR_CUDA;
   RecurrenceArgs ra = make_recurrence_args(shape, T, qn, kn, vc, g, beta, initial_state, cu_seqlens,
                                            o, final_state);
-  return cuda_status(run_recurrence(ra, static_cast<cudaStream_t>(stream_)));
+  ra.err = reinterpret_cast<int *>(ws + L.err);
+  return cuda_status(run_recurrence(ra, varlen, ws, L, stream));
 }
 
 kda_status kda_decode_step(const kda_shape *shape, const void *q, const void *k, const void *v,

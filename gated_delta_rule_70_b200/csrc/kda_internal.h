@@ -1,6 +1,7 @@
 // Internal launch interface between the C ABI (kda_api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -56,10 +57,84 @@ struct DecodeArgs {
   void *o;                   // [N, H, D]
 };
 
+// Tensor-core chunk path (bf16, head_dim 128): chunk_prep writes one record
+// per (chunk, head); state_pass runs the sequential state chain over them.
+struct PrepArgs {
+  int N, H, seq_len;
+  int64_t total_tokens;
+  const int32_t *cu;         // [N + 1] or nullptr (dense)
+  const int32_t *chunk_cu;   // [N + 1] chunk prefix (varlen) or nullptr (dense)
+  const void *qn, *kn, *vc;  // [T, H, 128] bf16
+  const float *g, *beta;     // [T, H, 128], [T, H]
+  void *records;             // [max_slots][H] records of chunkfmt::REC_STRIDE bytes
+  int64_t max_slots;         // record slots (set by the launcher)
+  int *err;
+};
+
+struct StateArgs {
+  int N, H, seq_len;
+  int64_t total_tokens;
+  const int32_t *cu, *chunk_cu;
+  const void *records;
+  int64_t max_slots;         // record slots in the workspace (chunks beyond are not read)
+  const float *state0;       // [N, H, 128, 128] or nullptr
+  float scale;
+  void *o;                   // [T, H, 128] bf16
+  float *state1;
+  int *err;
+};
+
+// Bytes of one chunk record and the number of record slots a shape needs.
+constexpr size_t kChunkRecordBytes = 74752;
+inline int64_t max_chunk_slots(int N, int64_t total_tokens, int seq_len, bool varlen) {
+  return varlen ? (total_tokens + 63) / 64 + N : (int64_t)N * ((seq_len + 63) / 64);
+}
+
+// Workspace layout (byte offsets, 256-aligned):
+//   error word | qn | kn | vc | g | beta   (prologue outputs; with_prologue only)
+//   | chunk table (N+1 int32) | chunk records    (tensor-core path only)
+struct WsLayout {
+  size_t err, qn, kn, vc, g, beta, chunk_cu, records, total;
+  bool tc;   // bf16 with head_dim 128: the tensor-core chunk path
+};
+inline WsLayout workspace_layout(int N, int H, int D, int seq_len, int64_t T, int io_dtype,
+                                 bool varlen, bool with_prologue) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t es = io_dtype == KDA_BF16 ? 2 : 4;
+  const size_t thd = (size_t)T * H * D;
+  WsLayout L{};
+  L.tc = io_dtype == KDA_BF16 && D == 128;
+  size_t off = 256;  // error word
+  L.err = 0;
+  if (with_prologue) {
+    L.qn = off; off = up(off + thd * es);
+    L.kn = off; off = up(off + thd * es);
+    L.vc = off; off = up(off + thd * es);
+    L.g = off; off = up(off + thd * 4);
+    L.beta = off; off = up(off + (size_t)T * H * 4);
+  }
+  if (L.tc) {
+    L.chunk_cu = off; off = up(off + (size_t)(N + 1) * 4);
+    off = (off + 1023) / 1024 * 1024;
+    L.records = off;
+    off += (size_t)max_chunk_slots(N, T, seq_len, varlen) * H * kChunkRecordBytes;
+  }
+  L.total = off;
+  return L;
+}
+
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t stream);
+cudaError_t launch_chunk_table(const int32_t *cu, int N, int64_t total, int32_t *chunk_cu,
+                               cudaStream_t stream);
+cudaError_t launch_chunk_prep(PrepArgs a, int64_t max_chunks, cudaStream_t stream);
+cudaError_t launch_state_pass(const StateArgs &a, cudaStream_t stream);
 cudaError_t launch_conv_state_out(const PrologueArgs &a, void *out, cudaStream_t stream);
 cudaError_t launch_recurrence(const RecurrenceArgs &a, cudaStream_t stream);
-cudaError_t launch_chunk_tc(const RecurrenceArgs &a, cudaStream_t stream);
+// The recurrence (a4-a8) for RecurrenceArgs `ra` with workspace `ws` laid out by
+// workspace_layout(): tensor-core chunk path for bf16 / head_dim 128, else the
+// CUDA-core token kernel.
+cudaError_t run_recurrence(const RecurrenceArgs &ra, bool varlen, char *ws, const WsLayout &L,
+                           cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 
 }  // namespace kda

@@ -47,8 +47,6 @@ cudaError_t scratch_address(void **out) {
   return cudaSuccess;
 }
 
-constexpr size_t kAlign = 256;
-inline size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 inline bool ok16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
@@ -65,13 +63,10 @@ extern "C" kda_status kda_prefill_noalloc(
   if (s->num_heads > 64) return KDA_ERR_UNSUPPORTED;
   if (s->num_seqs == 0) return KDA_OK;
   const int64_t T = cu_seqlens ? (int64_t)s->seq_len : (int64_t)s->num_seqs * s->seq_len;
-  const size_t es = s->io_dtype == KDA_BF16 ? 2 : 4;
-  const size_t thd = (size_t)T * s->num_heads * s->head_dim;
-  // scratch layout: error word | qn | kn | vc | g | beta
-  const size_t off_qn = kAlign, off_kn = up(off_qn + thd * es), off_vc = up(off_kn + thd * es);
-  const size_t off_g = up(off_vc + thd * es), off_b = up(off_g + thd * 4);
-  const size_t need = up(off_b + (size_t)T * s->num_heads * 4);
-  if (need > KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_WORKSPACE;
+  const bool varlen = cu_seqlens != nullptr;
+  const WsLayout L = workspace_layout(s->num_seqs, s->num_heads, s->head_dim, s->seq_len, T,
+                                      s->io_dtype, varlen, true);
+  if (L.total > KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_WORKSPACE;
   if (T > 0 && (!q || !k || !v || !alpha || !b || !o || !ok16(q) || !ok16(k) || !ok16(v) ||
                 !ok16(alpha) || !ok16(b) || !ok16(o)))
     return KDA_ERR_INVALID_ARGUMENT;
@@ -87,7 +82,7 @@ extern "C" kda_status kda_prefill_noalloc(
   char *ws = static_cast<char *>(base);
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   // The array keeps the previous call's contents; only the error word must start at zero.
-  if (cudaMemsetAsync(ws, 0, sizeof(int), stream) != cudaSuccess) return KDA_ERR_CUDA;
+  if (cudaMemsetAsync(ws + L.err, 0, sizeof(int), stream) != cudaSuccess) return KDA_ERR_CUDA;
 
   PrologueArgs pa{};
   pa.N = s->num_seqs; pa.H = s->num_heads; pa.D = s->head_dim; pa.seq_len = s->seq_len;
@@ -95,10 +90,10 @@ extern "C" kda_status kda_prefill_noalloc(
   pa.q = q; pa.k = k; pa.v = v; pa.conv_w = conv_w; pa.alpha = alpha; pa.b = b;
   pa.A_log = A_log; pa.dt_bias = dt_bias; pa.conv0 = initial_conv_state;
   pa.lower_bound = s->lower_bound; pa.eps = s->l2norm_eps;
-  pa.qn = ws + off_qn; pa.kn = ws + off_kn; pa.vc = ws + off_vc;
-  pa.g = reinterpret_cast<float *>(ws + off_g);
-  pa.beta = reinterpret_cast<float *>(ws + off_b);
-  pa.err = reinterpret_cast<int *>(ws);
+  pa.qn = ws + L.qn; pa.kn = ws + L.kn; pa.vc = ws + L.vc;
+  pa.g = reinterpret_cast<float *>(ws + L.g);
+  pa.beta = reinterpret_cast<float *>(ws + L.beta);
+  pa.err = reinterpret_cast<int *>(ws + L.err);
   if (launch_prologue(pa, stream) != cudaSuccess) return KDA_ERR_CUDA;
 
   RecurrenceArgs ra{};
@@ -107,12 +102,7 @@ extern "C" kda_status kda_prefill_noalloc(
   ra.qn = pa.qn; ra.kn = pa.kn; ra.vc = pa.vc; ra.g = pa.g; ra.beta = pa.beta;
   ra.state0 = initial_state; ra.scale = s->scale; ra.o = o; ra.state1 = final_state;
   ra.err = pa.err;
-#ifndef KDA_TOKEN_KERNEL_ONLY
-  const cudaError_t e = (s->io_dtype == KDA_BF16 && s->head_dim == 128) ? launch_chunk_tc(ra, stream)
-                                                                         : launch_recurrence(ra, stream);
-#else
-  const cudaError_t e = launch_recurrence(ra, stream);
-#endif
+  const cudaError_t e = run_recurrence(ra, varlen, ws, L, stream);
   if (e != cudaSuccess) return KDA_ERR_CUDA;
   if (final_conv_state != nullptr && launch_conv_state_out(pa, final_conv_state, stream) != cudaSuccess)
     return KDA_ERR_CUDA;

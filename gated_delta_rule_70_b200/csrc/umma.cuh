@@ -244,6 +244,16 @@ __device__ __forceinline__ void tma_load_3d(void *dst_smem, const CUtensorMap *m
          "r"(smem_u32(mbar))
       : "memory");
 }
+// Contiguous bulk copy global -> shared (addresses 16-byte aligned, bytes a multiple
+// of 16), completing on `mbar` as transaction bytes.
+__device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src, uint32_t bytes,
+                                         uint64_t *mbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      :: "r"(smem_u32(dst_smem)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes),
+         "r"(smem_u32(mbar))
+      : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -26,8 +26,8 @@ KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = 3, 4, 5
 KDA_BF16, KDA_FP32 = 0, 1
 
 EXPORTED = ["kda_prefill_workspace_size", "kda_prefill", "kda_prefill_status", "kda_prologue",
-            "kda_recurrence", "kda_decode_step", "kda_status_string", "kda_version",
-            "kda_prefill_noalloc"]
+            "kda_recurrence", "kda_recurrence_workspace_size", "kda_decode_step",
+            "kda_status_string", "kda_version", "kda_prefill_noalloc"]
 
 
 class KdaLibraryError(RuntimeError):
@@ -73,8 +73,10 @@ def load_library():
     lib.kda_prefill_status.restype = i32
     lib.kda_prologue.argtypes = [SP] + [P] * 16 + [P]
     lib.kda_prologue.restype = i32
-    lib.kda_recurrence.argtypes = [SP] + [P] * 9 + [P]
+    lib.kda_recurrence.argtypes = [SP] + [P] * 9 + [P, sz, P]
     lib.kda_recurrence.restype = i32
+    lib.kda_recurrence_workspace_size.argtypes = [SP, i32]
+    lib.kda_recurrence_workspace_size.restype = sz
     lib.kda_decode_step.argtypes = [SP] + [P] * 11 + [P]
     lib.kda_decode_step.restype = i32
     lib.kda_status_string.argtypes = [i32]
@@ -204,8 +206,13 @@ def prologue(q, k, v, conv_w, alpha, b, A_log, dt_bias, cu_seqlens=None, initial
     return qn, kn, vc, g, beta, fc
 
 
+def recurrence_workspace_size(shape: Shape, varlen: bool) -> int:
+    return int(load_library().kda_recurrence_workspace_size(ctypes.byref(shape), int(varlen)))
+
+
 def recurrence(qn, kn, vc, g, beta, initial_state=None, cu_seqlens=None, *,
-               num_seqs: Optional[int] = None, scale: float = 1.0, out=None, final_state=None):
+               num_seqs: Optional[int] = None, scale: float = 1.0, out=None, final_state=None,
+               workspace: Optional[torch.Tensor] = None):
     """The recurrence on prepared inputs (what ``prologue`` returns): (o [T,H,d], final_state)."""
     lib = load_library()
     T_total, H, d = qn.shape
@@ -218,8 +225,13 @@ def recurrence(qn, kn, vc, g, beta, initial_state=None, cu_seqlens=None, *,
     o = out if out is not None else torch.empty((T_total, H, d), dtype=qn.dtype, device=dev)
     fs = final_state if final_state is not None else torch.empty(
         (shape.num_seqs, H, d, d), dtype=torch.float32, device=dev)
+    ws_bytes = recurrence_workspace_size(shape, cu_seqlens is not None)
+    ws = workspace
+    if ws is None or ws.numel() < ws_bytes:
+        ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     st = lib.kda_recurrence(ctypes.byref(shape), _ptr(qn), _ptr(kn), _ptr(vc), _ptr(g), _ptr(beta),
-                            _ptr(initial_state), _ptr(cu_seqlens), _ptr(o), _ptr(fs), _stream(dev))
+                            _ptr(initial_state), _ptr(cu_seqlens), _ptr(o), _ptr(fs), _ptr(ws),
+                            ctypes.c_size_t(ws.numel()), _stream(dev))
     _check(st, "kda_recurrence")
     return o, fs
 

@@ -150,13 +150,18 @@ kda_status kda_prologue(const kda_shape *shape,
  *   cu_seqlens     [N + 1] int32 or NULL (dense)
  *   o              [T_total, H, d] io dtype, written
  *   final_state    [N, H, d, d]    fp32, written; may equal initial_state
- * kda_prefill is exactly kda_prologue followed by kda_recurrence.
+ *   workspace      >= kda_recurrence_workspace_size(shape, varlen) bytes,
+ *                  256-byte aligned (per-chunk records of the tensor-core path)
+ * kda_prefill is kda_prologue followed by kda_recurrence.  kda_prefill_status()
+ * reads this workspace's error word the same way.
  */
+size_t kda_recurrence_workspace_size(const kda_shape *shape, int is_varlen);
 kda_status kda_recurrence(const kda_shape *shape,
                           const void *qn, const void *kn, const void *vc,
                           const float *g, const float *beta,
                           const float *initial_state, const int32_t *cu_seqlens,
-                          void *o, float *final_state, void *stream);
+                          void *o, float *final_state,
+                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * kda_decode_step -- one new token for each of N sequences, in place.
@@ -190,7 +195,7 @@ kda_status kda_decode_step(const kda_shape *shape,
  * library holds until the library is unloaded.  The call allocates nothing.
  *
  *   - A shape whose intermediates need more than KDA_NOALLOC_SCRATCH_BYTES
- *     (bf16, d = 128: about 1.25 KiB per token per head, e.g. 800 tokens at
+ *     (bf16, d = 128: about 2.4 KiB per token per head, e.g. 400 tokens at
  *     32 heads) returns KDA_ERR_WORKSPACE and launches nothing.
  *   - The first call on each device looks up that device's address of the
  *     array (cudaGetSymbolAddress, with the device current).  Make that first

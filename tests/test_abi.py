@@ -99,8 +99,10 @@ def test_decode_and_prologue_validation(lib):
     sh = kda.make_shape(1, 8, 2, 64, torch.float32)
     assert lib.kda_prologue(ctypes.byref(sh), x, x, x, x, x, x, x, x, None, None,
                             x, x, P(260), x, x, None, None) == kda.KDA_ERR_INVALID_ARGUMENT
-    assert lib.kda_recurrence(ctypes.byref(sh), x, x, x, x, x, None, None, x, None, None) \
-        == kda.KDA_ERR_INVALID_ARGUMENT
+    assert lib.kda_recurrence(ctypes.byref(sh), x, x, x, x, x, None, None, x, None, x,
+                              ctypes.c_size_t(1 << 20), None) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert lib.kda_recurrence(ctypes.byref(sh), x, x, x, x, x, None, None, x, x, None,
+                              ctypes.c_size_t(0), None) == kda.KDA_ERR_WORKSPACE
 
 
 def test_binding_refuses_cpu_tensors(lib):
