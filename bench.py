@@ -8,12 +8,12 @@ Workloads (seeded, synthetic; see gated_delta_rule_70_b200/workloads.py):
   prefill  B=4, T=8192, H=32, d=128, bf16 I/O, fp32 state   (the step that `value` times)
   decode   256 sequences x 32 heads, d=128, state from a T=1024 prefill, 64 steps
 
-A "step" is one kda prefill over the whole batch: the prologue kernel
-(conv4+SiLU, L2 norm, gate, beta) followed by the recurrence kernel, issued
-through the C ABI with every input already resident in HBM.  The inputs
-(1.3 GB) are larger than L2, so no flush is needed between steps.  Per-kernel
-durations come from CUDA events recorded on the launching stream around each
-C-ABI call inside the timed region.  `e2e` repeats the step through the same
+A "step" is one kda_prefill call over the whole batch (chunk_prep with the
+fused prologue, the state pass, the final conv-state copy), issued through the
+C ABI with every input already resident in HBM.  The inputs (1.3 GB) are
+larger than L2, so no flush is needed between steps.  Per-kernel durations come
+from CUDA events the library records on the launching stream between its
+kernels (kda_kernel_timing) inside the timed region.  `e2e` repeats the step through the same
 C ABI with host (pinned) inputs: H2D copies, the prefill and the D2H read of
 o and the final state are all inside its timed region.
 
@@ -136,28 +136,22 @@ def run_ours(args, rank, world, local_rank):
     conv_w, alpha, b = up(inp["conv_w"]), up(inp["alpha"]), up(inp["b"])
     A_log, dt_bias, S0 = up(inp["A_log"]), up(inp["dt_bias"]), up(inp["S0"])
     bf = torch.bfloat16
-    qn, kn, vc = (torch.empty((T_total, H, d), dtype=bf, device=dev) for _ in range(3))
-    g = torch.empty((T_total, H, d), dtype=torch.float32, device=dev)
-    beta = torch.empty((T_total, H), dtype=torch.float32, device=dev)
     fc = torch.empty((N, 3, 3 * H * d), dtype=bf, device=dev)
     o = torch.empty((T_total, H, d), dtype=bf, device=dev)
     fs = torch.empty((N, H, d, d), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    rws = torch.empty(kda.recurrence_workspace_size(kda.make_shape(N, s.seq_lens[0], H, d, bf), False),
-                      dtype=torch.uint8, device=dev)
+    ws = torch.empty(kda.prefill_workspace_size(kda.make_shape(N, s.seq_lens[0], H, d, bf), False),
+                     dtype=torch.uint8, device=dev)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        kda.prologue(q, k, v, conv_w, alpha, b, A_log, dt_bias, num_seqs=N,
-                     out=(qn, kn, vc, g, beta, fc))
+        kda.prefill(q, k, v, conv_w, alpha, b, A_log, dt_bias, initial_state=S0, num_seqs=N,
+                    out=o, final_state=fs, final_conv_state=fc, workspace=ws, check=False)
         if ev is not None:
             ev[1].record(stream)
-        kda.recurrence(qn, kn, vc, g, beta, S0, num_seqs=N, out=o, final_state=fs, workspace=rws)
-        if ev is not None:
-            ev[2].record(stream)
 
-    launches_per_step = 4  # prologue, conv-state copy, chunk_prep, state_pass
+    launches_per_step = 3  # chunk_prep (with the prologue), state_pass, final conv-state copy
 
     for _ in range(args.warmup):
         step()
@@ -166,10 +160,11 @@ def run_ours(args, rank, world, local_rank):
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.3)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
+    kda.kernel_timing(True)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
@@ -180,13 +175,15 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
-    pro_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
-    rec_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    call_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    timed_calls, prep_ms, state_ms = kda.kernel_times()
+    kda.kernel_timing(False)
 
     if args.only == "prefill":
         clock_info = clocks.stop()
         line = {"metric": "prefill only (profiling run)", "ms_per_step": elapsed_ms / args.steps,
-                "kernels_ms": {"prologue": pro_ms, "recurrence": rec_ms}, "clocks": clock_info}
+                "kernels_ms": {"prefill_call": call_ms, "chunk_prep": prep_ms, "state_pass": state_ms},
+                "clocks": clock_info}
         return line if rank == 0 else None
 
     # ---- decode workload (state from a T=1024 prefill), timed per step
@@ -226,8 +223,6 @@ def run_ours(args, rank, world, local_rank):
     ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     hs = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
     e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, 5))
-    ws = torch.empty(kda.prefill_workspace_size(
-        kda.make_shape(N, s.seq_lens[0], H, d, bf), False), dtype=torch.uint8, device=dev)
 
     def e2e_step():
         q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True)
@@ -265,14 +260,18 @@ def run_ours(args, rank, world, local_rank):
     value = tokens / (ms_per_step * 1e-3)
     flops = prefill_flops_per_token_head(d) * T_total * H
     tc_tflops = flops / (ms_per_step * 1e-3) / 1e12
-    # algorithmic bytes per launch
+    # algorithmic bytes per launch ("Rooflines"): chunk_prep reads the raw
+    # q, k, v, alpha, b of every token and writes one record per (chunk, head); the state
+    # pass reads the records and the initial state and writes o and the final state.
     esz = 2
-    pro_bytes = T_total * H * (4 * d * esz + esz + 3 * d * esz + 4 * d + 4) + N * 9 * H * d * esz
-    rec_bytes = T_total * H * (3 * d * esz + 4 * d + 4 + d * esz) + 2 * N * H * d * d * 4
-    pro_gbs = pro_bytes / (pro_ms * 1e-3) / 1e9
-    rec_gbs = rec_bytes / (rec_ms * 1e-3) / 1e9
-    dominant = ("recurrence", rec_ms, rec_bytes, rec_gbs) if rec_ms >= pro_ms else \
-        ("prologue", pro_ms, pro_bytes, pro_gbs)
+    chunks = N * ((s.seq_lens[0] + 63) // 64)
+    rec_written = 74240
+    prep_bytes = T_total * H * (4 * d * esz + esz) + chunks * H * rec_written
+    state_bytes = chunks * H * rec_written + T_total * H * d * esz + 2 * N * H * d * d * 4
+    prep_gbs = prep_bytes / (prep_ms * 1e-3) / 1e9 if prep_ms > 0 else 0.0
+    state_gbs = state_bytes / (state_ms * 1e-3) / 1e9 if state_ms > 0 else 0.0
+    dominant = ("chunk_prep", prep_ms, prep_bytes, prep_gbs) if prep_ms >= state_ms else \
+        ("state_pass", state_ms, state_bytes, state_gbs)
     dec_step_ms = float(np.median(dec_ms))
     dec_bytes = decode_bytes(sd.num_seqs, sd.H, sd.d)
     dec_gbs = dec_bytes / (dec_step_ms * 1e-3) / 1e9
@@ -296,7 +295,8 @@ def run_ours(args, rank, world, local_rank):
         "tc": {"algorithmic_tflops": tc_tflops, "flop_per_token_head": prefill_flops_per_token_head(d),
                "frac_of_measured_bf16": tc_tflops / peaks["bf16_tflops"],
                "frac_of_2250_datasheet": tc_tflops / 2250.0},
-        "kernels_ms": {"prologue": pro_ms, "recurrence": rec_ms},
+        "kernels_ms": {"prefill_call": call_ms, "chunk_prep": prep_ms, "state_pass": state_ms,
+                       "timed_calls": timed_calls},
         "roofline": {"kernel": dominant[0], "bound": "hbm", "achieved": dominant[3],
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dominant[3] / peaks["hbm_gbs"],
                      "traffic": None, "algorithmic_bytes": dominant[2],

@@ -14,7 +14,6 @@ namespace {
 using namespace kda;
 
 constexpr size_t kAlign = 256;
-inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -35,8 +34,6 @@ kda_status check_shape(const kda_shape *s) {
 int64_t total_tokens(const kda_shape *s, const int32_t *cu) {
   return cu ? (int64_t)s->seq_len : (int64_t)s->num_seqs * s->seq_len;
 }
-
-size_t esize(const kda_shape *s) { return s->io_dtype == KDA_BF16 ? 2 : 4; }
 
 #define KDA_REQUIRE(p) do { if ((p) == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT; } while (0)
 #define KDA_OPTIONAL(p) do { if ((p) != nullptr && !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT; } while (0)
@@ -66,6 +63,7 @@ RecurrenceArgs make_recurrence_args(const kda_shape *s, int64_t T, const void *q
   ra.seq_len = s->seq_len; ra.total_tokens = T; ra.io_dtype = s->io_dtype;
   ra.cu = cu; ra.qn = qn; ra.kn = kn; ra.vc = vc; ra.g = g; ra.beta = beta;
   ra.state0 = state0; ra.scale = s->scale; ra.o = o; ra.state1 = state1;
+  ra.lower_bound = s->lower_bound;
   return ra;
 }
 
@@ -77,14 +75,14 @@ size_t kda_prefill_workspace_size(const kda_shape *shape, int is_varlen) {
   if (check_shape(shape) != KDA_OK) return 0;
   const int64_t T = is_varlen ? (int64_t)shape->seq_len : (int64_t)shape->num_seqs * shape->seq_len;
   return workspace_layout(shape->num_seqs, shape->num_heads, shape->head_dim, shape->seq_len, T,
-                          shape->io_dtype, is_varlen != 0, true).total;
+                          shape->io_dtype, shape->lower_bound, is_varlen != 0, true).total;
 }
 
 size_t kda_recurrence_workspace_size(const kda_shape *shape, int is_varlen) {
   if (check_shape(shape) != KDA_OK) return 0;
   const int64_t T = is_varlen ? (int64_t)shape->seq_len : (int64_t)shape->num_seqs * shape->seq_len;
   return workspace_layout(shape->num_seqs, shape->num_heads, shape->head_dim, shape->seq_len, T,
-                          shape->io_dtype, is_varlen != 0, false).total;
+                          shape->io_dtype, shape->lower_bound, is_varlen != 0, false).total;
 }
 
 kda_status kda_prefill(const kda_shape *shape, const void *q, const void *k, const void *v,
@@ -108,7 +106,8 @@ kda_status kda_prefill(const kda_shape *shape, const void *q, const void *k, con
     return KDA_ERR_WORKSPACE;
   const bool varlen = cu_seqlens != nullptr;
   const WsLayout L = workspace_layout(shape->num_seqs, shape->num_heads, shape->head_dim,
-                                      shape->seq_len, T, shape->io_dtype, varlen, true);
+                                      shape->seq_len, T, shape->io_dtype, shape->lower_bound,
+                                      varlen, true);
   if (workspace_bytes < L.total) return KDA_ERR_WORKSPACE;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   char *ws = static_cast<char *>(workspace);
@@ -119,20 +118,11 @@ kda_status kda_prefill(const kda_shape *shape, const void *q, const void *k, con
 
   PrologueArgs pa = make_prologue_args(shape, T, q, k, v, conv_w, alpha, b, A_log, dt_bias,
                                        initial_conv_state, cu_seqlens);
-  pa.qn = ws + L.qn; pa.kn = ws + L.kn; pa.vc = ws + L.vc;
-  pa.g = reinterpret_cast<float *>(ws + L.g);
-  pa.beta = reinterpret_cast<float *>(ws + L.beta);
   pa.err = err;
-  if ((e = launch_prologue(pa, stream)) != cudaSuccess) return KDA_ERR_CUDA;
-
-  RecurrenceArgs ra = make_recurrence_args(shape, T, pa.qn, pa.kn, pa.vc, pa.g, pa.beta,
+  RecurrenceArgs ra = make_recurrence_args(shape, T, nullptr, nullptr, nullptr, nullptr, nullptr,
                                            initial_state, cu_seqlens, o, final_state);
   ra.err = err;
-  if ((e = run_recurrence(ra, varlen, ws, L, stream)) != cudaSuccess) return KDA_ERR_CUDA;
-
-  if (final_conv_state != nullptr)
-    if ((e = launch_conv_state_out(pa, final_conv_state, stream)) != cudaSuccess) return KDA_ERR_CUDA;
-  return KDA_OK;
+  return cuda_status(run_prefill(pa, ra, final_conv_state, varlen, ws, L, stream));
 }
 
 kda_status kda_prefill_status(const void *workspace, void *stream_) {
@@ -191,7 +181,8 @@ kda_status kda_recurrence(const kda_shape *shape, const void *qn, const void *kn
     return KDA_ERR_WORKSPACE;
   const bool varlen = cu_seqlens != nullptr;
   const WsLayout L = workspace_layout(shape->num_seqs, shape->num_heads, shape->head_dim,
-                                      shape->seq_len, T, shape->io_dtype, varlen, false);
+                                      shape->seq_len, T, shape->io_dtype, shape->lower_bound,
+                                      varlen, false);
   if (workspace_bytes < L.total) return KDA_ERR_WORKSPACE;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   char *ws = static_cast<char *>(workspace);

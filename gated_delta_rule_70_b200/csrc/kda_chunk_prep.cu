@@ -15,26 +15,37 @@
 // e^{Gamma_C} of each (chunk, head) as one record, already in the
 // shared-memory image the state pass copies in.
 //
+// Prologue (fused variant, the prefill entry points): the chunk's raw q, k, v
+// (with the 3 tokens before it for the causal conv) and alpha arrive by TMA;
+// conv4 + SiLU, the L2 norm of q and k, the gate and beta are computed here,
+// so those intermediates never travel through device memory.  The other
+// variant reads them prepared (the recurrence entry point).
+//
 // Numerics: Gamma reaches 64 * (-5) = -320 inside a chunk, so e^{-Gamma}
 // overflows fp32.  The pairwise factor e^{Gamma_t - Gamma_s} is only ever split
 // around a reference close to both tokens: 16-token sub-blocks I with r_I =
-// Gamma at the end of block I-1.  Diagonal blocks use (q|k)_t e^{Gamma_t - r_I}
-// against k_s e^{r_I - Gamma_s} (factors within e^{+-80}); a row in block I
-// against earlier blocks uses r_I on both sides (factors <= 1).  Exponentials
-// run on the special-function unit in base 2; every other decay factor is a
-// product of terms ordered so that no intermediate overflows.
+// Gamma at the end of block I-1 (r_0 = 0).  Diagonal blocks use
+// (q|k)_t e^{Gamma_t - r_I} against k_s e^{r_I - Gamma_s} (factors within e^{+-88});
+// a row in block I against an earlier block J uses r_I on both sides (factors
+// <= 1).  Per element only two exponentials are taken, e^{Gamma_t - r_I} and
+// e^{r_{I+1} - Gamma_t}; every other factor is one of them times a per-channel
+// constant of the chunk (e^{r_I}, e^{r_I - r_{I+1}}, ...), all in base 2 on the
+// special-function unit.
 //
 // Structure: one CTA of 8 warps per (chunk, head), two CTAs per SM so that one
 // item's memory and tensor-core waits overlap the other's arithmetic.
 // Tensor-core work (tcgen05, fp32 accumulation in TMEM):
 //   [Lq; Lk] x R_all^T (M=128, N=160, K=128) -> A_qk and A_kk blocks
 //   W^T = K~^T T_b^T and U^T = V^T T_b^T      (M=128, N=64, K=64)
-// The 64x64 unit-lower-triangular solve runs in shared memory (16x16 blocks).
+// The 64x64 unit-lower-triangular solve runs in shared memory: 16x16 diagonal
+// blocks by forward substitution, then each warp owns a set of columns and
+// runs block forward substitution down them with no block-wide barrier.
 #include <algorithm>
 
 #include "chunk_common.cuh"
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "tma_host.h"
 
 namespace kda {
 namespace prep {
@@ -46,22 +57,43 @@ constexpr int TSS = 68;      // fp32 row stride of the solve scratch
 constexpr float LOG2E = 1.4426950408889634f;
 
 // Shared memory (byte offsets from a 1024-aligned base); two CTAs fit on one SM.
+// Prologue staging (fused variant), read before the operands are written:
+constexpr int RAW_ROWS = CH + 3;              // tokens c0-3 .. c0+63
+constexpr uint32_t RAW_ROW = DK * 2;          // 256 B per token row
+constexpr uint32_t OFF_RAWQ = 0;
+constexpr uint32_t OFF_RAWK = 17408;
+constexpr uint32_t OFF_RAWV = 34816;
+constexpr uint32_t OFF_RAWA = 52224;          // alpha: 64 rows
+// Intra-chunk MMA operands:
 constexpr uint32_t OFF_L = 0;                 // [q rows 0..63 | k rows 64..127] x 128 ch: 32 KB
 constexpr uint32_t OFF_R = 32768;             // R_all: 160 rows x 128 ch: 40 KB
-constexpr uint32_t OFF_SB = 0;                // diag(beta) A_kk fp32 [64][TSS] (after the intra MMA)
+// Once the intra-chunk MMA has completed:
+constexpr uint32_t OFF_SB = 0;                // diag(beta) A_kk fp32 [64][TSS]
 constexpr uint32_t OFF_ST = 64 * TSS * 4;     // T fp32 [64][TSS]
 constexpr uint32_t OFF_TB = 35840;            // T_b [t][s] bf16, 8 KB
 constexpr uint32_t OFF_KT = 73728;            // k e^{Gamma}: 16 KB
-constexpr uint32_t OFF_V = 90112;             // v: 16 KB
-constexpr uint32_t OFF_BETA = 106496;         // beta[64]
-constexpr uint32_t OFF_WTOT = OFF_BETA + 256; // per-warp gate sums [8][128], then their prefixes
-constexpr uint32_t OFF_RB = OFF_WTOT + 4096;  // Gamma at the end of blocks 0..3 [4][128]
-constexpr uint32_t OFF_BAR = OFF_RB + 2048;   // mbarrier + TMEM address
+constexpr uint32_t OFF_V = 90112;             // v: 16 KB (written as soon as v is known)
+// Per-channel constants of the chunk (after the prologue, which stages the conv
+// weights and dt_bias of the head in the same bytes):
+constexpr uint32_t OFF_C = 106496;
+constexpr uint32_t OFF_WCONV = OFF_C;         // [3][128][4] bf16
+constexpr uint32_t OFF_DTB = OFF_C + 3072;    // [128] fp32
+constexpr uint32_t C_R = OFF_C;               // r_I, I = 0..4 (r_0 = 0)         [5][128]
+constexpr uint32_t C_CR = OFF_C + 2560;       // 2^{r_2-r_1}, 2^{r_3-r_1}, 2^{r_3-r_2}  [3][128]
+constexpr uint32_t OFF_WTOT = OFF_C + 4096;   // per-warp gate sums [8][128], then their prefixes
+constexpr uint32_t OFF_BETA = OFF_C + 8192;   // beta[64]
+constexpr uint32_t OFF_BAR = OFF_BETA + 256;  // MMA barrier, TMA barrier, TMEM address
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64;
-constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
-static_assert(OFF_ST + 64 * TSS * 4 <= OFF_TB && OFF_TB + 8192 <= OFF_KT, "solve scratch overlaps");
-static_assert(OFF_TB % 1024 == 0 && OFF_KT % 1024 == 0 && OFF_V % 1024 == 0, "SW128 alignment");
-static_assert(2 * SMEM_ALLOC <= 231424, "two CTAs per SM");
+constexpr uint32_t TMA_BYTES = 3 * RAW_ROWS * RAW_ROW + CH * RAW_ROW + 3 * 1024 + 512;
+static_assert(OFF_RAWK >= RAW_ROWS * RAW_ROW && OFF_RAWV >= OFF_RAWK + RAW_ROWS * RAW_ROW &&
+              OFF_RAWA >= OFF_RAWV + RAW_ROWS * RAW_ROW && OFF_RAWA + CH * RAW_ROW <= OFF_KT,
+              "prologue staging overlaps");
+static_assert(OFF_ST + 64 * TSS * 4 <= OFF_TB && OFF_TB + 8192 <= OFF_KT && OFF_V + 16384 <= OFF_C,
+              "solve scratch overlaps");
+static_assert(OFF_TB % 1024 == 0 && OFF_KT % 1024 == 0 && OFF_V % 1024 == 0 && OFF_R % 1024 == 0,
+              "SW128 alignment");
+static_assert(OFF_DTB + 512 <= OFF_WTOT && C_CR + 1536 <= OFF_WTOT, "constant area");
+static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
 
 // R_all rows: [0,64) diagonal-reference rows, then R_1 (16 rows), R_2 (32), R_3 (48).
 __host__ __device__ constexpr int r_row0(int I) { return I == 1 ? 64 : (I == 2 ? 80 : 112); }
@@ -80,6 +112,72 @@ __device__ __forceinline__ bool wait_vote(uint64_t *bar, uint32_t parity, bool o
   return all;
 }
 
+__device__ __forceinline__ void lds8(const uint8_t *p, float (&x)[8]) {
+  const float4 u = *reinterpret_cast<const float4 *>(p);
+  const float4 w = *reinterpret_cast<const float4 *>(p + 16);
+  x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w; x[4] = w.x; x[5] = w.y; x[6] = w.z; x[7] = w.w;
+}
+
+// Off-diagonal blocks of T in the columns [col, col + NC) of column block J:
+// for I = J+1..3,  X = sum_{K=J}^{I-1} B_IK T_KJ,  T_IJ = -T_II X  (one warp;
+// lane = row r of the block and a group of NC columns).  X is parked where T_IJ
+// goes; no other warp touches these columns.
+template <int J, int NC>
+__device__ __forceinline__ void solve_columns(const float *sB, float *sT, int col, int r) {
+#pragma unroll
+  for (int I = J + 1; I < 4; ++I) {
+    float x[NC];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) x[c] = 0.f;
+#pragma unroll
+    for (int K = J; K < I; ++K) {
+#pragma unroll
+      for (int m4 = 0; m4 < 4; ++m4) {
+        const float4 bv = *reinterpret_cast<const float4 *>(sB + (16 * I + r) * TSS + 16 * K + 4 * m4);
+        const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float *trow = sT + (16 * K + 4 * m4 + e) * TSS + col;
+          if constexpr (NC == 2) {
+            const float2 tv = *reinterpret_cast<const float2 *>(trow);
+            x[0] = fmaf(bb[e], tv.x, x[0]);
+            x[1] = fmaf(bb[e], tv.y, x[1]);
+          } else {
+            const float4 tv = *reinterpret_cast<const float4 *>(trow);
+            x[0] = fmaf(bb[e], tv.x, x[0]);
+            x[1] = fmaf(bb[e], tv.y, x[1]);
+            x[2] = fmaf(bb[e], tv.z, x[2]);
+            x[3] = fmaf(bb[e], tv.w, x[3]);
+          }
+        }
+      }
+    }
+    float *dst = sT + (16 * I + r) * TSS + col;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) dst[c] = x[c];
+    __syncwarp();
+    float y[NC];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) y[c] = 0.f;
+#pragma unroll
+    for (int m4 = 0; m4 < 4; ++m4) {
+      const float4 tv = *reinterpret_cast<const float4 *>(sT + (16 * I + r) * TSS + 16 * I + 4 * m4);
+      const float tt[4] = {tv.x, tv.y, tv.z, tv.w};   // row r of T_II (zero right of the diagonal)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float *xrow = sT + (16 * I + 4 * m4 + e) * TSS + col;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) y[c] = fmaf(tt[e], xrow[c], y[c]);
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < NC; ++c) dst[c] = -y[c];
+    __syncwarp();
+  }
+}
+
+template <bool kFused>
 __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant__ PrepArgs a) {
   const int H = a.H;
   const int h = blockIdx.x % H;
@@ -106,65 +204,188 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   seq_bounds(a.cu, n, a.seq_len, a.total_tokens, s0, s1);
   const int64_t c0 = s0 + cidx * CH;
   if (c0 >= s1) return;   // only for malformed cu_seqlens / chunk tables
+  const int nt = (int)(s1 - c0 < CH ? s1 - c0 : CH);   // valid tokens in this chunk
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (umma::smem_u32(smem) & 1023u) {   // the swizzled operands need a 1024-byte aligned base
+    if (threadIdx.x == 0 && a.err) atomicExch(a.err, ERR_TIMEOUT);
+    return;
+  }
   uint8_t *rec = reinterpret_cast<uint8_t *>(a.records) + (gchunk * H + h) * (int64_t)REC_STRIDE;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int cg = tid & 15, tg = tid >> 4, blkI = warp >> 1;   // tokens 4tg..4tg+3; block warp/2
+  const int cg = tid & 15, tg = tid >> 4, blkI = warp >> 1;   // tokens 4tg..4tg+3, all in block warp/2
   float *beta_s = reinterpret_cast<float *>(smem + OFF_BETA);
   float *wtot = reinterpret_cast<float *>(smem + OFF_WTOT);
-  float *rbs = reinterpret_cast<float *>(smem + OFF_RB);
   float *sBm = reinterpret_cast<float *>(smem + OFF_SB);
   float *sTm = reinterpret_cast<float *>(smem + OFF_ST);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 8);
+  uint64_t *bar_mma = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  uint64_t *bar_tma = bar_mma + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 16);
   const uint32_t sbase = umma::smem_u32(smem);
   const uint32_t lane_base = (uint32_t)(warp & 3) * 32u << 16;
-  const __nv_bfloat16 *__restrict__ qn = reinterpret_cast<const __nv_bfloat16 *>(a.qn);
-  const __nv_bfloat16 *__restrict__ kn = reinterpret_cast<const __nv_bfloat16 *>(a.kn);
-  const __nv_bfloat16 *__restrict__ vc = reinterpret_cast<const __nv_bfloat16 *>(a.vc);
-
-  // ---------------------------------------------------------------- loads (all issued first)
-  uint4 qr[4], kr[4], vr[4];
-  float g2[4][8];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int t = tg * 4 + j;
-    const int64_t off = ((c0 + t) * H + h) * DK + cg * 8;
-    if (c0 + t < s1) {
-      qr[j] = __ldcs(reinterpret_cast<const uint4 *>(qn + off));
-      kr[j] = __ldcs(reinterpret_cast<const uint4 *>(kn + off));
-      vr[j] = __ldcs(reinterpret_cast<const uint4 *>(vc + off));
-      const float4 ga = __ldcs(reinterpret_cast<const float4 *>(a.g + off));
-      const float4 gb = __ldcs(reinterpret_cast<const float4 *>(a.g + off + 4));
-      g2[j][0] = ga.x; g2[j][1] = ga.y; g2[j][2] = ga.z; g2[j][3] = ga.w;
-      g2[j][4] = gb.x; g2[j][5] = gb.y; g2[j][6] = gb.z; g2[j][7] = gb.w;
-    } else {
-      qr[j] = kr[j] = vr[j] = make_uint4(0, 0, 0, 0);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) g2[j][i] = 0.f;
-    }
-  }
-  float btj = 0.f;
-  if (tid < 64 && c0 + tid < s1) btj = __ldcs(a.beta + (c0 + tid) * H + h);
 
   if (warp == 0) {
     umma::tmem_alloc(tmem_slot, 256);
     umma::tmem_relinquish();
   }
   if (tid == 32) {
-    umma::mbar_init(bar, 1);
+    umma::mbar_init(bar_mma, 1);
+    umma::mbar_init(bar_tma, 1);
     umma::mbar_fence_init();
   }
+  umma::fence_before_sync();
+  __syncthreads();
+  umma::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
 
-  // ---------------------------------------------------------------- cumulative gate (base 2)
+  // ---------------------------------------------------------------- inputs
+  uint4 qb[4], kb[4];          // bf16 q, k (normalised) of this thread's 4 tokens x 8 channels
+  float g2[4][8];              // gate in base 2
+  float btj = 0.f;             // beta of token tid (tid < 64)
+  if constexpr (kFused) {
+    if (tid == 0) {
+      umma::mbar_arrive_expect_tx(bar_tma, TMA_BYTES);
+      const int x = h * DK;
+      umma::tma_load_2d(smem + OFF_RAWQ, &a.map_q, x, (int)c0 - 3, bar_tma);
+      umma::tma_load_2d(smem + OFF_RAWK, &a.map_k, x, (int)c0 - 3, bar_tma);
+      umma::tma_load_2d(smem + OFF_RAWV, &a.map_v, x, (int)c0 - 3, bar_tma);
+      umma::tma_load_2d(smem + OFF_RAWA, &a.map_alpha, x, (int)c0, bar_tma);
+      const __nv_bfloat16 *cw = reinterpret_cast<const __nv_bfloat16 *>(a.conv_w);
+#pragma unroll
+      for (int blk = 0; blk < 3; ++blk)
+        umma::bulk_g2s(smem + OFF_WCONV + blk * 1024, cw + ((int64_t)blk * H + h) * DK * KCONV, 1024,
+                       bar_tma);
+      umma::bulk_g2s(smem + OFF_DTB, a.dt_bias + h * DK, 512, bar_tma);
+    }
+    const float negA = -expf(a.A_log[h]);
+    if (tid < 64 && tid < nt)
+      btj = sigmoid_f(__bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(a.b)[(c0 + tid) * H + h]));
+    // causal-conv history of a sequence's first chunk: the caller's conv state or zeros
+    const bool hist = cidx == 0 && tg == 0;
+    uint4 hraw[3][3];
+    if (hist) {
+      const __nv_bfloat16 *c0p = reinterpret_cast<const __nv_bfloat16 *>(a.conv0);
+#pragma unroll
+      for (int blk = 0; blk < 3; ++blk)
+#pragma unroll
+        for (int m = 0; m < 3; ++m)
+          hraw[blk][m] = c0p != nullptr
+                             ? *reinterpret_cast<const uint4 *>(
+                                   c0p + (((int64_t)n * 3 + m) * 3 + blk) * H * DK + h * DK + cg * 8)
+                             : make_uint4(0, 0, 0, 0);
+    }
+    ok = wait_vote(bar_tma, 0, ok);
+    if (hist) {
+#pragma unroll
+      for (int blk = 0; blk < 3; ++blk)
+#pragma unroll
+        for (int m = 0; m < 3; ++m)   // only this thread reads these 16 bytes
+          *reinterpret_cast<uint4 *>(smem + (blk == 0 ? OFF_RAWQ : blk == 1 ? OFF_RAWK : OFF_RAWV) +
+                                     m * RAW_ROW + cg * 16) = hraw[blk][m];
+    }
+    // gate g = max(-exp(A_log) softplus(alpha + dt_bias), lower_bound), kept in base 2
+    float bias[8];
+    lds8(smem + OFF_DTB + cg * 32, bias);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float al[8];
+      unpack8(*reinterpret_cast<const uint4 *>(smem + OFF_RAWA + (4 * tg + j) * RAW_ROW + cg * 16), al);
+      const bool valid = 4 * tg + j < nt;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        g2[j][i] = valid ? gate_f(al[i] + bias[i], negA, a.lower_bound) * LOG2E : 0.f;
+    }
+    // conv4 + SiLU (+ L2 norm over the head's 128 channels for q and k)
+#pragma unroll
+    for (int bi = 0; bi < 3; ++bi) {
+      const int blk = bi == 0 ? 2 : bi - 1;   // v first: it goes straight to its tile
+      const uint8_t *raw = smem + (blk == 0 ? OFF_RAWQ : blk == 1 ? OFF_RAWK : OFF_RAWV) + cg * 16;
+      // by channel pair: the pair's 4 taps x 2 channels (16 bytes) and its 7 input rows
+      float y[4][8];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        float wt[8];   // taps 0..3 of channel 2q4, then of channel 2q4+1
+        unpack8(*reinterpret_cast<const uint4 *>(smem + OFF_WCONV + blk * 1024 + cg * 64 + q4 * 16), wt);
+        float xa[7], xb[7];
+#pragma unroll
+        for (int r = 0; r < 7; ++r) {
+          const uint32_t u = *reinterpret_cast<const uint32_t *>(raw + (4 * tg + r) * RAW_ROW + q4 * 4);
+          xa[r] = __uint_as_float(u << 16);
+          xb[r] = __uint_as_float(u & 0xffff0000u);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float acc0 = wt[0] * xa[j], acc1 = wt[4] * xb[j];
+#pragma unroll
+          for (int m = 1; m < KCONV; ++m) {
+            acc0 = fmaf(wt[m], xa[j + m], acc0);
+            acc1 = fmaf(wt[4 + m], xb[j + m], acc1);
+          }
+          y[j][2 * q4] = silu_f(acc0);
+          y[j][2 * q4 + 1] = silu_f(acc1);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float yj[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) yj[i] = y[j][i];
+        if (blk < 2) {
+          float ss = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) ss = fmaf(yj[i], yj[i], ss);
+#pragma unroll
+          for (int off = 8; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+          const float rn = rsqrtf(ss + a.eps);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) yj[i] *= rn;
+        }
+        if (4 * tg + j >= nt) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) yj[i] = 0.f;
+        }
+        const uint4 packed = pack8(yj);
+        if (blk == 0) qb[j] = packed;
+        else if (blk == 1) kb[j] = packed;
+        else *reinterpret_cast<uint4 *>(smem + OFF_V + tr_off(64, tg * 4 + j, cg)) = packed;
+      }
+    }
+  } else {
+    const __nv_bfloat16 *__restrict__ qn = reinterpret_cast<const __nv_bfloat16 *>(a.qn);
+    const __nv_bfloat16 *__restrict__ kn = reinterpret_cast<const __nv_bfloat16 *>(a.kn);
+    const __nv_bfloat16 *__restrict__ vc = reinterpret_cast<const __nv_bfloat16 *>(a.vc);
+    uint4 vr[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = tg * 4 + j;
+      const int64_t off = ((c0 + t) * H + h) * DK + cg * 8;
+      if (t < nt) {
+        qb[j] = __ldcs(reinterpret_cast<const uint4 *>(qn + off));
+        kb[j] = __ldcs(reinterpret_cast<const uint4 *>(kn + off));
+        vr[j] = __ldcs(reinterpret_cast<const uint4 *>(vc + off));
+        const float4 ga = __ldcs(reinterpret_cast<const float4 *>(a.g + off));
+        const float4 gb = __ldcs(reinterpret_cast<const float4 *>(a.g + off + 4));
+        const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) g2[j][i] = fminf(fmaxf(gg[i], a.lower_bound), 0.f) * LOG2E;
+      } else {
+        qb[j] = kb[j] = vr[j] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) g2[j][i] = 0.f;
+      }
+    }
+    if (tid < 64 && tid < nt) btj = __ldcs(a.beta + (c0 + tid) * H + h);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)   // v is the U operand as it is: straight into its tile
+      *reinterpret_cast<uint4 *>(smem + OFF_V + tr_off(64, tg * 4 + j, cg)) = vr[j];
+  }
+
+  // ---------------------------------------------------------------- cumulative gate
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    g2[0][i] *= LOG2E;
 #pragma unroll
-    for (int j = 1; j < 4; ++j) g2[j][i] = fmaf(g2[j][i], LOG2E, g2[j - 1][i]);
+    for (int j = 1; j < 4; ++j) g2[j][i] += g2[j - 1][i];
     const float lo = __shfl_up_sync(0xffffffffu, g2[3][i], 16);
     if (lane >= 16) {
 #pragma unroll
@@ -175,85 +396,105 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
     *reinterpret_cast<float4 *>(wtot + warp * 128 + cg * 8) = make_float4(g2[3][0], g2[3][1], g2[3][2], g2[3][3]);
     *reinterpret_cast<float4 *>(wtot + warp * 128 + cg * 8 + 4) = make_float4(g2[3][4], g2[3][5], g2[3][6], g2[3][7]);
   }
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    *reinterpret_cast<uint4 *>(smem + OFF_V + tr_off(64, tg * 4 + j, cg)) = vr[j];
   if (tid < 64) beta_s[tid] = btj;
-  umma::fence_before_sync();
-  __syncthreads();
-  umma::fence_after_sync();
-  const uint32_t tmem = *tmem_slot;
-  // per channel: exclusive prefix of the warp sums (in place) and Gamma at block ends
+  __syncthreads();   // also: every read of the prologue staging is done
+  // per channel: exclusive prefix of the warp sums (in place), r_1..r_4 and the R-row constants
   if (tid < 128) {
-    float acc = 0.f;
+    float acc = 0.f, r[5];
+    r[0] = 0.f;
 #pragma unroll
     for (int w2 = 0; w2 < 8; ++w2) {
       const float x = wtot[w2 * 128 + tid];
       wtot[w2 * 128 + tid] = acc;
       acc += x;
-      if (w2 & 1) rbs[(w2 >> 1) * 128 + tid] = acc;
+      if (w2 & 1) r[(w2 >> 1) + 1] = acc;
     }
-    reinterpret_cast<float *>(rec + REC_EGC)[tid] = umma::ex2(acc);   // e^{Gamma_C}
+    float *cf = reinterpret_cast<float *>(smem);
+#pragma unroll
+    for (int I = 0; I < 5; ++I) cf[C_R / 4 + I * 128 + tid] = r[I];
+    cf[C_CR / 4 + 0 * 128 + tid] = umma::ex2(r[2] - r[1]);
+    cf[C_CR / 4 + 1 * 128 + tid] = umma::ex2(r[3] - r[1]);
+    cf[C_CR / 4 + 2 * 128 + tid] = umma::ex2(r[3] - r[2]);
+    reinterpret_cast<float *>(rec + REC_EGC)[tid] = umma::ex2(r[4]);   // e^{Gamma_C}
   }
   __syncthreads();
 
   // ---------------------------------------------------------------- operands
   {
-    float rI[8], rI1[8], rC[8];
-    {
-      const float4 p0 = *reinterpret_cast<const float4 *>(wtot + warp * 128 + cg * 8);
-      const float4 p1 = *reinterpret_cast<const float4 *>(wtot + warp * 128 + cg * 8 + 4);
-      const float pre[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    float pre[8];
+    lds8(smem + OFF_WTOT + (warp * 128 + cg * 8) * 4, pre);
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < 4; ++j)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) g2[j][i] += pre[i];
+      for (int i = 0; i < 8; ++i) g2[j][i] += pre[i];   // Gamma_t (base 2)
+  }
+  const uint32_t coff = (uint32_t)(cg * 8) * 4;
+  {  // L side: Lq = q e^{Gamma - r_I}, Lk likewise; q e^{Gamma}, k e^{Gamma}
+    float rI[8], eR[8];
+    lds8(smem + C_R + blkI * 512 + coff, rI);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        rI[i] = blkI == 0 ? 0.f : rbs[(blkI - 1) * 128 + cg * 8 + i];
-        rI1[i] = rbs[blkI * 128 + cg * 8 + i];
-        rC[i] = rbs[3 * 128 + cg * 8 + i];
-      }
-    }
-    float eR[8], cK[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      eR[i] = umma::ex2(rI[i]);            // e^{r_I}
-      cK[i] = umma::ex2(rC[i] - rI1[i]);   // e^{Gamma_C - r_{I+1}}
-    }
+    for (int i = 0; i < 8; ++i) eR[i] = umma::ex2(rI[i]);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int t = tg * 4 + j;
-      float q[8], k[8], Lq[8], Lk[8], Rd[8], Qt[8], Kt[8], Kh[8], u[8];
-      unpack8(qr[j], q);
-      unpack8(kr[j], k);
+      float q[8], k[8], Lq[8], Lk[8], Qt[8], Kt[8];
+      unpack8(qb[j], q);
+      unpack8(kb[j], k);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float e1 = umma::ex2(g2[j][i] - rI[i]);    // <= 1
-        const float rd = umma::ex2(rI[i] - g2[j][i]);    // in [1, 2^116)
-        u[i] = umma::ex2(rI1[i] - g2[j][i]);             // e^{r_{I+1} - Gamma_t} in (0, 1]
+        const float e1 = umma::ex2(g2[j][i] - rI[i]);   // in (2^-128, 1]
         Lq[i] = q[i] * e1;
         Lk[i] = k[i] * e1;
-        Rd[i] = k[i] * rd;
         Qt[i] = Lq[i] * eR[i];
         Kt[i] = Lk[i] * eR[i];
-        Kh[i] = k[i] * u[i] * cK[i];                      // e^{Gamma_C - Gamma_t}
       }
       *reinterpret_cast<uint4 *>(smem + OFF_L + tr_off(128, t, cg)) = pack8(Lq);
       *reinterpret_cast<uint4 *>(smem + OFF_L + tr_off(128, 64 + t, cg)) = pack8(Lk);
-      *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, t, cg)) = pack8(Rd);
       *reinterpret_cast<uint4 *>(smem + OFF_KT + tr_off(64, t, cg)) = pack8(Kt);
       *reinterpret_cast<uint4 *>(rec + REC_QT + tr_off(64, t, cg)) = pack8(Qt);
+    }
+  }
+  {  // R side: kd = k e^{r_{I+1} - Gamma}; Rd = kd e^{r_I - r_{I+1}}; R_{I+1..3} rows; k e^{Gamma_C - Gamma}
+    float rI1[8], cD[8], cK[8], cA[8], cB[8];
+    {
+      float rI[8], r4[8];
+      lds8(smem + C_R + blkI * 512 + coff, rI);
+      lds8(smem + C_R + (blkI + 1) * 512 + coff, rI1);
+      lds8(smem + C_R + 4 * 512 + coff, r4);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        cD[i] = umma::ex2(rI[i] - rI1[i]);   // 2^{r_I - r_{I+1}}
+        cK[i] = umma::ex2(r4[i] - rI1[i]);   // 2^{r_4 - r_{I+1}}
+      }
+    }
+    if (blkI < 2) lds8(smem + C_CR + (blkI == 0 ? 0 : 2) * 512 + coff, cA);   // 2^{r_{I+2} - r_{I+1}}
+    if (blkI == 0) lds8(smem + C_CR + 512 + coff, cB);                       // 2^{r_3 - r_1}
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = tg * 4 + j;
+      float k[8], kd[8], Rd[8], Kh[8];
+      unpack8(kb[j], k);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        kd[i] = k[i] * umma::ex2(rI1[i] - g2[j][i]);   // |kd| <= |k|
+        Rd[i] = kd[i] * cD[i];
+        Kh[i] = kd[i] * cK[i];
+      }
+      *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, t, cg)) = pack8(Rd);
       *reinterpret_cast<uint4 *>(rec + REC_KH + tr_off(64, t, cg)) = pack8(Kh);
+      if (blkI < 3)
+        *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, r_row0(blkI + 1) + t, cg)) = pack8(kd);
+      if (blkI < 2) {
+        float x[8];
 #pragma unroll
-      for (int ip = 1; ip < 4; ++ip) {   // rows of R_ip (reference r_ip) for later blocks
-        if (ip > blkI) {
-          float Rx[8];
+        for (int i = 0; i < 8; ++i) x[i] = kd[i] * cA[i];
+        *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, r_row0(blkI + 2) + t, cg)) = pack8(x);
+      }
+      if (blkI == 0) {
+        float x[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            Rx[i] = k[i] * umma::ex2(rbs[(ip - 1) * 128 + cg * 8 + i] - g2[j][i]);   // e^{r_ip - Gamma_t} <= 1
-          *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, r_row0(ip) + t, cg)) = pack8(Rx);
-        }
+        for (int i = 0; i < 8; ++i) x[i] = kd[i] * cB[i];
+        *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, r_row0(3) + t, cg)) = pack8(x);
       }
     }
   }
@@ -261,7 +502,6 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   __syncthreads();
 
   // ---------------------------------------------------------------- intra MMA
-  bool ok = true;
   uint32_t phase = 0;
   if (tid == 0) {
     umma::fence_after_sync();
@@ -270,57 +510,82 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
     for (int s = 0; s < DK / 16; ++s)
       umma::mma_ss(tmem + TM_P, desc_k128(sbase + OFF_L, 128, s), desc_k128(sbase + OFF_R, 160, s),
                    idesc, s > 0);
-    umma::mma_commit(bar);
+    umma::mma_commit(bar_mma);
   }
-  ok = wait_vote(bar, phase, ok);
+  ok = wait_vote(bar_mma, phase, ok);
   phase ^= 1u;
 
   // ---------------------------------------------------------------- A_qk (bf16) and diag(beta) A_kk
+  // Warp w reads TMEM lanes 32(w&3)..: q rows (warps 0-1) or k rows (2-3) of
+  // tokens 32p..32p+31, p = w & 1; lane half hh gives the block I = 2p + hh.
+  // Column group gi (s = 16gi..16gi+15) of row t comes from the diagonal product
+  // (gi == I) or from R_I (gi < I); tcgen05.ld is warp-uniform, so both halves
+  // load both candidates and keep their own.
   if (ok && warp < 4) {
-    const int r = warp * 32 + lane;
-    const int t = r & 63;
-    const bool is_q = r < 64;
-    const int I = t >> 4;
-    float rowv[64];
+    const int p = warp & 1, hh = lane >> 4;
+    const int t = 32 * p + lane;
+    const bool is_q = warp < 2;
+    const float bt = is_q ? 1.f : beta_s[t];
+    const uint32_t tb = tmem + lane_base + TM_P;
+    auto emit = [&](int gi, const uint32_t (&v)[16], bool zero, bool diag) {
+      float x[16];
 #pragma unroll
-    for (int s = 0; s < 64; ++s) rowv[s] = 0.f;
-    // P columns in 16-wide groups: 0..3 diagonal blocks, 4 = R_1, 5..6 = R_2, 7..9 = R_3.
-    // tcgen05.ld is warp-uniform: every lane loads every group and keeps its own.
+      for (int e = 0; e < 16; ++e) {
+        const int s = 16 * gi + e;
+        const bool keep = !zero && (!diag || (is_q ? s <= t : s < t));
+        x[e] = keep ? __uint_as_float(v[e]) * bt : 0.f;
+      }
+      if (is_q) {
+        float lo8[8], hi8[8];
 #pragma unroll
-    for (int c32 = 0; c32 < 5; ++c32) {
-      uint32_t rr[32];
-      umma::tmem_ld32(tmem + lane_base + TM_P + c32 * 32, rr);
+        for (int e = 0; e < 8; ++e) { lo8[e] = x[e]; hi8[e] = x[8 + e]; }
+        *reinterpret_cast<uint4 *>(rec + REC_AQ + tr_off(64, t, 2 * gi)) = pack8(lo8);
+        *reinterpret_cast<uint4 *>(rec + REC_AQ + tr_off(64, t, 2 * gi + 1)) = pack8(hi8);
+      } else {
+        float4 *dst = reinterpret_cast<float4 *>(sBm + t * TSS + 16 * gi);
+#pragma unroll
+        for (int e4 = 0; e4 < 4; ++e4)
+          dst[e4] = make_float4(x[4 * e4], x[4 * e4 + 1], x[4 * e4 + 2], x[4 * e4 + 3]);
+      }
+    };
+    uint32_t va[16], vb2[16], v[16];
+    if (p == 0) {
+      // gi 0: lo = diagonal (col 0), hi = R_1 (col 64); gi 1: hi = diagonal (col 16)
+      umma::tmem_ld16(tb + 0, va);
+      umma::tmem_ld16(tb + 64, vb2);
       umma::tmem_wait_ld();
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int cc = c32 * 2 + half;
-        const int want = cc < 4 ? cc : (cc == 4 ? 1 : (cc < 7 ? 2 : 3));
-        const int sblk = cc < 4 ? cc : (cc == 4 ? 0 : (cc < 7 ? cc - 5 : cc - 7));
-        if (I == want) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) rowv[sblk * 16 + e] = __uint_as_float(rr[half * 16 + e]);
-        }
-      }
-    }
-    if (is_q) {
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        float x8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x8[i] = (c8 * 8 + i <= t) ? rowv[c8 * 8 + i] : 0.f;
-        *reinterpret_cast<uint4 *>(rec + REC_AQ + tr_off(64, t, c8)) = pack8(x8);
-      }
+      for (int e = 0; e < 16; ++e) v[e] = hh ? vb2[e] : va[e];
+      emit(0, v, false, hh == 0);
+      umma::tmem_ld16(tb + 16, va);
+      umma::tmem_wait_ld();
+      emit(1, va, hh == 0, true);
+      emit(2, va, true, false);
+      emit(3, va, true, false);
     } else {
-      const float bt = beta_s[t];
+      // gi 0: lo = R_2 (col 80), hi = R_3 (col 112); gi 1: 96 / 128;
+      // gi 2: lo = diagonal (col 32), hi = R_3 (col 144); gi 3: hi = diagonal (col 48)
+      umma::tmem_ld16(tb + 80, va);
+      umma::tmem_ld16(tb + 112, vb2);
+      umma::tmem_wait_ld();
 #pragma unroll
-      for (int s4 = 0; s4 < 16; ++s4) {
-        float4 v;
-        v.x = (4 * s4 + 0 < t) ? rowv[4 * s4 + 0] * bt : 0.f;
-        v.y = (4 * s4 + 1 < t) ? rowv[4 * s4 + 1] * bt : 0.f;
-        v.z = (4 * s4 + 2 < t) ? rowv[4 * s4 + 2] * bt : 0.f;
-        v.w = (4 * s4 + 3 < t) ? rowv[4 * s4 + 3] * bt : 0.f;
-        *reinterpret_cast<float4 *>(sBm + t * TSS + 4 * s4) = v;
-      }
+      for (int e = 0; e < 16; ++e) v[e] = hh ? vb2[e] : va[e];
+      emit(0, v, false, false);
+      umma::tmem_ld16(tb + 96, va);
+      umma::tmem_ld16(tb + 128, vb2);
+      umma::tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[e] = hh ? vb2[e] : va[e];
+      emit(1, v, false, false);
+      umma::tmem_ld16(tb + 32, va);
+      umma::tmem_ld16(tb + 144, vb2);
+      umma::tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[e] = hh ? vb2[e] : va[e];
+      emit(2, v, false, hh == 0);
+      umma::tmem_ld16(tb + 48, va);
+      umma::tmem_wait_ld();
+      emit(3, va, hh == 0, true);
     }
   }
   umma::fence_before_sync();
@@ -343,56 +608,22 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
     }
   }
   __syncthreads();
-  // Off-diagonal blocks by distance d = I - J: X_IJ = sum_K B_IK T_KJ (kept in the unused
-  // upper block (J, I)), then T_IJ = -T_II X_IJ.  B rows are read as float4.
-#pragma unroll
-  for (int d = 1; d < 4; ++d) {
-    for (int e = tid; e < (4 - d) * 256; e += NT) {
-      const int J = e >> 8, I = J + d, r = (e >> 4) & 15, cc = e & 15;
-      float acc = 0.f;
-#pragma unroll
-      for (int kb = 0; kb < d; ++kb) {
-        const int K = J + kb;
-        const float4 *brow = reinterpret_cast<const float4 *>(sBm + (I * 16 + r) * TSS + K * 16);
-#pragma unroll
-        for (int m4 = 0; m4 < 4; ++m4) {
-          const float4 bv = brow[m4];
-          acc = fmaf(bv.x, sTm[(K * 16 + 4 * m4 + 0) * TSS + J * 16 + cc], acc);
-          acc = fmaf(bv.y, sTm[(K * 16 + 4 * m4 + 1) * TSS + J * 16 + cc], acc);
-          acc = fmaf(bv.z, sTm[(K * 16 + 4 * m4 + 2) * TSS + J * 16 + cc], acc);
-          acc = fmaf(bv.w, sTm[(K * 16 + 4 * m4 + 3) * TSS + J * 16 + cc], acc);
-        }
-      }
-      sBm[(J * 16 + r) * TSS + I * 16 + cc] = acc;
-    }
-    __syncthreads();
-    for (int e = tid; e < (4 - d) * 256; e += NT) {
-      const int J = e >> 8, I = J + d, r = (e >> 4) & 15, cc = e & 15;
-      const float4 *trow = reinterpret_cast<const float4 *>(sTm + (I * 16 + r) * TSS + I * 16);
-      float acc = 0.f;
-#pragma unroll
-      for (int m4 = 0; m4 < 4; ++m4) {
-        const float4 tv = trow[m4];   // row r of T_II (entries right of the diagonal masked)
-        const int m = 4 * m4;
-        acc = fmaf(m + 0 <= r ? tv.x : 0.f, sBm[(J * 16 + m + 0) * TSS + I * 16 + cc], acc);
-        acc = fmaf(m + 1 <= r ? tv.y : 0.f, sBm[(J * 16 + m + 1) * TSS + I * 16 + cc], acc);
-        acc = fmaf(m + 2 <= r ? tv.z : 0.f, sBm[(J * 16 + m + 2) * TSS + I * 16 + cc], acc);
-        acc = fmaf(m + 3 <= r ? tv.w : 0.f, sBm[(J * 16 + m + 3) * TSS + I * 16 + cc], acc);
-      }
-      sTm[(I * 16 + r) * TSS + J * 16 + cc] = -acc;
-    }
-    __syncthreads();
+  {  // off-diagonal blocks, column by column (column block 3 has none)
+    const int r = lane & 15, hh = lane >> 4;
+    if (warp < 4) solve_columns<0, 2>(sBm, sTm, 4 * warp + 2 * hh, r);
+    else if (warp < 6) solve_columns<1, 4>(sBm, sTm, 16 + 8 * (warp - 4) + 4 * hh, r);
+    else solve_columns<2, 4>(sBm, sTm, 32 + 8 * (warp - 6) + 4 * hh, r);
   }
+  __syncthreads();
 #pragma unroll
   for (int it = 0; it < 2; ++it) {  // T_b rows as bf16, K-major [t][s]
     const int e = tid + it * NT;
     const int t = e >> 3, c8 = e & 7;
-    float x8[8];
+    float tv[8], bv[8], x8[8];
+    lds8(reinterpret_cast<const uint8_t *>(sTm + t * TSS + c8 * 8), tv);
+    lds8(reinterpret_cast<const uint8_t *>(beta_s + c8 * 8), bv);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int s = c8 * 8 + i;
-      x8[i] = s <= t ? sTm[t * TSS + s] * beta_s[s] : 0.f;
-    }
+    for (int i = 0; i < 8; ++i) x8[i] = c8 * 8 + i <= t ? tv[i] * bv[i] : 0.f;
     *reinterpret_cast<uint4 *>(smem + OFF_TB + tr_off(64, t, c8)) = pack8(x8);
   }
   umma::fence_proxy_async_smem();
@@ -408,9 +639,9 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
       umma::mma_ss(tmem + TM_W, desc_mn_tok(sbase + OFF_KT, s), desc_k64(sbase + OFF_TB, s), idesc, s > 0);
       umma::mma_ss(tmem + TM_U, desc_mn_tok(sbase + OFF_V, s), desc_k64(sbase + OFF_TB, s), idesc, s > 0);
     }
-    umma::mma_commit(bar);
+    umma::mma_commit(bar_mma);
   }
-  ok = wait_vote(bar, phase, ok);
+  ok = wait_vote(bar_mma, phase, ok);
 
   // ---------------------------------------------------------------- -W^T (warps 0-3), U^T (4-7) rows
   if (ok) {
@@ -441,38 +672,58 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   }
 }
 
-// chunk_cu[n] = number of 64-token chunks in sequences 0..n-1 (one thread; N is small).
-__global__ void chunk_table_kernel(const int32_t *cu, int N, int64_t total, int32_t *chunk_cu) {
+// chunk_cu[n] = number of 64-token chunks before sequence n (varlen batches);
+// also checks cu_seqlens: starts at 0, never decreases, ends at the token total.
+__global__ void chunk_table_kernel(const int32_t *cu, int N, int64_t total, int32_t *chunk_cu, int *err) {
   if (blockIdx.x != 0 || threadIdx.x != 0) return;
+  bool good = cu[0] == 0 && (int64_t)cu[N] == total;
   int32_t acc = 0;
   for (int n = 0; n < N; ++n) {
+    good = good && cu[n + 1] >= cu[n];
     int64_t s, e;
     seq_bounds(cu, n, 0, total, s, e);
     chunk_cu[n] = acc;
     acc += (int32_t)((e - s + CH - 1) / CH);
   }
   chunk_cu[N] = acc;
+  if (!good && err != nullptr) atomicExch(err, ERR_BAD_CU_SEQLENS);
 }
 
 }  // namespace prep
 
 static_assert(kChunkRecordBytes == chunkfmt::REC_STRIDE, "record size");
 
-cudaError_t launch_chunk_table(const int32_t *cu, int N, int64_t total, int32_t *chunk_cu,
+cudaError_t launch_chunk_table(const int32_t *cu, int N, int64_t total, int32_t *chunk_cu, int *err,
                                cudaStream_t stream) {
-  prep::chunk_table_kernel<<<1, 32, 0, stream>>>(cu, N, total, chunk_cu);
+  prep::chunk_table_kernel<<<1, 32, 0, stream>>>(cu, N, total, chunk_cu, err);
   return cudaGetLastError();
 }
 
-cudaError_t launch_chunk_prep(PrepArgs a, int64_t max_chunks, cudaStream_t stream) {
-  if (max_chunks == 0 || a.H == 0) return cudaSuccess;
-  a.max_slots = max_chunks;
-  cudaError_t e = cudaFuncSetAttribute(prep::chunk_prep_kernel,
+namespace {
+template <bool kFused>
+cudaError_t launch_prep_variant(const PrepArgs &a, int64_t max_chunks, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(prep::chunk_prep_kernel<kFused>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)prep::SMEM_ALLOC);
+                                       (int)prep::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  prep::chunk_prep_kernel<<<(unsigned)(max_chunks * a.H), prep::NT, prep::SMEM_ALLOC, stream>>>(a);
+  prep::chunk_prep_kernel<kFused><<<(unsigned)(max_chunks * a.H), prep::NT, prep::SMEM_BYTES, stream>>>(a);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_chunk_prep(PrepArgs a, int64_t max_chunks, bool fused, const void *q,
+                              const void *k, const void *v, const void *alpha, cudaStream_t stream) {
+  if (max_chunks == 0 || a.H == 0 || a.total_tokens == 0) return cudaSuccess;
+  a.max_slots = max_chunks;
+  if (!fused) return launch_prep_variant<false>(a, max_chunks, stream);
+  const uint64_t rows = (uint64_t)a.total_tokens, cols = (uint64_t)a.H * chunkfmt::DK;
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!encode_rows(&a.map_q, q, bf, 2, rows, cols, cols, prep::RAW_ROWS, chunkfmt::DK) ||
+      !encode_rows(&a.map_k, k, bf, 2, rows, cols, cols, prep::RAW_ROWS, chunkfmt::DK) ||
+      !encode_rows(&a.map_v, v, bf, 2, rows, cols, cols, prep::RAW_ROWS, chunkfmt::DK) ||
+      !encode_rows(&a.map_alpha, alpha, bf, 2, rows, cols, cols, chunkfmt::CH, chunkfmt::DK))
+    return cudaErrorInvalidValue;
+  return launch_prep_variant<true>(a, max_chunks, stream);
 }
 
 }  // namespace kda

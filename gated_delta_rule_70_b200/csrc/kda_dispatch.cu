@@ -1,37 +1,144 @@
-// Recurrence dispatch: bf16 with head_dim 128 runs the tensor-core chunk path
-// (chunk_prep over every (chunk, head), then the sequential state pass); every
-// other shape runs the CUDA-core token kernel.
+// Dispatch of the recurrence and of the whole prefill.
+//
+// bf16 with head_dim 128 (and a gate bound the chunk factorisation can hold)
+// runs the tensor-core chunk path: chunk_prep over every (chunk, head), then
+// the sequential state pass.  For a prefill chunk_prep also runs the prologue
+// on the raw inputs, so conv'd / normalised q, k, v and the gates never travel
+// through device memory.  Every other shape runs the prologue kernel and the
+// CUDA-core token kernel.
+#include <mutex>
+#include <vector>
+
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
 namespace kda {
 
+namespace {
+
+// Optional per-kernel timing of the chunk path (kda_kernel_timing / kda_kernel_times).
+struct KernelClock {
+  std::mutex mu;
+  bool on = false;
+  std::vector<cudaEvent_t> ev;   // 3 per recorded call
+};
+KernelClock g_clock;
+constexpr size_t kMaxTimedCalls = 4096;
+
+void drop_events_locked() {
+  for (cudaEvent_t e : g_clock.ev) cudaEventDestroy(e);
+  g_clock.ev.clear();
+}
+
+// Records one event on `stream` when timing is on and this call is being timed.
+void clock_mark(bool timed, cudaStream_t stream) {
+  if (!timed) return;
+  cudaEvent_t e;
+  if (cudaEventCreate(&e) != cudaSuccess) return;
+  cudaEventRecord(e, stream);
+  std::lock_guard<std::mutex> lock(g_clock.mu);
+  g_clock.ev.push_back(e);
+}
+
+bool clock_begin() {
+  std::lock_guard<std::mutex> lock(g_clock.mu);
+  return g_clock.on && g_clock.ev.size() / 3 < kMaxTimedCalls;
+}
+
+cudaError_t run_chunk_path(PrepArgs pa, const RecurrenceArgs &ra, bool varlen, bool fused,
+                           const PrologueArgs *raw, char *ws, const WsLayout &L,
+                           cudaStream_t stream) {
+  int32_t *chunk_cu = nullptr;
+  if (varlen) {
+    chunk_cu = reinterpret_cast<int32_t *>(ws + L.chunk_cu);
+    cudaError_t e = launch_chunk_table(ra.cu, ra.N, ra.total_tokens, chunk_cu, ra.err, stream);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t slots = max_chunk_slots(ra.N, ra.total_tokens, ra.seq_len, varlen);
+  pa.N = ra.N; pa.H = ra.H; pa.seq_len = ra.seq_len; pa.total_tokens = ra.total_tokens;
+  pa.cu = ra.cu; pa.chunk_cu = chunk_cu;
+  pa.records = ws + L.records; pa.err = ra.err;
+  const bool timed = clock_begin();
+  clock_mark(timed, stream);
+  cudaError_t e = launch_chunk_prep(pa, slots, fused, raw ? raw->q : nullptr, raw ? raw->k : nullptr,
+                                    raw ? raw->v : nullptr, raw ? raw->alpha : nullptr, stream);
+  clock_mark(timed, stream);
+  if (e != cudaSuccess) {
+    clock_mark(timed, stream);   // keep the events in triples
+    return e;
+  }
+  StateArgs sa{};
+  sa.N = ra.N; sa.H = ra.H; sa.seq_len = ra.seq_len; sa.total_tokens = ra.total_tokens;
+  sa.cu = ra.cu; sa.chunk_cu = chunk_cu; sa.records = ws + L.records; sa.max_slots = slots;
+  sa.state0 = ra.state0; sa.scale = ra.scale; sa.o = ra.o; sa.state1 = ra.state1; sa.err = ra.err;
+  e = launch_state_pass(sa, stream);
+  clock_mark(timed, stream);
+  return e;
+}
+
+}  // namespace
+
 cudaError_t run_recurrence(const RecurrenceArgs &ra, bool varlen, char *ws, const WsLayout &L,
                            cudaStream_t stream) {
 #ifndef KDA_TOKEN_KERNEL_ONLY
   if (L.tc) {
-    int32_t *chunk_cu = nullptr;
-    if (varlen) {
-      chunk_cu = reinterpret_cast<int32_t *>(ws + L.chunk_cu);
-      cudaError_t e = launch_chunk_table(ra.cu, ra.N, ra.total_tokens, chunk_cu, stream);
-      if (e != cudaSuccess) return e;
-    }
-    const int64_t slots = max_chunk_slots(ra.N, ra.total_tokens, ra.seq_len, varlen);
     PrepArgs pa{};
-    pa.N = ra.N; pa.H = ra.H; pa.seq_len = ra.seq_len; pa.total_tokens = ra.total_tokens;
-    pa.cu = ra.cu; pa.chunk_cu = chunk_cu;
     pa.qn = ra.qn; pa.kn = ra.kn; pa.vc = ra.vc; pa.g = ra.g; pa.beta = ra.beta;
-    pa.records = ws + L.records; pa.err = ra.err;
-    cudaError_t e = launch_chunk_prep(pa, slots, stream);
-    if (e != cudaSuccess) return e;
-    StateArgs sa{};
-    sa.N = ra.N; sa.H = ra.H; sa.seq_len = ra.seq_len; sa.total_tokens = ra.total_tokens;
-    sa.cu = ra.cu; sa.chunk_cu = chunk_cu; sa.records = ws + L.records; sa.max_slots = slots;
-    sa.state0 = ra.state0; sa.scale = ra.scale; sa.o = ra.o; sa.state1 = ra.state1; sa.err = ra.err;
-    return launch_state_pass(sa, stream);
+    pa.lower_bound = ra.lower_bound;
+    return run_chunk_path(pa, ra, varlen, false, nullptr, ws, L, stream);
   }
 #endif
   return launch_recurrence(ra, stream);
 }
 
+cudaError_t run_prefill(PrologueArgs pa, RecurrenceArgs ra, void *final_conv_state, bool varlen,
+                        char *ws, const WsLayout &L, cudaStream_t stream) {
+  cudaError_t e = cudaSuccess;
+#ifndef KDA_TOKEN_KERNEL_ONLY
+  if (L.tc) {
+    PrepArgs p{};
+    p.lower_bound = pa.lower_bound; p.eps = pa.eps;
+    p.conv_w = pa.conv_w; p.b = pa.b; p.A_log = pa.A_log; p.dt_bias = pa.dt_bias; p.conv0 = pa.conv0;
+    e = run_chunk_path(p, ra, varlen, true, &pa, ws, L, stream);
+  } else
+#endif
+  {
+    pa.qn = ws + L.qn; pa.kn = ws + L.kn; pa.vc = ws + L.vc;
+    pa.g = reinterpret_cast<float *>(ws + L.g);
+    pa.beta = reinterpret_cast<float *>(ws + L.beta);
+    if ((e = launch_prologue(pa, stream)) != cudaSuccess) return e;
+    ra.qn = pa.qn; ra.kn = pa.kn; ra.vc = pa.vc; ra.g = pa.g; ra.beta = pa.beta;
+    e = launch_recurrence(ra, stream);
+  }
+  if (e != cudaSuccess) return e;
+  if (final_conv_state != nullptr) e = launch_conv_state_out(pa, final_conv_state, stream);
+  return e;
+}
+
 }  // namespace kda
+
+extern "C" int kda_kernel_timing(int enable) {
+  std::lock_guard<std::mutex> lock(kda::g_clock.mu);
+  kda::g_clock.on = enable != 0;
+  if (!kda::g_clock.on) kda::drop_events_locked();
+  return 0;
+}
+
+extern "C" int kda_kernel_times(float *prep_ms, float *state_ms) {
+  std::lock_guard<std::mutex> lock(kda::g_clock.mu);
+  const size_t calls = kda::g_clock.ev.size() / 3;
+  double a = 0.0, b = 0.0;
+  bool ok = true;
+  for (size_t c = 0; c < calls && ok; ++c) {
+    cudaEvent_t *e = &kda::g_clock.ev[3 * c];
+    float x = 0.f, y = 0.f;
+    ok = cudaEventSynchronize(e[2]) == cudaSuccess && cudaEventElapsedTime(&x, e[0], e[1]) == cudaSuccess &&
+         cudaEventElapsedTime(&y, e[1], e[2]) == cudaSuccess;
+    a += x;
+    b += y;
+  }
+  kda::drop_events_locked();
+  if (prep_ms) *prep_ms = calls && ok ? (float)(a / calls) : 0.f;
+  if (state_ms) *state_ms = calls && ok ? (float)(b / calls) : 0.f;
+  return ok ? (int)calls : -1;
+}

@@ -38,6 +38,7 @@ struct RecurrenceArgs {
   const float *beta;         // [T, H]
   const float *state0;       // [N, H, D, D] or nullptr
   float scale;
+  float lower_bound;         // gates are taken as clamped into [lower_bound, 0]
   void *o;                   // [T, H, D] io dtype
   float *state1;             // [N, H, D, D]
   int *err;
@@ -59,16 +60,28 @@ struct DecodeArgs {
 
 // Tensor-core chunk path (bf16, head_dim 128): chunk_prep writes one record
 // per (chunk, head); state_pass runs the sequential state chain over them.
+// chunk_prep either runs the prologue itself on the raw inputs (fused: the
+// prefill entry points) or reads prepared inputs (the recurrence entry point).
 struct PrepArgs {
   int N, H, seq_len;
   int64_t total_tokens;
   const int32_t *cu;         // [N + 1] or nullptr (dense)
   const int32_t *chunk_cu;   // [N + 1] chunk prefix (varlen) or nullptr (dense)
+  float lower_bound, eps;
+  // fused prologue: raw inputs (q, k, v, alpha read through the tensor maps)
+  const void *conv_w;        // [3, H*128, 4] bf16
+  const void *b;             // [T, H] bf16
+  const float *A_log;        // [H]
+  const float *dt_bias;      // [H, 128]
+  const void *conv0;         // [N, 3, 3*H*128] bf16 or nullptr
+  // prepared inputs
   const void *qn, *kn, *vc;  // [T, H, 128] bf16
   const float *g, *beta;     // [T, H, 128], [T, H]
   void *records;             // [max_slots][H] records of chunkfmt::REC_STRIDE bytes
   int64_t max_slots;         // record slots (set by the launcher)
   int *err;
+  // [T rows][H*128] bf16: q, k, v (67-row boxes: 3 history rows + 64) and alpha (64 rows)
+  CUtensorMap map_q, map_k, map_v, map_alpha;
 };
 
 struct StateArgs {
@@ -91,22 +104,29 @@ inline int64_t max_chunk_slots(int N, int64_t total_tokens, int seq_len, bool va
 }
 
 // Workspace layout (byte offsets, 256-aligned):
-//   error word | qn | kn | vc | g | beta   (prologue outputs; with_prologue only)
+//   error word | qn | kn | vc | g | beta   (prologue outputs; token-kernel prefill only)
 //   | chunk table (N+1 int32) | chunk records    (tensor-core path only)
 struct WsLayout {
   size_t err, qn, kn, vc, g, beta, chunk_cu, records, total;
   bool tc;   // bf16 with head_dim 128: the tensor-core chunk path
 };
+// The tensor-core path splits e^{Gamma_t - Gamma_s} around references at most 16
+// tokens away, which stays inside fp32 / bf16 range for gates >= -5.5 (16 * 5.5 *
+// log2 e < 127); shapes with a lower gate bound run the token kernel.
+constexpr float kTcMinLowerBound = -5.5f;
+inline bool use_tensor_core_path(int io_dtype, int D, float lower_bound) {
+  return io_dtype == KDA_BF16 && D == 128 && lower_bound >= kTcMinLowerBound;
+}
 inline WsLayout workspace_layout(int N, int H, int D, int seq_len, int64_t T, int io_dtype,
-                                 bool varlen, bool with_prologue) {
+                                 float lower_bound, bool varlen, bool with_prologue) {
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t es = io_dtype == KDA_BF16 ? 2 : 4;
   const size_t thd = (size_t)T * H * D;
   WsLayout L{};
-  L.tc = io_dtype == KDA_BF16 && D == 128;
+  L.tc = use_tensor_core_path(io_dtype, D, lower_bound);
   size_t off = 256;  // error word
   L.err = 0;
-  if (with_prologue) {
+  if (with_prologue && !L.tc) {  // the tensor-core path runs the prologue inside chunk_prep
     L.qn = off; off = up(off + thd * es);
     L.kn = off; off = up(off + thd * es);
     L.vc = off; off = up(off + thd * es);
@@ -124,9 +144,14 @@ inline WsLayout workspace_layout(int N, int H, int D, int seq_len, int64_t T, in
 }
 
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t stream);
-cudaError_t launch_chunk_table(const int32_t *cu, int N, int64_t total, int32_t *chunk_cu,
+// chunk_cu[n] = 64-token chunks before sequence n; also checks cu_seqlens
+// (starts at 0, non-decreasing, ends at total) and flags ERR_BAD_CU_SEQLENS in *err.
+cudaError_t launch_chunk_table(const int32_t *cu, int N, int64_t total, int32_t *chunk_cu, int *err,
                                cudaStream_t stream);
-cudaError_t launch_chunk_prep(PrepArgs a, int64_t max_chunks, cudaStream_t stream);
+// fused: run the prologue on the raw inputs in a.{conv_w, b, A_log, dt_bias, conv0}
+// and q, k, v, alpha (tensor maps built here); else read a.{qn, kn, vc, g, beta}.
+cudaError_t launch_chunk_prep(PrepArgs a, int64_t max_chunks, bool fused, const void *q,
+                              const void *k, const void *v, const void *alpha, cudaStream_t stream);
 cudaError_t launch_state_pass(const StateArgs &a, cudaStream_t stream);
 cudaError_t launch_conv_state_out(const PrologueArgs &a, void *out, cudaStream_t stream);
 cudaError_t launch_recurrence(const RecurrenceArgs &a, cudaStream_t stream);
@@ -135,6 +160,11 @@ cudaError_t launch_recurrence(const RecurrenceArgs &a, cudaStream_t stream);
 // CUDA-core token kernel.
 cudaError_t run_recurrence(const RecurrenceArgs &ra, bool varlen, char *ws, const WsLayout &L,
                            cudaStream_t stream);
+// The whole prefill (prologue + recurrence + final conv state) for PrologueArgs
+// `pa` (inputs, err) and RecurrenceArgs `ra` (state0, scale, o, state1) in a
+// workspace laid out by workspace_layout(..., with_prologue = true).
+cudaError_t run_prefill(PrologueArgs pa, RecurrenceArgs ra, void *final_conv_state, bool varlen,
+                        char *ws, const WsLayout &L, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 
 }  // namespace kda

@@ -65,7 +65,7 @@ extern "C" kda_status kda_prefill_noalloc(
   const int64_t T = cu_seqlens ? (int64_t)s->seq_len : (int64_t)s->num_seqs * s->seq_len;
   const bool varlen = cu_seqlens != nullptr;
   const WsLayout L = workspace_layout(s->num_seqs, s->num_heads, s->head_dim, s->seq_len, T,
-                                      s->io_dtype, varlen, true);
+                                      s->io_dtype, s->lower_bound, varlen, true);
   if (L.total > KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_WORKSPACE;
   if (T > 0 && (!q || !k || !v || !alpha || !b || !o || !ok16(q) || !ok16(k) || !ok16(v) ||
                 !ok16(alpha) || !ok16(b) || !ok16(o)))
@@ -90,21 +90,13 @@ extern "C" kda_status kda_prefill_noalloc(
   pa.q = q; pa.k = k; pa.v = v; pa.conv_w = conv_w; pa.alpha = alpha; pa.b = b;
   pa.A_log = A_log; pa.dt_bias = dt_bias; pa.conv0 = initial_conv_state;
   pa.lower_bound = s->lower_bound; pa.eps = s->l2norm_eps;
-  pa.qn = ws + L.qn; pa.kn = ws + L.kn; pa.vc = ws + L.vc;
-  pa.g = reinterpret_cast<float *>(ws + L.g);
-  pa.beta = reinterpret_cast<float *>(ws + L.beta);
   pa.err = reinterpret_cast<int *>(ws + L.err);
-  if (launch_prologue(pa, stream) != cudaSuccess) return KDA_ERR_CUDA;
 
   RecurrenceArgs ra{};
   ra.N = s->num_seqs; ra.H = s->num_heads; ra.D = s->head_dim; ra.seq_len = s->seq_len;
   ra.total_tokens = T; ra.io_dtype = s->io_dtype; ra.cu = cu_seqlens;
-  ra.qn = pa.qn; ra.kn = pa.kn; ra.vc = pa.vc; ra.g = pa.g; ra.beta = pa.beta;
   ra.state0 = initial_state; ra.scale = s->scale; ra.o = o; ra.state1 = final_state;
-  ra.err = pa.err;
-  const cudaError_t e = run_recurrence(ra, varlen, ws, L, stream);
-  if (e != cudaSuccess) return KDA_ERR_CUDA;
-  if (final_conv_state != nullptr && launch_conv_state_out(pa, final_conv_state, stream) != cudaSuccess)
-    return KDA_ERR_CUDA;
+  ra.lower_bound = s->lower_bound; ra.err = pa.err;
+  if (run_prefill(pa, ra, final_conv_state, varlen, ws, L, stream) != cudaSuccess) return KDA_ERR_CUDA;
   return KDA_OK;
 }

@@ -27,7 +27,8 @@ KDA_BF16, KDA_FP32 = 0, 1
 
 EXPORTED = ["kda_prefill_workspace_size", "kda_prefill", "kda_prefill_status", "kda_prologue",
             "kda_recurrence", "kda_recurrence_workspace_size", "kda_decode_step",
-            "kda_status_string", "kda_version", "kda_prefill_noalloc"]
+            "kda_status_string", "kda_version", "kda_prefill_noalloc", "kda_kernel_timing",
+            "kda_kernel_times"]
 
 
 class KdaLibraryError(RuntimeError):
@@ -83,6 +84,10 @@ def load_library():
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_version.argtypes = []
     lib.kda_version.restype = i32
+    lib.kda_kernel_timing.argtypes = [i32]
+    lib.kda_kernel_timing.restype = i32
+    lib.kda_kernel_times.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]
+    lib.kda_kernel_times.restype = i32
     _lib = lib
     return lib
 
@@ -134,7 +139,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, conv_w: torch.Ten
             initial_conv_state: Optional[torch.Tensor] = None, *, num_seqs: Optional[int] = None,
             lower_bound: float = -5.0, l2norm_eps: float = 1e-6,
             scale: float = 1.0, want_conv_state: bool = True, out: Optional[torch.Tensor] = None,
-            final_state: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+            final_state: Optional[torch.Tensor] = None,
+            final_conv_state: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
             check: bool = True) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
     """KDA prefill.  q, k, v: [T_total, H*d] (or [B, T, H*d] dense); alpha: [.., H, d];
     b: [.., H].  Returns (o [T_total, H, d], final_state [N, H, d, d], final_conv_state
@@ -157,7 +163,9 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, conv_w: torch.Ten
     o = out if out is not None else torch.empty((T_total, H, d), dtype=q.dtype, device=dev)
     fs = final_state if final_state is not None else torch.empty((N, H, d, d), dtype=torch.float32,
                                                                  device=dev)
-    fc = (torch.empty((N, 3, 3 * H * d), dtype=q.dtype, device=dev) if want_conv_state else None)
+    fc = final_conv_state
+    if fc is None and want_conv_state:
+        fc = torch.empty((N, 3, 3 * H * d), dtype=q.dtype, device=dev)
     ws_bytes = prefill_workspace_size(shape, cu_seqlens is not None)
     ws = workspace
     if ws is None or ws.numel() < ws_bytes:
@@ -250,3 +258,17 @@ def decode_step(q, k, v, alpha, b, conv_w, A_log, dt_bias, state: torch.Tensor,
                              _ptr(conv_state), _ptr(o), _stream(q.device))
     _check(st, "kda_decode_step")
     return o
+
+
+def kernel_timing(enable: bool) -> None:
+    """Start (True) or stop (False) per-kernel event timing of the chunk path."""
+    load_library().kda_kernel_timing(1 if enable else 0)
+
+
+def kernel_times() -> Tuple[int, float, float]:
+    """(calls, mean chunk_prep ms, mean state-pass ms) over the calls timed since the last read."""
+    a, b = ctypes.c_float(0.0), ctypes.c_float(0.0)
+    n = load_library().kda_kernel_times(ctypes.byref(a), ctypes.byref(b))
+    if n < 0:
+        raise KdaError(KDA_ERR_CUDA, "kda_kernel_times")
+    return n, float(a.value), float(b.value)

@@ -216,6 +216,25 @@ kda_status kda_prefill_noalloc(const kda_shape *shape,
                                void *o, float *final_state, void *final_conv_state,
                                void *stream);
 
+/*
+ * kda_kernel_timing / kda_kernel_times -- per-kernel device time of the
+ * tensor-core chunk path, for benchmarks.  The pages describe no such facility.
+ *
+ * kda_kernel_timing(1) makes every later kda_prefill / kda_prefill_noalloc /
+ * kda_recurrence call that takes the chunk path record CUDA events on its
+ * stream before chunk_prep, between chunk_prep and the state pass, and after
+ * the state pass (up to 4096 calls are kept; later ones are not timed).
+ * kda_kernel_timing(0) stops recording and drops what was kept.
+ * kda_kernel_times() waits for the recorded events, writes the mean duration
+ * in milliseconds of chunk_prep to *prep_ms and of the state pass to *state_ms
+ * over the calls recorded since the last read (both 0 when there were none),
+ * returns the number of calls, and forgets them.  Recording is process-wide and
+ * not meant for concurrent use from several host threads.  Returns -1 when a
+ * CUDA call fails.
+ */
+int kda_kernel_timing(int enable);
+int kda_kernel_times(float *prep_ms, float *state_ms);
+
 /* Static description of a status code (never NULL). */
 const char *kda_status_string(kda_status status);
 

@@ -47,13 +47,26 @@ def test_status_strings(lib):
 
 
 def test_workspace_size_rules(lib):
-    sh = kda.make_shape(4, 8192, 32, 128, __import__("torch").bfloat16)
+    import torch
+    record = 74752  # bytes per (chunk, head) record of the tensor-core path
+    # bf16, d=128: chunk records only (the prologue runs inside chunk_prep)
+    sh = kda.make_shape(4, 8192, 32, 128, torch.bfloat16)
     dense = kda.prefill_workspace_size(sh, False)
     varlen = kda.prefill_workspace_size(sh, True)
     T = 4 * 8192
-    assert dense >= T * 32 * 128 * (3 * 2 + 4) + T * 32 * 4
-    assert varlen < dense
-    bad = kda.make_shape(4, 8192, 32, 96, __import__("torch").bfloat16)
+    assert dense >= 4 * (8192 // 64) * 32 * record
+    assert dense < 4 * (8192 // 64) * 32 * record + (1 << 20)
+    assert varlen < dense  # 8192 packed tokens: ceil(8192/64) + 4 chunk slots
+    assert kda.recurrence_workspace_size(sh, False) == dense
+    # a gate bound the chunk factorisation cannot hold takes the token kernel:
+    # the prologue's intermediates, no records
+    low = kda.make_shape(4, 8192, 32, 128, torch.bfloat16, lower_bound=-8.0)
+    assert kda.prefill_workspace_size(low, False) >= T * 32 * 128 * (3 * 2 + 4) + T * 32 * 4
+    assert kda.recurrence_workspace_size(low, False) < 4096
+    # fp32 runs the token kernel
+    f32 = kda.make_shape(1, 256, 2, 64, torch.float32)
+    assert kda.prefill_workspace_size(f32, False) >= 256 * 2 * 64 * (3 * 4 + 4) + 256 * 2 * 4
+    bad = kda.make_shape(4, 8192, 32, 96, torch.bfloat16)
     assert kda.prefill_workspace_size(bad, False) == 0
 
 
