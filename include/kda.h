@@ -44,8 +44,11 @@
  *     [2*H*d, 3*H*d) is v; conv_w[blk][c][3] multiplies the current token.
  *
  * Supported shapes: head_dim 64 or 128; num_heads 1..64; any sequence
- * length >= 0.  bf16 with head_dim 128 runs the tensor-core chunk kernel;
- * other combinations run the CUDA-core token kernel (fp32 test mode).
+ * length >= 0.  bf16 with head_dim 128 and lower_bound >= -5.5 runs the
+ * tensor-core chunk path (chunk_prep, with the prologue fused in, then the
+ * state pass); other combinations run the prologue kernel and the CUDA-core
+ * token kernel (fp32 test mode).  The bound keeps the chunk path's split decay
+ * factors, which span up to 16 tokens of gate, inside fp32 and bf16 range.
  */
 #ifndef KDA_H
 #define KDA_H
@@ -144,7 +147,8 @@ kda_status kda_prologue(const kda_shape *shape,
  * kda_recurrence -- the recurrence alone, on prepared per-token inputs
  * (what kda_prologue writes):
  *   qn, kn, vc     [T_total, H, d] io dtype
- *   g              [T_total, H, d] fp32, gate values (log-decay, <= 0)
+ *   g              [T_total, H, d] fp32, gate values in [lower_bound, 0] (what
+ *                  kda_prologue writes; the tensor-core path clamps into that range)
  *   beta           [T_total, H]    fp32
  *   initial_state  [N, H, d, d]    fp32 or NULL (zeros)
  *   cu_seqlens     [N + 1] int32 or NULL (dense)
@@ -152,8 +156,10 @@ kda_status kda_prologue(const kda_shape *shape,
  *   final_state    [N, H, d, d]    fp32, written; may equal initial_state
  *   workspace      >= kda_recurrence_workspace_size(shape, varlen) bytes,
  *                  256-byte aligned (per-chunk records of the tensor-core path)
- * kda_prefill is kda_prologue followed by kda_recurrence.  kda_prefill_status()
- * reads this workspace's error word the same way.
+ * kda_prologue followed by kda_recurrence computes what kda_prefill computes
+ * (kda_prefill fuses the two on the tensor-core path).  kda_prefill_status()
+ * reads this workspace's error word the same way; on the tensor-core path it
+ * also reports bad cu_seqlens.
  */
 size_t kda_recurrence_workspace_size(const kda_shape *shape, int is_varlen);
 kda_status kda_recurrence(const kda_shape *shape,
@@ -189,14 +195,17 @@ kda_status kda_decode_step(const kda_shape *shape,
  * memory and lends the library only its inputs and outputs, code running
  * under an allocator that must not grow, a host callback).
  *
- * Same arguments and results as kda_prefill minus the workspace: the
- * prologue's intermediate tensors live in a library-owned array of
- * KDA_NOALLOC_SCRATCH_BYTES in device memory, which every GPU that loads the
- * library holds until the library is unloaded.  The call allocates nothing.
+ * Same arguments and results as kda_prefill minus the workspace: what
+ * kda_prefill keeps in its workspace (the per-chunk records of the
+ * tensor-core path, or the prologue's outputs on the token-kernel path) lives
+ * in a library-owned array of KDA_NOALLOC_SCRATCH_BYTES in device memory,
+ * which every GPU that loads the library holds until the library is unloaded.
+ * The call allocates nothing.
  *
  *   - A shape whose intermediates need more than KDA_NOALLOC_SCRATCH_BYTES
- *     (bf16, d = 128: about 2.4 KiB per token per head, e.g. 400 tokens at
- *     32 heads) returns KDA_ERR_WORKSPACE and launches nothing.
+ *     (bf16, d = 128: a 74,752-byte record per 64-token chunk and head, about
+ *     1.2 KiB per token per head, e.g. 896 tokens at 32 heads) returns
+ *     KDA_ERR_WORKSPACE and launches nothing.
  *   - The first call on each device looks up that device's address of the
  *     array (cudaGetSymbolAddress, with the device current).  Make that first
  *     call before any stream capture.
