@@ -11,6 +11,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "umma.cuh"
@@ -57,6 +58,35 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&x)[8]) {
     x[2 * i] = f.x;
     x[2 * i + 1] = f.y;
   }
+}
+
+// ---- two-lane fp32 arithmetic (sm_100 FFMA2 / FMUL2 / FADD2: each lane rounds
+// exactly like the scalar instruction) and bf16 pair conversions
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+// bf16 pair in one 32-bit word (lower address in the low half) -> (low, high) as fp32
+__device__ __forceinline__ float2 bf2_f2(uint32_t u) {
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+__device__ __forceinline__ uint32_t f2_bf2(float2 v) { return pack_bf16(v.x, v.y); }
+__device__ __forceinline__ uint32_t word(const uint4 &u, int i) {
+  return i == 0 ? u.x : (i == 1 ? u.y : (i == 2 ? u.z : u.w));
+}
+__device__ __forceinline__ float2 ex2_2(float2 x) {
+  return make_float2(umma::ex2(x.x), umma::ex2(x.y));
+}
+// SiLU(x) = x sigmoid(x) with sigmoid(x) = 1/2 + tanh(x/2)/2, the tanh taken two
+// lanes at a time in half precision on the special-function unit (absolute
+// error of the sigmoid about 2^-12, below the bf16 rounding of the result).
+__device__ __forceinline__ float2 silu2(float2 x) {
+  const float2 hx = mul2(x, f2(0.5f));
+  uint32_t h, t;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(hx.y), "f"(hx.x));
+  asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(h));
+  const float2 th = __half22float2(*reinterpret_cast<const __half2 *>(&t));
+  return mul2(x, fma2(th, f2(0.5f), f2(0.5f)));
 }
 
 // K-major descriptor over a token-rows operand with `rows` rows, K = 128 channels, k-step s.

@@ -19,7 +19,11 @@
 // (with the 3 tokens before it for the causal conv) and alpha arrive by TMA;
 // conv4 + SiLU, the L2 norm of q and k, the gate and beta are computed here,
 // so those intermediates never travel through device memory.  The other
-// variant reads them prepared (the recurrence entry point).
+// variant reads them prepared (the recurrence entry point).  Elementwise work
+// runs two fp32 lanes per instruction; the SiLU's sigmoid is 1/2 + tanh(x/2)/2
+// with the tanh in half precision on the special-function unit (absolute
+// error about 2^-12, under the bf16 rounding of q, k, v); the gate and every
+// decay factor stay in fp32.
 //
 // Numerics: Gamma reaches 64 * (-5) = -320 inside a chunk, so e^{-Gamma}
 // overflows fp32.  The pairwise factor e^{Gamma_t - Gamma_s} is only ever split
@@ -76,8 +80,9 @@ constexpr uint32_t OFF_V = 90112;             // v: 16 KB (written as soon as v 
 // Per-channel constants of the chunk (after the prologue, which stages the conv
 // weights and dt_bias of the head in the same bytes):
 constexpr uint32_t OFF_C = 106496;
-constexpr uint32_t OFF_WCONV = OFF_C;         // [3][128][4] bf16
-constexpr uint32_t OFF_DTB = OFF_C + 3072;    // [128] fp32
+constexpr uint32_t OFF_WCONV = OFF_C;         // [3][8 x 144 B]: 16 channels x 4 taps bf16 per 144 B
+constexpr uint32_t WSEG = 144;                // padded segment stride: conflict-free 16-byte reads
+constexpr uint32_t OFF_DTB = OFF_C + 3 * 8 * WSEG;   // [128] fp32
 constexpr uint32_t C_R = OFF_C;               // r_I, I = 0..4 (r_0 = 0)         [5][128]
 constexpr uint32_t C_CR = OFF_C + 2560;       // 2^{r_2-r_1}, 2^{r_3-r_1}, 2^{r_3-r_2}  [3][128]
 constexpr uint32_t OFF_WTOT = OFF_C + 4096;   // per-warp gate sums [8][128], then their prefixes
@@ -93,6 +98,12 @@ static_assert(OFF_ST + 64 * TSS * 4 <= OFF_TB && OFF_TB + 8192 <= OFF_KT && OFF_
 static_assert(OFF_TB % 1024 == 0 && OFF_KT % 1024 == 0 && OFF_V % 1024 == 0 && OFF_R % 1024 == 0,
               "SW128 alignment");
 static_assert(OFF_DTB + 512 <= OFF_WTOT && C_CR + 1536 <= OFF_WTOT, "constant area");
+static_assert(OFF_DTB % 16 == 0 && WSEG % 16 == 0, "bulk copy alignment");
+
+// A per-channel vector of 128 floats is stored as two halves: channels 8c..8c+3
+// of every channel group c, then channels 8c+4..8c+7, so that the 8-channel
+// group of a thread is two 16-byte reads that fall in distinct banks.
+__device__ __forceinline__ int cpos(int ch) { return ((ch & 7) >> 2) * 64 + (ch >> 3) * 4 + (ch & 3); }
 static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
 
 // R_all rows: [0,64) diagonal-reference rows, then R_1 (16 rows), R_2 (32), R_3 (48).
@@ -112,23 +123,18 @@ __device__ __forceinline__ bool wait_vote(uint64_t *bar, uint32_t parity, bool o
   return all;
 }
 
-__device__ __forceinline__ void lds8(const uint8_t *p, float (&x)[8]) {
-  const float4 u = *reinterpret_cast<const float4 *>(p);
-  const float4 w = *reinterpret_cast<const float4 *>(p + 16);
-  x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w; x[4] = w.x; x[5] = w.y; x[6] = w.z; x[7] = w.w;
-}
-
 // Off-diagonal blocks of T in the columns [col, col + NC) of column block J:
 // for I = J+1..3,  X = sum_{K=J}^{I-1} B_IK T_KJ,  T_IJ = -T_II X  (one warp;
 // lane = row r of the block and a group of NC columns).  X is parked where T_IJ
 // goes; no other warp touches these columns.
 template <int J, int NC>
 __device__ __forceinline__ void solve_columns(const float *sB, float *sT, int col, int r) {
+  constexpr int NP = NC / 2;   // column pairs
 #pragma unroll
   for (int I = J + 1; I < 4; ++I) {
-    float x[NC];
+    float2 x[NP];
 #pragma unroll
-    for (int c = 0; c < NC; ++c) x[c] = 0.f;
+    for (int c = 0; c < NP; ++c) x[c] = f2(0.f);
 #pragma unroll
     for (int K = J; K < I; ++K) {
 #pragma unroll
@@ -139,26 +145,22 @@ __device__ __forceinline__ void solve_columns(const float *sB, float *sT, int co
         for (int e = 0; e < 4; ++e) {
           const float *trow = sT + (16 * K + 4 * m4 + e) * TSS + col;
           if constexpr (NC == 2) {
-            const float2 tv = *reinterpret_cast<const float2 *>(trow);
-            x[0] = fmaf(bb[e], tv.x, x[0]);
-            x[1] = fmaf(bb[e], tv.y, x[1]);
+            x[0] = fma2(f2(bb[e]), *reinterpret_cast<const float2 *>(trow), x[0]);
           } else {
             const float4 tv = *reinterpret_cast<const float4 *>(trow);
-            x[0] = fmaf(bb[e], tv.x, x[0]);
-            x[1] = fmaf(bb[e], tv.y, x[1]);
-            x[2] = fmaf(bb[e], tv.z, x[2]);
-            x[3] = fmaf(bb[e], tv.w, x[3]);
+            x[0] = fma2(f2(bb[e]), make_float2(tv.x, tv.y), x[0]);
+            x[1] = fma2(f2(bb[e]), make_float2(tv.z, tv.w), x[1]);
           }
         }
       }
     }
     float *dst = sT + (16 * I + r) * TSS + col;
 #pragma unroll
-    for (int c = 0; c < NC; ++c) dst[c] = x[c];
+    for (int c = 0; c < NP; ++c) *reinterpret_cast<float2 *>(dst + 2 * c) = x[c];
     __syncwarp();
-    float y[NC];
+    float2 y[NP];
 #pragma unroll
-    for (int c = 0; c < NC; ++c) y[c] = 0.f;
+    for (int c = 0; c < NP; ++c) y[c] = f2(0.f);
 #pragma unroll
     for (int m4 = 0; m4 < 4; ++m4) {
       const float4 tv = *reinterpret_cast<const float4 *>(sT + (16 * I + r) * TSS + 16 * I + 4 * m4);
@@ -167,12 +169,12 @@ __device__ __forceinline__ void solve_columns(const float *sB, float *sT, int co
       for (int e = 0; e < 4; ++e) {
         const float *xrow = sT + (16 * I + 4 * m4 + e) * TSS + col;
 #pragma unroll
-        for (int c = 0; c < NC; ++c) y[c] = fmaf(tt[e], xrow[c], y[c]);
+        for (int c = 0; c < NP; ++c) y[c] = fma2(f2(tt[e]), *reinterpret_cast<const float2 *>(xrow + 2 * c), y[c]);
       }
     }
     __syncwarp();
 #pragma unroll
-    for (int c = 0; c < NC; ++c) dst[c] = -y[c];
+    for (int c = 0; c < NP; ++c) *reinterpret_cast<float2 *>(dst + 2 * c) = mul2(y[c], f2(-1.f));
     __syncwarp();
   }
 }
@@ -241,24 +243,30 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
 
   // ---------------------------------------------------------------- inputs
   uint4 qb[4], kb[4];          // bf16 q, k (normalised) of this thread's 4 tokens x 8 channels
-  float g2[4][8];              // gate in base 2
+  float2 g2[4][4];             // gate in base 2, [token][channel pair]
   float btj = 0.f;             // beta of token tid (tid < 64)
   if constexpr (kFused) {
-    if (tid == 0) {
-      umma::mbar_arrive_expect_tx(bar_tma, TMA_BYTES);
-      const int x = h * DK;
-      umma::tma_load_2d(smem + OFF_RAWQ, &a.map_q, x, (int)c0 - 3, bar_tma);
-      umma::tma_load_2d(smem + OFF_RAWK, &a.map_k, x, (int)c0 - 3, bar_tma);
-      umma::tma_load_2d(smem + OFF_RAWV, &a.map_v, x, (int)c0 - 3, bar_tma);
-      umma::tma_load_2d(smem + OFF_RAWA, &a.map_alpha, x, (int)c0, bar_tma);
-      const __nv_bfloat16 *cw = reinterpret_cast<const __nv_bfloat16 *>(a.conv_w);
-#pragma unroll
-      for (int blk = 0; blk < 3; ++blk)
-        umma::bulk_g2s(smem + OFF_WCONV + blk * 1024, cw + ((int64_t)blk * H + h) * DK * KCONV, 1024,
-                       bar_tma);
-      umma::bulk_g2s(smem + OFF_DTB, a.dt_bias + h * DK, 512, bar_tma);
+    if (warp == 0) {
+      if (lane == 0) {
+        umma::mbar_arrive_expect_tx(bar_tma, TMA_BYTES);
+        const int x = h * DK;
+        umma::tma_load_2d(smem + OFF_RAWQ, &a.map_q, x, (int)c0 - 3, bar_tma);
+        umma::tma_load_2d(smem + OFF_RAWK, &a.map_k, x, (int)c0 - 3, bar_tma);
+        umma::tma_load_2d(smem + OFF_RAWV, &a.map_v, x, (int)c0 - 3, bar_tma);
+        umma::tma_load_2d(smem + OFF_RAWA, &a.map_alpha, x, (int)c0, bar_tma);
+      }
+      __syncwarp();
+      if (lane < 24) {   // conv weights: 3 tensors x 8 segments of 16 channels
+        const int blk = lane >> 3, sg = lane & 7;
+        const __nv_bfloat16 *cw = reinterpret_cast<const __nv_bfloat16 *>(a.conv_w);
+        umma::bulk_g2s(smem + OFF_WCONV + (blk * 8 + sg) * WSEG,
+                       cw + (((int64_t)blk * H + h) * DK + sg * 16) * KCONV, 128, bar_tma);
+      } else if (lane == 24) {
+        umma::bulk_g2s(smem + OFF_DTB, a.dt_bias + h * DK, 512, bar_tma);
+      }
     }
-    const float negA = -expf(a.A_log[h]);
+    const float negA2 = -expf(a.A_log[h]) * LOG2E;   // the gate is kept in base 2
+    const float lb2 = a.lower_bound * LOG2E;
     if (tid < 64 && tid < nt)
       btj = sigmoid_f(__bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(a.b)[(c0 + tid) * H + h]));
     // causal-conv history of a sequence's first chunk: the caller's conv state or zeros
@@ -284,71 +292,79 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
           *reinterpret_cast<uint4 *>(smem + (blk == 0 ? OFF_RAWQ : blk == 1 ? OFF_RAWK : OFF_RAWV) +
                                      m * RAW_ROW + cg * 16) = hraw[blk][m];
     }
-    // gate g = max(-exp(A_log) softplus(alpha + dt_bias), lower_bound), kept in base 2
-    float bias[8];
-    lds8(smem + OFF_DTB + cg * 32, bias);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      float al[8];
-      unpack8(*reinterpret_cast<const uint4 *>(smem + OFF_RAWA + (4 * tg + j) * RAW_ROW + cg * 16), al);
-      const bool valid = 4 * tg + j < nt;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        g2[j][i] = valid ? gate_f(al[i] + bias[i], negA, a.lower_bound) * LOG2E : 0.f;
-    }
-    // conv4 + SiLU (+ L2 norm over the head's 128 channels for q and k)
+    // conv4 + SiLU (+ L2 norm over the head's 128 channels for q and k), two
+    // channels at a time; v first, it goes straight into its operand tile
 #pragma unroll
     for (int bi = 0; bi < 3; ++bi) {
-      const int blk = bi == 0 ? 2 : bi - 1;   // v first: it goes straight to its tile
+      const int blk = bi == 0 ? 2 : bi - 1;
       const uint8_t *raw = smem + (blk == 0 ? OFF_RAWQ : blk == 1 ? OFF_RAWK : OFF_RAWV) + cg * 16;
-      // by channel pair: the pair's 4 taps x 2 channels (16 bytes) and its 7 input rows
-      float y[4][8];
+      uint4 xr[7];   // input rows 4tg .. 4tg+6 (tokens 4tg-3 .. 4tg+3), 8 channels each
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        float wt[8];   // taps 0..3 of channel 2q4, then of channel 2q4+1
-        unpack8(*reinterpret_cast<const uint4 *>(smem + OFF_WCONV + blk * 1024 + cg * 64 + q4 * 16), wt);
-        float xa[7], xb[7];
+      for (int r = 0; r < 7; ++r) xr[r] = *reinterpret_cast<const uint4 *>(raw + (4 * tg + r) * RAW_ROW);
+      float2 y[4][4];
 #pragma unroll
-        for (int r = 0; r < 7; ++r) {
-          const uint32_t u = *reinterpret_cast<const uint32_t *>(raw + (4 * tg + r) * RAW_ROW + q4 * 4);
-          xa[r] = __uint_as_float(u << 16);
-          xb[r] = __uint_as_float(u & 0xffff0000u);
-        }
+      for (int p = 0; p < 4; ++p) {
+        // taps of channels 2p and 2p+1: (t0 t1), (t2 t3) of each, 16 bytes
+        const uint4 wq = *reinterpret_cast<const uint4 *>(smem + OFF_WCONV + (blk * 8 + (cg >> 1)) * WSEG +
+                                                          (cg & 1) * 64 + p * 16);
+        const float2 wa = bf2_f2(wq.x), wb = bf2_f2(wq.y), wc = bf2_f2(wq.z), wd = bf2_f2(wq.w);
+        const float2 w0 = make_float2(wa.x, wc.x), w1 = make_float2(wa.y, wc.y);
+        const float2 w2 = make_float2(wb.x, wd.x), w3 = make_float2(wb.y, wd.y);
+        float2 x[7];
+#pragma unroll
+        for (int r = 0; r < 7; ++r) x[r] = bf2_f2(word(xr[r], p));
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          float acc0 = wt[0] * xa[j], acc1 = wt[4] * xb[j];
-#pragma unroll
-          for (int m = 1; m < KCONV; ++m) {
-            acc0 = fmaf(wt[m], xa[j + m], acc0);
-            acc1 = fmaf(wt[4 + m], xb[j + m], acc1);
-          }
-          y[j][2 * q4] = silu_f(acc0);
-          y[j][2 * q4 + 1] = silu_f(acc1);
+          float2 acc = mul2(w0, x[j]);
+          acc = fma2(w1, x[j + 1], acc);
+          acc = fma2(w2, x[j + 2], acc);
+          acc = fma2(w3, x[j + 3], acc);
+          y[j][p] = silu2(acc);
         }
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        float yj[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) yj[i] = y[j][i];
         if (blk < 2) {
-          float ss = 0.f;
+          float2 ss = mul2(y[j][0], y[j][0]);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) ss = fmaf(yj[i], yj[i], ss);
+          for (int p = 1; p < 4; ++p) ss = fma2(y[j][p], y[j][p], ss);
+          float s1 = ss.x + ss.y;
 #pragma unroll
-          for (int off = 8; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-          const float rn = rsqrtf(ss + a.eps);
+          for (int off = 8; off >= 1; off >>= 1) s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+          const float2 rn = f2(rsqrtf(s1 + a.eps));
 #pragma unroll
-          for (int i = 0; i < 8; ++i) yj[i] *= rn;
+          for (int p = 0; p < 4; ++p) y[j][p] = mul2(y[j][p], rn);
         }
-        if (4 * tg + j >= nt) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) yj[i] = 0.f;
-        }
-        const uint4 packed = pack8(yj);
+        const bool valid = 4 * tg + j < nt;
+        const uint4 packed = valid ? make_uint4(f2_bf2(y[j][0]), f2_bf2(y[j][1]), f2_bf2(y[j][2]), f2_bf2(y[j][3]))
+                                   : make_uint4(0, 0, 0, 0);
         if (blk == 0) qb[j] = packed;
         else if (blk == 1) kb[j] = packed;
         else *reinterpret_cast<uint4 *>(smem + OFF_V + tr_off(64, tg * 4 + j, cg)) = packed;
+      }
+    }
+    // gate g = max(-exp(A_log) softplus(alpha + dt_bias), lower_bound), in base 2;
+    // softplus(x) = max(x, 0) + ln 2 * log2(1 + 2^{-|x| log2 e})
+    float2 bias[4];
+    {
+      const float4 b0 = *reinterpret_cast<const float4 *>(smem + OFF_DTB + cg * 32);
+      const float4 b1 = *reinterpret_cast<const float4 *>(smem + OFF_DTB + cg * 32 + 16);
+      bias[0] = make_float2(b0.x, b0.y); bias[1] = make_float2(b0.z, b0.w);
+      bias[2] = make_float2(b1.x, b1.y); bias[3] = make_float2(b1.z, b1.w);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 ar = *reinterpret_cast<const uint4 *>(smem + OFF_RAWA + (4 * tg + j) * RAW_ROW + cg * 16);
+      const bool valid = 4 * tg + j < nt;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const float2 x = add2(bf2_f2(word(ar, p)), bias[p]);
+        const float2 e = ex2_2(mul2(make_float2(fabsf(x.x), fabsf(x.y)), f2(-LOG2E)));
+        const float2 l = add2(e, f2(1.f));
+        const float2 lg = make_float2(lg2_approx(l.x), lg2_approx(l.y));
+        const float2 sp = fma2(lg, f2(kLn2), make_float2(fmaxf(x.x, 0.f), fmaxf(x.y, 0.f)));
+        const float2 g = mul2(sp, f2(negA2));
+        g2[j][p] = valid ? make_float2(fmaxf(g.x, lb2), fmaxf(g.y, lb2)) : f2(0.f);
       }
     }
   } else {
@@ -368,11 +384,13 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
         const float4 gb = __ldcs(reinterpret_cast<const float4 *>(a.g + off + 4));
         const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) g2[j][i] = fminf(fmaxf(gg[i], a.lower_bound), 0.f) * LOG2E;
+        for (int p = 0; p < 4; ++p)
+          g2[j][p] = make_float2(fminf(fmaxf(gg[2 * p], a.lower_bound), 0.f) * LOG2E,
+                                 fminf(fmaxf(gg[2 * p + 1], a.lower_bound), 0.f) * LOG2E);
       } else {
         qb[j] = kb[j] = vr[j] = make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) g2[j][i] = 0.f;
+        for (int p = 0; p < 4; ++p) g2[j][p] = f2(0.f);
       }
     }
     if (tid < 64 && tid < nt) btj = __ldcs(a.beta + (c0 + tid) * H + h);
@@ -383,119 +401,129 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
 
   // ---------------------------------------------------------------- cumulative gate
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int p = 0; p < 4; ++p) {
 #pragma unroll
-    for (int j = 1; j < 4; ++j) g2[j][i] += g2[j - 1][i];
-    const float lo = __shfl_up_sync(0xffffffffu, g2[3][i], 16);
+    for (int j = 1; j < 4; ++j) g2[j][p] = add2(g2[j][p], g2[j - 1][p]);
+    const float2 lo = make_float2(__shfl_up_sync(0xffffffffu, g2[3][p].x, 16),
+                                  __shfl_up_sync(0xffffffffu, g2[3][p].y, 16));
     if (lane >= 16) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) g2[j][i] += lo;
+      for (int j = 0; j < 4; ++j) g2[j][p] = add2(g2[j][p], lo);
     }
   }
   if (lane >= 16) {
-    *reinterpret_cast<float4 *>(wtot + warp * 128 + cg * 8) = make_float4(g2[3][0], g2[3][1], g2[3][2], g2[3][3]);
-    *reinterpret_cast<float4 *>(wtot + warp * 128 + cg * 8 + 4) = make_float4(g2[3][4], g2[3][5], g2[3][6], g2[3][7]);
+    *reinterpret_cast<float4 *>(wtot + warp * 128 + cg * 4) = make_float4(g2[3][0].x, g2[3][0].y, g2[3][1].x, g2[3][1].y);
+    *reinterpret_cast<float4 *>(wtot + warp * 128 + 64 + cg * 4) = make_float4(g2[3][2].x, g2[3][2].y, g2[3][3].x, g2[3][3].y);
   }
   if (tid < 64) beta_s[tid] = btj;
   __syncthreads();   // also: every read of the prologue staging is done
   // per channel: exclusive prefix of the warp sums (in place), r_1..r_4 and the R-row constants
   if (tid < 128) {
+    const int pc = cpos(tid);   // this thread's channel, in the split-half layout
     float acc = 0.f, r[5];
     r[0] = 0.f;
 #pragma unroll
     for (int w2 = 0; w2 < 8; ++w2) {
-      const float x = wtot[w2 * 128 + tid];
-      wtot[w2 * 128 + tid] = acc;
+      const float x = wtot[w2 * 128 + pc];
+      wtot[w2 * 128 + pc] = acc;
       acc += x;
       if (w2 & 1) r[(w2 >> 1) + 1] = acc;
     }
     float *cf = reinterpret_cast<float *>(smem);
 #pragma unroll
-    for (int I = 0; I < 5; ++I) cf[C_R / 4 + I * 128 + tid] = r[I];
-    cf[C_CR / 4 + 0 * 128 + tid] = umma::ex2(r[2] - r[1]);
-    cf[C_CR / 4 + 1 * 128 + tid] = umma::ex2(r[3] - r[1]);
-    cf[C_CR / 4 + 2 * 128 + tid] = umma::ex2(r[3] - r[2]);
+    for (int I = 0; I < 5; ++I) cf[C_R / 4 + I * 128 + pc] = r[I];
+    cf[C_CR / 4 + 0 * 128 + pc] = umma::ex2(r[2] - r[1]);
+    cf[C_CR / 4 + 1 * 128 + pc] = umma::ex2(r[3] - r[1]);
+    cf[C_CR / 4 + 2 * 128 + pc] = umma::ex2(r[3] - r[2]);
     reinterpret_cast<float *>(rec + REC_EGC)[tid] = umma::ex2(r[4]);   // e^{Gamma_C}
   }
   __syncthreads();
 
   // ---------------------------------------------------------------- operands
+  const uint32_t coff = (uint32_t)cg * 16;
+  auto lds_pairs = [&](uint32_t off, float2 (&x)[4]) {   // this thread's 8 channels of a split-half vector
+    const float4 u = *reinterpret_cast<const float4 *>(smem + off + coff);
+    const float4 w = *reinterpret_cast<const float4 *>(smem + off + 256 + coff);
+    x[0] = make_float2(u.x, u.y); x[1] = make_float2(u.z, u.w);
+    x[2] = make_float2(w.x, w.y); x[3] = make_float2(w.z, w.w);
+  };
   {
-    float pre[8];
-    lds8(smem + OFF_WTOT + (warp * 128 + cg * 8) * 4, pre);
+    float2 pre[4];
+    lds_pairs(OFF_WTOT + warp * 512, pre);
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) g2[j][i] += pre[i];   // Gamma_t (base 2)
+      for (int p = 0; p < 4; ++p) g2[j][p] = add2(g2[j][p], pre[p]);   // Gamma_t (base 2)
   }
-  const uint32_t coff = (uint32_t)(cg * 8) * 4;
   {  // L side: Lq = q e^{Gamma - r_I}, Lk likewise; q e^{Gamma}, k e^{Gamma}
-    float rI[8], eR[8];
-    lds8(smem + C_R + blkI * 512 + coff, rI);
+    float2 nrI[4], eR[4];
+    lds_pairs(C_R + blkI * 512, nrI);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) eR[i] = umma::ex2(rI[i]);
+    for (int p = 0; p < 4; ++p) {
+      eR[p] = ex2_2(nrI[p]);
+      nrI[p] = mul2(nrI[p], f2(-1.f));
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int t = tg * 4 + j;
-      float q[8], k[8], Lq[8], Lk[8], Qt[8], Kt[8];
-      unpack8(qb[j], q);
-      unpack8(kb[j], k);
+      uint32_t Lq[4], Lk[4], Qt[4], Kt[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float e1 = umma::ex2(g2[j][i] - rI[i]);   // in (2^-128, 1]
-        Lq[i] = q[i] * e1;
-        Lk[i] = k[i] * e1;
-        Qt[i] = Lq[i] * eR[i];
-        Kt[i] = Lk[i] * eR[i];
+      for (int p = 0; p < 4; ++p) {
+        const float2 e1 = ex2_2(add2(g2[j][p], nrI[p]));   // in (2^-128, 1]
+        const float2 lq = mul2(bf2_f2(word(qb[j], p)), e1);
+        const float2 lk = mul2(bf2_f2(word(kb[j], p)), e1);
+        Lq[p] = f2_bf2(lq);
+        Lk[p] = f2_bf2(lk);
+        Qt[p] = f2_bf2(mul2(lq, eR[p]));
+        Kt[p] = f2_bf2(mul2(lk, eR[p]));
       }
-      *reinterpret_cast<uint4 *>(smem + OFF_L + tr_off(128, t, cg)) = pack8(Lq);
-      *reinterpret_cast<uint4 *>(smem + OFF_L + tr_off(128, 64 + t, cg)) = pack8(Lk);
-      *reinterpret_cast<uint4 *>(smem + OFF_KT + tr_off(64, t, cg)) = pack8(Kt);
-      *reinterpret_cast<uint4 *>(rec + REC_QT + tr_off(64, t, cg)) = pack8(Qt);
+      *reinterpret_cast<uint4 *>(smem + OFF_L + tr_off(128, t, cg)) = make_uint4(Lq[0], Lq[1], Lq[2], Lq[3]);
+      *reinterpret_cast<uint4 *>(smem + OFF_L + tr_off(128, 64 + t, cg)) = make_uint4(Lk[0], Lk[1], Lk[2], Lk[3]);
+      *reinterpret_cast<uint4 *>(smem + OFF_KT + tr_off(64, t, cg)) = make_uint4(Kt[0], Kt[1], Kt[2], Kt[3]);
+      *reinterpret_cast<uint4 *>(rec + REC_QT + tr_off(64, t, cg)) = make_uint4(Qt[0], Qt[1], Qt[2], Qt[3]);
     }
   }
   {  // R side: kd = k e^{r_{I+1} - Gamma}; Rd = kd e^{r_I - r_{I+1}}; R_{I+1..3} rows; k e^{Gamma_C - Gamma}
-    float rI1[8], cD[8], cK[8], cA[8], cB[8];
+    float2 rI1[4], cD[4], cK[4], cA[4], cB[4];
     {
-      float rI[8], r4[8];
-      lds8(smem + C_R + blkI * 512 + coff, rI);
-      lds8(smem + C_R + (blkI + 1) * 512 + coff, rI1);
-      lds8(smem + C_R + 4 * 512 + coff, r4);
+      float2 rI[4], r4[4];
+      lds_pairs(C_R + blkI * 512, rI);
+      lds_pairs(C_R + (blkI + 1) * 512, rI1);
+      lds_pairs(C_R + 4 * 512, r4);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        cD[i] = umma::ex2(rI[i] - rI1[i]);   // 2^{r_I - r_{I+1}}
-        cK[i] = umma::ex2(r4[i] - rI1[i]);   // 2^{r_4 - r_{I+1}}
+      for (int p = 0; p < 4; ++p) {
+        const float2 nr = mul2(rI1[p], f2(-1.f));
+        cD[p] = ex2_2(add2(rI[p], nr));   // 2^{r_I - r_{I+1}}
+        cK[p] = ex2_2(add2(r4[p], nr));   // 2^{r_4 - r_{I+1}}
       }
     }
-    if (blkI < 2) lds8(smem + C_CR + (blkI == 0 ? 0 : 2) * 512 + coff, cA);   // 2^{r_{I+2} - r_{I+1}}
-    if (blkI == 0) lds8(smem + C_CR + 512 + coff, cB);                       // 2^{r_3 - r_1}
+    if (blkI < 2) lds_pairs(C_CR + (blkI == 0 ? 0 : 2) * 512, cA);   // 2^{r_{I+2} - r_{I+1}}
+    if (blkI == 0) lds_pairs(C_CR + 512, cB);                       // 2^{r_3 - r_1}
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int t = tg * 4 + j;
-      float k[8], kd[8], Rd[8], Kh[8];
-      unpack8(kb[j], k);
+      uint32_t Rd[4], Kh[4], K1[4], K2[4], K3[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        kd[i] = k[i] * umma::ex2(rI1[i] - g2[j][i]);   // |kd| <= |k|
-        Rd[i] = kd[i] * cD[i];
-        Kh[i] = kd[i] * cK[i];
+      for (int p = 0; p < 4; ++p) {
+        const float2 kd = mul2(bf2_f2(word(kb[j], p)),
+                               ex2_2(add2(rI1[p], mul2(g2[j][p], f2(-1.f)))));   // |kd| <= |k|
+        Rd[p] = f2_bf2(mul2(kd, cD[p]));
+        Kh[p] = f2_bf2(mul2(kd, cK[p]));
+        K1[p] = f2_bf2(kd);
+        K2[p] = blkI < 2 ? f2_bf2(mul2(kd, cA[p])) : 0u;
+        K3[p] = blkI == 0 ? f2_bf2(mul2(kd, cB[p])) : 0u;
       }
-      *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, t, cg)) = pack8(Rd);
-      *reinterpret_cast<uint4 *>(rec + REC_KH + tr_off(64, t, cg)) = pack8(Kh);
+      *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, t, cg)) = make_uint4(Rd[0], Rd[1], Rd[2], Rd[3]);
+      *reinterpret_cast<uint4 *>(rec + REC_KH + tr_off(64, t, cg)) = make_uint4(Kh[0], Kh[1], Kh[2], Kh[3]);
       if (blkI < 3)
-        *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, r_row0(blkI + 1) + t, cg)) = pack8(kd);
-      if (blkI < 2) {
-        float x[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = kd[i] * cA[i];
-        *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, r_row0(blkI + 2) + t, cg)) = pack8(x);
-      }
-      if (blkI == 0) {
-        float x[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = kd[i] * cB[i];
-        *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, r_row0(3) + t, cg)) = pack8(x);
-      }
+        *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, r_row0(blkI + 1) + t, cg)) =
+            make_uint4(K1[0], K1[1], K1[2], K1[3]);
+      if (blkI < 2)
+        *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, r_row0(blkI + 2) + t, cg)) =
+            make_uint4(K2[0], K2[1], K2[2], K2[3]);
+      if (blkI == 0)
+        *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, r_row0(3) + t, cg)) =
+            make_uint4(K3[0], K3[1], K3[2], K3[3]);
     }
   }
   umma::fence_proxy_async_smem();
@@ -528,24 +556,27 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
     const float bt = is_q ? 1.f : beta_s[t];
     const uint32_t tb = tmem + lane_base + TM_P;
     auto emit = [&](int gi, const uint32_t (&v)[16], bool zero, bool diag) {
-      float x[16];
+      if (is_q) {   // A_qk row t, s <= t, bf16 into the record
+        uint32_t w8[8];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int s = 16 * gi + e;
-        const bool keep = !zero && (!diag || (is_q ? s <= t : s < t));
-        x[e] = keep ? __uint_as_float(v[e]) * bt : 0.f;
-      }
-      if (is_q) {
-        float lo8[8], hi8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) { lo8[e] = x[e]; hi8[e] = x[8 + e]; }
-        *reinterpret_cast<uint4 *>(rec + REC_AQ + tr_off(64, t, 2 * gi)) = pack8(lo8);
-        *reinterpret_cast<uint4 *>(rec + REC_AQ + tr_off(64, t, 2 * gi + 1)) = pack8(hi8);
-      } else {
+        for (int e2 = 0; e2 < 8; ++e2) {
+          const int s = 16 * gi + 2 * e2;
+          const bool k0 = !zero && (!diag || s <= t), k1 = !zero && (!diag || s + 1 <= t);
+          w8[e2] = pack_bf16(k0 ? __uint_as_float(v[2 * e2]) : 0.f, k1 ? __uint_as_float(v[2 * e2 + 1]) : 0.f);
+        }
+        *reinterpret_cast<uint4 *>(rec + REC_AQ + tr_off(64, t, 2 * gi)) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+        *reinterpret_cast<uint4 *>(rec + REC_AQ + tr_off(64, t, 2 * gi + 1)) = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+      } else {      // beta_t A_kk row t, s < t, fp32 into the solve scratch
         float4 *dst = reinterpret_cast<float4 *>(sBm + t * TSS + 16 * gi);
 #pragma unroll
-        for (int e4 = 0; e4 < 4; ++e4)
-          dst[e4] = make_float4(x[4 * e4], x[4 * e4 + 1], x[4 * e4 + 2], x[4 * e4 + 3]);
+        for (int e4 = 0; e4 < 4; ++e4) {
+          const int s = 16 * gi + 4 * e4;
+          const float2 lo = mul2(make_float2(__uint_as_float(v[4 * e4]), __uint_as_float(v[4 * e4 + 1])), f2(bt));
+          const float2 hi = mul2(make_float2(__uint_as_float(v[4 * e4 + 2]), __uint_as_float(v[4 * e4 + 3])), f2(bt));
+          const bool k0 = !zero && (!diag || s < t), k1 = !zero && (!diag || s + 1 < t);
+          const bool k2 = !zero && (!diag || s + 2 < t), k3 = !zero && (!diag || s + 3 < t);
+          dst[e4] = make_float4(k0 ? lo.x : 0.f, k1 ? lo.y : 0.f, k2 ? hi.x : 0.f, k3 ? hi.y : 0.f);
+        }
       }
     };
     uint32_t va[16], vb2[16], v[16];
@@ -619,12 +650,22 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   for (int it = 0; it < 2; ++it) {  // T_b rows as bf16, K-major [t][s]
     const int e = tid + it * NT;
     const int t = e >> 3, c8 = e & 7;
-    float tv[8], bv[8], x8[8];
-    lds8(reinterpret_cast<const uint8_t *>(sTm + t * TSS + c8 * 8), tv);
-    lds8(reinterpret_cast<const uint8_t *>(beta_s + c8 * 8), bv);
+    const float4 t0 = *reinterpret_cast<const float4 *>(sTm + t * TSS + c8 * 8);
+    const float4 t1 = *reinterpret_cast<const float4 *>(sTm + t * TSS + c8 * 8 + 4);
+    const float4 b0 = *reinterpret_cast<const float4 *>(beta_s + c8 * 8);
+    const float4 b1 = *reinterpret_cast<const float4 *>(beta_s + c8 * 8 + 4);
+    const float2 p0 = mul2(make_float2(t0.x, t0.y), make_float2(b0.x, b0.y));
+    const float2 p1 = mul2(make_float2(t0.z, t0.w), make_float2(b0.z, b0.w));
+    const float2 p2 = mul2(make_float2(t1.x, t1.y), make_float2(b1.x, b1.y));
+    const float2 p3 = mul2(make_float2(t1.z, t1.w), make_float2(b1.z, b1.w));
+    const float x8[8] = {p0.x, p0.y, p1.x, p1.y, p2.x, p2.y, p3.x, p3.y};
+    uint32_t w4[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) x8[i] = c8 * 8 + i <= t ? tv[i] * bv[i] : 0.f;
-    *reinterpret_cast<uint4 *>(smem + OFF_TB + tr_off(64, t, c8)) = pack8(x8);
+    for (int i = 0; i < 4; ++i) {
+      const int s0 = c8 * 8 + 2 * i;
+      w4[i] = pack_bf16(s0 <= t ? x8[2 * i] : 0.f, s0 + 1 <= t ? x8[2 * i + 1] : 0.f);
+    }
+    *reinterpret_cast<uint4 *>(smem + OFF_TB + tr_off(64, t, c8)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
   }
   umma::fence_proxy_async_smem();
   umma::fence_before_sync();
@@ -633,11 +674,12 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   // ---------------------------------------------------------------- W^T, U^T (P has been read)
   if (tid == 0) {
     umma::fence_after_sync();
-    const uint32_t idesc = umma::make_idesc_bf16(128, 64, 1, 0);
+    const uint32_t idesc_w = umma::make_idesc_bf16(128, 64, 1, 0, 1);   // -W^T: A negated
+    const uint32_t idesc_u = umma::make_idesc_bf16(128, 64, 1, 0);
 #pragma unroll
     for (int s = 0; s < CH / 16; ++s) {
-      umma::mma_ss(tmem + TM_W, desc_mn_tok(sbase + OFF_KT, s), desc_k64(sbase + OFF_TB, s), idesc, s > 0);
-      umma::mma_ss(tmem + TM_U, desc_mn_tok(sbase + OFF_V, s), desc_k64(sbase + OFF_TB, s), idesc, s > 0);
+      umma::mma_ss(tmem + TM_W, desc_mn_tok(sbase + OFF_KT, s), desc_k64(sbase + OFF_TB, s), idesc_w, s > 0);
+      umma::mma_ss(tmem + TM_U, desc_mn_tok(sbase + OFF_V, s), desc_k64(sbase + OFF_TB, s), idesc_u, s > 0);
     }
     umma::mma_commit(bar_mma);
   }
@@ -647,7 +689,6 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   if (ok) {
     const int i = (warp & 3) * 32 + lane;   // TMEM lane: key channel (W^T) / value channel (U^T)
     const bool isW = warp < 4;
-    const float sign = isW ? -1.f : 1.f;
     uint8_t *dst = rec + (isW ? REC_WT : REC_U);
 #pragma unroll
     for (int c32 = 0; c32 < 2; ++c32) {
@@ -656,10 +697,11 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
       umma::tmem_wait_ld();
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
-        float x8[8];
+        uint32_t w4[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x8[e] = sign * __uint_as_float(rr[q4 * 8 + e]);
-        *reinterpret_cast<uint4 *>(dst + row64_off(i, c32 * 4 + q4)) = pack8(x8);
+        for (int e = 0; e < 4; ++e)
+          w4[e] = pack_bf16(__uint_as_float(rr[q4 * 8 + 2 * e]), __uint_as_float(rr[q4 * 8 + 2 * e + 1]));
+        *reinterpret_cast<uint4 *>(dst + row64_off(i, c32 * 4 + q4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
     }
   }

@@ -4,7 +4,7 @@
 //
 // Per 64-token chunk, with the record chunk_prep wrote (-W^T, U^T, A_qk,
 // q e^{Gamma}, k e^{Gamma_C - Gamma}, e^{Gamma_C}):
-//   D^T = U^T - S^T W^T                  (U^T enters the accumulator exactly: U^T x I)
+//   D^T = U^T - S^T W^T
 //   O^T = S^T (q e^{Gamma})^T + D^T A_qk^T
 //   S^T <- S^T diag(e^{Gamma_C}) + D^T (k e^{Gamma_C - Gamma})
 // i.e. the per-token loop of the AliceAI-Foundation KDA write-up ("二、KDA
@@ -15,6 +15,13 @@
 // Records arrive by one contiguous bulk copy each (they are stored as their
 // shared-memory image), double-buffered: the copy of chunk c+2 starts as soon
 // as chunk c's MMAs have read its buffer.
+//
+// Only D stands between one chunk's state and the next, so the chain per chunk
+// is: the S^T W^T MMA -> D + U to bf16 -> the state-update MMA -> the state's
+// bf16 copy.  The pass that makes that copy also applies the next chunk's decay
+// to the fp32 state (the next record is normally resident by then), and O is
+// double-buffered in TMEM so that chunk c-1's output leaves while chunk c's
+// MMAs run: transposed through shared memory into 16-byte row stores.
 #include "chunk_common.cuh"
 #include "kda_common.cuh"
 #include "kda_internal.h"
@@ -27,22 +34,21 @@ using namespace chunkfmt;
 constexpr int NT = 128;
 constexpr uint32_t OFF_REC0 = 0;
 constexpr uint32_t OFF_REC1 = REC_STRIDE;
-constexpr uint32_t OFF_ID = 2 * REC_STRIDE;        // 64x64 identity, K-major image: 8 KB
-constexpr uint32_t OFF_BAR = OFF_ID + 8192;
+constexpr uint32_t OFF_OST = 2 * REC_STRIDE;   // o of one chunk, bf16 [64 t][128 j]: 16 KB
+constexpr uint32_t OFF_BAR = OFF_OST + CH * DK * 2;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
-static_assert(REC_STRIDE % 1024 == 0 && OFF_ID % 1024 == 0, "SW128 alignment");
+static_assert(REC_STRIDE % 1024 == 0, "SW128 alignment");
 
 // TMEM columns (512 allocated)
 constexpr uint32_t TM_S32 = 0;     // S^T fp32, 128 cols
 constexpr uint32_t TM_S16 = 128;   // S^T bf16 A operand, 64 cols
-constexpr uint32_t TM_D = 192;     // D^T fp32, 64 cols
-constexpr uint32_t TM_D16 = 256;   // D^T bf16 A operand, 32 cols
-constexpr uint32_t TM_O = 288;     // O^T fp32, 64 cols
+constexpr uint32_t TM_D = 192;     // D^T fp32, 64 cols; its bf16 copy (32 cols) is packed in place
+constexpr uint32_t TM_O = 256;     // O^T fp32, 2 x 64 cols (chunk parity)
 
 constexpr uint32_t WAIT_POLLS = 1u << 22;
-enum { B_FULL0 = 0, B_FULL1, B_MMA, B_COUNT };
+enum { B_FULL0 = 0, B_FULL1, B_D, B_S, B_COUNT };
 
 __device__ __forceinline__ bool wait_vote(uint64_t *bar, uint32_t parity, bool ok) {
   const bool mine = ok && umma::mbar_wait_bounded(bar, parity, WAIT_POLLS);
@@ -84,17 +90,6 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(StateArgs a) {
     for (int i = 0; i < B_COUNT; ++i) umma::mbar_init(&bar[i], 1);
     umma::mbar_fence_init();
   }
-  // identity [64][64] as a K-major B operand (row t holds e_t)
-#pragma unroll
-  for (int it = 0; it < 4; ++it) {
-    const int e = tid + it * NT;         // 512 chunks of 16 bytes
-    const int t = e >> 3, c8 = e & 7;
-    float x8[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) x8[i] = (c8 * 8 + i == t) ? 1.f : 0.f;
-    *reinterpret_cast<uint4 *>(smem + OFF_ID + row64_off(t, c8)) = pack8(x8);
-  }
-  umma::fence_proxy_async_smem();
   umma::fence_before_sync();
   __syncthreads();
   umma::fence_after_sync();
@@ -123,58 +118,112 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(StateArgs a) {
   umma::fence_before_sync();
   __syncthreads();
 
+  // o of chunk cc (its O^T in TMEM columns ocol): lane j holds column j of the
+  // chunk's 64 rows; a shared-memory transpose turns them into 16-byte row stores
+  __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_OST);
+  auto emit_o = [&](int cc, uint32_t ocol) {
+    uint32_t r[2][32];
+    umma::tmem_ld32(tmem + lane_base + ocol, r[0]);
+    umma::tmem_ld32(tmem + lane_base + ocol + 32, r[1]);
+    umma::tmem_wait_ld();
+#pragma unroll
+    for (int t = 0; t < CH; ++t) ost[t * DK + j] = __float2bfloat16_rn(a.scale * __uint_as_float(r[t >> 5][t & 31]));
+    __syncthreads();
+    const int64_t c0 = s0 + (int64_t)cc * CH;
+    const int nvalid = (int)min((int64_t)CH, s1 - c0);
+#pragma unroll
+    for (int k = 0; k < CH * DK / 8 / NT; ++k) {
+      const int q = tid + k * NT, t = q >> 4, c16 = q & 15;
+      if (t < nvalid)
+        *reinterpret_cast<uint4 *>(o + ((c0 + t) * H + h) * DK + c16 * 8) =
+            *reinterpret_cast<const uint4 *>(ost + t * DK + c16 * 8);
+    }
+    __syncthreads();
+  };
+  // S^T columns *= e^{Gamma_C} of the record at rb; with bf16: also refresh the bf16 copy first
+  auto state_pass_over = [&](uint32_t rb, bool decay, bool bf16) {
+    const float4 *egc = reinterpret_cast<const float4 *>(smem + rb + REC_EGC);
+#pragma unroll
+    for (int cc = 0; cc < DK; cc += 64) {
+      uint32_t x[2][32];
+      umma::tmem_ld32(tmem + lane_base + TM_S32 + cc, x[0]);
+      umma::tmem_ld32(tmem + lane_base + TM_S32 + cc + 32, x[1]);
+      umma::tmem_wait_ld();
+      if (bf16) {
+        uint32_t p[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          p[e] = pack_bf16(__uint_as_float(x[e >> 4][(e & 15) * 2]), __uint_as_float(x[e >> 4][(e & 15) * 2 + 1]));
+        umma::tmem_st32(tmem + lane_base + TM_S16 + cc / 2, p);
+      }
+      if (decay) {
+#pragma unroll
+        for (int e4 = 0; e4 < 16; ++e4) {
+          const float4 g = egc[cc / 4 + e4];
+          uint32_t *y = &x[e4 >> 3][(e4 & 7) * 4];
+          const float2 lo = mul2(make_float2(__uint_as_float(y[0]), __uint_as_float(y[1])), make_float2(g.x, g.y));
+          const float2 hi = mul2(make_float2(__uint_as_float(y[2]), __uint_as_float(y[3])), make_float2(g.z, g.w));
+          y[0] = __float_as_uint(lo.x); y[1] = __float_as_uint(lo.y);
+          y[2] = __float_as_uint(hi.x); y[3] = __float_as_uint(hi.y);
+        }
+        umma::tmem_st32(tmem + lane_base + TM_S32 + cc, x[0]);
+        umma::tmem_st32(tmem + lane_base + TM_S32 + cc + 32, x[1]);
+      }
+    }
+    umma::tmem_wait_st();
+  };
+
   bool ok = true;
-  uint32_t ph_mma = 0;
 #pragma unroll 1
   for (int c = 0; c < nchunks; ++c) {
     const int b = c & 1;
     const uint32_t rb = b ? OFF_REC1 : OFF_REC0;
-    const int64_t c0 = s0 + (int64_t)c * CH;
+    const uint32_t ocol = TM_O + (uint32_t)b * 64;
     ok = wait_vote(&bar[B_FULL0 + b], (c >> 1) & 1, ok);
     if (!ok) break;
-    // D^T = U^T I + S^T (-W^T)   (committed alone: the next step needs only D^T); O^T = S^T Q~^T
+    if (c == 0) {   // the first chunk's decay (later ones ride on the previous chunk's last pass)
+      state_pass_over(rb, true, false);
+      umma::fence_before_sync();
+      __syncthreads();
+      umma::fence_after_sync();
+    }
+    // D^T = S^T (-W^T) (committed alone: the chain needs only D^T); O^T = S^T Q~^T
     if (tid == 0) {
-      const uint32_t id_u = umma::make_idesc_bf16(128, 64, 0, 0);
       const uint32_t id_d = umma::make_idesc_bf16(128, 64, 0, 1);
       const uint32_t id_o = umma::make_idesc_bf16(128, 64, 0, 0);
 #pragma unroll
-      for (int s = 0; s < CH / 16; ++s)
-        umma::mma_ss(tmem + TM_D, desc_k64(sbase + rb + REC_U, s), desc_k64(sbase + OFF_ID, s), id_u, s > 0);
-#pragma unroll
       for (int s = 0; s < DK / 16; ++s)
         umma::mma_ts(tmem + TM_D, tmem + TM_S16 + (uint32_t)(s * 8), desc_mn_rows(sbase + rb + REC_WT, s),
-                     id_d, 1);
-      umma::mma_commit(&bar[B_MMA]);
+                     id_d, s > 0);
+      umma::mma_commit(&bar[B_D]);
 #pragma unroll
       for (int s = 0; s < DK / 16; ++s)
-        umma::mma_ts(tmem + TM_O, tmem + TM_S16 + (uint32_t)(s * 8), desc_k128(sbase + rb + REC_QT, 64, s),
+        umma::mma_ts(tmem + ocol, tmem + TM_S16 + (uint32_t)(s * 8), desc_k128(sbase + rb + REC_QT, 64, s),
                      id_o, s > 0);
     }
-    ok = wait_vote(&bar[B_MMA], ph_mma, ok);
-    ph_mma ^= 1u;
+    // while those run: the previous chunk's o
+    if (c > 0) emit_o(c - 1, TM_O + (uint32_t)(b ^ 1) * 64);
+    ok = wait_vote(&bar[B_D], c & 1, ok);
     if (!ok) break;
-    // D^T -> bf16 A operand; decay the columns of S^T by e^{Gamma_C}
+    // D^T + U^T -> bf16 A operand, packed over the first 32 columns of D
     {
-      uint32_t r0[32], r1[32], p[32];
-      umma::tmem_ld32(tmem + lane_base + TM_D, r0);
-      umma::tmem_ld32(tmem + lane_base + TM_D + 32, r1);
+      uint32_t r[2][32], p[32];
+      umma::tmem_ld32(tmem + lane_base + TM_D, r[0]);
+      umma::tmem_ld32(tmem + lane_base + TM_D + 32, r[1]);
       umma::tmem_wait_ld();
+      const uint8_t *urow = smem + rb + REC_U;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        p[e] = pack_bf16(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
-        p[16 + e] = pack_bf16(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1]));
-      }
-      umma::tmem_st32(tmem + lane_base + TM_D16, p);
-      const float *egc = reinterpret_cast<const float *>(smem + rb + REC_EGC);
-#pragma unroll 1
-      for (int cc = 0; cc < DK; cc += 32) {
-        uint32_t s[32];
-        umma::tmem_ld32(tmem + lane_base + TM_S32 + cc, s);
-        umma::tmem_wait_ld();
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(urow + row64_off(j, c8));   // tokens 8c8 .. 8c8+7
+        const uint32_t *x = &r[c8 >> 2][(c8 & 3) * 8];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) s[e] = __float_as_uint(__uint_as_float(s[e]) * egc[cc + e]);
-        umma::tmem_st32(tmem + lane_base + TM_S32 + cc, s);
+        for (int w = 0; w < 4; ++w) {
+          const float2 d = add2(make_float2(__uint_as_float(x[2 * w]), __uint_as_float(x[2 * w + 1])),
+                                bf2_f2(word(u, w)));
+          p[4 * c8 + w] = f2_bf2(d);
+        }
       }
+      umma::tmem_st32(tmem + lane_base + TM_D, p);
       umma::tmem_wait_st();
     }
     umma::fence_before_sync();
@@ -186,53 +235,32 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(StateArgs a) {
       const uint32_t id_o = umma::make_idesc_bf16(128, 64, 0, 0);
 #pragma unroll
       for (int s = 0; s < CH / 16; ++s)
-        umma::mma_ts(tmem + TM_S32, tmem + TM_D16 + (uint32_t)(s * 8), desc_mn_tok(sbase + rb + REC_KH, s),
+        umma::mma_ts(tmem + TM_S32, tmem + TM_D + (uint32_t)(s * 8), desc_mn_tok(sbase + rb + REC_KH, s),
                      id_s, 1);
 #pragma unroll
       for (int s = 0; s < CH / 16; ++s)
-        umma::mma_ts(tmem + TM_O, tmem + TM_D16 + (uint32_t)(s * 8), desc_k64(sbase + rb + REC_AQ, s),
-                     id_o, 1);
-      umma::mma_commit(&bar[B_MMA]);
+        umma::mma_ts(tmem + ocol, tmem + TM_D + (uint32_t)(s * 8), desc_k64(sbase + rb + REC_AQ, s), id_o, 1);
+      umma::mma_commit(&bar[B_S]);
     }
-    ok = wait_vote(&bar[B_MMA], ph_mma, ok);
-    ph_mma ^= 1u;
+    ok = wait_vote(&bar[B_S], c & 1, ok);
     if (!ok) break;
     // this buffer has been read: start the copy of chunk c+2 into it
     if (tid == 0 && c + 2 < nchunks) {
       umma::mbar_arrive_expect_tx(&bar[B_FULL0 + b], REC_BYTES);
       umma::bulk_g2s(smem + rb, rec_ptr(c + 2), REC_BYTES, &bar[B_FULL0 + b]);
     }
-    // refresh the bf16 state copy (next chunk's A operand), then store O
-    {
-#pragma unroll 1
-      for (int cc = 0; cc < DK; cc += 32) {
-        uint32_t s[32], p[16];
-        umma::tmem_ld32(tmem + lane_base + TM_S32 + cc, s);
-        umma::tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) p[e] = pack_bf16(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1]));
-        umma::tmem_st16(tmem + lane_base + TM_S16 + cc / 2, p);
-      }
-      uint32_t r0[32], r1[32];
-      umma::tmem_ld32(tmem + lane_base + TM_O, r0);
-      umma::tmem_ld32(tmem + lane_base + TM_O + 32, r1);
-      umma::tmem_wait_ld();
-      umma::tmem_wait_st();
-      const int nvalid = (int)min((int64_t)CH, s1 - c0);
-      __nv_bfloat16 *orow = o + (c0 * H + h) * DK + j;
-#pragma unroll
-      for (int t = 0; t < 32; ++t)
-        if (t < nvalid) orow[(int64_t)t * H * DK] = __float2bfloat16_rn(a.scale * __uint_as_float(r0[t]));
-#pragma unroll
-      for (int t = 0; t < 32; ++t)
-        if (t + 32 < nvalid)
-          orow[(int64_t)(t + 32) * H * DK] = __float2bfloat16_rn(a.scale * __uint_as_float(r1[t]));
+    // the next chunk's A operand (bf16 copy of the state) and its decay, in one pass
+    if (c + 1 < nchunks) {
+      ok = wait_vote(&bar[B_FULL0 + (b ^ 1)], ((c + 1) >> 1) & 1, ok);
+      if (!ok) break;
+      state_pass_over(b ? OFF_REC0 : OFF_REC1, true, true);
     }
     umma::fence_before_sync();
     __syncthreads();
   }
-  // final state: S[i][j] = S^T[j][i]
   if (ok) {
+    if (nchunks > 0) emit_o(nchunks - 1, TM_O + (uint32_t)((nchunks - 1) & 1) * 64);
+    // final state: S[i][j] = S^T[j][i]
 #pragma unroll 1
     for (int cc = 0; cc < DK; cc += 32) {
       uint32_t s[32];
