@@ -18,10 +18,14 @@
 //
 // Only D stands between one chunk's state and the next, so the chain per chunk
 // is: the S^T W^T MMA -> D + U to bf16 -> the state-update MMA -> the state's
-// bf16 copy.  The pass that makes that copy also applies the next chunk's decay
-// to the fp32 state (the next record is normally resident by then), and O is
-// double-buffered in TMEM so that chunk c-1's output leaves while chunk c's
-// MMAs run: transposed through shared memory into 16-byte row stores.
+// bf16 copy.  Warp-specialised: warp 4 only issues MMAs, warp 5 only record
+// copies; warps 0-3 (one per TMEM lane quadrant) run the epilogues.  They hand off
+// through mbarriers: the MMA commits, "D in bf16 is ready" and "the next bf16
+// state copy is ready".  The bf16 state copy is double-buffered so the O MMAs
+// of chunk c can still read it while chunk c+1's copy is written; the pass that
+// writes it also applies the next chunk's decay to the fp32 state.  O is
+// triple-buffered: chunk c-1's output leaves, transposed through shared memory
+// into 16-byte row stores, while chunk c+1's first MMAs run.
 #include "chunk_common.cuh"
 #include "kda_common.cuh"
 #include "kda_internal.h"
@@ -31,37 +35,33 @@ namespace spass {
 
 using namespace chunkfmt;
 
-constexpr int NT = 128;
+constexpr int NT = 192;          // warps 0-3: epilogues (TMEM lanes); warp 4: MMA issue; warp 5: record copies
+constexpr int NE = 128;          // epilogue threads
+constexpr uint32_t BAR_EPI = 1;  // named barrier of the epilogue warps
 constexpr uint32_t OFF_REC0 = 0;
 constexpr uint32_t OFF_REC1 = REC_STRIDE;
 constexpr uint32_t OFF_OST = 2 * REC_STRIDE;   // o of one chunk, bf16 [64 t][128 j]: 16 KB
 constexpr uint32_t OFF_BAR = OFF_OST + CH * DK * 2;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 64;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 128;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 static_assert(REC_STRIDE % 1024 == 0, "SW128 alignment");
 
 // TMEM columns (512 allocated)
 constexpr uint32_t TM_S32 = 0;     // S^T fp32, 128 cols
-constexpr uint32_t TM_S16 = 128;   // S^T bf16 A operand, 64 cols
-constexpr uint32_t TM_D = 192;     // D^T fp32, 64 cols; its bf16 copy (32 cols) is packed in place
-constexpr uint32_t TM_O = 256;     // O^T fp32, 2 x 64 cols (chunk parity)
+constexpr uint32_t TM_S16 = 128;   // S^T bf16 A operand, 2 x 64 cols (chunk parity)
+constexpr uint32_t TM_D = 256;     // D^T fp32, 64 cols; its bf16 copy (32 cols) is packed in place
+constexpr uint32_t TM_O = 320;     // O^T fp32, 3 x 64 cols (chunk index mod 3)
 
 constexpr uint32_t WAIT_POLLS = 1u << 22;
-enum { B_FULL0 = 0, B_FULL1, B_D, B_S, B_COUNT };
-
-__device__ __forceinline__ bool wait_vote(uint64_t *bar, uint32_t parity, bool ok) {
-  const bool mine = ok && umma::mbar_wait_bounded(bar, parity, WAIT_POLLS);
-  const bool all = __syncthreads_and(mine) != 0;
-  umma::fence_after_sync();
-  return all;
-}
+enum { B_FULL0 = 0, B_FULL1, B_D, B_S, B_O, B_D16, B_S16, B_COUNT };
+__device__ __forceinline__ uint32_t o_cols(int c) { return TM_O + (uint32_t)(c % 3) * 64; }
 
 __global__ void __launch_bounds__(NT, 1) state_pass_kernel(StateArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
   const int n = blockIdx.x / H, h = blockIdx.x % H;
   int64_t s0, s1;
@@ -73,209 +73,252 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(StateArgs a) {
   if (chunk0 + nchunks > a.max_slots) nchunks = (int)(a.max_slots - chunk0);
   const uint8_t *recs = reinterpret_cast<const uint8_t *>(a.records);
   auto rec_ptr = [&](int c) { return recs + ((chunk0 + c) * H + h) * (int64_t)REC_STRIDE; };
+  auto rec_off = [](int c) { return (c & 1) ? OFF_REC1 : OFF_REC0; };
 
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_BAR + 8 * B_COUNT);
+  int *fail = reinterpret_cast<int *>(smem + OFF_BAR + 8 * B_COUNT + 8);
   const uint32_t sbase = umma::smem_u32(smem);
-  const int j = tid;                                  // TMEM lane = value channel
-  const uint32_t lane_base = (uint32_t)warp * 32u << 16;
-  const int64_t sg = ((int64_t)n * H + h) * DK * DK;
-  __nv_bfloat16 *__restrict__ o = reinterpret_cast<__nv_bfloat16 *>(a.o);
 
   if (warp == 0) {
     umma::tmem_alloc(tmem_slot, 512);
     umma::tmem_relinquish();
   }
   if (tid == 32) {
-    for (int i = 0; i < B_COUNT; ++i) umma::mbar_init(&bar[i], 1);
+    for (int i = 0; i < B_COUNT; ++i) umma::mbar_init(&bar[i], (i == B_D16 || i == B_S16) ? 4 : 1);
     umma::mbar_fence_init();
+    *fail = 0;
   }
   umma::fence_before_sync();
   __syncthreads();
   umma::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  // first two records in flight
-  if (tid == 0) {
-    for (int c = 0; c < 2 && c < nchunks; ++c) {
-      umma::mbar_arrive_expect_tx(&bar[B_FULL0 + c], REC_BYTES);
-      umma::bulk_g2s(smem + (c ? OFF_REC1 : OFF_REC0), rec_ptr(c), REC_BYTES, &bar[B_FULL0 + c]);
-    }
-  }
-  // initial state: S^T[j][i] = S0[i][j] (fp32 and bf16 copies)
-#pragma unroll 1
-  for (int c = 0; c < DK; c += 32) {
-    uint32_t r[32], p[16];
-#pragma unroll
-    for (int e = 0; e < 32; ++e)
-      r[e] = __float_as_uint(a.state0 ? a.state0[sg + (int64_t)(c + e) * DK + j] : 0.f);
-#pragma unroll
-    for (int e = 0; e < 16; ++e) p[e] = pack_bf16(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
-    umma::tmem_st32(tmem + lane_base + TM_S32 + c, r);
-    umma::tmem_st16(tmem + lane_base + TM_S16 + c / 2, p);
-  }
-  umma::tmem_wait_st();
-  umma::fence_before_sync();
-  __syncthreads();
-
-  // o of chunk cc (its O^T in TMEM columns ocol): lane j holds column j of the
-  // chunk's 64 rows; a shared-memory transpose turns them into 16-byte row stores
-  __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_OST);
-  auto emit_o = [&](int cc, uint32_t ocol) {
-    uint32_t r[2][32];
-    umma::tmem_ld32(tmem + lane_base + ocol, r[0]);
-    umma::tmem_ld32(tmem + lane_base + ocol + 32, r[1]);
-    umma::tmem_wait_ld();
-#pragma unroll
-    for (int t = 0; t < CH; ++t) ost[t * DK + j] = __float2bfloat16_rn(a.scale * __uint_as_float(r[t >> 5][t & 31]));
-    __syncthreads();
-    const int64_t c0 = s0 + (int64_t)cc * CH;
-    const int nvalid = (int)min((int64_t)CH, s1 - c0);
-#pragma unroll
-    for (int k = 0; k < CH * DK / 8 / NT; ++k) {
-      const int q = tid + k * NT, t = q >> 4, c16 = q & 15;
-      if (t < nvalid)
-        *reinterpret_cast<uint4 *>(o + ((c0 + t) * H + h) * DK + c16 * 8) =
-            *reinterpret_cast<const uint4 *>(ost + t * DK + c16 * 8);
-    }
-    __syncthreads();
-  };
-  // S^T columns *= e^{Gamma_C} of the record at rb; with bf16: also refresh the bf16 copy first
-  auto state_pass_over = [&](uint32_t rb, bool decay, bool bf16) {
-    const float4 *egc = reinterpret_cast<const float4 *>(smem + rb + REC_EGC);
-#pragma unroll
-    for (int cc = 0; cc < DK; cc += 64) {
-      uint32_t x[2][32];
-      umma::tmem_ld32(tmem + lane_base + TM_S32 + cc, x[0]);
-      umma::tmem_ld32(tmem + lane_base + TM_S32 + cc + 32, x[1]);
-      umma::tmem_wait_ld();
-      if (bf16) {
-        uint32_t p[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          p[e] = pack_bf16(__uint_as_float(x[e >> 4][(e & 15) * 2]), __uint_as_float(x[e >> 4][(e & 15) * 2 + 1]));
-        umma::tmem_st32(tmem + lane_base + TM_S16 + cc / 2, p);
+  if (warp >= 4) {
+    if (warp == 5 && lane == 0) {
+      // ---------------------------------------------------------- record copies
+      // chunk c+2 goes into chunk c's buffer once every MMA of chunk c is done (the
+      // epilogues read U and e^{Gamma_C} from it before their hand-offs)
+      int c = 0;
+      for (; c < 2 && c < nchunks; ++c) {
+        umma::mbar_arrive_expect_tx(&bar[B_FULL0 + c], REC_BYTES);
+        umma::bulk_g2s(smem + rec_off(c), rec_ptr(c), REC_BYTES, &bar[B_FULL0 + c]);
       }
-      if (decay) {
-#pragma unroll
-        for (int e4 = 0; e4 < 16; ++e4) {
-          const float4 g = egc[cc / 4 + e4];
-          uint32_t *y = &x[e4 >> 3][(e4 & 7) * 4];
-          const float2 lo = mul2(make_float2(__uint_as_float(y[0]), __uint_as_float(y[1])), make_float2(g.x, g.y));
-          const float2 hi = mul2(make_float2(__uint_as_float(y[2]), __uint_as_float(y[3])), make_float2(g.z, g.w));
-          y[0] = __float_as_uint(lo.x); y[1] = __float_as_uint(lo.y);
-          y[2] = __float_as_uint(hi.x); y[3] = __float_as_uint(hi.y);
-        }
-        umma::tmem_st32(tmem + lane_base + TM_S32 + cc, x[0]);
-        umma::tmem_st32(tmem + lane_base + TM_S32 + cc + 32, x[1]);
+      int issued = c;
+      bool ok = true;
+      for (c = 0; c + 2 < nchunks; ++c) {
+        ok = umma::mbar_wait_bounded(&bar[B_O], c & 1, WAIT_POLLS) && *(volatile int *)fail == 0;
+        if (!ok) break;
+        umma::mbar_arrive_expect_tx(&bar[B_FULL0 + (c & 1)], REC_BYTES);
+        umma::bulk_g2s(smem + rec_off(c), rec_ptr(c + 2), REC_BYTES, &bar[B_FULL0 + (c & 1)]);
+        issued = c + 3;
       }
-    }
-    umma::tmem_wait_st();
-  };
-
-  bool ok = true;
-#pragma unroll 1
-  for (int c = 0; c < nchunks; ++c) {
-    const int b = c & 1;
-    const uint32_t rb = b ? OFF_REC1 : OFF_REC0;
-    const uint32_t ocol = TM_O + (uint32_t)b * 64;
-    ok = wait_vote(&bar[B_FULL0 + b], (c >> 1) & 1, ok);
-    if (!ok) break;
-    if (c == 0) {   // the first chunk's decay (later ones ride on the previous chunk's last pass)
-      state_pass_over(rb, true, false);
-      umma::fence_before_sync();
-      __syncthreads();
-      umma::fence_after_sync();
-    }
-    // D^T = S^T (-W^T) (committed alone: the chain needs only D^T); O^T = S^T Q~^T
-    if (tid == 0) {
+      if (!ok) {
+        atomicExch(fail, 1);
+        // copies still in flight into this CTA's shared memory: wait (bounded) for them
+        for (int k = issued - 2 < 0 ? 0 : issued - 2; k < issued; ++k)
+          (void)umma::mbar_wait_bounded(&bar[B_FULL0 + (k & 1)], (k >> 1) & 1, WAIT_POLLS);
+      }
+    } else if (warp == 4 && lane == 0) {
+      // ---------------------------------------------------------- MMA issue
+      bool ok = true;
       const uint32_t id_d = umma::make_idesc_bf16(128, 64, 0, 1);
       const uint32_t id_o = umma::make_idesc_bf16(128, 64, 0, 0);
-#pragma unroll
-      for (int s = 0; s < DK / 16; ++s)
-        umma::mma_ts(tmem + TM_D, tmem + TM_S16 + (uint32_t)(s * 8), desc_mn_rows(sbase + rb + REC_WT, s),
-                     id_d, s > 0);
-      umma::mma_commit(&bar[B_D]);
-#pragma unroll
-      for (int s = 0; s < DK / 16; ++s)
-        umma::mma_ts(tmem + ocol, tmem + TM_S16 + (uint32_t)(s * 8), desc_k128(sbase + rb + REC_QT, 64, s),
-                     id_o, s > 0);
-    }
-    // while those run: the previous chunk's o
-    if (c > 0) emit_o(c - 1, TM_O + (uint32_t)(b ^ 1) * 64);
-    ok = wait_vote(&bar[B_D], c & 1, ok);
-    if (!ok) break;
-    // D^T + U^T -> bf16 A operand, packed over the first 32 columns of D
-    {
-      uint32_t r[2][32], p[32];
-      umma::tmem_ld32(tmem + lane_base + TM_D, r[0]);
-      umma::tmem_ld32(tmem + lane_base + TM_D + 32, r[1]);
-      umma::tmem_wait_ld();
-      const uint8_t *urow = smem + rb + REC_U;
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(urow + row64_off(j, c8));   // tokens 8c8 .. 8c8+7
-        const uint32_t *x = &r[c8 >> 2][(c8 & 3) * 8];
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const float2 d = add2(make_float2(__uint_as_float(x[2 * w]), __uint_as_float(x[2 * w + 1])),
-                                bf2_f2(word(u, w)));
-          p[4 * c8 + w] = f2_bf2(d);
-        }
-      }
-      umma::tmem_st32(tmem + lane_base + TM_D, p);
-      umma::tmem_wait_st();
-    }
-    umma::fence_before_sync();
-    __syncthreads();
-    if (tid == 0) {
-      umma::fence_after_sync();
-      // S^T += D^T K^ first (the chain), then O^T += D^T A_qk^T
       const uint32_t id_s = umma::make_idesc_bf16(128, 128, 0, 1);
-      const uint32_t id_o = umma::make_idesc_bf16(128, 64, 0, 0);
+      for (int c = 0; c < nchunks && ok; ++c) {
+        const int b = c & 1;
+        const uint32_t rb = sbase + rec_off(c);
+        const uint32_t s16 = tmem + TM_S16 + (uint32_t)b * 64;
+        const uint32_t ocol = tmem + o_cols(c);
+        ok = umma::mbar_wait_bounded(&bar[B_FULL0 + b], (c >> 1) & 1, WAIT_POLLS) &&
+             umma::mbar_wait_bounded(&bar[B_S16], c & 1, WAIT_POLLS) &&
+             (c == 0 || umma::mbar_wait_bounded(&bar[B_O], (c - 1) & 1, WAIT_POLLS)) &&
+             *(volatile int *)fail == 0;
+        if (!ok) break;
+        umma::fence_after_sync();
+        // D^T = S^T (-W^T); O^T = S^T Q~^T
 #pragma unroll
-      for (int s = 0; s < CH / 16; ++s)
-        umma::mma_ts(tmem + TM_S32, tmem + TM_D + (uint32_t)(s * 8), desc_mn_tok(sbase + rb + REC_KH, s),
-                     id_s, 1);
+        for (int s = 0; s < DK / 16; ++s)
+          umma::mma_ts(tmem + TM_D, s16 + (uint32_t)(s * 8), desc_mn_rows(rb + REC_WT, s), id_d, s > 0);
+        umma::mma_commit(&bar[B_D]);
 #pragma unroll
-      for (int s = 0; s < CH / 16; ++s)
-        umma::mma_ts(tmem + ocol, tmem + TM_D + (uint32_t)(s * 8), desc_k64(sbase + rb + REC_AQ, s), id_o, 1);
-      umma::mma_commit(&bar[B_S]);
-    }
-    ok = wait_vote(&bar[B_S], c & 1, ok);
-    if (!ok) break;
-    // this buffer has been read: start the copy of chunk c+2 into it
-    if (tid == 0 && c + 2 < nchunks) {
-      umma::mbar_arrive_expect_tx(&bar[B_FULL0 + b], REC_BYTES);
-      umma::bulk_g2s(smem + rb, rec_ptr(c + 2), REC_BYTES, &bar[B_FULL0 + b]);
-    }
-    // the next chunk's A operand (bf16 copy of the state) and its decay, in one pass
-    if (c + 1 < nchunks) {
-      ok = wait_vote(&bar[B_FULL0 + (b ^ 1)], ((c + 1) >> 1) & 1, ok);
-      if (!ok) break;
-      state_pass_over(b ? OFF_REC0 : OFF_REC1, true, true);
-    }
-    umma::fence_before_sync();
-    __syncthreads();
-  }
-  if (ok) {
-    if (nchunks > 0) emit_o(nchunks - 1, TM_O + (uint32_t)((nchunks - 1) & 1) * 64);
-    // final state: S[i][j] = S^T[j][i]
-#pragma unroll 1
-    for (int cc = 0; cc < DK; cc += 32) {
-      uint32_t s[32];
-      umma::tmem_ld32(tmem + lane_base + TM_S32 + cc, s);
-      umma::tmem_wait_ld();
+        for (int s = 0; s < DK / 16; ++s)
+          umma::mma_ts(ocol, s16 + (uint32_t)(s * 8), desc_k128(rb + REC_QT, 64, s), id_o, s > 0);
+        ok = umma::mbar_wait_bounded(&bar[B_D16], c & 1, WAIT_POLLS) && *(volatile int *)fail == 0;
+        if (!ok) break;
+        umma::fence_after_sync();
+        // S^T += D^T K^ (the chain), then O^T += D^T A_qk^T
 #pragma unroll
-      for (int e = 0; e < 32; ++e) a.state1[sg + (int64_t)(cc + e) * DK + j] = __uint_as_float(s[e]);
+        for (int s = 0; s < CH / 16; ++s)
+          umma::mma_ts(tmem + TM_S32, tmem + TM_D + (uint32_t)(s * 8), desc_mn_tok(rb + REC_KH, s), id_s, 1);
+        umma::mma_commit(&bar[B_S]);
+#pragma unroll
+        for (int s = 0; s < CH / 16; ++s)
+          umma::mma_ts(ocol, tmem + TM_D + (uint32_t)(s * 8), desc_k64(rb + REC_AQ, s), id_o, 1);
+        umma::mma_commit(&bar[B_O]);
+      }
+      if (!ok) atomicExch(fail, 1);
     }
   } else {
-    // a copy may still be in flight into this CTA's shared memory: wait (bounded) for it
-    for (int c = 0; c < 2; ++c) (void)umma::mbar_wait_bounded(&bar[B_FULL0 + c], 0, WAIT_POLLS);
-    if (tid == 0 && a.err) atomicExch(a.err, ERR_TIMEOUT);
+    // ------------------------------------------------------------ epilogues (warps 0-3)
+    const int j = tid;                                  // TMEM lane = value channel
+    const uint32_t lane_base = (uint32_t)warp * 32u << 16;
+    const int64_t sg = ((int64_t)n * H + h) * DK * DK;
+    __nv_bfloat16 *__restrict__ o = reinterpret_cast<__nv_bfloat16 *>(a.o);
+    __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_OST);
+    // Each thread waits on its own (bounded); a wait that gives up sets the shared
+    // fail flag and the thread carries on along the same path (its values are
+    // garbage, but every address and every barrier stays the same), so the
+    // warps never diverge around a barrier.  The flag is checked where all
+    // epilogue threads have just passed the same named barrier.
+    auto wait_one = [&](uint64_t *bb, uint32_t parity) {
+      if (!umma::mbar_wait_bounded(bb, parity, WAIT_POLLS)) *(volatile int *)fail = 1;
+      umma::fence_after_sync();
+    };
+    auto handoff = [&](uint64_t *bb) {   // this warp's TMEM stores are done: tell the issuer
+      umma::tmem_wait_st();
+      umma::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) umma::mbar_arrive(bb);
+    };
+    // o of chunk cc (its O^T in TMEM columns ocol): lane j holds column j of the chunk's
+    // 64 rows; a shared-memory transpose turns them into 16-byte row stores
+    auto emit_o = [&](int cc, uint32_t ocol) {
+      uint32_t r[2][32];
+      umma::tmem_ld32(tmem + lane_base + ocol, r[0]);
+      umma::tmem_ld32(tmem + lane_base + ocol + 32, r[1]);
+      umma::tmem_wait_ld();
+#pragma unroll
+      for (int t = 0; t < CH; ++t) ost[t * DK + j] = __float2bfloat16_rn(a.scale * __uint_as_float(r[t >> 5][t & 31]));
+      umma::named_sync(BAR_EPI, NE);
+      const int64_t c0 = s0 + (int64_t)cc * CH;
+      const int nvalid = (int)min((int64_t)CH, s1 - c0);
+#pragma unroll
+      for (int k = 0; k < CH * DK / 8 / NE; ++k) {
+        const int q = tid + k * NE, t = q >> 4, c16 = q & 15;
+        if (t < nvalid)
+          *reinterpret_cast<uint4 *>(o + ((c0 + t) * H + h) * DK + c16 * 8) =
+              *reinterpret_cast<const uint4 *>(ost + t * DK + c16 * 8);
+      }
+      umma::named_sync(BAR_EPI, NE);
+    };
+    // S^T columns *= e^{Gamma_C} of the record at rb; with s16: also write the bf16 copy there first
+    auto state_pass_over = [&](uint32_t rb, int s16) {
+      const float4 *egc = reinterpret_cast<const float4 *>(smem + rb + REC_EGC);
+      uint32_t x[4][32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) umma::tmem_ld32(tmem + lane_base + TM_S32 + q * 32, x[q]);
+      umma::tmem_wait_ld();
+      if (s16 >= 0) {
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+          uint32_t p[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            p[e] = pack_bf16(__uint_as_float(x[2 * q2 + (e >> 4)][(e & 15) * 2]),
+                             __uint_as_float(x[2 * q2 + (e >> 4)][(e & 15) * 2 + 1]));
+          umma::tmem_st32(tmem + lane_base + TM_S16 + (uint32_t)s16 * 64 + q2 * 32, p);
+        }
+        handoff(&bar[B_S16]);   // the next D / O MMAs need only this copy
+      }
+#pragma unroll
+      for (int e4 = 0; e4 < 32; ++e4) {
+        const float4 g = egc[e4];
+        uint32_t *y = &x[e4 >> 3][(e4 & 7) * 4];
+        const float2 lo = mul2(make_float2(__uint_as_float(y[0]), __uint_as_float(y[1])), make_float2(g.x, g.y));
+        const float2 hi = mul2(make_float2(__uint_as_float(y[2]), __uint_as_float(y[3])), make_float2(g.z, g.w));
+        y[0] = __float_as_uint(lo.x); y[1] = __float_as_uint(lo.y);
+        y[2] = __float_as_uint(hi.x); y[3] = __float_as_uint(hi.y);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) umma::tmem_st32(tmem + lane_base + TM_S32 + q * 32, x[q]);
+    };
+
+    // initial state: S^T[j][i] = S0[i][j] (fp32, and bf16 copy 0)
+#pragma unroll 1
+    for (int c = 0; c < DK; c += 32) {
+      uint32_t r[32], p[16];
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        r[e] = __float_as_uint(a.state0 ? a.state0[sg + (int64_t)(c + e) * DK + j] : 0.f);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) p[e] = pack_bf16(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+      umma::tmem_st32(tmem + lane_base + TM_S32 + c, r);
+      umma::tmem_st16(tmem + lane_base + TM_S16 + c / 2, p);
+    }
+    if (nchunks > 0) {   // chunk 0's decay
+      wait_one(&bar[B_FULL0], 0);
+      umma::tmem_wait_st();
+      state_pass_over(OFF_REC0, -1);
+    }
+    handoff(&bar[B_S16]);
+#pragma unroll 1
+    for (int c = 0; c < nchunks; ++c) {
+      const int b = c & 1;
+      const uint32_t rb = rec_off(c);
+      wait_one(&bar[B_D], c & 1);
+      wait_one(&bar[B_FULL0 + b], (c >> 1) & 1);   // (complete already: makes U visible here)
+      // (before this chunk's hand-off below: after it, chunk c's O commit could land
+      // first and the parity of the wait would then name the wrong phase)
+      if (c > 0) wait_one(&bar[B_O], (c - 1) & 1);
+      // D^T + U^T -> bf16 A operand, packed over the first 32 columns of D
+      {
+        uint32_t r[2][32], p[32];
+        umma::tmem_ld32(tmem + lane_base + TM_D, r[0]);
+        umma::tmem_ld32(tmem + lane_base + TM_D + 32, r[1]);
+        uint4 u[8];
+        const uint8_t *urow = smem + rb + REC_U;
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) u[c8] = *reinterpret_cast<const uint4 *>(urow + row64_off(j, c8));
+        umma::tmem_wait_ld();
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {   // tokens 8c8 .. 8c8+7
+          const uint32_t *x = &r[c8 >> 2][(c8 & 3) * 8];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const float2 d = add2(make_float2(__uint_as_float(x[2 * w]), __uint_as_float(x[2 * w + 1])),
+                                  bf2_f2(word(u[c8], w)));
+            p[4 * c8 + w] = f2_bf2(d);
+          }
+        }
+        umma::tmem_st32(tmem + lane_base + TM_D, p);
+      }
+      handoff(&bar[B_D16]);
+      wait_one(&bar[B_S], c & 1);
+      // the next chunk's bf16 state copy (handed off first), then its decay
+      if (c + 1 < nchunks) {
+        wait_one(&bar[B_FULL0 + (b ^ 1)], ((c + 1) >> 1) & 1);
+        state_pass_over(rec_off(c + 1), b ^ 1);
+      }
+      // the previous chunk's o, while the next chunk's first MMAs run (its barriers
+      // make the fail flag uniform: stop here when a wait anywhere has given up)
+      if (c > 0) {
+        emit_o(c - 1, o_cols(c - 1));
+        if (*(volatile int *)fail != 0) break;
+      }
+    }
+    umma::named_sync(BAR_EPI, NE);
+    const bool ok = *(volatile int *)fail == 0;
+    if (ok && nchunks > 0) {
+      wait_one(&bar[B_O], (nchunks - 1) & 1);
+      emit_o(nchunks - 1, o_cols(nchunks - 1));
+    }
+    if (ok) {
+      // final state: S[i][j] = S^T[j][i]
+      umma::tmem_wait_st();
+#pragma unroll 1
+      for (int cc = 0; cc < DK; cc += 32) {
+        uint32_t x[32];
+        umma::tmem_ld32(tmem + lane_base + TM_S32 + cc, x);
+        umma::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) a.state1[sg + (int64_t)(cc + e) * DK + j] = __uint_as_float(x[e]);
+      }
+    }
   }
   umma::fence_before_sync();
   __syncthreads();
+  if (tid == 0 && *(volatile int *)fail != 0 && a.err) atomicExch(a.err, ERR_TIMEOUT);
   if (warp == 0) {
     umma::fence_after_sync();
     umma::tmem_dealloc(tmem, 512);
