@@ -39,6 +39,11 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+# DRAM bytes (read + write) of one chunk_prep launch on 4x8192x32, from the ncu capture in
+# profiles/chunk_prep_prefill_1x8k.md scaled by the chunk-heads (x4); None when the kernel
+# has changed since that capture.
+CHUNK_PREP_TRAFFIC_BYTES = 4 * (269.257728e6 + 256.303616e6)
+
 HBM_FALLBACK_GBS = 6650.0
 BF16_FALLBACK_TFLOPS = 1590.0
 C = 64  # chunk length used for the algorithmic flop count
@@ -299,7 +304,8 @@ def run_ours(args, rank, world, local_rank):
                        "timed_calls": timed_calls},
         "roofline": {"kernel": dominant[0], "bound": "hbm", "achieved": dominant[3],
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dominant[3] / peaks["hbm_gbs"],
-                     "traffic": None, "algorithmic_bytes": dominant[2],
+                     "traffic": CHUNK_PREP_TRAFFIC_BYTES if dominant[0] == "chunk_prep" else None,
+                     "algorithmic_bytes": dominant[2],
                      "peak_source": peaks["source"] + " (burst copy)"},
         "decode": {"workload": "256 seqs x 32 heads, d=128, fp32 state, 64 steps",
                    "ms_per_step": dec_step_ms, "algorithmic_bytes": dec_bytes, "GB_s": dec_gbs,
