@@ -129,12 +129,12 @@ __device__ __forceinline__ bool wait_vote(uint64_t *bar, uint32_t parity, bool o
 // goes; no other warp touches these columns.
 template <int J, int NC>
 __device__ __forceinline__ void solve_columns(const float *sB, float *sT, int col, int r) {
-  constexpr int NP = NC / 2;   // column pairs
+  constexpr int NP = NC / 2;   // column pairs; two accumulators each (even / odd terms) for ILP
 #pragma unroll
   for (int I = J + 1; I < 4; ++I) {
-    float2 x[NP];
+    float2 x[2][NP];
 #pragma unroll
-    for (int c = 0; c < NP; ++c) x[c] = f2(0.f);
+    for (int c = 0; c < NP; ++c) x[0][c] = x[1][c] = f2(0.f);
 #pragma unroll
     for (int K = J; K < I; ++K) {
 #pragma unroll
@@ -145,22 +145,22 @@ __device__ __forceinline__ void solve_columns(const float *sB, float *sT, int co
         for (int e = 0; e < 4; ++e) {
           const float *trow = sT + (16 * K + 4 * m4 + e) * TSS + col;
           if constexpr (NC == 2) {
-            x[0] = fma2(f2(bb[e]), *reinterpret_cast<const float2 *>(trow), x[0]);
+            x[e & 1][0] = fma2(f2(bb[e]), *reinterpret_cast<const float2 *>(trow), x[e & 1][0]);
           } else {
             const float4 tv = *reinterpret_cast<const float4 *>(trow);
-            x[0] = fma2(f2(bb[e]), make_float2(tv.x, tv.y), x[0]);
-            x[1] = fma2(f2(bb[e]), make_float2(tv.z, tv.w), x[1]);
+            x[e & 1][0] = fma2(f2(bb[e]), make_float2(tv.x, tv.y), x[e & 1][0]);
+            x[e & 1][1] = fma2(f2(bb[e]), make_float2(tv.z, tv.w), x[e & 1][1]);
           }
         }
       }
     }
     float *dst = sT + (16 * I + r) * TSS + col;
 #pragma unroll
-    for (int c = 0; c < NP; ++c) *reinterpret_cast<float2 *>(dst + 2 * c) = x[c];
+    for (int c = 0; c < NP; ++c) *reinterpret_cast<float2 *>(dst + 2 * c) = add2(x[0][c], x[1][c]);
     __syncwarp();
-    float2 y[NP];
+    float2 y[2][NP];
 #pragma unroll
-    for (int c = 0; c < NP; ++c) y[c] = f2(0.f);
+    for (int c = 0; c < NP; ++c) y[0][c] = y[1][c] = f2(0.f);
 #pragma unroll
     for (int m4 = 0; m4 < 4; ++m4) {
       const float4 tv = *reinterpret_cast<const float4 *>(sT + (16 * I + r) * TSS + 16 * I + 4 * m4);
@@ -169,12 +169,13 @@ __device__ __forceinline__ void solve_columns(const float *sB, float *sT, int co
       for (int e = 0; e < 4; ++e) {
         const float *xrow = sT + (16 * I + 4 * m4 + e) * TSS + col;
 #pragma unroll
-        for (int c = 0; c < NP; ++c) y[c] = fma2(f2(tt[e]), *reinterpret_cast<const float2 *>(xrow + 2 * c), y[c]);
+        for (int c = 0; c < NP; ++c)
+          y[e & 1][c] = fma2(f2(tt[e]), *reinterpret_cast<const float2 *>(xrow + 2 * c), y[e & 1][c]);
       }
     }
     __syncwarp();
 #pragma unroll
-    for (int c = 0; c < NP; ++c) *reinterpret_cast<float2 *>(dst + 2 * c) = mul2(y[c], f2(-1.f));
+    for (int c = 0; c < NP; ++c) *reinterpret_cast<float2 *>(dst + 2 * c) = mul2(add2(y[0][c], y[1][c]), f2(-1.f));
     __syncwarp();
   }
 }
@@ -544,15 +545,18 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   phase ^= 1u;
 
   // ---------------------------------------------------------------- A_qk (bf16) and diag(beta) A_kk
-  // Warp w reads TMEM lanes 32(w&3)..: q rows (warps 0-1) or k rows (2-3) of
+  // Warp w reads TMEM lanes 32(w&3)..: q rows (w&3 = 0, 1) or k rows (2, 3) of
   // tokens 32p..32p+31, p = w & 1; lane half hh gives the block I = 2p + hh.
   // Column group gi (s = 16gi..16gi+15) of row t comes from the diagonal product
   // (gi == I) or from R_I (gi < I); tcgen05.ld is warp-uniform, so both halves
-  // load both candidates and keep their own.
-  if (ok && warp < 4) {
+  // load both candidates and keep their own.  Warps 0-3 take column groups 0-1,
+  // warps 4-7 (the same lane quadrants) groups 2-3.  Blocks of diag(beta) A_kk
+  // right of the diagonal are never read, so only A_qk gets explicit zeros.
+  if (ok) {
     const int p = warp & 1, hh = lane >> 4;
     const int t = 32 * p + lane;
-    const bool is_q = warp < 2;
+    const bool is_q = (warp & 3) < 2;
+    const bool upper = warp >= 4;
     const float bt = is_q ? 1.f : beta_s[t];
     const uint32_t tb = tmem + lane_base + TM_P;
     auto emit = [&](int gi, const uint32_t (&v)[16], bool zero, bool diag) {
@@ -581,21 +585,25 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
     };
     uint32_t va[16], vb2[16], v[16];
     if (p == 0) {
-      // gi 0: lo = diagonal (col 0), hi = R_1 (col 64); gi 1: hi = diagonal (col 16)
-      umma::tmem_ld16(tb + 0, va);
-      umma::tmem_ld16(tb + 64, vb2);
-      umma::tmem_wait_ld();
+      if (!upper) {
+        // gi 0: lo = diagonal (col 0), hi = R_1 (col 64); gi 1: hi = diagonal (col 16)
+        umma::tmem_ld16(tb + 0, va);
+        umma::tmem_ld16(tb + 64, vb2);
+        umma::tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = hh ? vb2[e] : va[e];
-      emit(0, v, false, hh == 0);
-      umma::tmem_ld16(tb + 16, va);
-      umma::tmem_wait_ld();
-      emit(1, va, hh == 0, true);
-      emit(2, va, true, false);
-      emit(3, va, true, false);
-    } else {
-      // gi 0: lo = R_2 (col 80), hi = R_3 (col 112); gi 1: 96 / 128;
-      // gi 2: lo = diagonal (col 32), hi = R_3 (col 144); gi 3: hi = diagonal (col 48)
+        for (int e = 0; e < 16; ++e) v[e] = hh ? vb2[e] : va[e];
+        emit(0, v, false, hh == 0);
+        umma::tmem_ld16(tb + 16, va);
+        umma::tmem_wait_ld();
+        emit(1, va, hh == 0, true);
+      } else if (is_q) {   // groups 2-3 of blocks 0-1: zero
+#pragma unroll
+        for (int e = 0; e < 16; ++e) va[e] = 0u;
+        emit(2, va, true, false);
+        emit(3, va, true, false);
+      }
+    } else if (!upper) {
+      // gi 0: lo = R_2 (col 80), hi = R_3 (col 112); gi 1: 96 / 128
       umma::tmem_ld16(tb + 80, va);
       umma::tmem_ld16(tb + 112, vb2);
       umma::tmem_wait_ld();
@@ -608,6 +616,8 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
 #pragma unroll
       for (int e = 0; e < 16; ++e) v[e] = hh ? vb2[e] : va[e];
       emit(1, v, false, false);
+    } else {
+      // gi 2: lo = diagonal (col 32), hi = R_3 (col 144); gi 3: hi = diagonal (col 48)
       umma::tmem_ld16(tb + 32, va);
       umma::tmem_ld16(tb + 144, vb2);
       umma::tmem_wait_ld();
