@@ -222,6 +222,13 @@ def run_ours(args, rank, world, local_rank):
     dec_ms = [de[i].elapsed_time(de[i + 1]) for i in range(64)]
     clock_info = clocks.stop()
 
+    # ---- the other prefill workloads (reported beside the headline, not in `value`)
+    extra = {}
+    if not args.no_extra:
+        for wname in ("long_256k", "varlen_32"):
+            extra[wname] = time_prefill_workload(W.spec(wname), dev, stream, args.warmup,
+                                                 max(3, min(args.steps, 5)), peaks)
+
     # ---- e2e through the C ABI with host buffers
     pin = lambda t: t.detach().cpu().pin_memory()
     hq, hk, hv, ha, hb = pin(q), pin(k), pin(v), pin(alpha), pin(b)
@@ -315,6 +322,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": None if args.no_e2e else {
             "value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "other_workloads": extra,
         "gpu_launches": launches_per_step * args.steps + 64,
         "clocks": clock_info,
         "peaks": peaks,
@@ -322,6 +330,68 @@ def run_ours(args, rank, world, local_rank):
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
     return line
+
+
+def time_prefill_workload(s, dev, stream, warmup, steps, peaks):
+    """One kda_prefill over a whole workload (inputs resident in HBM), timed with CUDA
+    events on the launching stream; chunk_prep / state-pass split from the library's
+    kernel timing."""
+    import torch
+    from gated_delta_rule_70_b200 import kda
+    from gated_delta_rule_70_b200 import workloads as W
+
+    params = {k: W.to_device(v, dev) for k, v in W.make_params(s).items()}
+    T = s.total_tokens
+    H, d = s.H, s.d
+    bf = torch.bfloat16
+    q, k, v = (torch.empty((T, H * d), dtype=bf, device=dev) for _ in range(3))
+    alpha = torch.empty((T, H, d), dtype=bf, device=dev)
+    b = torch.empty((T, H), dtype=bf, device=dev)
+    blk = 65536
+    for t0 in range(0, T, blk):   # host generation in slices, uploaded as they come
+        t1 = min(T, t0 + blk)
+        tok = W.make_tokens(s, t0, t1)
+        for name, dst in (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("b", b)):
+            dst[t0:t1].copy_(W.to_device(tok[name], dev))
+        del tok
+    S0 = W.make_initial_state(s)
+    S0 = W.to_device(S0, dev) if S0 is not None else None
+    cu = W.to_device(s.cu_seqlens, dev) if s.varlen else None
+    N = s.num_seqs
+    o = torch.empty((T, H, d), dtype=bf, device=dev)
+    fs = torch.empty((N, H, d, d), dtype=torch.float32, device=dev)
+    fc = torch.empty((N, 3, 3 * H * d), dtype=bf, device=dev)
+    seq_len = T if s.varlen else s.seq_lens[0]
+    ws = torch.empty(kda.prefill_workspace_size(kda.make_shape(N, seq_len, H, d, bf), s.varlen),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        kda.prefill(q, k, v, params["conv_w"], alpha, b, params["A_log"], params["dt_bias"],
+                    initial_state=S0, cu_seqlens=cu, num_seqs=N, out=o, final_state=fs,
+                    final_conv_state=fc, workspace=ws, check=False)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    kda.kernel_timing(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    _, prep_ms, state_ms = kda.kernel_times()
+    kda.kernel_timing(False)
+    ms = e0.elapsed_time(e1) / steps
+    flops = prefill_flops_per_token_head(d) * T * H
+    out = {"tokens": T, "sequences": N, "heads": H, "head_dim": d, "ms_per_step": ms,
+           "tokens_per_s": T / (ms * 1e-3), "algorithmic_tflops": flops / (ms * 1e-3) / 1e12,
+           "frac_of_measured_bf16": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+           "kernels_ms": {"chunk_prep": prep_ms, "state_pass": state_ms}, "steps": steps,
+           "warmup": warmup}
+    del q, k, v, alpha, b, o, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def decode_bytes(N, H, d, esz=2):
@@ -335,28 +405,43 @@ def decode_bytes(N, H, d, esz=2):
 # ---------------------------------------------------------------- CPU oracle timing
 
 def cpu_baseline(seconds: float = 15.0, tokens: int = None):
-    """Time the fp64 oracle on a bounded sample of the prefill workload (first sequence, all 32
-    heads, the first `tokens` tokens; default the whole 8192-token sequence, about 17
-    core-seconds) on all host cores; tokens/s counts every head."""
+    """Time the fp64 oracle on host cores, tokens/s counting every head.  Default: whole
+    sequences of the prefill workload (8192 tokens x 32 heads each), as many as fit in
+    about `seconds` of wall time (at least one, at most all four); with `tokens`: the first
+    `tokens` tokens of sequence 0 (the reference arm's per-step sample)."""
     from gated_delta_rule_70_b200 import workloads as W
     from oracle import oracle
 
     s = W.spec("prefill_4x8k")
-    cores = os.cpu_count() or 1
-    if tokens is None:
-        tokens = s.seq_lens[0]
-    t1 = tokens
     params = W.make_params(s)
-    tok = W.make_tokens(s, 0, t1)
-    f = {kk: W.as_f64(vv) for kk, vv in {**params, **tok}.items()}
-    S0 = W.make_initial_state(s)[:1].astype(np.float64)
-    t0 = time.perf_counter()
-    _, _, _, used = oracle.forward([0, t1], s.H, s.d, f["q"], f["k"], f["v"], f["conv_w"],
-                                   f["alpha"], f["b"], f["A_log"], f["dt_bias"], state0=S0)
-    dt = time.perf_counter() - t0
-    return {"value": t1 / dt, "unit": "tokens/s", "cores": int(used), "kind": "oracle",
-            "sample": "sequence 0 of prefill B=4 T=8192 H=32 d=128: first %d tokens, all 32 heads, "
-                      "fp64 C oracle, %d threads over heads, %.1f s" % (t1, used, dt)}
+    S0_all = W.make_initial_state(s).astype(np.float64)
+    L = s.seq_lens[0]
+    f_par = {kk: W.as_f64(vv) for kk, vv in params.items()}
+
+    def run_seq(n, t1):
+        tok = W.make_tokens(s, n * L, n * L + t1)
+        f = {kk: W.as_f64(vv) for kk, vv in tok.items()}
+        t0 = time.perf_counter()
+        _, _, _, used = oracle.forward([0, t1], s.H, s.d, f["q"], f["k"], f["v"], f_par["conv_w"],
+                                       f["alpha"], f["b"], f_par["A_log"], f_par["dt_bias"],
+                                       state0=S0_all[n:n + 1])
+        return time.perf_counter() - t0, used
+
+    if tokens is not None:
+        dt, used = run_seq(0, tokens)
+        return {"value": tokens / dt, "unit": "tokens/s", "cores": int(used), "kind": "oracle",
+                "sample": "sequence 0 of prefill B=4 T=8192 H=32 d=128: first %d tokens, all 32 heads, "
+                          "fp64 C oracle, %d threads over heads, %.1f s" % (tokens, used, dt)}
+    total, done, used = 0.0, 0, 1
+    for n in range(s.num_seqs):
+        dt, used = run_seq(n, L)
+        total += dt
+        done += 1
+        if total >= seconds:
+            break
+    return {"value": done * L / total, "unit": "tokens/s", "cores": int(used), "kind": "oracle",
+            "sample": "%d of the 4 sequences of prefill B=4 T=8192 H=32 d=128 (%d tokens x 32 heads), "
+                      "fp64 C oracle, %d threads over heads, %.1f s" % (done, done * L, used, total)}
 
 
 def run_reference(args, rank):
@@ -400,6 +485,8 @@ def main():
                     help="prefill sequences (the measured workload is 4; smaller only for profiling)")
     ap.add_argument("--only", choices=["all", "prefill"], default="all")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the long (1x262144) and varlen (32 sequences) prefill workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
