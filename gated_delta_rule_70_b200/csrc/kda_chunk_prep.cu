@@ -27,14 +27,15 @@
 //
 // Numerics: Gamma reaches 64 * (-5) = -320 inside a chunk, so e^{-Gamma}
 // overflows fp32.  The pairwise factor e^{Gamma_t - Gamma_s} is only ever split
-// around a reference close to both tokens: 16-token sub-blocks I with r_I =
-// Gamma at the end of block I-1 (r_0 = 0).  Diagonal blocks use
-// (q|k)_t e^{Gamma_t - r_I} against k_s e^{r_I - Gamma_s} (factors within e^{+-88});
-// a row in block I against an earlier block J uses r_I on both sides (factors
-// <= 1).  Per element only two exponentials are taken, e^{Gamma_t - r_I} and
-// e^{r_{I+1} - Gamma_t}; every other factor is one of them times a per-channel
-// constant of the chunk (e^{r_I}, e^{r_I - r_{I+1}}, ...), all in base 2 on the
-// special-function unit.
+// around a reference close to both tokens: the 16-token sub-block I of a token
+// has the reference m_I = Gamma after its 8th token.  A token's L-side factor
+// e^{Gamma_t - m_I} and R-side factor e^{m_I - Gamma_t} then stay within
+// e^{+-8 |g|max} (2^{+-116} at a gate bound of -10), so neither overflows nor
+// drops to a subnormal the exponential would flush.  A row in block I against an
+// earlier block J uses k_s e^{m_J - Gamma_s} times e^{m_I - m_J} <= 1.  Per
+// element only two exponentials are taken, e^{Gamma_t - m_I} and e^{m_I - Gamma_t};
+// every other factor is one of them times a per-channel constant of the chunk,
+// all in base 2 on the special-function unit.
 //
 // Structure: one CTA of 8 warps per (chunk, head), two CTAs per SM so that one
 // item's memory and tensor-core waits overlap the other's arithmetic.
@@ -83,8 +84,7 @@ constexpr uint32_t OFF_C = 106496;
 constexpr uint32_t OFF_WCONV = OFF_C;         // [3][8 x 144 B]: 16 channels x 4 taps bf16 per 144 B
 constexpr uint32_t WSEG = 144;                // padded segment stride: conflict-free 16-byte reads
 constexpr uint32_t OFF_DTB = OFF_C + 3 * 8 * WSEG;   // [128] fp32
-constexpr uint32_t C_R = OFF_C;               // r_I, I = 0..4 (r_0 = 0)         [5][128]
-constexpr uint32_t C_CR = OFF_C + 2560;       // 2^{r_2-r_1}, 2^{r_3-r_1}, 2^{r_3-r_2}  [3][128]
+constexpr uint32_t C_M = OFF_C;               // m_0..m_3 (block references), Gamma_C  [5][128]
 constexpr uint32_t OFF_WTOT = OFF_C + 4096;   // per-warp gate sums [8][128], then their prefixes
 constexpr uint32_t OFF_BETA = OFF_C + 8192;   // beta[64]
 constexpr uint32_t OFF_BAR = OFF_BETA + 256;  // MMA barrier, TMA barrier, TMEM address
@@ -97,7 +97,7 @@ static_assert(OFF_ST + 64 * TSS * 4 <= OFF_TB && OFF_TB + 8192 <= OFF_KT && OFF_
               "solve scratch overlaps");
 static_assert(OFF_TB % 1024 == 0 && OFF_KT % 1024 == 0 && OFF_V % 1024 == 0 && OFF_R % 1024 == 0,
               "SW128 alignment");
-static_assert(OFF_DTB + 512 <= OFF_WTOT && C_CR + 1536 <= OFF_WTOT, "constant area");
+static_assert(OFF_DTB + 512 <= OFF_WTOT && C_M + 2560 <= OFF_WTOT, "constant area");
 static_assert(OFF_DTB % 16 == 0 && WSEG % 16 == 0, "bulk copy alignment");
 
 // A per-channel vector of 128 floats is stored as two halves: channels 8c..8c+3
@@ -106,7 +106,9 @@ static_assert(OFF_DTB % 16 == 0 && WSEG % 16 == 0, "bulk copy alignment");
 __device__ __forceinline__ int cpos(int ch) { return ((ch & 7) >> 2) * 64 + (ch >> 3) * 4 + (ch & 3); }
 static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
 
-// R_all rows: [0,64) diagonal-reference rows, then R_1 (16 rows), R_2 (32), R_3 (48).
+// R_all rows: [0,64) diagonal-block rows (every token against its own block's
+// reference), then R_1 (16 rows), R_2 (32), R_3 (48): R_I holds the tokens of blocks
+// before I against block I's reference.
 __host__ __device__ constexpr int r_row0(int I) { return I == 1 ? 64 : (I == 2 ? 80 : 112); }
 
 // TMEM columns (256 allocated): intra products; after they are read, W^T and U^T
@@ -418,25 +420,23 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   }
   if (tid < 64) beta_s[tid] = btj;
   __syncthreads();   // also: every read of the prologue staging is done
-  // per channel: exclusive prefix of the warp sums (in place), r_1..r_4 and the R-row constants
+  // per channel: exclusive prefix of the warp sums (in place), the block references
+  // m_I (Gamma after token 16I+7, the end of warp 2I's tokens) and Gamma_C
   if (tid < 128) {
     const int pc = cpos(tid);   // this thread's channel, in the split-half layout
-    float acc = 0.f, r[5];
-    r[0] = 0.f;
+    float acc = 0.f, m[4];
 #pragma unroll
     for (int w2 = 0; w2 < 8; ++w2) {
       const float x = wtot[w2 * 128 + pc];
       wtot[w2 * 128 + pc] = acc;
       acc += x;
-      if (w2 & 1) r[(w2 >> 1) + 1] = acc;
+      if ((w2 & 1) == 0) m[w2 >> 1] = acc;
     }
     float *cf = reinterpret_cast<float *>(smem);
 #pragma unroll
-    for (int I = 0; I < 5; ++I) cf[C_R / 4 + I * 128 + pc] = r[I];
-    cf[C_CR / 4 + 0 * 128 + pc] = umma::ex2(r[2] - r[1]);
-    cf[C_CR / 4 + 1 * 128 + pc] = umma::ex2(r[3] - r[1]);
-    cf[C_CR / 4 + 2 * 128 + pc] = umma::ex2(r[3] - r[2]);
-    reinterpret_cast<float *>(rec + REC_EGC)[tid] = umma::ex2(r[4]);   // e^{Gamma_C}
+    for (int I = 0; I < 4; ++I) cf[C_M / 4 + I * 128 + pc] = m[I];
+    cf[C_M / 4 + 4 * 128 + pc] = acc;
+    reinterpret_cast<float *>(rec + REC_EGC)[tid] = umma::ex2(acc);   // e^{Gamma_C}
   }
   __syncthreads();
 
@@ -456,13 +456,13 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
 #pragma unroll
       for (int p = 0; p < 4; ++p) g2[j][p] = add2(g2[j][p], pre[p]);   // Gamma_t (base 2)
   }
-  {  // L side: Lq = q e^{Gamma - r_I}, Lk likewise; q e^{Gamma}, k e^{Gamma}
-    float2 nrI[4], eR[4];
-    lds_pairs(C_R + blkI * 512, nrI);
+  {  // L side: Lq = q e^{Gamma - m_I}, Lk likewise; q e^{Gamma}, k e^{Gamma}
+    float2 nm[4], eM[4];
+    lds_pairs(C_M + blkI * 512, nm);
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      eR[p] = ex2_2(nrI[p]);
-      nrI[p] = mul2(nrI[p], f2(-1.f));
+      eM[p] = ex2_2(nm[p]);
+      nm[p] = mul2(nm[p], f2(-1.f));
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -470,13 +470,13 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
       uint32_t Lq[4], Lk[4], Qt[4], Kt[4];
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
-        const float2 e1 = ex2_2(add2(g2[j][p], nrI[p]));   // in (2^-128, 1]
+        const float2 e1 = ex2_2(add2(g2[j][p], nm[p]));   // within 2^{+-8|g|max}
         const float2 lq = mul2(bf2_f2(word(qb[j], p)), e1);
         const float2 lk = mul2(bf2_f2(word(kb[j], p)), e1);
         Lq[p] = f2_bf2(lq);
         Lk[p] = f2_bf2(lk);
-        Qt[p] = f2_bf2(mul2(lq, eR[p]));
-        Kt[p] = f2_bf2(mul2(lk, eR[p]));
+        Qt[p] = f2_bf2(mul2(lq, eM[p]));
+        Kt[p] = f2_bf2(mul2(lk, eM[p]));
       }
       *reinterpret_cast<uint4 *>(smem + OFF_L + tr_off(128, t, cg)) = make_uint4(Lq[0], Lq[1], Lq[2], Lq[3]);
       *reinterpret_cast<uint4 *>(smem + OFF_L + tr_off(128, 64 + t, cg)) = make_uint4(Lk[0], Lk[1], Lk[2], Lk[3]);
@@ -484,22 +484,25 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
       *reinterpret_cast<uint4 *>(rec + REC_QT + tr_off(64, t, cg)) = make_uint4(Qt[0], Qt[1], Qt[2], Qt[3]);
     }
   }
-  {  // R side: kd = k e^{r_{I+1} - Gamma}; Rd = kd e^{r_I - r_{I+1}}; R_{I+1..3} rows; k e^{Gamma_C - Gamma}
-    float2 rI1[4], cD[4], cK[4], cA[4], cB[4];
+  {  // R side: kd = k e^{m_I - Gamma} (the diagonal-block row); R rows of the later
+     // blocks I' = kd e^{m_I' - m_I}; k e^{Gamma_C - Gamma} = kd e^{Gamma_C - m_I}
+    float2 m[4], cK[4], c1[4], c2[4], c3[4];
+    lds_pairs(C_M + blkI * 512, m);
     {
-      float2 rI[4], r4[4];
-      lds_pairs(C_R + blkI * 512, rI);
-      lds_pairs(C_R + (blkI + 1) * 512, rI1);
-      lds_pairs(C_R + 4 * 512, r4);
+      float2 gc[4];
+      lds_pairs(C_M + 4 * 512, gc);
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const float2 nr = mul2(rI1[p], f2(-1.f));
-        cD[p] = ex2_2(add2(rI[p], nr));   // 2^{r_I - r_{I+1}}
-        cK[p] = ex2_2(add2(r4[p], nr));   // 2^{r_4 - r_{I+1}}
-      }
+      for (int p = 0; p < 4; ++p) cK[p] = ex2_2(add2(gc[p], mul2(m[p], f2(-1.f))));   // <= 1
     }
-    if (blkI < 2) lds_pairs(C_CR + (blkI == 0 ? 0 : 2) * 512, cA);   // 2^{r_{I+2} - r_{I+1}}
-    if (blkI == 0) lds_pairs(C_CR + 512, cB);                       // 2^{r_3 - r_1}
+    auto later = [&](int I2, float2 (&c)[4]) {   // 2^{m_I2 - m_I} <= 1
+      float2 mi[4];
+      lds_pairs(C_M + I2 * 512, mi);
+#pragma unroll
+      for (int p = 0; p < 4; ++p) c[p] = ex2_2(add2(mi[p], mul2(m[p], f2(-1.f))));
+    };
+    if (blkI < 3) later(blkI + 1, c1);
+    if (blkI < 2) later(blkI + 2, c2);
+    if (blkI < 1) later(3, c3);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int t = tg * 4 + j;
@@ -507,12 +510,12 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         const float2 kd = mul2(bf2_f2(word(kb[j], p)),
-                               ex2_2(add2(rI1[p], mul2(g2[j][p], f2(-1.f)))));   // |kd| <= |k|
-        Rd[p] = f2_bf2(mul2(kd, cD[p]));
+                               ex2_2(add2(m[p], mul2(g2[j][p], f2(-1.f)))));   // within 2^{+-8|g|max}
+        Rd[p] = f2_bf2(kd);
         Kh[p] = f2_bf2(mul2(kd, cK[p]));
-        K1[p] = f2_bf2(kd);
-        K2[p] = blkI < 2 ? f2_bf2(mul2(kd, cA[p])) : 0u;
-        K3[p] = blkI == 0 ? f2_bf2(mul2(kd, cB[p])) : 0u;
+        K1[p] = blkI < 3 ? f2_bf2(mul2(kd, c1[p])) : 0u;
+        K2[p] = blkI < 2 ? f2_bf2(mul2(kd, c2[p])) : 0u;
+        K3[p] = blkI < 1 ? f2_bf2(mul2(kd, c3[p])) : 0u;
       }
       *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, t, cg)) = make_uint4(Rd[0], Rd[1], Rd[2], Rd[3]);
       *reinterpret_cast<uint4 *>(rec + REC_KH + tr_off(64, t, cg)) = make_uint4(Kh[0], Kh[1], Kh[2], Kh[3]);
@@ -522,7 +525,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
       if (blkI < 2)
         *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, r_row0(blkI + 2) + t, cg)) =
             make_uint4(K2[0], K2[1], K2[2], K2[3]);
-      if (blkI == 0)
+      if (blkI < 1)
         *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, r_row0(3) + t, cg)) =
             make_uint4(K3[0], K3[1], K3[2], K3[3]);
     }

@@ -110,10 +110,11 @@ struct WsLayout {
   size_t err, qn, kn, vc, g, beta, chunk_cu, records, total;
   bool tc;   // bf16 with head_dim 128: the tensor-core chunk path
 };
-// The tensor-core path splits e^{Gamma_t - Gamma_s} around references at most 16
-// tokens away, which stays inside fp32 / bf16 range for gates >= -5.5 (16 * 5.5 *
-// log2 e < 127); shapes with a lower gate bound run the token kernel.
-constexpr float kTcMinLowerBound = -5.5f;
+// The tensor-core path splits e^{Gamma_t - Gamma_s} around a reference in the middle
+// of each 16-token block, so each factor spans at most 8 gates: for gates >= -10 that is
+// within 2^{+-116}, inside fp32 / bf16 normal range; shapes with a lower gate bound run
+// the token kernel.
+constexpr float kTcMinLowerBound = -10.0f;
 inline bool use_tensor_core_path(int io_dtype, int D, float lower_bound) {
   return io_dtype == KDA_BF16 && D == 128 && lower_bound >= kTcMinLowerBound;
 }

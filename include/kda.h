@@ -44,11 +44,11 @@
  *     [2*H*d, 3*H*d) is v; conv_w[blk][c][3] multiplies the current token.
  *
  * Supported shapes: head_dim 64 or 128; num_heads 1..64; any sequence
- * length >= 0.  bf16 with head_dim 128 and lower_bound >= -5.5 runs the
+ * length >= 0.  bf16 with head_dim 128 and lower_bound >= -10 runs the
  * tensor-core chunk path (chunk_prep, with the prologue fused in, then the
  * state pass); other combinations run the prologue kernel and the CUDA-core
  * token kernel (fp32 test mode).  The bound keeps the chunk path's split decay
- * factors, which span up to 16 tokens of gate, inside fp32 and bf16 range.
+ * factors, which span up to 8 tokens of gate, inside fp32 and bf16 normal range.
  */
 #ifndef KDA_H
 #define KDA_H

@@ -60,7 +60,7 @@ def test_workspace_size_rules(lib):
     assert kda.recurrence_workspace_size(sh, False) == dense
     # a gate bound the chunk factorisation cannot hold takes the token kernel:
     # the prologue's intermediates, no records
-    low = kda.make_shape(4, 8192, 32, 128, torch.bfloat16, lower_bound=-8.0)
+    low = kda.make_shape(4, 8192, 32, 128, torch.bfloat16, lower_bound=-12.0)
     assert kda.prefill_workspace_size(low, False) >= T * 32 * 128 * (3 * 2 + 4) + T * 32 * 4
     assert kda.recurrence_workspace_size(low, False) < 4096
     # fp32 runs the token kernel

@@ -152,6 +152,62 @@ def test_prefill_fp32_varlen_with_conv_history():
     check_prefill(s, conv0)
 
 
+def test_prefill_bf16_varlen_with_conv_history():
+    """The tensor-core path's first chunks take the caller's conv history (fused prologue)."""
+    s = W.small("bf16v", [5, 70, 2, 130], H=2, d=128, seed=24, s0_std=0.02, varlen=True)
+    conv0 = W._store(np.random.default_rng(5).standard_normal((4, 3, 3 * 2 * 128)).astype(np.float32),
+                     "bf16")
+    check_prefill(s, conv0)
+
+
+def test_prefill_bf16_continuation():
+    """prefill(T1) then prefill(T2) from its final state and conv history == prefill(T1 + T2)."""
+    H, d, T1, T2 = 2, 128, 150, 97
+    s = W.small("cont", [T1 + T2], H=H, d=d, seed=25, s0_std=0.02)
+    inp = W.make_inputs(s)
+    o_all, s_all, c_all = gpu_prefill(s, inp)
+    part = lambda a, z: {k: (v[a:z] if k in ("q", "k", "v", "alpha", "b") else v) for k, v in inp.items()}
+    s1 = W.small("cont", [T1], H=H, d=d, seed=25, s0_std=0.02)
+    o1, st1, cs1 = gpu_prefill(s1, part(0, T1))
+    p2 = part(T1, T1 + T2)
+    o2, st2, cs2 = kda.prefill(_dev(p2["q"]), _dev(p2["k"]), _dev(p2["v"]), _dev(p2["conv_w"]),
+                               _dev(p2["alpha"]), _dev(p2["b"]), _dev(p2["A_log"]), _dev(p2["dt_bias"]),
+                               initial_state=st1, initial_conv_state=cs1, num_seqs=1)
+    torch.cuda.synchronize()
+    o_cat = np.concatenate([W.from_device(o1), W.from_device(o2)])
+    o_ref, s_ref, c_ref, _ = oracle_prefill(s, inp)
+    for h in range(H):
+        assert rel_l2(o_cat[:, h], o_ref[:, h]) <= TOL["bf16"]
+        assert rel_l2(o_cat[:, h], W.from_device(o_all)[:, h]) <= TOL["bf16"]
+    assert max_state_err(W.from_device(st2), s_ref) <= TOL["bf16"]
+    np.testing.assert_array_equal(W.from_device(cs2), c_ref)
+
+
+def test_recurrence_entry_bf16():
+    """kda_prologue + kda_recurrence (chunk_prep on prepared inputs) against the oracle."""
+    s = W.small("rec", [130, 64, 3], H=2, d=128, seed=26, s0_std=0.02, varlen=True)
+    inp = W.make_inputs(s)
+    cu = _dev(inp["cu_seqlens"])
+    qn, kn, vc, g, beta, _ = kda.prologue(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]),
+                                       _dev(inp["conv_w"]), _dev(inp["alpha"]), _dev(inp["b"]),
+                                       _dev(inp["A_log"]), _dev(inp["dt_bias"]), cu_seqlens=cu,
+                                       num_seqs=s.num_seqs)
+    o, fs = kda.recurrence(qn, kn, vc, g, beta, _dev(inp["S0"]), cu_seqlens=cu, num_seqs=s.num_seqs)
+    torch.cuda.synchronize()
+    o_ref, s_ref, _, _ = oracle_prefill(s, inp)
+    assert max_pair_err(W.from_device(o), o_ref, inp["cu_seqlens"], s.H) <= TOL["bf16"]
+    assert max_state_err(W.from_device(fs), s_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("lower_bound", [-5.5, -8.0, -10.0, -12.0])
+def test_prefill_bf16_saturated_gates(lower_bound):
+    """Gates pinned at the lower bound.  Down to -10 the tensor-core path runs (its split
+    decay factors span at most 8 gates: within 2^{+-116}); -12 runs the token kernel."""
+    s = W.small("sat", [200], H=2, d=128, seed=27, alpha_mu=3.0, s0_std=0.02)
+    s.lower_bound = lower_bound
+    check_prefill(s)
+
+
 def test_prefill_in_place_state():
     """final_state may be the same buffer as initial_state."""
     s = W.small("inplace", [100, 100], H=2, d=128, seed=18, s0_std=0.02)
