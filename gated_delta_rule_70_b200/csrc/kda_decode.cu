@@ -14,6 +14,7 @@
 // reductions.
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "umma.cuh"
 
 namespace kda {
 
@@ -154,7 +155,276 @@ decode_kernel(DecodeArgs a) {
   }
 }
 
+cudaError_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream);
+
+// ---------------------------------------------------------------------------
+// bf16, head_dim 128, H % 8 == 0: persistent and pipelined.  One CTA per SM walks
+// the (sequence, head) items.  A producer warp brings each item's 64 KB state and
+// its token's inputs (q, k, v, the 3-token conv history, alpha, the sequence's
+// row of b, the head's conv weights and dt_bias) by bulk copy two items ahead
+// into a 3-slot ring, and sends the updated state back by an asynchronous bulk
+// store; eight compute warps run the prologue and the state update in shared
+// memory.  Under a saturated HBM the bulk-copy issue itself stalls for about as
+// long as an item's arithmetic, so it lives in its own warp.
+namespace dec {
+
+constexpr int NC = 256;                             // compute threads (warps 0-7)
+constexpr int NT = NC + 32;                         // + the producer warp (warp 8)
+constexpr int D = 128;
+constexpr uint32_t S_STATE = 0;                     // fp32 [128][128]
+constexpr uint32_t S_QKV = 65536;                   // bf16 q, k, v of the token: 3 x 256 B
+constexpr uint32_t S_HIST = S_QKV + 768;            // bf16 conv history [slot m][tensor]: 9 x 256 B
+constexpr uint32_t S_ALPHA = S_HIST + 2304;         // bf16 [128]
+constexpr uint32_t S_W = S_ALPHA + 256;             // bf16 conv weights [tensor][128][4]: 3 x 1 KB
+constexpr uint32_t S_DTB = S_W + 3072;              // fp32 dt_bias [128]
+constexpr uint32_t S_B = S_DTB + 512;               // bf16 b of the token's sequence row [H <= 64]
+constexpr uint32_t SLOT = S_B + 128;                // 72,576 B per item
+constexpr int NSLOT = 3;
+constexpr uint32_t OFF_SCR = NSLOT * SLOT;
+struct Scratch {
+  float q[D], k[D], eg[D], v[D];
+  float red_p[NC / 32][D], red_r[NC / 32][D], red_qk[NC / 32];
+  float norm_part[2][4];
+  float alog[64];
+  float beta;
+  int fail;
+  int req[NSLOT];   // requests issued per slot (for the error path)
+  uint64_t full[NSLOT], empty[NSLOT];
+};
+constexpr uint32_t SMEM_BYTES = OFF_SCR + sizeof(Scratch);
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(SLOT % 16 == 0 && S_QKV % 16 == 0 && S_HIST % 16 == 0 && S_W % 16 == 0 && S_DTB % 16 == 0 &&
+              S_B % 16 == 0, "bulk copy alignment");
+constexpr uint32_t WAIT_POLLS = 1u << 22;
+constexpr uint32_t BAR_COMPUTE = 1;                 // named barrier of the compute warps
+
+__global__ void __launch_bounds__(NT, 1) decode_tma_kernel(DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  Scratch &sc = *reinterpret_cast<Scratch *>(smem + OFF_SCR);
+  const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+  const int H = a.H;
+  const int64_t HD = (int64_t)H * D;
+  const int items = a.N * H;
+  const int G = gridDim.x;
+  const __nv_bfloat16 *cw = reinterpret_cast<const __nv_bfloat16 *>(a.conv_w);
+  __nv_bfloat16 *cs = reinterpret_cast<__nv_bfloat16 *>(a.conv_state);
+
+  if (tid == 0) {
+    for (int i = 0; i < NSLOT; ++i) {
+      umma::mbar_init(&sc.full[i], 1);
+      umma::mbar_init(&sc.empty[i], NC);
+      sc.req[i] = 0;
+    }
+    umma::mbar_fence_init();
+    sc.fail = 0;
+  }
+  // A_log of every head, once: a plain load inside the loop would queue behind
+  // the bulk traffic for about one item's time
+  if (tid < H) sc.alog[tid] = a.A_log[tid];
+  __syncthreads();
+
+  if (w == NC / 32) {
+    // ---------------- producer warp
+    // everything item `it` reads, into ring slot `slot` (lanes 0-18: one copy each)
+    auto request = [&](int it, int slot) {
+      const int n = it / H, h = it % H;
+      uint8_t *base = smem + slot * SLOT;
+      uint64_t *bar = &sc.full[slot];
+      if (l == 0) {
+        umma::mbar_arrive_expect_tx(bar, S_B + 2 * H);
+        ++sc.req[slot];
+      }
+      __syncwarp();
+      if (l == 0) {
+        umma::bulk_g2s(base + S_STATE, a.state + (int64_t)it * D * D, D * D * 4, bar);
+      } else if (l < 4) {
+        const void *tok = l == 1 ? a.q : (l == 2 ? a.k : a.v);
+        umma::bulk_g2s(base + S_QKV + (l - 1) * 256,
+                       reinterpret_cast<const __nv_bfloat16 *>(tok) + (int64_t)n * HD + h * D, 256, bar);
+      } else if (l < 13) {
+        const int m = (l - 4) / 3, blk = (l - 4) % 3;
+        umma::bulk_g2s(base + S_HIST + (m * 3 + blk) * 256,
+                       cs + ((int64_t)n * 3 + m) * 3 * HD + blk * HD + h * D, 256, bar);
+      } else if (l == 13) {
+        umma::bulk_g2s(base + S_ALPHA, reinterpret_cast<const __nv_bfloat16 *>(a.alpha) + (int64_t)it * D, 256, bar);
+      } else if (l < 17) {
+        const int blk = l - 14;
+        umma::bulk_g2s(base + S_W + blk * 1024, cw + ((int64_t)blk * HD + h * D) * KCONV, 1024, bar);
+      } else if (l == 17) {
+        umma::bulk_g2s(base + S_DTB, a.dt_bias + h * D, 512, bar);
+      } else if (l == 18) {   // the row of b for sequence n (2H bytes, 16-byte aligned for H % 8 == 0)
+        umma::bulk_g2s(base + S_B, reinterpret_cast<const __nv_bfloat16 *>(a.b) + (int64_t)n * H, 2 * H, bar);
+      }
+      __syncwarp();
+    };
+    int it = blockIdx.x;
+    if (it < items) request(it, 0);
+    if (it + G < items) request(it + G, 1);
+#pragma unroll 1
+    for (int j = 0; it < items; ++j, it += G) {
+      const int slot = j % NSLOT;
+      // item j's state is final in its slot: store it
+      int ok = l == 0 ? (int)umma::mbar_wait_bounded(&sc.empty[slot], (j / NSLOT) & 1, WAIT_POLLS) : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) { sc.fail = 1; break; }
+      if (l == 0) {
+        umma::bulk_s2g(a.state + (int64_t)it * D * D, smem + slot * SLOT + S_STATE, D * D * 4);
+        umma::bulk_commit();
+      }
+      // two items ahead, into the slot item j-1 used: only its store (not item j's)
+      // must have finished reading shared memory
+      if (it + 2 * G < items) {
+        if (l == 0) umma::bulk_wait_read<1>();
+        __syncwarp();
+        request(it + 2 * G, (j + 2) % NSLOT);
+      }
+      if (*(volatile int *)&sc.fail) break;
+    }
+    // the stores read shared memory until they finish: wait before the CTA can leave
+    if (l == 0) umma::bulk_wait<0>();
+    if (*(volatile int *)&sc.fail) {
+      // copies requested into a slot may still be landing: wait (bounded) for each slot's last
+      if (l < NSLOT && sc.req[l] > 0) (void)umma::mbar_wait_bounded(&sc.full[l], (sc.req[l] - 1) & 1, WAIT_POLLS);
+    }
+  } else {
+    // ---------------- compute warps
+    const bool first = tid < D;
+    const int i = tid % D;   // q/k channel (first half) or v / gate channel (second half)
+#pragma unroll 1
+    for (int k = 0, it = blockIdx.x; it < items; ++k, it += G) {
+      const int slot = k % NSLOT;
+      const int n = it / H, h = it % H;
+      uint8_t *base = smem + slot * SLOT;
+      float *S_s = reinterpret_cast<float *>(base + S_STATE);
+      // all compute threads agree to go on: the slot has landed and nobody failed.
+      // The barrier also closes every read of the previous item's scratch values.
+      const bool landed = umma::mbar_wait_bounded(&sc.full[slot], (k / NSLOT) & 1, WAIT_POLLS);
+      if (!umma::named_sync_and(BAR_COMPUTE, NC, landed && !*(volatile int *)&sc.fail)) {
+        if (tid == 0) sc.fail = 1;
+        break;
+      }
+
+      // 1. prologue of this token: conv4 + SiLU per channel; the history shifts by one
+      const __nv_bfloat16 *qkv = reinterpret_cast<const __nv_bfloat16 *>(base + S_QKV);
+      const __nv_bfloat16 *hist = reinterpret_cast<const __nv_bfloat16 *>(base + S_HIST);
+      const __nv_bfloat16 *wts = reinterpret_cast<const __nv_bfloat16 *>(base + S_W);
+      auto conv_channel = [&](int blk) -> float {
+        const __nv_bfloat16 *wc = wts + (blk * D + i) * KCONV;
+        const __nv_bfloat16 h0 = hist[(0 * 3 + blk) * D + i], h1 = hist[(1 * 3 + blk) * D + i];
+        const __nv_bfloat16 h2 = hist[(2 * 3 + blk) * D + i], xn = qkv[blk * D + i];
+        float acc = __bfloat162float(wc[0]) * __bfloat162float(h0);
+        acc = fmaf(__bfloat162float(wc[1]), __bfloat162float(h1), acc);
+        acc = fmaf(__bfloat162float(wc[2]), __bfloat162float(h2), acc);
+        acc = fmaf(__bfloat162float(wc[3]), __bfloat162float(xn), acc);
+        __nv_bfloat16 *c = cs + (int64_t)n * 3 * 3 * HD + blk * HD + h * D + i;   // slot m at + m * 3 * HD
+        c[0] = h1;
+        c[3 * HD] = h2;
+        c[6 * HD] = xn;
+        return silu_f(acc);
+      };
+      float qv = 0.f, kv = 0.f;
+      if (first) {
+        qv = conv_channel(0);
+        kv = conv_channel(1);
+        float sq = qv * qv, sk = kv * kv;
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+          sq += __shfl_xor_sync(0xffffffffu, sq, off);
+          sk += __shfl_xor_sync(0xffffffffu, sk, off);
+        }
+        if (l == 0) { sc.norm_part[0][w] = sq; sc.norm_part[1][w] = sk; }
+      } else {
+        sc.v[i] = conv_channel(2);
+        const float al = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base + S_ALPHA)[i]);
+        const float g = gate_f(al + reinterpret_cast<const float *>(base + S_DTB)[i], -expf(sc.alog[h]),
+                               a.lower_bound);
+        sc.eg[i] = expf(g);
+        if (i == 0) sc.beta = sigmoid_f(__bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base + S_B)[h]));
+      }
+      umma::named_sync(BAR_COMPUTE, NC);
+      if (first) {
+        const float sq = sc.norm_part[0][0] + sc.norm_part[0][1] + sc.norm_part[0][2] + sc.norm_part[0][3];
+        const float sk = sc.norm_part[1][0] + sc.norm_part[1][1] + sc.norm_part[1][2] + sc.norm_part[1][3];
+        sc.q[i] = qv * rsqrtf(sq + a.eps);
+        sc.k[i] = kv * rsqrtf(sk + a.eps);
+      }
+      umma::named_sync(BAR_COMPUTE, NC);
+
+      // 2. decay, then the column reductions p = S'^T k and r = S'^T q
+      //    (warp w: rows 16w..16w+15; lane l: columns 4l..4l+3)
+      float S[16][4];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const float4 x = *reinterpret_cast<const float4 *>(S_s + (16 * w + r) * D + 4 * l);
+        S[r][0] = x.x; S[r][1] = x.y; S[r][2] = x.z; S[r][3] = x.w;
+      }
+      float p[4] = {0.f, 0.f, 0.f, 0.f}, rr[4] = {0.f, 0.f, 0.f, 0.f}, qk = 0.f;
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const int ii = 16 * w + r;
+        const float e = sc.eg[ii], kk = sc.k[ii], qq = sc.q[ii];
+        qk = fmaf(qq, kk, qk);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          S[r][c] *= e;
+          p[c] = fmaf(kk, S[r][c], p[c]);
+          rr[c] = fmaf(qq, S[r][c], rr[c]);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) { sc.red_p[w][4 * l + c] = p[c]; sc.red_r[w][4 * l + c] = rr[c]; }
+      if (l == 0) sc.red_qk[w] = qk;
+      umma::named_sync(BAR_COMPUTE, NC);
+      float P[4] = {0.f, 0.f, 0.f, 0.f}, R[4] = {0.f, 0.f, 0.f, 0.f}, QK = 0.f;
+#pragma unroll
+      for (int ww = 0; ww < NC / 32; ++ww) {
+        QK += sc.red_qk[ww];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) { P[c] += sc.red_p[ww][4 * l + c]; R[c] += sc.red_r[ww][4 * l + c]; }
+      }
+      const float bt = sc.beta;
+      float dl[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) dl[c] = bt * (sc.v[4 * l + c] - P[c]);
+      if (w == 0) {
+        __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o) + (int64_t)it * D + 4 * l;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) o[c] = __float2bfloat16_rn(a.scale * fmaf(QK, dl[c], R[c]));
+      }
+      // 3. S = S' + k d^T, back into the slot; the producer stores it
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const float kk = sc.k[16 * w + r];
+        *reinterpret_cast<float4 *>(S_s + (16 * w + r) * D + 4 * l) =
+            make_float4(fmaf(kk, dl[0], S[r][0]), fmaf(kk, dl[1], S[r][1]), fmaf(kk, dl[2], S[r][2]),
+                        fmaf(kk, dl[3], S[r][3]));
+      }
+      umma::fence_proxy_async_smem();
+      umma::mbar_arrive(&sc.empty[slot]);
+    }
+  }
+  __syncthreads();
+}
+
+}  // namespace dec
+
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
+  if ((int64_t)a.N * a.H == 0) return cudaSuccess;
+  if (a.io_dtype == KDA_BF16 && a.D == 128 && a.H % 8 == 0) {
+    cudaError_t e = cudaFuncSetAttribute(dec::decode_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)dec::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const int items = a.N * a.H;
+    dec::decode_tma_kernel<<<items < sms ? items : sms, dec::NT, dec::SMEM_BYTES, stream>>>(a);
+    return cudaGetLastError();
+  }
+  return launch_decode_simt(a, stream);
+}
+
+cudaError_t launch_decode_simt(const DecodeArgs &a, cudaStream_t stream) {
   if ((int64_t)a.N * a.H == 0) return cudaSuccess;
   const unsigned grid = (unsigned)(a.N * a.H);
   if (a.io_dtype == KDA_BF16) {

@@ -254,6 +254,22 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src, uint32
          "r"(smem_u32(mbar))
       : "memory");
 }
+// Contiguous bulk copy shared -> global (16-byte aligned addresses, bytes a multiple of
+// 16), tracked in the issuing thread's bulk-async groups.
+__device__ __forceinline__ void bulk_s2g(void *dst_global, const void *src_smem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               :: "l"(reinterpret_cast<uint64_t>(dst_global)), "r"(smem_u32(src_smem)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Until at most N of this thread's committed bulk groups are still reading shared memory.
+template <int N> __device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" :: "n"(N) : "memory");
+}
+// Until at most N of this thread's committed bulk groups are still in flight.
+template <int N> __device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" :: "n"(N) : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

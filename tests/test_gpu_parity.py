@@ -241,9 +241,11 @@ def _decode_inputs(s: W.Spec, step):
     return W.make_decode_step(s, step)
 
 
-def test_decode_parity_and_handoff():
-    """prefill(T1) -> decode steps on GPU vs the oracle, and against one long GPU prefill."""
-    H, d, N, T1, steps = 3, 128, 5, 70, 4
+@pytest.mark.parametrize("H,N,T1", [(3, 5, 70), (16, 40, 20)])
+def test_decode_parity_and_handoff(H, N, T1):
+    """prefill(T1) -> decode steps on GPU vs the oracle.  H=3 takes the per-item kernel;
+    H=16 with 640 items takes the persistent one, several items per CTA around its ring."""
+    d, steps = 128, 4
     s = W.small("dec", [T1] * N, H=H, d=d, seed=21, s0_std=0.02)
     inp = W.make_inputs(s)
     o, st, cs = gpu_prefill(s, inp)
