@@ -300,8 +300,8 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "prefill B=4 T=8192 H=32 d=128 bf16 I/O fp32 state (S0~N(0,0.02))",
-                   "global_batch": 4 * world, "seq_len": 8192, "heads": H, "head_dim": d,
+        "config": {"workload": "prefill B=%d T=8192 H=32 d=128 bf16 I/O fp32 state (S0~N(0,0.02))" % args.batch,
+                   "global_batch": args.batch * world, "seq_len": 8192, "heads": H, "head_dim": d,
                    "parallelism": "dp%d (independent sequences per rank)" % world,
                    "l2": "inputs 1.3 GB > 126 MB L2, no flush"},
         "tc": {"algorithmic_tflops": tc_tflops, "flop_per_token_head": prefill_flops_per_token_head(d),
@@ -311,7 +311,8 @@ def run_ours(args, rank, world, local_rank):
                        "timed_calls": timed_calls},
         "roofline": {"kernel": dominant[0], "bound": "hbm", "achieved": dominant[3],
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dominant[3] / peaks["hbm_gbs"],
-                     "traffic": CHUNK_PREP_TRAFFIC_BYTES if dominant[0] == "chunk_prep" else None,
+                     "traffic": (CHUNK_PREP_TRAFFIC_BYTES * args.batch / 4
+                                 if dominant[0] == "chunk_prep" and CHUNK_PREP_TRAFFIC_BYTES else None),
                      "algorithmic_bytes": dominant[2],
                      "peak_source": peaks["source"] + " (burst copy)"},
         "decode": {"workload": "256 seqs x 32 heads, d=128, fp32 state, 64 steps",

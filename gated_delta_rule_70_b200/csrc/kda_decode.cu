@@ -1,17 +1,20 @@
 // KDA decode step: one new token per sequence, fused prologue + in-place state
-// update, one CTA per (sequence, head).
+// update.
 //
 // The operation is one iteration of the per-token loop of the AliceAI-Foundation
 // KDA write-up ("二、KDA 线性注意力"), on the state a prefill left behind (section
 // "五": prefill and decode share initial_state / final_state) with the conv
 // history advanced by one token (section "四": 3 conv states per channel).
 //
-// HBM-bound by construction: the CTA issues all loads of its 128x128 fp32 state
-// slice (16 x 16-byte loads per thread, fully coalesced rows) before doing the
-// token's prologue, so the prologue's latency hides under the state stream;
-// each state element is then decayed, reduced, corrected and written back
-// exactly once.  o = S'^T q + (q.k) d lets one __syncthreads carry all column
-// reductions.
+// HBM-bound by construction: each state element is read once, decayed, reduced,
+// corrected and written back once; o = S'^T q + (q.k) d lets one barrier carry
+// all column reductions.  Two kernels:
+//   - dec::decode_tma_kernel (bf16, head_dim 128, heads a multiple of 8): one
+//     persistent CTA per SM, a producer warp streaming (sequence, head) items
+//     through a 3-slot shared-memory ring by bulk copy;
+//   - decode_kernel (every other shape): one CTA per (sequence, head), which
+//     issues all loads of its state slice before the token's prologue so the
+//     prologue's latency hides under the state stream.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "umma.cuh"
