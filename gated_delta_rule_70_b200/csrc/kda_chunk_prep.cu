@@ -81,9 +81,8 @@ constexpr uint32_t OFF_V = 90112;             // v: 16 KB (written as soon as v 
 // Per-channel constants of the chunk (after the prologue, which stages the conv
 // weights and dt_bias of the head in the same bytes):
 constexpr uint32_t OFF_C = 106496;
-constexpr uint32_t OFF_WCONV = OFF_C;         // [3][8 x 144 B]: 16 channels x 4 taps bf16 per 144 B
-constexpr uint32_t WSEG = 144;                // padded segment stride: conflict-free 16-byte reads
-constexpr uint32_t OFF_DTB = OFF_C + 3 * 8 * WSEG;   // [128] fp32
+constexpr uint32_t OFF_WCONV = OFF_C;         // [3][128 channels][4 taps] bf16, 1 KB per tensor
+constexpr uint32_t OFF_DTB = OFF_C + 3 * 1024;   // [128] fp32
 constexpr uint32_t C_M = OFF_C;               // m_0..m_3 (block references), Gamma_C  [5][128]
 constexpr uint32_t OFF_WTOT = OFF_C + 4096;   // per-warp gate sums [8][128], then their prefixes
 constexpr uint32_t OFF_BETA = OFF_C + 8192;   // beta[64]
@@ -98,7 +97,7 @@ static_assert(OFF_ST + 64 * TSS * 4 <= OFF_TB && OFF_TB + 8192 <= OFF_KT && OFF_
 static_assert(OFF_TB % 1024 == 0 && OFF_KT % 1024 == 0 && OFF_V % 1024 == 0 && OFF_R % 1024 == 0,
               "SW128 alignment");
 static_assert(OFF_DTB + 512 <= OFF_WTOT && C_M + 2560 <= OFF_WTOT, "constant area");
-static_assert(OFF_DTB % 16 == 0 && WSEG % 16 == 0, "bulk copy alignment");
+static_assert(OFF_DTB % 16 == 0 && OFF_WCONV % 16 == 0, "bulk copy alignment");
 
 // A per-channel vector of 128 floats is stored as two halves: channels 8c..8c+3
 // of every channel group c, then channels 8c+4..8c+7, so that the 8-channel
@@ -182,21 +181,17 @@ __device__ __forceinline__ void solve_columns(const float *sB, float *sT, int co
   }
 }
 
-template <bool kFused>
-__global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant__ PrepArgs a) {
-  const int H = a.H;
-  const int h = blockIdx.x % H;
-  const int64_t gchunk = blockIdx.x / H;
-  // locate (sequence, chunk): dense batches by division, varlen by the chunk table
-  int n;
-  int64_t cidx;
+// The (sequence, chunk) of chunk slot `gchunk`: dense batches by division, varlen
+// by the chunk table.  False for slots past the last chunk.
+__device__ __forceinline__ bool locate(const PrepArgs &a, int64_t gchunk, int &n, int64_t &c0, int &nt,
+                                       int64_t &cidx) {
   if (a.chunk_cu == nullptr) {
     const int64_t per = (a.seq_len + CH - 1) / CH;
-    if (per == 0 || gchunk >= per * a.N) return;
+    if (per == 0 || gchunk >= per * a.N) return false;
     n = (int)(gchunk / per);
     cidx = gchunk % per;
   } else {
-    if (gchunk >= a.chunk_cu[a.N] || gchunk >= a.max_slots) return;
+    if (gchunk >= a.chunk_cu[a.N] || gchunk >= a.max_slots) return false;
     int lo = 0, hi = a.N - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -207,9 +202,20 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   }
   int64_t s0, s1;
   seq_bounds(a.cu, n, a.seq_len, a.total_tokens, s0, s1);
-  const int64_t c0 = s0 + cidx * CH;
-  if (c0 >= s1) return;   // only for malformed cu_seqlens / chunk tables
-  const int nt = (int)(s1 - c0 < CH ? s1 - c0 : CH);   // valid tokens in this chunk
+  c0 = s0 + cidx * CH;
+  if (c0 >= s1) return false;   // only for malformed cu_seqlens / chunk tables
+  nt = (int)(s1 - c0 < CH ? s1 - c0 : CH);   // valid tokens in this chunk
+  return true;
+}
+
+template <bool kFused>
+__global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant__ PrepArgs a) {
+  const int H = a.H;
+  const int h = blockIdx.x % H;
+  const int64_t gchunk = blockIdx.x / H;
+  int n, nt;
+  int64_t c0, cidx;
+  if (!locate(a, gchunk, n, c0, nt, cidx)) return;
 
   extern __shared__ __align__(1024) uint8_t smem[];
   if (umma::smem_u32(smem) & 1023u) {   // the swizzled operands need a 1024-byte aligned base
@@ -229,14 +235,38 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   const uint32_t sbase = umma::smem_u32(smem);
   const uint32_t lane_base = (uint32_t)(warp & 3) * 32u << 16;
 
+  if (warp == 1) {
+    // barriers, then at once the chunk's input copies: their latency overlaps the
+    // TMEM allocation and the first block barrier
+    if (lane == 0) {
+      umma::mbar_init(bar_mma, 1);
+      umma::mbar_init(bar_tma, 1);
+      umma::mbar_fence_init();
+    }
+    __syncwarp();
+    if constexpr (kFused) {
+      if (lane == 0) {
+        umma::mbar_arrive_expect_tx(bar_tma, TMA_BYTES);
+        const int x = h * DK;
+        umma::tma_load_2d(smem + OFF_RAWQ, &a.map_q, x, (int)c0 - 3, bar_tma);
+        umma::tma_load_2d(smem + OFF_RAWK, &a.map_k, x, (int)c0 - 3, bar_tma);
+        umma::tma_load_2d(smem + OFF_RAWV, &a.map_v, x, (int)c0 - 3, bar_tma);
+        umma::tma_load_2d(smem + OFF_RAWA, &a.map_alpha, x, (int)c0, bar_tma);
+      }
+      __syncwarp();
+      // one copy per tensor: under load every copy instruction costs about as much
+      // to issue as a few KB of data, so the weights come as 3 x 1 KB
+      if (lane < 3) {   // conv weights of tensor `lane`
+        const __nv_bfloat16 *cw = reinterpret_cast<const __nv_bfloat16 *>(a.conv_w);
+        umma::bulk_g2s(smem + OFF_WCONV + lane * 1024, cw + ((int64_t)lane * H + h) * DK * KCONV, 1024, bar_tma);
+      } else if (lane == 3) {
+        umma::bulk_g2s(smem + OFF_DTB, a.dt_bias + h * DK, 512, bar_tma);
+      }
+    }
+  }
   if (warp == 0) {
     umma::tmem_alloc(tmem_slot, 256);
     umma::tmem_relinquish();
-  }
-  if (tid == 32) {
-    umma::mbar_init(bar_mma, 1);
-    umma::mbar_init(bar_tma, 1);
-    umma::mbar_fence_init();
   }
   umma::fence_before_sync();
   __syncthreads();
@@ -249,25 +279,6 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   float2 g2[4][4];             // gate in base 2, [token][channel pair]
   float btj = 0.f;             // beta of token tid (tid < 64)
   if constexpr (kFused) {
-    if (warp == 0) {
-      if (lane == 0) {
-        umma::mbar_arrive_expect_tx(bar_tma, TMA_BYTES);
-        const int x = h * DK;
-        umma::tma_load_2d(smem + OFF_RAWQ, &a.map_q, x, (int)c0 - 3, bar_tma);
-        umma::tma_load_2d(smem + OFF_RAWK, &a.map_k, x, (int)c0 - 3, bar_tma);
-        umma::tma_load_2d(smem + OFF_RAWV, &a.map_v, x, (int)c0 - 3, bar_tma);
-        umma::tma_load_2d(smem + OFF_RAWA, &a.map_alpha, x, (int)c0, bar_tma);
-      }
-      __syncwarp();
-      if (lane < 24) {   // conv weights: 3 tensors x 8 segments of 16 channels
-        const int blk = lane >> 3, sg = lane & 7;
-        const __nv_bfloat16 *cw = reinterpret_cast<const __nv_bfloat16 *>(a.conv_w);
-        umma::bulk_g2s(smem + OFF_WCONV + (blk * 8 + sg) * WSEG,
-                       cw + (((int64_t)blk * H + h) * DK + sg * 16) * KCONV, 128, bar_tma);
-      } else if (lane == 24) {
-        umma::bulk_g2s(smem + OFF_DTB, a.dt_bias + h * DK, 512, bar_tma);
-      }
-    }
     const float negA2 = -expf(a.A_log[h]) * LOG2E;   // the gate is kept in base 2
     const float lb2 = a.lower_bound * LOG2E;
     if (tid < 64 && tid < nt)
@@ -308,8 +319,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         // taps of channels 2p and 2p+1: (t0 t1), (t2 t3) of each, 16 bytes
-        const uint4 wq = *reinterpret_cast<const uint4 *>(smem + OFF_WCONV + (blk * 8 + (cg >> 1)) * WSEG +
-                                                          (cg & 1) * 64 + p * 16);
+        const uint4 wq = *reinterpret_cast<const uint4 *>(smem + OFF_WCONV + blk * 1024 + cg * 64 + p * 16);
         const float2 wa = bf2_f2(wq.x), wb = bf2_f2(wq.y), wc = bf2_f2(wq.z), wd = bf2_f2(wq.w);
         const float2 w0 = make_float2(wa.x, wc.x), w1 = make_float2(wa.y, wc.y);
         const float2 w2 = make_float2(wb.x, wd.x), w3 = make_float2(wb.y, wd.y);
