@@ -25,6 +25,7 @@ kda_status check_shape(const kda_shape *s) {
   if (!std::isfinite(s->lower_bound) || !std::isfinite(s->l2norm_eps) || s->l2norm_eps < 0.f ||
       !std::isfinite(s->scale))
     return KDA_ERR_INVALID_ARGUMENT;
+  if (s->flags & ~KDA_FLAGS_KNOWN) return KDA_ERR_INVALID_ARGUMENT;
   if (s->head_dim != 64 && s->head_dim != 128) return KDA_ERR_UNSUPPORTED;
   if (s->num_heads > 64) return KDA_ERR_UNSUPPORTED;
   return KDA_OK;
@@ -51,6 +52,7 @@ PrologueArgs make_prologue_args(const kda_shape *s, int64_t T, const void *q, co
   a.q = q; a.k = k; a.v = v; a.conv_w = conv_w; a.alpha = alpha; a.b = b;
   a.A_log = A_log; a.dt_bias = dt_bias; a.conv0 = conv0;
   a.lower_bound = s->lower_bound; a.eps = s->l2norm_eps;
+  a.beta2 = (s->flags & KDA_FLAG_NEGATIVE_EIGENVALUES) != 0;
   return a;
 }
 
@@ -209,6 +211,7 @@ kda_status kda_decode_step(const kda_shape *shape, const void *q, const void *k,
   a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.b = b; a.conv_w = conv_w;
   a.A_log = A_log; a.dt_bias = dt_bias;
   a.lower_bound = shape->lower_bound; a.eps = shape->l2norm_eps; a.scale = shape->scale;
+  a.beta2 = (shape->flags & KDA_FLAG_NEGATIVE_EIGENVALUES) != 0;
   a.state = state; a.conv_state = conv_state; a.o = o;
   return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream_)));
 }

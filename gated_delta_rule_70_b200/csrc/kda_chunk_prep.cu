@@ -282,7 +282,8 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
     const float negA2 = -expf(a.A_log[h]) * LOG2E;   // the gate is kept in base 2
     const float lb2 = a.lower_bound * LOG2E;
     if (tid < 64 && tid < nt)
-      btj = sigmoid_f(__bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(a.b)[(c0 + tid) * H + h]));
+      btj = (a.beta2 ? 2.f : 1.f) *
+            sigmoid_f(__bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(a.b)[(c0 + tid) * H + h]));
     // causal-conv history of a sequence's first chunk: the caller's conv state or zeros
     const bool hist = cidx == 0 && tg == 0;
     uint4 hraw[3][3];

@@ -91,7 +91,7 @@ decode_kernel(DecodeArgs a) {
     const float al = to_f32(reinterpret_cast<const T *>(a.alpha)[((int64_t)n * H + h) * D + i]);
     const float g = gate_f(al + a.dt_bias[h * D + i], -expf(a.A_log[h]), a.lower_bound);
     sm.eg[i] = expf(g);
-    if (i == 0) sm.beta = sigmoid_f(to_f32(reinterpret_cast<const T *>(a.b)[(int64_t)n * H + h]));
+    if (i == 0) sm.beta = (a.beta2 ? 2.f : 1.f) * sigmoid_f(to_f32(reinterpret_cast<const T *>(a.b)[(int64_t)n * H + h]));
   }
   __syncthreads();
   if (first) {
@@ -342,7 +342,9 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_kernel(DecodeArgs a) {
         const float g = gate_f(al + reinterpret_cast<const float *>(base + S_DTB)[i], -expf(sc.alog[h]),
                                a.lower_bound);
         sc.eg[i] = expf(g);
-        if (i == 0) sc.beta = sigmoid_f(__bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base + S_B)[h]));
+        if (i == 0)
+          sc.beta = (a.beta2 ? 2.f : 1.f) *
+                    sigmoid_f(__bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base + S_B)[h]));
       }
       umma::named_sync(BAR_COMPUTE, NC);
       if (first) {

@@ -97,7 +97,7 @@ cudaError_t run_prefill(PrologueArgs pa, RecurrenceArgs ra, void *final_conv_sta
 #ifndef KDA_TOKEN_KERNEL_ONLY
   if (L.tc) {
     PrepArgs p{};
-    p.lower_bound = pa.lower_bound; p.eps = pa.eps;
+    p.lower_bound = pa.lower_bound; p.eps = pa.eps; p.beta2 = pa.beta2;
     p.conv_w = pa.conv_w; p.b = pa.b; p.A_log = pa.A_log; p.dt_bias = pa.dt_bias; p.conv0 = pa.conv0;
     e = run_chunk_path(p, ra, varlen, true, &pa, ws, L, stream);
   } else

@@ -22,6 +22,7 @@ struct PrologueArgs {
   const float *dt_bias;      // [H, D]
   const void *conv0;         // [N, 3, 3*H*D] or nullptr
   float lower_bound, eps;
+  int beta2;                 // beta = 2 sigmoid(b) (negative eigenvalues allowed); 0: sigmoid(b)
   void *qn, *kn, *vc;        // [T, H, D] io dtype
   float *g;                  // [T, H, D]
   float *beta;               // [T, H]
@@ -53,6 +54,7 @@ struct DecodeArgs {
   const void *conv_w;        // [3, H*D, 4]
   const float *A_log, *dt_bias;
   float lower_bound, eps, scale;
+  int beta2;                 // beta = 2 sigmoid(b); 0: sigmoid(b)
   float *state;              // [N, H, D, D] in place
   void *conv_state;          // [N, 3, 3*H*D] in place
   void *o;                   // [N, H, D]
@@ -68,6 +70,7 @@ struct PrepArgs {
   const int32_t *cu;         // [N + 1] or nullptr (dense)
   const int32_t *chunk_cu;   // [N + 1] chunk prefix (varlen) or nullptr (dense)
   float lower_bound, eps;
+  int beta2;                 // fused: beta = 2 sigmoid(b); 0: sigmoid(b)
   // fused prologue: raw inputs (q, k, v, alpha read through the tensor maps)
   const void *conv_w;        // [3, H*128, 4] bf16
   const void *b;             // [T, H] bf16

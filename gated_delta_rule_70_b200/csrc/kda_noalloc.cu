@@ -57,7 +57,7 @@ extern "C" kda_status kda_prefill_noalloc(
     const float *initial_state, const void *initial_conv_state, const int32_t *cu_seqlens, void *o,
     float *final_state, void *final_conv_state, void *stream_) {
   if (s == nullptr || s->num_seqs < 0 || s->seq_len < 0 || s->num_heads < 1 ||
-      (s->io_dtype != KDA_BF16 && s->io_dtype != KDA_FP32))
+      (s->io_dtype != KDA_BF16 && s->io_dtype != KDA_FP32) || (s->flags & ~KDA_FLAGS_KNOWN))
     return KDA_ERR_INVALID_ARGUMENT;
   if (s->head_dim != 64 && s->head_dim != 128) return KDA_ERR_UNSUPPORTED;
   if (s->num_heads > 64) return KDA_ERR_UNSUPPORTED;
@@ -90,6 +90,7 @@ extern "C" kda_status kda_prefill_noalloc(
   pa.q = q; pa.k = k; pa.v = v; pa.conv_w = conv_w; pa.alpha = alpha; pa.b = b;
   pa.A_log = A_log; pa.dt_bias = dt_bias; pa.conv0 = initial_conv_state;
   pa.lower_bound = s->lower_bound; pa.eps = s->l2norm_eps;
+  pa.beta2 = (s->flags & KDA_FLAG_NEGATIVE_EIGENVALUES) != 0;
   pa.err = reinterpret_cast<int *>(ws + L.err);
 
   RecurrenceArgs ra{};

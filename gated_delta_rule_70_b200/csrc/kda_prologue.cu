@@ -186,7 +186,7 @@ prologue_kernel(PrologueArgs a) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) gt[i] = gate_f(al[i] + bias[i], negA, a.lower_bound);
     store8(a.g + (t * H + h) * D + lane_in_group * 8, gt);
-    if (lane_in_group == 0) a.beta[t * H + h] = sigmoid_f(bvals[j]);
+    if (lane_in_group == 0) a.beta[t * H + h] = (a.beta2 ? 2.f : 1.f) * sigmoid_f(bvals[j]);
   }
 }
 

@@ -45,7 +45,10 @@ class Shape(ctypes.Structure):
     _fields_ = [("num_seqs", ctypes.c_int32), ("seq_len", ctypes.c_int32),
                 ("num_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("lower_bound", ctypes.c_float), ("l2norm_eps", ctypes.c_float),
-                ("scale", ctypes.c_float), ("io_dtype", ctypes.c_int32)]
+                ("scale", ctypes.c_float), ("io_dtype", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+
+
+KDA_FLAG_NEGATIVE_EIGENVALUES = 0x1
 
 
 def library_path() -> str:
@@ -119,9 +122,10 @@ def _dtype_code(dt: torch.dtype) -> int:
 
 
 def make_shape(num_seqs: int, seq_len: int, num_heads: int, head_dim: int, io_dtype: torch.dtype,
-               lower_bound: float = -5.0, l2norm_eps: float = 1e-6, scale: float = 1.0) -> Shape:
+               lower_bound: float = -5.0, l2norm_eps: float = 1e-6, scale: float = 1.0,
+               negative_eigenvalues: bool = False) -> Shape:
     return Shape(num_seqs, seq_len, num_heads, head_dim, lower_bound, l2norm_eps, scale,
-                 _dtype_code(io_dtype))
+                 _dtype_code(io_dtype), KDA_FLAG_NEGATIVE_EIGENVALUES if negative_eigenvalues else 0)
 
 
 def prefill_workspace_size(shape: Shape, varlen: bool) -> int:
@@ -138,19 +142,22 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, conv_w: torch.Ten
             initial_state: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None,
             initial_conv_state: Optional[torch.Tensor] = None, *, num_seqs: Optional[int] = None,
             lower_bound: float = -5.0, l2norm_eps: float = 1e-6,
-            scale: float = 1.0, want_conv_state: bool = True, out: Optional[torch.Tensor] = None,
+            scale: float = 1.0, negative_eigenvalues: bool = False,
+            want_conv_state: bool = True, out: Optional[torch.Tensor] = None,
             final_state: Optional[torch.Tensor] = None,
             final_conv_state: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
             check: bool = True) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
     """KDA prefill.  q, k, v: [T_total, H*d] (or [B, T, H*d] dense); alpha: [.., H, d];
     b: [.., H].  Returns (o [T_total, H, d], final_state [N, H, d, d], final_conv_state
-    [N, 3, 3*H*d] or None).  ``check`` synchronises and raises on device-side errors."""
+    [N, 3, 3*H*d] or None).  ``negative_eigenvalues``: beta = 2 sigmoid(b).  ``check``
+    synchronises and raises on device-side errors."""
     lib = load_library()
     H, d = alpha.shape[-2], alpha.shape[-1]
     if cu_seqlens is not None:
         N = cu_seqlens.numel() - 1
         T_total = q.numel() // (H * d)
-        shape = make_shape(N, T_total, H, d, q.dtype, lower_bound, l2norm_eps, scale)
+        shape = make_shape(N, T_total, H, d, q.dtype, lower_bound, l2norm_eps, scale,
+                           negative_eigenvalues)
     else:
         if q.dim() == 3:
             N, T = q.shape[0], q.shape[1]
@@ -158,7 +165,7 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, conv_w: torch.Ten
             N = 1 if num_seqs is None else num_seqs
             T = q.numel() // (H * d) // N
         T_total = N * T
-        shape = make_shape(N, T, H, d, q.dtype, lower_bound, l2norm_eps, scale)
+        shape = make_shape(N, T, H, d, q.dtype, lower_bound, l2norm_eps, scale, negative_eigenvalues)
     dev = q.device
     o = out if out is not None else torch.empty((T_total, H, d), dtype=q.dtype, device=dev)
     fs = final_state if final_state is not None else torch.empty((N, H, d, d), dtype=torch.float32,
@@ -180,23 +187,26 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, conv_w: torch.Ten
     return o, fs, fc
 
 
-def _prefill_shape(q, alpha, cu_seqlens, num_seqs, lower_bound, l2norm_eps, scale):
+def _prefill_shape(q, alpha, cu_seqlens, num_seqs, lower_bound, l2norm_eps, scale,
+                   negative_eigenvalues=False):
     H, d = alpha.shape[-2], alpha.shape[-1]
     T_total = q.numel() // (H * d)
     if cu_seqlens is not None:
         return make_shape(cu_seqlens.numel() - 1, T_total, H, d, q.dtype, lower_bound, l2norm_eps,
-                          scale), T_total
+                          scale, negative_eigenvalues), T_total
     N = (q.shape[0] if q.dim() == 3 else 1) if num_seqs is None else num_seqs
-    return make_shape(N, T_total // max(N, 1), H, d, q.dtype, lower_bound, l2norm_eps, scale), T_total
+    return make_shape(N, T_total // max(N, 1), H, d, q.dtype, lower_bound, l2norm_eps, scale,
+                      negative_eigenvalues), T_total
 
 
 def prologue(q, k, v, conv_w, alpha, b, A_log, dt_bias, cu_seqlens=None, initial_conv_state=None,
              *, num_seqs: Optional[int] = None, lower_bound: float = -5.0, l2norm_eps: float = 1e-6,
-             want_conv_state: bool = False, out=None):
+             negative_eigenvalues: bool = False, want_conv_state: bool = False, out=None):
     """The prologue alone: returns (qn, kn, vc [T,H,d] io dtype, g [T,H,d] fp32, beta [T,H] fp32,
     final_conv_state [N,3,3*H*d] or None).  ``out`` may pass those six buffers preallocated."""
     lib = load_library()
-    shape, T_total = _prefill_shape(q, alpha, cu_seqlens, num_seqs, lower_bound, l2norm_eps, 1.0)
+    shape, T_total = _prefill_shape(q, alpha, cu_seqlens, num_seqs, lower_bound, l2norm_eps, 1.0,
+                                    negative_eigenvalues)
     H, d, N = shape.num_heads, shape.head_dim, shape.num_seqs
     dev = q.device
     if out is None:
@@ -246,12 +256,13 @@ def recurrence(qn, kn, vc, g, beta, initial_state=None, cu_seqlens=None, *,
 
 def decode_step(q, k, v, alpha, b, conv_w, A_log, dt_bias, state: torch.Tensor,
                 conv_state: torch.Tensor, *, lower_bound: float = -5.0, l2norm_eps: float = 1e-6,
-                scale: float = 1.0, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                scale: float = 1.0, negative_eigenvalues: bool = False,
+                out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """One token per sequence; updates ``state`` [N,H,d,d] and ``conv_state`` [N,3,3*H*d] in
     place and returns o [N, H, d]."""
     lib = load_library()
     N, H, d = state.shape[0], state.shape[1], state.shape[2]
-    shape = make_shape(N, 1, H, d, q.dtype, lower_bound, l2norm_eps, scale)
+    shape = make_shape(N, 1, H, d, q.dtype, lower_bound, l2norm_eps, scale, negative_eigenvalues)
     o = out if out is not None else torch.empty((N, H, d), dtype=q.dtype, device=q.device)
     st = lib.kda_decode_step(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b),
                              _ptr(conv_w), _ptr(A_log), _ptr(dt_bias), _ptr(state),

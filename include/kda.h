@@ -80,7 +80,15 @@ typedef struct {
     float l2norm_eps;    /* added to |x|^2 inside the square root: 1e-6f */
     float scale;         /* output scale on S^T q: 1.0f (the pages apply none) */
     int32_t io_dtype;    /* kda_dtype */
+    uint32_t flags;      /* KDA_FLAG_* bits; 0 is the configuration the pages run */
 } kda_shape;
+
+/* beta = 2 sigmoid(b), in (0, 2), instead of sigmoid(b): the write's transition
+ * I - beta k k^T then has eigenvalue 1 - beta in (-1, 1) along k.  The KDA layer's
+ * kda_allow_negative_eigenvalues switch (AliceAI-Foundation KDA write-up, section
+ * "二": with the switch off, beta is not doubled and stays in (0, 1)). */
+#define KDA_FLAG_NEGATIVE_EIGENVALUES 0x1u
+#define KDA_FLAGS_KNOWN 0x1u
 
 /* Bytes of device workspace kda_prefill() needs for this shape (0 on a bad
  * shape).  is_varlen != 0: shape->seq_len is the packed token total (the call

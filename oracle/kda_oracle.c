@@ -43,6 +43,7 @@ typedef struct {
     const double *q, *k, *v, *conv_w, *alpha, *b, *A_log, *dt_bias;
     const double *state0, *conv0;
     double lower_bound, eps, scale;
+    int beta2;              /* kda_allow_negative_eigenvalues: beta = 2 sigmoid(b) */
     double *o, *state1, *conv1;
     /* prologue-only outputs (any may be NULL) */
     double *qn, *kn, *vc, *g, *beta;
@@ -106,13 +107,15 @@ static void run_pair(const job_t *J, int64_t n, int64_t h)
         for (int64_t i = 0; i < D; ++i) { sq += qt[i] * qt[i]; sk += kt[i] * kt[i]; }
         double rq = 1.0 / sqrt(sq + J->eps), rk = 1.0 / sqrt(sk + J->eps);
         for (int64_t i = 0; i < D; ++i) { qt[i] *= rq; kt[i] *= rk; }
-        /* gate g = max(-exp(A_log) * softplus(alpha + dt_bias), lower_bound); beta = sigmoid(b) */
+        /* gate g = max(-exp(A_log) * softplus(alpha + dt_bias), lower_bound); beta = sigmoid(b),
+         * doubled when negative eigenvalues are allowed (section "二": with
+         * kda_allow_negative_eigenvalues off, beta is not multiplied by 2) */
         for (int64_t i = 0; i < D; ++i) {
             double x = J->alpha[(row * H + h) * D + i] + J->dt_bias[h * D + i];
             double g = -A * softplus(x);
             gt[i] = g < J->lower_bound ? J->lower_bound : g;
         }
-        const double beta = sigmoid(J->b[row * H + h]);
+        const double beta = (J->beta2 ? 2.0 : 1.0) * sigmoid(J->b[row * H + h]);
 
         if (J->qn) for (int64_t i = 0; i < D; ++i) J->qn[(row * H + h) * D + i] = qt[i];
         if (J->kn) for (int64_t i = 0; i < D; ++i) J->kn[(row * H + h) * D + i] = kt[i];
@@ -193,7 +196,7 @@ int kda_oracle_forward(int64_t N, const int64_t *cu_seqlens, int64_t H, int64_t 
                        const double *conv_w, const double *alpha, const double *b,
                        const double *A_log, const double *dt_bias,
                        const double *state0, const double *conv0,
-                       double lower_bound, double eps, double scale,
+                       double lower_bound, double eps, double scale, int beta2,
                        double *o, double *state1, double *conv1, int nthreads)
 {
     job_t J;
@@ -201,7 +204,7 @@ int kda_oracle_forward(int64_t N, const int64_t *cu_seqlens, int64_t H, int64_t 
     J.N = N; J.H = H; J.D = D; J.cu = cu_seqlens;
     J.q = q; J.k = k; J.v = v; J.conv_w = conv_w; J.alpha = alpha; J.b = b;
     J.A_log = A_log; J.dt_bias = dt_bias; J.state0 = state0; J.conv0 = conv0;
-    J.lower_bound = lower_bound; J.eps = eps; J.scale = scale;
+    J.lower_bound = lower_bound; J.eps = eps; J.scale = scale; J.beta2 = beta2;
     J.o = o; J.state1 = state1; J.conv1 = conv1;
     J.run_recurrence = 1;
     return run_all(&J, nthreads);
@@ -212,7 +215,7 @@ int kda_oracle_prologue(int64_t N, const int64_t *cu_seqlens, int64_t H, int64_t
                         const double *q, const double *k, const double *v,
                         const double *conv_w, const double *alpha, const double *b,
                         const double *A_log, const double *dt_bias, const double *conv0,
-                        double lower_bound, double eps,
+                        double lower_bound, double eps, int beta2,
                         double *qn, double *kn, double *vc, double *g, double *beta,
                         int nthreads)
 {
@@ -221,7 +224,7 @@ int kda_oracle_prologue(int64_t N, const int64_t *cu_seqlens, int64_t H, int64_t
     J.N = N; J.H = H; J.D = D; J.cu = cu_seqlens;
     J.q = q; J.k = k; J.v = v; J.conv_w = conv_w; J.alpha = alpha; J.b = b;
     J.A_log = A_log; J.dt_bias = dt_bias; J.conv0 = conv0;
-    J.lower_bound = lower_bound; J.eps = eps; J.scale = 1.0;
+    J.lower_bound = lower_bound; J.eps = eps; J.scale = 1.0; J.beta2 = beta2;
     J.qn = qn; J.kn = kn; J.vc = vc; J.g = g; J.beta = beta;
     J.run_recurrence = 0;
     return run_all(&J, nthreads);

@@ -48,10 +48,10 @@ def _bind(lib):
     I = ctypes.POINTER(ctypes.c_int64)
     i64, f64 = ctypes.c_int64, ctypes.c_double
     lib.kda_oracle_forward.argtypes = [i64, I, i64, i64, D, D, D, D, D, D, D, D, D, D,
-                                       f64, f64, f64, D, D, D, ctypes.c_int]
+                                       f64, f64, f64, ctypes.c_int, D, D, D, ctypes.c_int]
     lib.kda_oracle_forward.restype = ctypes.c_int
     lib.kda_oracle_prologue.argtypes = [i64, I, i64, i64, D, D, D, D, D, D, D, D, D,
-                                        f64, f64, D, D, D, D, D, ctypes.c_int]
+                                        f64, f64, ctypes.c_int, D, D, D, D, D, ctypes.c_int]
     lib.kda_oracle_prologue.restype = ctypes.c_int
     lib.kda_oracle_recurrence.argtypes = [i64, I, i64, i64, D, D, D, D, D, D, f64, D, D]
     lib.kda_oracle_recurrence.restype = ctypes.c_int
@@ -91,10 +91,11 @@ def _cu(cu_seqlens) -> np.ndarray:
 
 def forward(cu_seqlens, H: int, D: int, q, k, v, conv_w, alpha, b, A_log, dt_bias,
             state0=None, conv0=None, lower_bound: float = -5.0, eps: float = 1e-6,
-            scale: float = 1.0, nthreads: int = 0
+            scale: float = 1.0, nthreads: int = 0, negative_eigenvalues: bool = False
             ) -> Tuple[np.ndarray, np.ndarray, np.ndarray, int]:
     """Prefill over packed sequences.  Returns (o [T,H,D], final_state [N,H,D,D],
-    final_conv_state [N,3,3*H*D], threads used)."""
+    final_conv_state [N,3,3*H*D], threads used).  ``negative_eigenvalues``: beta =
+    2 sigmoid(b) (the kda_allow_negative_eigenvalues switch, section "二")."""
     cu = _cu(cu_seqlens)
     N, T = len(cu) - 1, int(cu[-1])
     q, k, v, conv_w, alpha, b = map(_f, (q, k, v, conv_w, alpha, b))
@@ -105,12 +106,14 @@ def forward(cu_seqlens, H: int, D: int, q, k, v, conv_w, alpha, b, A_log, dt_bia
     used = _load().kda_oracle_forward(
         N, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), H, D,
         _p(q), _p(k), _p(v), _p(conv_w), _p(alpha), _p(b), _p(A_log), _p(dt_bias),
-        _p(state0), _p(conv0), lower_bound, eps, scale, _p(o), _p(s1), _p(c1), nthreads)
+        _p(state0), _p(conv0), lower_bound, eps, scale, int(negative_eigenvalues), _p(o), _p(s1),
+        _p(c1), nthreads)
     return o, s1, c1, used
 
 
 def prologue(cu_seqlens, H: int, D: int, q, k, v, conv_w, alpha, b, A_log, dt_bias,
-             conv0=None, lower_bound: float = -5.0, eps: float = 1e-6, nthreads: int = 0):
+             conv0=None, lower_bound: float = -5.0, eps: float = 1e-6, nthreads: int = 0,
+             negative_eigenvalues: bool = False):
     """Prepared per-token inputs: (qn, kn, vc [T,H,D], g [T,H,D], beta [T,H])."""
     cu = _cu(cu_seqlens)
     N, T = len(cu) - 1, int(cu[-1])
@@ -121,7 +124,8 @@ def prologue(cu_seqlens, H: int, D: int, q, k, v, conv_w, alpha, b, A_log, dt_bi
     _load().kda_oracle_prologue(
         N, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), H, D,
         _p(q), _p(k), _p(v), _p(conv_w), _p(alpha), _p(b), _p(A_log), _p(dt_bias),
-        _p(conv0), lower_bound, eps, _p(qn), _p(kn), _p(vc), _p(g), _p(beta), nthreads)
+        _p(conv0), lower_bound, eps, int(negative_eigenvalues), _p(qn), _p(kn), _p(vc), _p(g),
+        _p(beta), nthreads)
     return qn, kn, vc, g, beta
 
 
@@ -141,14 +145,15 @@ def recurrence(cu_seqlens, q, k, v, g, beta, state0=None, scale: float = 1.0):
 
 def decode_step(H: int, D: int, state, conv_state, q, k, v, alpha, b, conv_w, A_log,
                 dt_bias, lower_bound: float = -5.0, eps: float = 1e-6, scale: float = 1.0,
-                nthreads: int = 0):
+                nthreads: int = 0, negative_eigenvalues: bool = False):
     """One token per sequence (q, k, v [N, H*D], alpha [N,H,D], b [N,H]) on top of
     (state [N,H,D,D], conv_state [N,3,3*H*D]).  Returns (o [N,H,D], state', conv_state')."""
     N = np.asarray(state).shape[0]
     cu = np.arange(N + 1, dtype=np.int64)
     o, s1, c1, _ = forward(cu, H, D, q, k, v, conv_w, alpha, b, A_log, dt_bias,
                            state0=state, conv0=conv_state, lower_bound=lower_bound,
-                           eps=eps, scale=scale, nthreads=nthreads)
+                           eps=eps, scale=scale, nthreads=nthreads,
+                           negative_eigenvalues=negative_eigenvalues)
     return o, s1, c1
 
 

@@ -88,6 +88,9 @@ def test_host_validation_codes(lib):
     bad_dtype = kda.make_shape(1, 16, 2, 64, torch.float32)
     bad_dtype.io_dtype = 7
     assert _call_prefill(lib, bad_dtype) == kda.KDA_ERR_INVALID_ARGUMENT
+    bad_flags = kda.make_shape(1, 16, 2, 64, torch.float32)
+    bad_flags.flags = 0x80
+    assert _call_prefill(lib, bad_flags) == kda.KDA_ERR_INVALID_ARGUMENT
     nan_lb = kda.make_shape(1, 16, 2, 64, torch.float32, lower_bound=float("nan"))
     assert _call_prefill(lib, nan_lb) == kda.KDA_ERR_INVALID_ARGUMENT
     # misaligned tensor pointer

@@ -26,14 +26,14 @@ def _dev(arr):
     return W.to_device(arr)
 
 
-def gpu_prefill(s: W.Spec, inp: dict, conv0=None, want_conv=True):
+def gpu_prefill(s: W.Spec, inp: dict, conv0=None, want_conv=True, neg=False):
     cu = _dev(inp["cu_seqlens"]) if s.varlen else None
     o, fs, fc = kda.prefill(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["conv_w"]),
                             _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]),
                             _dev(inp["dt_bias"]), initial_state=_dev(inp["S0"]), cu_seqlens=cu,
                             initial_conv_state=_dev(conv0), num_seqs=s.num_seqs,
                             lower_bound=s.lower_bound, l2norm_eps=s.eps, scale=s.scale,
-                            want_conv_state=want_conv)
+                            negative_eigenvalues=neg, want_conv_state=want_conv)
     torch.cuda.synchronize()
     return o, fs, fc
 
@@ -42,12 +42,12 @@ def f64_inputs(inp):
     return {k: W.as_f64(v) for k, v in inp.items() if k != "cu_seqlens"}
 
 
-def oracle_prefill(s: W.Spec, inp: dict, conv0=None):
+def oracle_prefill(s: W.Spec, inp: dict, conv0=None, neg=False):
     f = f64_inputs(inp)
     return oracle.forward(inp["cu_seqlens"], s.H, s.d, f["q"], f["k"], f["v"], f["conv_w"],
                           f["alpha"], f["b"], f["A_log"], f["dt_bias"], state0=f["S0"],
                           conv0=W.as_f64(conv0), lower_bound=s.lower_bound, eps=s.eps,
-                          scale=s.scale)
+                          scale=s.scale, negative_eigenvalues=neg)
 
 
 def rel_l2(x, ref):
@@ -74,10 +74,10 @@ def max_state_err(s_gpu, s_ref):
     return max(rel_l2(s_gpu[n, h], s_ref[n, h]) for n in range(N) for h in range(H))
 
 
-def check_prefill(s: W.Spec, conv0=None):
+def check_prefill(s: W.Spec, conv0=None, neg=False):
     inp = W.make_inputs(s)
-    o, fs, fc = gpu_prefill(s, inp, conv0)
-    o_ref, s_ref, c_ref, _ = oracle_prefill(s, inp, conv0)
+    o, fs, fc = gpu_prefill(s, inp, conv0, neg=neg)
+    o_ref, s_ref, c_ref, _ = oracle_prefill(s, inp, conv0, neg=neg)
     tol = TOL[s.io_dtype]
     eo = max_pair_err(W.from_device(o), o_ref, inp["cu_seqlens"], s.H)
     es = max_state_err(W.from_device(fs), s_ref)
@@ -241,25 +241,27 @@ def _decode_inputs(s: W.Spec, step):
     return W.make_decode_step(s, step)
 
 
-@pytest.mark.parametrize("H,N,T1", [(3, 5, 70), (16, 40, 20)])
-def test_decode_parity_and_handoff(H, N, T1):
+@pytest.mark.parametrize("H,N,T1,neg", [(3, 5, 70, False), (16, 40, 20, False), (3, 4, 30, True),
+                                        (16, 40, 20, True)])
+def test_decode_parity_and_handoff(H, N, T1, neg):
     """prefill(T1) -> decode steps on GPU vs the oracle.  H=3 takes the per-item kernel;
-    H=16 with 640 items takes the persistent one, several items per CTA around its ring."""
+    H=16 with 640 items takes the persistent one, several items per CTA around its ring.
+    neg: beta = 2 sigmoid(b) in the prefill and every step."""
     d, steps = 128, 4
     s = W.small("dec", [T1] * N, H=H, d=d, seed=21, s0_std=0.02)
     inp = W.make_inputs(s)
-    o, st, cs = gpu_prefill(s, inp)
+    o, st, cs = gpu_prefill(s, inp, neg=neg)
     f = f64_inputs(inp)
-    o_ref, s_ref, c_ref, _ = oracle_prefill(s, inp)
+    o_ref, s_ref, c_ref, _ = oracle_prefill(s, inp, neg=neg)
     for step in range(steps):
         x = _decode_inputs(s, step)
         o_t = kda.decode_step(_dev(x["q"]), _dev(x["k"]), _dev(x["v"]), _dev(x["alpha"]),
                               _dev(x["b"]), _dev(inp["conv_w"]), _dev(inp["A_log"]),
-                              _dev(inp["dt_bias"]), st, cs)
+                              _dev(inp["dt_bias"]), st, cs, negative_eigenvalues=neg)
         xf = {k: W.as_f64(v) for k, v in x.items()}
         o_r, s_ref, c_ref = oracle.decode_step(H, d, s_ref, c_ref, xf["q"], xf["k"], xf["v"],
                                                xf["alpha"], xf["b"], f["conv_w"], f["A_log"],
-                                               f["dt_bias"])
+                                               f["dt_bias"], negative_eigenvalues=neg)
         torch.cuda.synchronize()
         og = W.from_device(o_t)
         worst = max(rel_l2(og[n, h], o_r[n, h]) for n in range(N) for h in range(H))
@@ -309,3 +311,29 @@ def test_prefill_plus_decode_equals_long_prefill_gpu():
     for h in range(H):
         assert rel_l2(o_cat[:, h], ol[:, h]) <= TOL["bf16"]
     assert max_state_err(W.from_device(st), W.from_device(s_long)) <= TOL["bf16"]
+
+
+# ------------------------------------------------------------------ negative eigenvalues
+
+@pytest.mark.parametrize("io,d,lens", [("bf16", 128, [1, 70, 200]), ("fp32", 64, [33, 90]),
+                                       ("fp32", 128, [65])])
+def test_prefill_negative_eigenvalues(io, d, lens):
+    """beta = 2 sigmoid(b) (kda_allow_negative_eigenvalues): the bf16 chunk path and the
+    fp32 token kernel against the switched oracle."""
+    s = W.small("neg", lens, H=3, d=d, io_dtype=io, seed=41, s0_std=0.02, varlen=len(lens) > 1)
+    check_prefill(s, neg=True)
+
+
+def test_prologue_negative_eigenvalues_beta():
+    s = W.small("negpro", [9, 30], H=2, d=128, io_dtype="bf16", seed=42)
+    inp = W.make_inputs(s)
+    out = kda.prologue(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["conv_w"]),
+                       _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]), _dev(inp["dt_bias"]),
+                       cu_seqlens=_dev(inp["cu_seqlens"]), num_seqs=s.num_seqs,
+                       negative_eigenvalues=True)
+    torch.cuda.synchronize()
+    f = f64_inputs(inp)
+    ref = oracle.prologue(inp["cu_seqlens"], s.H, s.d, f["q"], f["k"], f["v"], f["conv_w"],
+                          f["alpha"], f["b"], f["A_log"], f["dt_bias"], negative_eigenvalues=True)
+    np.testing.assert_allclose(W.from_device(out[4]), ref[4], rtol=1e-5, atol=1e-6)
+    assert float(W.from_device(out[4]).max()) > 1.0   # the doubled range is in use

@@ -31,8 +31,10 @@ MUTATIONS = {
     "decay_exp_of_neg": ("double e = exp(gt[i]);", "double e = exp(-gt[i]);"),
     "eps_outside_root": ("1.0 / sqrt(sq + J->eps)", "1.0 / (sqrt(sq) + J->eps)"),
     "conv_history_shift": ("raw_at(J, n, t - (KCONV - 1) + j, c)", "raw_at(J, n, t - KCONV + j, c)"),
-    "beta_not_sigmoid": ("const double beta = sigmoid(J->b[row * H + h]);",
-                         "const double beta = J->b[row * H + h];"),
+    "beta_not_sigmoid": ("const double beta = (J->beta2 ? 2.0 : 1.0) * sigmoid(J->b[row * H + h]);",
+                         "const double beta = (J->beta2 ? 2.0 : 1.0) * J->b[row * H + h];"),
+    "beta2_ignored": ("(J->beta2 ? 2.0 : 1.0) * sigmoid", "1.0 * sigmoid"),
+    "beta2_squared": ("(J->beta2 ? 2.0 : 1.0) * sigmoid", "(J->beta2 ? 4.0 : 1.0) * sigmoid"),
 }
 
 PIN_TESTS = [
@@ -45,6 +47,9 @@ PIN_TESTS = [
     pins.test_lower_bound_decay_closed_form,
     pins.test_forward_equals_prologue_then_recurrence,
     lambda: [pins.test_prefill_then_decode_equals_long_prefill(a, b) for a, b in [(7, 5), (1, 4)]],
+    pins.test_negative_eigenvalues_beta_is_twice_sigmoid,
+    pins.test_negative_eigenvalues_write_is_a_householder_reflection,
+    pins.test_negative_eigenvalues_equal_plain_run_with_rescaled_b,
 ]
 
 

@@ -191,6 +191,80 @@ def test_lower_bound_decay_closed_form():
 
 # ---------------------------------------------------------------- composition
 
+# ---------------------------------------------------------------- negative eigenvalues
+# The kda_allow_negative_eigenvalues switch (AliceAI-Foundation KDA write-up, section
+# "二": with it off, beta is not multiplied by 2 and stays in (0, 1)): beta = 2 sigmoid(b).
+
+def test_negative_eigenvalues_beta_is_twice_sigmoid():
+    """The prologue's beta doubles; q, k, v and g do not change."""
+    H, D, lens = 2, 8, [7, 3]
+    I = _prologue_inputs(31, lens, H, D)
+    args = (I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"], I["alpha"], I["b"], I["A_log"],
+            I["dt_bias"])
+    plain = oracle.prologue(*args)
+    neg = oracle.prologue(*args, negative_eigenvalues=True)
+    for x, y in zip(plain[:4], neg[:4]):
+        np.testing.assert_array_equal(x, y)
+    np.testing.assert_allclose(neg[4], 2.0 * sp.expit(I["b"]), rtol=1e-14)
+
+
+def test_negative_eigenvalues_write_is_a_householder_reflection():
+    """beta = 2 (b -> +inf), no decay (alpha -> -inf), unit key (eps = 0), v = 0: one
+    write maps S to (I - 2 k k^T) S, the reflection through the plane normal to k,
+    whose eigenvalue along k is -1."""
+    H, D = 1, 6
+    I = _prologue_inputs(32, [1], H, D)
+    I["b"][:] = 50.0          # sigmoid -> 1 in fp64
+    I["alpha"][:] = -800.0    # softplus -> 0, g = 0
+    I["v"][:] = 0.0
+    S0 = _rng(33).standard_normal((1, H, D, D))
+    o, S1, _, _ = oracle.forward(I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"], I["alpha"],
+                                 I["b"], I["A_log"], I["dt_bias"], state0=S0, eps=0.0,
+                                 negative_eigenvalues=True)
+    # the unit key, from the conv + SiLU + norm of token 0 (only the newest tap sees it)
+    y = I["k"][0] * I["conv_w"][1][:, 3]
+    k = y * sp.expit(y)
+    k /= np.linalg.norm(k)
+    R = np.eye(D) - 2.0 * np.outer(k, k)
+    np.testing.assert_allclose(S1[0, 0], R @ S0[0, 0], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(k @ S1[0, 0], -(k @ S0[0, 0]), rtol=1e-12, atol=1e-13)
+    # without the switch the same write is a projection: k^T S' = 0
+    _, S1p, _, _ = oracle.forward(I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"], I["alpha"],
+                                  I["b"], I["A_log"], I["dt_bias"], state0=S0, eps=0.0)
+    np.testing.assert_allclose(k @ S1p[0, 0], 0.0, atol=1e-13)
+
+
+def test_negative_eigenvalues_equal_plain_run_with_rescaled_b():
+    """For b < 0, 2 sigmoid(b) < 1 is itself a sigmoid: the switched run equals the plain
+    run on b' = logit(2 sigmoid(b))."""
+    H, D, lens = 2, 8, [9, 5]
+    I = _prologue_inputs(34, lens, H, D)
+    I["b"] = -np.abs(I["b"]) - 0.1
+    S0 = _rng(35).standard_normal((2, H, D, D)) * 0.1
+    common = (I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"], I["alpha"])
+    o1, S1, _, _ = oracle.forward(*common, I["b"], I["A_log"], I["dt_bias"], state0=S0,
+                                  negative_eigenvalues=True)
+    b2 = sp.logit(2.0 * sp.expit(I["b"]))
+    o2, S2, _, _ = oracle.forward(*common, b2, I["A_log"], I["dt_bias"], state0=S0)
+    np.testing.assert_allclose(o1, o2, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(S1, S2, rtol=1e-10, atol=1e-12)
+
+
+def test_recurrence_with_beta_above_one_matches_unrolled_product():
+    """beta in (1, 2): the transition has a negative eigenvalue; the product form still holds."""
+    r = _rng(36)
+    T, D = 6, 4
+    q, k, v = (r.standard_normal((T, 1, D)) for _ in range(3))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    g = -r.uniform(0, 1, (T, 1, D))
+    beta = r.uniform(1.05, 1.95, (T, 1))
+    S0 = r.standard_normal((1, 1, D, D))
+    o, S = oracle.recurrence([0, T], q, k, v, g, beta, S0)
+    o_ref, S_ref = _brute_force(q[:, 0], k[:, 0], v[:, 0], g[:, 0], beta[:, 0], S0[0, 0])
+    np.testing.assert_allclose(o[:, 0], o_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(S[0, 0], S_ref, rtol=1e-12, atol=1e-12)
+
+
 def test_forward_equals_prologue_then_recurrence():
     H, D, lens = 2, 8, [9, 4]
     I = _prologue_inputs(16, lens, H, D)
