@@ -27,6 +27,15 @@
  *   conv_state     [N, 3, 3*H*D]   raw inputs of the 3 tokens before the
  *                                  sequence start, oldest first
  *   o              [Ttot, H, D]
+ *   ogate          [Ttot, H, D]    output gate (pre-sigmoid), optional
+ *   onw            [D]             o_norm weight, shared by the heads
+ *
+ * Output epilogue (optional): the layer's o_norm and sigmoid output gating
+ * (same write-up: the KDA layer projects an output_gate, section "二", and ends
+ * in o_norm plus sigmoid gating, section "三"; the Ling-3.0-flash-VL weight list
+ * names o_norm and g_proj).  Read as an RMS norm over the head's D channels with
+ * a per-channel weight, then the elementwise sigmoid gate:
+ *   o[j] <- o[j] / sqrt(mean_j o^2 + oeps) * onw[j] * sigmoid(ogate[j]).
  */
 #include <math.h>
 #include <pthread.h>
@@ -44,6 +53,8 @@ typedef struct {
     const double *state0, *conv0;
     double lower_bound, eps, scale;
     int beta2;              /* kda_allow_negative_eigenvalues: beta = 2 sigmoid(b) */
+    const double *ogate, *onw;   /* output epilogue, or NULL */
+    double oeps;
     double *o, *state1, *conv1;
     /* prologue-only outputs (any may be NULL) */
     double *qn, *kn, *vc, *g, *beta;
@@ -137,10 +148,18 @@ static void run_pair(const job_t *J, int64_t n, int64_t h)
         for (int64_t j = 0; j < D; ++j) dl[j] = (vt[j] - p[j]) * beta;
         for (int64_t i = 0; i < D; ++i)
             for (int64_t j = 0; j < D; ++j) S[i * D + j] += kt[i] * dl[j];
+        double *ot = J->o + (row * H + h) * D;
         for (int64_t j = 0; j < D; ++j) {
             double acc = 0.0;
             for (int64_t i = 0; i < D; ++i) acc += qt[i] * S[i * D + j];
-            J->o[(row * H + h) * D + j] = J->scale * acc;
+            ot[j] = J->scale * acc;
+        }
+        if (J->ogate) {   /* o_norm (RMS over the head's D channels, weighted), then the gate */
+            double ms = 0.0;
+            for (int64_t j = 0; j < D; ++j) ms += ot[j] * ot[j];
+            const double r = 1.0 / sqrt(ms / (double)D + J->oeps);
+            for (int64_t j = 0; j < D; ++j)
+                ot[j] = ot[j] * r * J->onw[j] * sigmoid(J->ogate[(row * H + h) * D + j]);
         }
     }
 
@@ -197,6 +216,7 @@ int kda_oracle_forward(int64_t N, const int64_t *cu_seqlens, int64_t H, int64_t 
                        const double *A_log, const double *dt_bias,
                        const double *state0, const double *conv0,
                        double lower_bound, double eps, double scale, int beta2,
+                       const double *ogate, const double *onw, double oeps,
                        double *o, double *state1, double *conv1, int nthreads)
 {
     job_t J;
@@ -205,6 +225,7 @@ int kda_oracle_forward(int64_t N, const int64_t *cu_seqlens, int64_t H, int64_t 
     J.q = q; J.k = k; J.v = v; J.conv_w = conv_w; J.alpha = alpha; J.b = b;
     J.A_log = A_log; J.dt_bias = dt_bias; J.state0 = state0; J.conv0 = conv0;
     J.lower_bound = lower_bound; J.eps = eps; J.scale = scale; J.beta2 = beta2;
+    J.ogate = ogate; J.onw = onw; J.oeps = oeps;
     J.o = o; J.state1 = state1; J.conv1 = conv1;
     J.run_recurrence = 1;
     return run_all(&J, nthreads);

@@ -48,7 +48,7 @@ def _bind(lib):
     I = ctypes.POINTER(ctypes.c_int64)
     i64, f64 = ctypes.c_int64, ctypes.c_double
     lib.kda_oracle_forward.argtypes = [i64, I, i64, i64, D, D, D, D, D, D, D, D, D, D,
-                                       f64, f64, f64, ctypes.c_int, D, D, D, ctypes.c_int]
+                                       f64, f64, f64, ctypes.c_int, D, D, f64, D, D, D, ctypes.c_int]
     lib.kda_oracle_forward.restype = ctypes.c_int
     lib.kda_oracle_prologue.argtypes = [i64, I, i64, i64, D, D, D, D, D, D, D, D, D,
                                         f64, f64, ctypes.c_int, D, D, D, D, D, ctypes.c_int]
@@ -91,23 +91,28 @@ def _cu(cu_seqlens) -> np.ndarray:
 
 def forward(cu_seqlens, H: int, D: int, q, k, v, conv_w, alpha, b, A_log, dt_bias,
             state0=None, conv0=None, lower_bound: float = -5.0, eps: float = 1e-6,
-            scale: float = 1.0, nthreads: int = 0, negative_eigenvalues: bool = False
+            scale: float = 1.0, nthreads: int = 0, negative_eigenvalues: bool = False,
+            out_gate=None, o_norm_weight=None, o_norm_eps: float = 1e-5
             ) -> Tuple[np.ndarray, np.ndarray, np.ndarray, int]:
     """Prefill over packed sequences.  Returns (o [T,H,D], final_state [N,H,D,D],
     final_conv_state [N,3,3*H*D], threads used).  ``negative_eigenvalues``: beta =
-    2 sigmoid(b) (the kda_allow_negative_eigenvalues switch, section "二")."""
+    2 sigmoid(b) (the kda_allow_negative_eigenvalues switch, section "二").  ``out_gate``
+    [T,H,D] with ``o_norm_weight`` [D]: the output epilogue o <- rmsnorm(o) * w * sigmoid(gate)."""
     cu = _cu(cu_seqlens)
     N, T = len(cu) - 1, int(cu[-1])
     q, k, v, conv_w, alpha, b = map(_f, (q, k, v, conv_w, alpha, b))
     A_log, dt_bias, state0, conv0 = map(_f, (A_log, dt_bias, state0, conv0))
+    out_gate, o_norm_weight = _f(out_gate), _f(o_norm_weight)
+    if (out_gate is None) != (o_norm_weight is None):
+        raise ValueError("out_gate and o_norm_weight go together")
     o = np.zeros((T, H, D))
     s1 = np.zeros((N, H, D, D))
     c1 = np.zeros((N, 3, 3 * H * D))
     used = _load().kda_oracle_forward(
         N, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), H, D,
         _p(q), _p(k), _p(v), _p(conv_w), _p(alpha), _p(b), _p(A_log), _p(dt_bias),
-        _p(state0), _p(conv0), lower_bound, eps, scale, int(negative_eigenvalues), _p(o), _p(s1),
-        _p(c1), nthreads)
+        _p(state0), _p(conv0), lower_bound, eps, scale, int(negative_eigenvalues), _p(out_gate),
+        _p(o_norm_weight), o_norm_eps, _p(o), _p(s1), _p(c1), nthreads)
     return o, s1, c1, used
 
 
@@ -145,7 +150,8 @@ def recurrence(cu_seqlens, q, k, v, g, beta, state0=None, scale: float = 1.0):
 
 def decode_step(H: int, D: int, state, conv_state, q, k, v, alpha, b, conv_w, A_log,
                 dt_bias, lower_bound: float = -5.0, eps: float = 1e-6, scale: float = 1.0,
-                nthreads: int = 0, negative_eigenvalues: bool = False):
+                nthreads: int = 0, negative_eigenvalues: bool = False, out_gate=None,
+                o_norm_weight=None, o_norm_eps: float = 1e-5):
     """One token per sequence (q, k, v [N, H*D], alpha [N,H,D], b [N,H]) on top of
     (state [N,H,D,D], conv_state [N,3,3*H*D]).  Returns (o [N,H,D], state', conv_state')."""
     N = np.asarray(state).shape[0]
@@ -153,7 +159,8 @@ def decode_step(H: int, D: int, state, conv_state, q, k, v, alpha, b, conv_w, A_
     o, s1, c1, _ = forward(cu, H, D, q, k, v, conv_w, alpha, b, A_log, dt_bias,
                            state0=state, conv0=conv_state, lower_bound=lower_bound,
                            eps=eps, scale=scale, nthreads=nthreads,
-                           negative_eigenvalues=negative_eigenvalues)
+                           negative_eigenvalues=negative_eigenvalues, out_gate=out_gate,
+                           o_norm_weight=o_norm_weight, o_norm_eps=o_norm_eps)
     return o, s1, c1
 
 

@@ -35,6 +35,11 @@ MUTATIONS = {
                          "const double beta = (J->beta2 ? 2.0 : 1.0) * J->b[row * H + h];"),
     "beta2_ignored": ("(J->beta2 ? 2.0 : 1.0) * sigmoid", "1.0 * sigmoid"),
     "beta2_squared": ("(J->beta2 ? 2.0 : 1.0) * sigmoid", "(J->beta2 ? 4.0 : 1.0) * sigmoid"),
+    "onorm_sum_not_mean": ("sqrt(ms / (double)D + J->oeps)", "sqrt(ms + J->oeps)"),
+    "onorm_eps_outside_root": ("1.0 / sqrt(ms / (double)D + J->oeps)", "1.0 / (sqrt(ms / (double)D) + J->oeps)"),
+    "onorm_no_weight": ("ot[j] * r * J->onw[j] * sigmoid", "ot[j] * r * sigmoid"),
+    "ogate_not_sigmoid": ("* sigmoid(J->ogate[(row * H + h) * D + j])", "* exp(J->ogate[(row * H + h) * D + j])"),
+    "ogate_channel_shift": ("J->ogate[(row * H + h) * D + j]", "J->ogate[(row * H + h) * D + (j + 1) % D]"),
 }
 
 PIN_TESTS = [
@@ -50,6 +55,11 @@ PIN_TESTS = [
     pins.test_negative_eigenvalues_beta_is_twice_sigmoid,
     pins.test_negative_eigenvalues_write_is_a_householder_reflection,
     pins.test_negative_eigenvalues_equal_plain_run_with_rescaled_b,
+    pins.test_output_gate_unit_rms_and_direction,
+    pins.test_output_gate_is_a_sigmoid,
+    pins.test_output_gate_acts_channel_by_channel,
+    pins.test_output_gate_weight_is_per_channel,
+    pins.test_output_gate_eps_inside_the_mean_square,
 ]
 
 

@@ -265,6 +265,93 @@ def test_recurrence_with_beta_above_one_matches_unrolled_product():
     np.testing.assert_allclose(S[0, 0], S_ref, rtol=1e-12, atol=1e-12)
 
 
+# ---------------------------------------------------------------- output epilogue
+# o_norm then sigmoid output gating (write-up sections "二" and "三"):
+# properties that hold for an RMS norm with a per-channel weight followed by a sigmoid gate.
+
+def _gated(I, H, D, S0, gate, w, eps=0.0, scale=1.0):
+    return oracle.forward(I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"], I["alpha"], I["b"],
+                          I["A_log"], I["dt_bias"], state0=S0, scale=scale, out_gate=gate,
+                          o_norm_weight=w, o_norm_eps=eps)
+
+
+def test_output_gate_unit_rms_and_direction():
+    """w = 1, gate -> +inf, eps = 0: each head's output has RMS exactly 1 over its D
+    channels and points the way the plain output does; the state is untouched."""
+    H, D, lens = 2, 8, [6, 3]
+    I = _prologue_inputs(51, lens, H, D)
+    S0 = _rng(52).standard_normal((2, H, D, D))
+    T = sum(lens)
+    og, S1g, _, _ = _gated(I, H, D, S0, np.full((T, H, D), 60.0), np.ones(D))
+    op, S1p, _, _ = oracle.forward(I["cu"], H, D, I["q"], I["k"], I["v"], I["conv_w"], I["alpha"],
+                                   I["b"], I["A_log"], I["dt_bias"], state0=S0)
+    np.testing.assert_allclose(np.sqrt((og * og).mean(-1)), 1.0, rtol=1e-12)
+    cos = (og * op).sum(-1) / np.linalg.norm(og, axis=-1) / np.linalg.norm(op, axis=-1)
+    np.testing.assert_allclose(cos, 1.0, rtol=1e-12)
+    np.testing.assert_array_equal(S1g, S1p)
+
+
+def test_output_gate_is_a_sigmoid():
+    """sigmoid(x) + sigmoid(-x) = 1 and sigmoid(0) = 1/2, elementwise in the gate."""
+    H, D, lens = 2, 8, [7]
+    I = _prologue_inputs(53, lens, H, D)
+    S0 = _rng(54).standard_normal((1, H, D, D))
+    w = _rng(55).uniform(0.5, 1.5, D)
+    g = _rng(56).standard_normal((7, H, D)) * 2.0
+    o_pos, _, _, _ = _gated(I, H, D, S0, g, w, eps=1e-5)
+    o_neg, _, _, _ = _gated(I, H, D, S0, -g, w, eps=1e-5)
+    o_inf, _, _, _ = _gated(I, H, D, S0, np.full_like(g, 60.0), w, eps=1e-5)
+    o_zero, _, _, _ = _gated(I, H, D, S0, np.zeros_like(g), w, eps=1e-5)
+    np.testing.assert_allclose(o_pos + o_neg, o_inf, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(o_zero, 0.5 * o_inf, rtol=1e-13, atol=1e-15)
+
+
+def test_output_gate_acts_channel_by_channel():
+    """A one-hot gate (+60 on channel m, -60 elsewhere) keeps channel m of the fully open
+    output and closes the rest (sigmoid(-60) ~ 1e-26)."""
+    H, D, lens = 2, 8, [4]
+    I = _prologue_inputs(65, lens, H, D)
+    S0 = _rng(66).standard_normal((1, H, D, D))
+    w = _rng(67).uniform(0.5, 1.5, D)
+    o_inf, _, _, _ = _gated(I, H, D, S0, np.full((4, H, D), 60.0), w, eps=1e-5)
+    for m in (0, 3, D - 1):
+        g = np.full((4, H, D), -60.0)
+        g[..., m] = 60.0
+        o_m, _, _, _ = _gated(I, H, D, S0, g, w, eps=1e-5)
+        np.testing.assert_allclose(o_m[..., m], o_inf[..., m], rtol=1e-14)
+        others = np.delete(o_m, m, axis=-1)
+        assert np.abs(others).max() <= 1e-20 * np.abs(o_inf).max()
+
+
+def test_output_gate_weight_is_per_channel():
+    H, D, lens = 1, 8, [5]
+    I = _prologue_inputs(57, lens, H, D)
+    S0 = _rng(58).standard_normal((1, H, D, D))
+    g = _rng(59).standard_normal((5, H, D))
+    w = _rng(60).uniform(-2, 2, D)
+    o_w, _, _, _ = _gated(I, H, D, S0, g, w, eps=1e-5)
+    o_1, _, _, _ = _gated(I, H, D, S0, g, np.ones(D), eps=1e-5)
+    np.testing.assert_allclose(o_w, o_1 * w, rtol=1e-13, atol=1e-15)
+
+
+def test_output_gate_eps_inside_the_mean_square():
+    """o scales with `scale`; the norm is homogeneous when eps scales with the mean
+    square: out(scale c, eps c^2) == out(scale 1, eps), and eps = 0 makes it scale-free."""
+    H, D, lens = 2, 8, [6]
+    I = _prologue_inputs(61, lens, H, D)
+    S0 = _rng(62).standard_normal((1, H, D, D)) * 0.1
+    g = _rng(63).standard_normal((6, H, D))
+    w = _rng(64).uniform(0.5, 1.5, D)
+    c = 7.0
+    a, _, _, _ = _gated(I, H, D, S0, g, w, eps=0.3, scale=1.0)
+    b_, _, _, _ = _gated(I, H, D, S0, g, w, eps=0.3 * c * c, scale=c)
+    np.testing.assert_allclose(a, b_, rtol=1e-12, atol=1e-14)
+    z1, _, _, _ = _gated(I, H, D, S0, g, w, eps=0.0, scale=1.0)
+    zc, _, _, _ = _gated(I, H, D, S0, g, w, eps=0.0, scale=c)
+    np.testing.assert_allclose(z1, zc, rtol=1e-12, atol=1e-14)
+    assert not np.allclose(a, z1, rtol=1e-3)   # the eps in use does matter at this size
+
+
 def test_forward_equals_prologue_then_recurrence():
     H, D, lens = 2, 8, [9, 4]
     I = _prologue_inputs(16, lens, H, D)
