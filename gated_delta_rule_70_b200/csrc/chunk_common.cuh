@@ -89,6 +89,17 @@ __device__ __forceinline__ float2 silu2(float2 x) {
   return mul2(x, fma2(th, f2(0.5f), f2(0.5f)));
 }
 
+// sigmoid(x) = 1/2 + tanh(x/2)/2 two lanes at a time, the tanh in half precision
+// on the special-function unit (absolute error about 2^-12).
+__device__ __forceinline__ float2 sigmoid2(float2 x) {
+  const float2 hx = mul2(x, f2(0.5f));
+  uint32_t h, t;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(hx.y), "f"(hx.x));
+  asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(h));
+  const float2 th = __half22float2(*reinterpret_cast<const __half2 *>(&t));
+  return fma2(th, f2(0.5f), f2(0.5f));
+}
+
 // K-major descriptor over a token-rows operand with `rows` rows, K = 128 channels, k-step s.
 __device__ __forceinline__ uint64_t desc_k128(uint32_t base, int rows, int s) {
   return umma::make_desc(base + (uint32_t)((s >> 2) * rows * 128 + (s & 3) * 32), 16, 1024,

@@ -41,6 +41,15 @@ int64_t total_tokens(const kda_shape *s, const int32_t *cu) {
 
 kda_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
 
+// The output epilogue's arguments (nullptr: no epilogue).
+kda_status check_out_gate(const kda_output_gate *og, int64_t rows) {
+  if (og == nullptr) return KDA_OK;
+  if (rows > 0 && (og->gate == nullptr || !aligned16(og->gate))) return KDA_ERR_INVALID_ARGUMENT;
+  if (og->weight == nullptr || !aligned16(og->weight)) return KDA_ERR_INVALID_ARGUMENT;
+  if (!std::isfinite(og->eps) || og->eps < 0.f) return KDA_ERR_INVALID_ARGUMENT;
+  return KDA_OK;
+}
+
 PrologueArgs make_prologue_args(const kda_shape *s, int64_t T, const void *q, const void *k,
                                 const void *v, const void *conv_w, const void *alpha, const void *b,
                                 const float *A_log, const float *dt_bias, const void *conv0,
@@ -93,10 +102,24 @@ kda_status kda_prefill(const kda_shape *shape, const void *q, const void *k, con
                        const void *initial_conv_state, const int32_t *cu_seqlens, void *o,
                        float *final_state, void *final_conv_state, void *workspace,
                        size_t workspace_bytes, void *stream_) {
+  return kda_prefill_gated(shape, q, k, v, conv_w, alpha, b, A_log, dt_bias, initial_state,
+                           initial_conv_state, cu_seqlens, nullptr, o, final_state,
+                           final_conv_state, workspace, workspace_bytes, stream_);
+}
+
+kda_status kda_prefill_gated(const kda_shape *shape, const void *q, const void *k, const void *v,
+                             const void *conv_w, const void *alpha, const void *b,
+                             const float *A_log, const float *dt_bias, const float *initial_state,
+                             const void *initial_conv_state, const int32_t *cu_seqlens,
+                             const kda_output_gate *out_gate, void *o, float *final_state,
+                             void *final_conv_state, void *workspace, size_t workspace_bytes,
+                             void *stream_) {
   kda_status st = check_shape(shape);
   if (st != KDA_OK) return st;
   if (shape->num_seqs == 0) return KDA_OK;
   const int64_t T = total_tokens(shape, cu_seqlens);
+  st = check_out_gate(out_gate, T);
+  if (st != KDA_OK) return st;
   if (T > 0) {
     KDA_REQUIRE(q); KDA_REQUIRE(k); KDA_REQUIRE(v); KDA_REQUIRE(alpha); KDA_REQUIRE(b);
     KDA_REQUIRE(o);
@@ -124,6 +147,9 @@ kda_status kda_prefill(const kda_shape *shape, const void *q, const void *k, con
   RecurrenceArgs ra = make_recurrence_args(shape, T, nullptr, nullptr, nullptr, nullptr, nullptr,
                                            initial_state, cu_seqlens, o, final_state);
   ra.err = err;
+  if (out_gate != nullptr) {
+    ra.ogate = out_gate->gate; ra.onw = out_gate->weight; ra.oeps = out_gate->eps;
+  }
   return cuda_status(run_prefill(pa, ra, final_conv_state, varlen, ws, L, stream));
 }
 
@@ -199,9 +225,20 @@ kda_status kda_decode_step(const kda_shape *shape, const void *q, const void *k,
                            const void *alpha, const void *b, const void *conv_w,
                            const float *A_log, const float *dt_bias, float *state,
                            void *conv_state, void *o, void *stream_) {
+  return kda_decode_step_gated(shape, q, k, v, alpha, b, conv_w, A_log, dt_bias, nullptr, state,
+                               conv_state, o, stream_);
+}
+
+kda_status kda_decode_step_gated(const kda_shape *shape, const void *q, const void *k,
+                                 const void *v, const void *alpha, const void *b,
+                                 const void *conv_w, const float *A_log, const float *dt_bias,
+                                 const kda_output_gate *out_gate, float *state, void *conv_state,
+                                 void *o, void *stream_) {
   kda_status st = check_shape(shape);
   if (st != KDA_OK) return st;
   if (shape->num_seqs == 0) return KDA_OK;
+  st = check_out_gate(out_gate, shape->num_seqs);
+  if (st != KDA_OK) return st;
   KDA_REQUIRE(q); KDA_REQUIRE(k); KDA_REQUIRE(v); KDA_REQUIRE(alpha); KDA_REQUIRE(b);
   KDA_REQUIRE(conv_w); KDA_REQUIRE(A_log); KDA_REQUIRE(dt_bias); KDA_REQUIRE(state);
   KDA_REQUIRE(conv_state); KDA_REQUIRE(o);
@@ -212,6 +249,9 @@ kda_status kda_decode_step(const kda_shape *shape, const void *q, const void *k,
   a.A_log = A_log; a.dt_bias = dt_bias;
   a.lower_bound = shape->lower_bound; a.eps = shape->l2norm_eps; a.scale = shape->scale;
   a.beta2 = (shape->flags & KDA_FLAG_NEGATIVE_EIGENVALUES) != 0;
+  if (out_gate != nullptr) {
+    a.ogate = out_gate->gate; a.onw = out_gate->weight; a.oeps = out_gate->eps;
+  }
   a.state = state; a.conv_state = conv_state; a.o = o;
   return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream_)));
 }

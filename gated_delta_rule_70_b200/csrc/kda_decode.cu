@@ -24,6 +24,7 @@ namespace kda {
 template <int D>
 struct DecSmem {
   float q[D], k[D], eg[D], v[D];
+  float gate[D];   // output gate (epilogue only)
   float red_p[D / 16][D], red_r[D / 16][D], red_qk[D / 16];
   float norm_part[2][D / 32];
   float beta;
@@ -92,6 +93,7 @@ decode_kernel(DecodeArgs a) {
     const float g = gate_f(al + a.dt_bias[h * D + i], -expf(a.A_log[h]), a.lower_bound);
     sm.eg[i] = expf(g);
     if (i == 0) sm.beta = (a.beta2 ? 2.f : 1.f) * sigmoid_f(to_f32(reinterpret_cast<const T *>(a.b)[(int64_t)n * H + h]));
+    if (a.ogate) sm.gate[i] = to_f32(reinterpret_cast<const T *>(a.ogate)[((int64_t)n * H + h) * D + i]);
   }
   __syncthreads();
   if (first) {
@@ -138,8 +140,21 @@ decode_kernel(DecodeArgs a) {
   for (int c = 0; c < CPL; ++c) dl[c] = bt * (sm.v[CPL * l + c] - P[c]);
   if (w == 0) {
     T *o = reinterpret_cast<T *>(a.o) + ((int64_t)n * H + h) * D + CPL * l;
+    float ov[CPL];
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) o[c] = from_f32<T>(a.scale * fmaf(QK, dl[c], R[c]));
+    for (int c = 0; c < CPL; ++c) ov[c] = a.scale * fmaf(QK, dl[c], R[c]);
+    if (a.ogate) {   // output epilogue: o_norm over the row, then the sigmoid gate
+      float ss = 0.f;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) ss = fmaf(ov[c], ov[c], ss);
+#pragma unroll
+      for (int sh = 16; sh >= 1; sh >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, sh);
+      const float rn = rsqrtf(ss * (1.f / D) + a.oeps);
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) ov[c] = ov[c] * rn * a.onw[CPL * l + c] * sigmoid_f(sm.gate[CPL * l + c]);
+    }
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) o[c] = from_f32<T>(ov[c]);
   }
 
   // 4. write S = S' + k d^T back in place
@@ -181,7 +196,8 @@ constexpr uint32_t S_ALPHA = S_HIST + 2304;         // bf16 [128]
 constexpr uint32_t S_W = S_ALPHA + 256;             // bf16 conv weights [tensor][128][4]: 3 x 1 KB
 constexpr uint32_t S_DTB = S_W + 3072;              // fp32 dt_bias [128]
 constexpr uint32_t S_B = S_DTB + 512;               // bf16 b of the token's sequence row [H <= 64]
-constexpr uint32_t SLOT = S_B + 128;                // 72,576 B per item
+constexpr uint32_t S_GATE = S_B + 128;              // bf16 output gate [128] (epilogue only)
+constexpr uint32_t SLOT = S_GATE + 256;             // 72,832 B per item
 constexpr int NSLOT = 3;
 constexpr uint32_t OFF_SCR = NSLOT * SLOT;
 struct Scratch {
@@ -189,6 +205,7 @@ struct Scratch {
   float red_p[NC / 32][D], red_r[NC / 32][D], red_qk[NC / 32];
   float norm_part[2][4];
   float alog[64];
+  float onw[D];     // output epilogue weight
   float beta;
   int fail;
   int req[NSLOT];   // requests issued per slot (for the error path)
@@ -197,7 +214,7 @@ struct Scratch {
 constexpr uint32_t SMEM_BYTES = OFF_SCR + sizeof(Scratch);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(SLOT % 16 == 0 && S_QKV % 16 == 0 && S_HIST % 16 == 0 && S_W % 16 == 0 && S_DTB % 16 == 0 &&
-              S_B % 16 == 0, "bulk copy alignment");
+              S_B % 16 == 0 && S_GATE % 16 == 0, "bulk copy alignment");
 constexpr uint32_t WAIT_POLLS = 1u << 22;
 constexpr uint32_t BAR_COMPUTE = 1;                 // named barrier of the compute warps
 
@@ -224,6 +241,8 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_kernel(DecodeArgs a) {
   // A_log of every head, once: a plain load inside the loop would queue behind
   // the bulk traffic for about one item's time
   if (tid < H) sc.alog[tid] = a.A_log[tid];
+  const bool gated = a.ogate != nullptr;
+  if (gated && tid < D) sc.onw[tid] = a.onw[tid];
   __syncthreads();
 
   if (w == NC / 32) {
@@ -234,7 +253,7 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_kernel(DecodeArgs a) {
       uint8_t *base = smem + slot * SLOT;
       uint64_t *bar = &sc.full[slot];
       if (l == 0) {
-        umma::mbar_arrive_expect_tx(bar, S_B + 2 * H);
+        umma::mbar_arrive_expect_tx(bar, S_B + 2 * H + (gated ? 2 * D : 0));
         ++sc.req[slot];
       }
       __syncwarp();
@@ -257,6 +276,9 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_kernel(DecodeArgs a) {
         umma::bulk_g2s(base + S_DTB, a.dt_bias + h * D, 512, bar);
       } else if (l == 18) {   // the row of b for sequence n (2H bytes, 16-byte aligned for H % 8 == 0)
         umma::bulk_g2s(base + S_B, reinterpret_cast<const __nv_bfloat16 *>(a.b) + (int64_t)n * H, 2 * H, bar);
+      } else if (l == 19 && gated) {
+        umma::bulk_g2s(base + S_GATE, reinterpret_cast<const __nv_bfloat16 *>(a.ogate) + (int64_t)it * D,
+                       2 * D, bar);
       }
       __syncwarp();
     };
@@ -393,8 +415,23 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_kernel(DecodeArgs a) {
       for (int c = 0; c < 4; ++c) dl[c] = bt * (sc.v[4 * l + c] - P[c]);
       if (w == 0) {
         __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o) + (int64_t)it * D + 4 * l;
+        float ov[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) o[c] = __float2bfloat16_rn(a.scale * fmaf(QK, dl[c], R[c]));
+        for (int c = 0; c < 4; ++c) ov[c] = a.scale * fmaf(QK, dl[c], R[c]);
+        if (gated) {   // output epilogue: o_norm over the row, then the sigmoid gate
+          float ss = 0.f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) ss = fmaf(ov[c], ov[c], ss);
+#pragma unroll
+          for (int sh = 16; sh >= 1; sh >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, sh);
+          const float rn = rsqrtf(ss * (1.f / D) + a.oeps);
+          const __nv_bfloat16 *gr = reinterpret_cast<const __nv_bfloat16 *>(base + S_GATE) + 4 * l;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            ov[c] = ov[c] * rn * sc.onw[4 * l + c] * sigmoid_f(__bfloat162float(gr[c]));
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) o[c] = __float2bfloat16_rn(ov[c]);
       }
       // 3. S = S' + k d^T, back into the slot; the producer stores it
 #pragma unroll

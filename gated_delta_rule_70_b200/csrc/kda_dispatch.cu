@@ -71,7 +71,8 @@ cudaError_t run_chunk_path(PrepArgs pa, const RecurrenceArgs &ra, bool varlen, b
   sa.N = ra.N; sa.H = ra.H; sa.seq_len = ra.seq_len; sa.total_tokens = ra.total_tokens;
   sa.cu = ra.cu; sa.chunk_cu = chunk_cu; sa.records = ws + L.records; sa.max_slots = slots;
   sa.state0 = ra.state0; sa.scale = ra.scale; sa.o = ra.o; sa.state1 = ra.state1; sa.err = ra.err;
-  e = launch_state_pass(sa, stream);
+  if (ra.ogate != nullptr) { sa.onw = ra.onw; sa.oeps = ra.oeps; }
+  e = launch_state_pass(sa, ra.ogate, stream);
   clock_mark(timed, stream);
   return e;
 }

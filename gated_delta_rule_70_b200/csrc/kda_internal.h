@@ -43,6 +43,10 @@ struct RecurrenceArgs {
   void *o;                   // [T, H, D] io dtype
   float *state1;             // [N, H, D, D]
   int *err;
+  // output epilogue: o <- o / sqrt(mean o^2 + oeps) * onw * sigmoid(ogate), or ogate == nullptr
+  const void *ogate;         // [T, H, D] io dtype
+  const float *onw;          // [D]
+  float oeps;
 };
 
 struct DecodeArgs {
@@ -55,6 +59,9 @@ struct DecodeArgs {
   const float *A_log, *dt_bias;
   float lower_bound, eps, scale;
   int beta2;                 // beta = 2 sigmoid(b); 0: sigmoid(b)
+  const void *ogate;         // output epilogue [N, H, D] io dtype, or nullptr
+  const float *onw;          // [D]
+  float oeps;
   float *state;              // [N, H, D, D] in place
   void *conv_state;          // [N, 3, 3*H*D] in place
   void *o;                   // [N, H, D]
@@ -98,6 +105,9 @@ struct StateArgs {
   void *o;                   // [T, H, 128] bf16
   float *state1;
   int *err;
+  const float *onw;          // output epilogue weight [128], with map_gate; nullptr: off
+  float oeps;
+  CUtensorMap map_gate;      // gate [T rows][H*128] bf16, 64-row boxes
 };
 
 // Bytes of one chunk record and the number of record slots a shape needs.
@@ -156,7 +166,7 @@ cudaError_t launch_chunk_table(const int32_t *cu, int N, int64_t total, int32_t 
 // and q, k, v, alpha (tensor maps built here); else read a.{qn, kn, vc, g, beta}.
 cudaError_t launch_chunk_prep(PrepArgs a, int64_t max_chunks, bool fused, const void *q,
                               const void *k, const void *v, const void *alpha, cudaStream_t stream);
-cudaError_t launch_state_pass(const StateArgs &a, cudaStream_t stream);
+cudaError_t launch_state_pass(StateArgs a, const void *gate, cudaStream_t stream);
 cudaError_t launch_conv_state_out(const PrologueArgs &a, void *out, cudaStream_t stream);
 cudaError_t launch_recurrence(const RecurrenceArgs &a, cudaStream_t stream);
 // The recurrence (a4-a8) for RecurrenceArgs `ra` with workspace `ws` laid out by

@@ -11,6 +11,11 @@
 // Thread layout (D = 128: 8 warps): warp w owns key rows [16w, 16w + 16),
 // lane l owns value columns [CPL*l, CPL*l + CPL) with CPL = D/32; the state
 // slice lives in registers for the whole sequence.
+//
+// Optional output epilogue (the layer's o_norm and sigmoid output gate, same
+// write-up sections "二" and "三"): warp 0 holds a token's whole o row, so
+// o <- o / sqrt(mean o^2 + eps) * w * sigmoid(gate) takes one warp reduction;
+// the gate rows are staged with the token tile.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -23,6 +28,7 @@ struct RecSmem {
   float k[REC_TT][D], q[REC_TT][D], eg[REC_TT][D], v[REC_TT][D];
   float beta[REC_TT];
   float red_p[2][D / 16][D], red_r[2][D / 16][D], red_qk[2][D / 16];
+  float gate[REC_TT][D];     // output gate of the tile (epilogue only)
 };
 
 template <typename T, int D>
@@ -51,6 +57,10 @@ recurrence_kernel(RecurrenceArgs a) {
   const T *__restrict__ kn = reinterpret_cast<const T *>(a.kn);
   const T *__restrict__ vc = reinterpret_cast<const T *>(a.vc);
   T *__restrict__ o = reinterpret_cast<T *>(a.o);
+  const T *__restrict__ og = reinterpret_cast<const T *>(a.ogate);
+  float onw[CPL];   // epilogue weight of this lane's channels
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) onw[c] = og ? a.onw[CPL * l + c] : 0.f;
   int buf = 0;
 
   for (int64_t tile0 = s0; tile0 < s1; tile0 += REC_TT) {
@@ -63,6 +73,7 @@ recurrence_kernel(RecurrenceArgs a) {
       sm.q[tt][i] = to_f32(qn[off]);
       sm.v[tt][i] = to_f32(vc[off]);
       sm.eg[tt][i] = expf(a.g[off]);
+      if (og) sm.gate[tt][i] = to_f32(og[off]);
     }
     for (int tt = threadIdx.x; tt < nt; tt += NT) sm.beta[tt] = a.beta[(tile0 + tt) * H + h];
     __syncthreads();
@@ -108,8 +119,21 @@ recurrence_kernel(RecurrenceArgs a) {
       for (int c = 0; c < CPL; ++c) dl[c] = bt * (sm.v[tt][CPL * l + c] - P[c]);
       if (w == 0) {
         const int64_t off = ((tile0 + tt) * H + h) * D + CPL * l;
+        float ov[CPL];
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) o[off + c] = from_f32<T>(a.scale * fmaf(QK, dl[c], R[c]));
+        for (int c = 0; c < CPL; ++c) ov[c] = a.scale * fmaf(QK, dl[c], R[c]);
+        if (og) {   // o_norm over the row (RMS with the weight), then the sigmoid gate
+          float ss = 0.f;
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) ss = fmaf(ov[c], ov[c], ss);
+#pragma unroll
+          for (int sh = 16; sh >= 1; sh >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, sh);
+          const float rn = rsqrtf(ss * (1.f / D) + a.oeps);
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) ov[c] = ov[c] * rn * onw[c] * sigmoid_f(sm.gate[tt][CPL * l + c]);
+        }
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) o[off + c] = from_f32<T>(ov[c]);
       }
 #pragma unroll
       for (int r = 0; r < 16; ++r) {

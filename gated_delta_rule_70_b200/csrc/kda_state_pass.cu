@@ -26,22 +26,32 @@
 // writes it also applies the next chunk's decay to the fp32 state.  O is
 // triple-buffered: chunk c-1's output leaves, transposed through shared memory
 // into 16-byte row stores, while chunk c+1's first MMAs run.
+//
+// Optional output epilogue (the layer's o_norm and sigmoid output gate, same
+// write-up sections "二" and "三"): o <- o / sqrt(mean o^2 + eps) * w * sigmoid(gate)
+// per (token, head).  Warp 6 streams the chunk's gate tile by TMA into one of two
+// slots; the transpose then stages o in fp32 so that the norm sees it unrounded.
 #include "chunk_common.cuh"
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "tma_host.h"
+#include "umma.cuh"
 
 namespace kda {
 namespace spass {
 
 using namespace chunkfmt;
 
-constexpr int NT = 192;          // warps 0-3: epilogues (TMEM lanes); warp 4: MMA issue; warp 5: record copies
+constexpr int NT = 224;          // warps 0-3: epilogues (TMEM lanes); warp 4: MMA issue; warp 5: record
+                                 // copies; warp 6: output-gate copies
 constexpr int NE = 128;          // epilogue threads
 constexpr uint32_t BAR_EPI = 1;  // named barrier of the epilogue warps
 constexpr uint32_t OFF_REC0 = 0;
 constexpr uint32_t OFF_REC1 = REC_STRIDE;
-constexpr uint32_t OFF_OST = 2 * REC_STRIDE;   // o of one chunk, bf16 [64 t][128 j]: 16 KB
-constexpr uint32_t OFF_BAR = OFF_OST + CH * DK * 2;
+constexpr uint32_t OFF_OST = 2 * REC_STRIDE;   // o of one chunk, [64 t][128 j]: bf16, or fp32 when gated
+constexpr uint32_t OFF_GATE = OFF_OST + CH * DK * 4;   // output gate tiles, 2 x bf16 [64 t][128 j]
+constexpr uint32_t GATE_BYTES = CH * DK * 2;
+constexpr uint32_t OFF_BAR = OFF_GATE + 2 * GATE_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 128;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
@@ -54,10 +64,11 @@ constexpr uint32_t TM_D = 256;     // D^T fp32, 64 cols; its bf16 copy (32 cols)
 constexpr uint32_t TM_O = 320;     // O^T fp32, 3 x 64 cols (chunk index mod 3)
 
 constexpr uint32_t WAIT_POLLS = 1u << 22;
-enum { B_FULL0 = 0, B_FULL1, B_D, B_S, B_O, B_D16, B_S16, B_COUNT };
+enum { B_FULL0 = 0, B_FULL1, B_D, B_S, B_O, B_D16, B_S16, B_G0, B_G1, B_EMIT, B_COUNT };
+static_assert(8 * B_COUNT + 16 <= 128, "barrier area");
 __device__ __forceinline__ uint32_t o_cols(int c) { return TM_O + (uint32_t)(c % 3) * 64; }
 
-__global__ void __launch_bounds__(NT, 1) state_pass_kernel(StateArgs a) {
+__global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant__ StateArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -85,7 +96,8 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(StateArgs a) {
     umma::tmem_relinquish();
   }
   if (tid == 32) {
-    for (int i = 0; i < B_COUNT; ++i) umma::mbar_init(&bar[i], (i == B_D16 || i == B_S16) ? 4 : 1);
+    for (int i = 0; i < B_COUNT; ++i)
+      umma::mbar_init(&bar[i], (i == B_D16 || i == B_S16 || i == B_EMIT) ? 4 : 1);
     umma::mbar_fence_init();
     *fail = 0;
   }
@@ -94,8 +106,29 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(StateArgs a) {
   umma::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
+  const bool gated = a.onw != nullptr;
   if (warp >= 4) {
-    if (warp == 5 && lane == 0) {
+    if (warp == 6 && lane == 0 && gated) {
+      // ---------------------------------------------------------- output-gate copies
+      // chunk c's 64 gate rows into slot c % 2 once chunk c-2's o has left it
+      bool ok = true;
+      int issued = 0;
+      for (int c = 0; c < nchunks; ++c) {
+        if (c >= 2) {
+          ok = umma::mbar_wait_bounded(&bar[B_EMIT], (c - 2) & 1, WAIT_POLLS) && *(volatile int *)fail == 0;
+          if (!ok) break;
+        }
+        umma::mbar_arrive_expect_tx(&bar[B_G0 + (c & 1)], GATE_BYTES);
+        umma::tma_load_2d(smem + OFF_GATE + (c & 1) * GATE_BYTES, &a.map_gate, h * DK,
+                          (int)(s0 + (int64_t)c * CH), &bar[B_G0 + (c & 1)]);
+        issued = c + 1;
+      }
+      if (!ok) {
+        atomicExch(fail, 1);
+        for (int k = issued - 2 < 0 ? 0 : issued - 2; k < issued; ++k)
+          (void)umma::mbar_wait_bounded(&bar[B_G0 + (k & 1)], (k >> 1) & 1, WAIT_POLLS);
+      }
+    } else if (warp == 5 && lane == 0) {
       // ---------------------------------------------------------- record copies
       // chunk c+2 goes into chunk c's buffer once every MMA of chunk c is done (the
       // epilogues read U and e^{Gamma_C} from it before their hand-offs)
@@ -166,6 +199,16 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(StateArgs a) {
     const int64_t sg = ((int64_t)n * H + h) * DK * DK;
     __nv_bfloat16 *__restrict__ o = reinterpret_cast<__nv_bfloat16 *>(a.o);
     __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(smem + OFF_OST);
+    float *ost32 = reinterpret_cast<float *>(smem + OFF_OST);
+    float2 onw[4];   // epilogue weight of this thread's 8 channels (c16 = tid & 15 in every row pass)
+    if (gated) {
+      const float4 w0 = *reinterpret_cast<const float4 *>(a.onw + (tid & 15) * 8);
+      const float4 w1 = *reinterpret_cast<const float4 *>(a.onw + (tid & 15) * 8 + 4);
+      onw[0] = make_float2(w0.x, w0.y); onw[1] = make_float2(w0.z, w0.w);
+      onw[2] = make_float2(w1.x, w1.y); onw[3] = make_float2(w1.z, w1.w);
+    } else {
+      onw[0] = onw[1] = onw[2] = onw[3] = f2(0.f);
+    }
     // Each thread waits on its own (bounded); a wait that gives up sets the shared
     // fail flag and the thread carries on along the same path (its values are
     // garbage, but every address and every barrier stays the same), so the
@@ -188,19 +231,55 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(StateArgs a) {
       umma::tmem_ld32(tmem + lane_base + ocol, r[0]);
       umma::tmem_ld32(tmem + lane_base + ocol + 32, r[1]);
       umma::tmem_wait_ld();
-#pragma unroll
-      for (int t = 0; t < CH; ++t) ost[t * DK + j] = __float2bfloat16_rn(a.scale * __uint_as_float(r[t >> 5][t & 31]));
-      umma::named_sync(BAR_EPI, NE);
       const int64_t c0 = s0 + (int64_t)cc * CH;
       const int nvalid = (int)min((int64_t)CH, s1 - c0);
+      if (!gated) {
 #pragma unroll
-      for (int k = 0; k < CH * DK / 8 / NE; ++k) {
-        const int q = tid + k * NE, t = q >> 4, c16 = q & 15;
-        if (t < nvalid)
-          *reinterpret_cast<uint4 *>(o + ((c0 + t) * H + h) * DK + c16 * 8) =
-              *reinterpret_cast<const uint4 *>(ost + t * DK + c16 * 8);
+        for (int t = 0; t < CH; ++t) ost[t * DK + j] = __float2bfloat16_rn(a.scale * __uint_as_float(r[t >> 5][t & 31]));
+        umma::named_sync(BAR_EPI, NE);
+#pragma unroll
+        for (int k = 0; k < CH * DK / 8 / NE; ++k) {
+          const int q = tid + k * NE, t = q >> 4, c16 = q & 15;
+          if (t < nvalid)
+            *reinterpret_cast<uint4 *>(o + ((c0 + t) * H + h) * DK + c16 * 8) =
+                *reinterpret_cast<const uint4 *>(ost + t * DK + c16 * 8);
+        }
+        umma::named_sync(BAR_EPI, NE);
+      } else {
+        // o in fp32 through shared memory; a token's 128 channels then sit in 16
+        // consecutive lanes (8 each): the mean square by a 16-lane butterfly
+#pragma unroll
+        for (int t = 0; t < CH; ++t) ost32[t * DK + j] = a.scale * __uint_as_float(r[t >> 5][t & 31]);
+        wait_one(&bar[B_G0 + (cc & 1)], (cc >> 1) & 1);
+        umma::named_sync(BAR_EPI, NE);
+        const uint8_t *gt = smem + OFF_GATE + (cc & 1) * GATE_BYTES;
+#pragma unroll 2
+        for (int k = 0; k < CH * DK / 8 / NE; ++k) {
+          const int q = tid + k * NE, t = q >> 4, c16 = q & 15;
+          const float4 x0 = *reinterpret_cast<const float4 *>(ost32 + t * DK + c16 * 8);
+          const float4 x1 = *reinterpret_cast<const float4 *>(ost32 + t * DK + c16 * 8 + 4);
+          const uint4 graw = *reinterpret_cast<const uint4 *>(gt + t * (DK * 2) + c16 * 16);
+          float2 x[4] = {make_float2(x0.x, x0.y), make_float2(x0.z, x0.w), make_float2(x1.x, x1.y),
+                         make_float2(x1.z, x1.w)};
+          float2 ss = mul2(x[0], x[0]);
+#pragma unroll
+          for (int e = 1; e < 4; ++e) ss = fma2(x[e], x[e], ss);
+          float s2 = ss.x + ss.y;
+#pragma unroll
+          for (int off = 8; off >= 1; off >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, off);
+          const float rn = rsqrtf(s2 * (1.f / DK) + a.oeps);
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 sg = sigmoid2(bf2_f2(word(graw, e)));
+            w4[e] = f2_bf2(mul2(mul2(x[e], f2(rn)), mul2(onw[e], sg)));
+          }
+          if (t < nvalid)
+            *reinterpret_cast<uint4 *>(o + ((c0 + t) * H + h) * DK + c16 * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+        umma::named_sync(BAR_EPI, NE);
+        if (lane == 0) umma::mbar_arrive(&bar[B_EMIT]);   // gate slot cc % 2 is free again
       }
-      umma::named_sync(BAR_EPI, NE);
     };
     // S^T columns *= e^{Gamma_C} of the record at rb; with s16: also write the bf16 copy there first
     auto state_pass_over = [&](uint32_t rb, int s16) {
@@ -327,8 +406,18 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(StateArgs a) {
 
 }  // namespace spass
 
-cudaError_t launch_state_pass(const StateArgs &a, cudaStream_t stream) {
+cudaError_t launch_state_pass(StateArgs a, const void *gate, cudaStream_t stream) {
   if ((int64_t)a.N * a.H == 0) return cudaSuccess;
+  if (a.onw != nullptr) {   // output epilogue: the gate [T rows][H * 128] in 64-row tiles
+    if (gate == nullptr || a.total_tokens == 0) {
+      a.onw = nullptr;
+    } else {
+      const uint64_t rows = (uint64_t)a.total_tokens, cols = (uint64_t)a.H * chunkfmt::DK;
+      if (!encode_rows(&a.map_gate, gate, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, cols,
+                       chunkfmt::CH, chunkfmt::DK))
+        return cudaErrorInvalidValue;
+    }
+  }
   cudaError_t e = cudaFuncSetAttribute(spass::state_pass_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)spass::SMEM_ALLOC);

@@ -28,7 +28,7 @@ KDA_BF16, KDA_FP32 = 0, 1
 EXPORTED = ["kda_prefill_workspace_size", "kda_prefill", "kda_prefill_status", "kda_prologue",
             "kda_recurrence", "kda_recurrence_workspace_size", "kda_decode_step",
             "kda_status_string", "kda_version", "kda_prefill_noalloc", "kda_kernel_timing",
-            "kda_kernel_times"]
+            "kda_kernel_times", "kda_prefill_gated", "kda_decode_step_gated"]
 
 
 class KdaLibraryError(RuntimeError):
@@ -49,6 +49,11 @@ class Shape(ctypes.Structure):
 
 
 KDA_FLAG_NEGATIVE_EIGENVALUES = 0x1
+
+
+class OutputGate(ctypes.Structure):
+    """kda_output_gate: o <- o / sqrt(mean o^2 + eps) * weight * sigmoid(gate)."""
+    _fields_ = [("gate", ctypes.c_void_p), ("weight", ctypes.c_void_p), ("eps", ctypes.c_float)]
 
 
 def library_path() -> str:
@@ -83,6 +88,11 @@ def load_library():
     lib.kda_recurrence_workspace_size.restype = sz
     lib.kda_decode_step.argtypes = [SP] + [P] * 11 + [P]
     lib.kda_decode_step.restype = i32
+    OG = ctypes.POINTER(OutputGate)
+    lib.kda_prefill_gated.argtypes = [SP] + [P] * 11 + [OG] + [P] * 3 + [P, sz, P]
+    lib.kda_prefill_gated.restype = i32
+    lib.kda_decode_step_gated.argtypes = [SP] + [P] * 8 + [OG] + [P] * 3 + [P]
+    lib.kda_decode_step_gated.restype = i32
     lib.kda_status_string.argtypes = [i32]
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_version.argtypes = []
@@ -143,14 +153,18 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, conv_w: torch.Ten
             initial_conv_state: Optional[torch.Tensor] = None, *, num_seqs: Optional[int] = None,
             lower_bound: float = -5.0, l2norm_eps: float = 1e-6,
             scale: float = 1.0, negative_eigenvalues: bool = False,
+            out_gate: Optional[torch.Tensor] = None, o_norm_weight: Optional[torch.Tensor] = None,
+            o_norm_eps: float = 1e-5,
             want_conv_state: bool = True, out: Optional[torch.Tensor] = None,
             final_state: Optional[torch.Tensor] = None,
             final_conv_state: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
             check: bool = True) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
     """KDA prefill.  q, k, v: [T_total, H*d] (or [B, T, H*d] dense); alpha: [.., H, d];
     b: [.., H].  Returns (o [T_total, H, d], final_state [N, H, d, d], final_conv_state
-    [N, 3, 3*H*d] or None).  ``negative_eigenvalues``: beta = 2 sigmoid(b).  ``check``
-    synchronises and raises on device-side errors."""
+    [N, 3, 3*H*d] or None).  ``negative_eigenvalues``: beta = 2 sigmoid(b).  ``out_gate``
+    [.., H, d] with ``o_norm_weight`` [d] fp32: the output epilogue o <- o / sqrt(mean o^2 +
+    o_norm_eps) * weight * sigmoid(out_gate).  ``check`` synchronises and raises on
+    device-side errors."""
     lib = load_library()
     H, d = alpha.shape[-2], alpha.shape[-1]
     if cu_seqlens is not None:
@@ -177,14 +191,24 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, conv_w: torch.Ten
     ws = workspace
     if ws is None or ws.numel() < ws_bytes:
         ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
-    st = lib.kda_prefill(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w), _ptr(alpha),
-                         _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(initial_state),
-                         _ptr(initial_conv_state), _ptr(cu_seqlens), _ptr(o), _ptr(fs), _ptr(fc),
-                         _ptr(ws), ctypes.c_size_t(ws.numel()), _stream(dev))
+    og = _output_gate(out_gate, o_norm_weight, o_norm_eps)
+    st = lib.kda_prefill_gated(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
+                               _ptr(alpha), _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(initial_state),
+                               _ptr(initial_conv_state), _ptr(cu_seqlens), og, _ptr(o), _ptr(fs),
+                               _ptr(fc), _ptr(ws), ctypes.c_size_t(ws.numel()), _stream(dev))
     _check(st, "kda_prefill")
     if check:
         _check(lib.kda_prefill_status(_ptr(ws), _stream(dev)), "kda_prefill (device)")
     return o, fs, fc
+
+
+def _output_gate(gate, weight, eps):
+    """A kda_output_gate for the call, or None (no epilogue)."""
+    if gate is None and weight is None:
+        return None
+    if gate is None or weight is None:
+        raise ValueError("out_gate and o_norm_weight go together")
+    return ctypes.byref(OutputGate(_ptr(gate), _ptr(weight), float(eps)))
 
 
 def _prefill_shape(q, alpha, cu_seqlens, num_seqs, lower_bound, l2norm_eps, scale,
@@ -257,16 +281,18 @@ def recurrence(qn, kn, vc, g, beta, initial_state=None, cu_seqlens=None, *,
 def decode_step(q, k, v, alpha, b, conv_w, A_log, dt_bias, state: torch.Tensor,
                 conv_state: torch.Tensor, *, lower_bound: float = -5.0, l2norm_eps: float = 1e-6,
                 scale: float = 1.0, negative_eigenvalues: bool = False,
-                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                out_gate: Optional[torch.Tensor] = None, o_norm_weight: Optional[torch.Tensor] = None,
+                o_norm_eps: float = 1e-5, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """One token per sequence; updates ``state`` [N,H,d,d] and ``conv_state`` [N,3,3*H*d] in
     place and returns o [N, H, d]."""
     lib = load_library()
     N, H, d = state.shape[0], state.shape[1], state.shape[2]
     shape = make_shape(N, 1, H, d, q.dtype, lower_bound, l2norm_eps, scale, negative_eigenvalues)
     o = out if out is not None else torch.empty((N, H, d), dtype=q.dtype, device=q.device)
-    st = lib.kda_decode_step(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b),
-                             _ptr(conv_w), _ptr(A_log), _ptr(dt_bias), _ptr(state),
-                             _ptr(conv_state), _ptr(o), _stream(q.device))
+    og = _output_gate(out_gate, o_norm_weight, o_norm_eps)
+    st = lib.kda_decode_step_gated(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                   _ptr(b), _ptr(conv_w), _ptr(A_log), _ptr(dt_bias), og,
+                                   _ptr(state), _ptr(conv_state), _ptr(o), _stream(q.device))
     _check(st, "kda_decode_step")
     return o
 

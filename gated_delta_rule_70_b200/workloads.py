@@ -40,7 +40,7 @@ import numpy as np
 BLOCK = 4096
 
 _TAGS = {"q": 1, "k": 2, "v": 3, "alpha": 4, "b": 5, "conv_w": 6, "A_log": 7,
-         "dt_bias": 8, "S0": 9, "lens": 10, "step": 11}
+         "dt_bias": 8, "S0": 9, "lens": 10, "step": 11, "gate": 12, "o_norm_w": 13}
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -218,6 +218,16 @@ def make_decode_step(s: Spec, step: int) -> Dict[str, np.ndarray]:
     b = rng.standard_normal((N, s.H), dtype=np.float32)
     return {k_: _store(v_, s.io_dtype) for k_, v_ in
             (("q", q), ("k", k), ("v", v), ("alpha", alpha), ("b", b))}
+
+
+def make_output_gate(s: Spec, rows: int, tag: int = 0) -> Dict[str, np.ndarray]:
+    """Inputs of the output epilogue: gate ~ N(0,1) [rows, H, d] in the io dtype (rows =
+    the workload's tokens, or its sequences for a decode step; ``tag`` tells steps apart)
+    and the o_norm weight ~ U(0.5, 1.5) [d] fp32."""
+    rng = np.random.default_rng([s.seed, _TAGS["gate"], tag])
+    gate = rng.standard_normal((rows, s.H, s.d), dtype=np.float32)
+    w = np.random.default_rng([s.seed, _TAGS["o_norm_w"]]).uniform(0.5, 1.5, s.d).astype(np.float32)
+    return {"gate": _store(gate, s.io_dtype), "o_norm_weight": w}
 
 
 def small(name: str, seq_lens: List[int], H: int, d: int, io_dtype: str = "bf16",

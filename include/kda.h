@@ -128,6 +128,39 @@ kda_status kda_prefill(const kda_shape *shape,
                        void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Output epilogue of the KDA layer, fused into the store of o: the layer's
+ * o_norm followed by its sigmoid output gating (AliceAI-Foundation KDA
+ * write-up: the layer projects an output_gate, section "二", and ends in o_norm
+ * plus sigmoid gating, section "三"; the Ling-3.0-flash-VL weight list names
+ * o_norm and g_proj).  Per (token, head), over the head's d value channels:
+ *
+ *   o[j] <- o[j] / sqrt(mean_j o[j]^2 + eps) * weight[j] * sigmoid(gate[j])
+ *
+ *   gate    [T_total, H, d] io dtype (prefill) or [N, H, d] (decode): the
+ *           output gate before the sigmoid; 16-byte aligned
+ *   weight  [d] fp32, shared by the heads; 16-byte aligned
+ *   eps     inside the root, added to the mean square (1e-5f); finite, >= 0
+ */
+typedef struct {
+    const void *gate;
+    const float *weight;
+    float eps;
+} kda_output_gate;
+
+/*
+ * kda_prefill_gated -- kda_prefill with the output epilogue applied to o
+ * (out_gate NULL: exactly kda_prefill).  Same workspace size.
+ */
+kda_status kda_prefill_gated(const kda_shape *shape,
+                             const void *q, const void *k, const void *v,
+                             const void *conv_w, const void *alpha, const void *b,
+                             const float *A_log, const float *dt_bias,
+                             const float *initial_state, const void *initial_conv_state,
+                             const int32_t *cu_seqlens, const kda_output_gate *out_gate,
+                             void *o, float *final_state, void *final_conv_state,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * kda_prefill_status -- synchronises `stream` and reads the device error word
  * the last kda_prefill() on this workspace left: KDA_OK, KDA_ERR_INVALID_ARGUMENT
  * (bad cu_seqlens), KDA_ERR_TIMEOUT (a bounded wait gave up) or KDA_ERR_CUDA.
@@ -195,6 +228,15 @@ kda_status kda_decode_step(const kda_shape *shape,
                            const void *alpha, const void *b,
                            const void *conv_w, const float *A_log, const float *dt_bias,
                            float *state, void *conv_state, void *o, void *stream);
+
+/* kda_decode_step with the output epilogue (gate [N, H, d]); out_gate NULL:
+ * exactly kda_decode_step. */
+kda_status kda_decode_step_gated(const kda_shape *shape,
+                                 const void *q, const void *k, const void *v,
+                                 const void *alpha, const void *b,
+                                 const void *conv_w, const float *A_log, const float *dt_bias,
+                                 const kda_output_gate *out_gate,
+                                 float *state, void *conv_state, void *o, void *stream);
 
 /*
  * kda_prefill_noalloc -- kda_prefill for callers that cannot allocate device

@@ -126,3 +126,24 @@ def test_binding_refuses_cpu_tensors(lib):
     t = torch.zeros(16)
     with pytest.raises(ValueError):
         kda._ptr(t)
+
+
+def test_output_gate_validation(lib):
+    """kda_prefill_gated / kda_decode_step_gated reject a missing or misaligned gate or weight
+    and a bad eps before any launch."""
+    import torch
+    P = ctypes.c_void_p
+    x = P(256)
+    sh = kda.make_shape(1, 16, 2, 64, torch.float32)
+    def pre(og):
+        return lib.kda_prefill_gated(ctypes.byref(sh), x, x, x, x, x, x, x, x, None, None, None,
+                                     ctypes.byref(og), x, x, None, x, ctypes.c_size_t(1 << 30), None)
+    assert pre(kda.OutputGate(None, 512, 1e-5)) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert pre(kda.OutputGate(264, 512, 1e-5)) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert pre(kda.OutputGate(512, 520, 1e-5)) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert pre(kda.OutputGate(512, 512, float("nan"))) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert pre(kda.OutputGate(512, 512, -1.0)) == kda.KDA_ERR_INVALID_ARGUMENT
+    dsh = kda.make_shape(2, 1, 2, 128, torch.bfloat16)
+    assert lib.kda_decode_step_gated(ctypes.byref(dsh), x, x, x, x, x, x, x, x,
+                                     ctypes.byref(kda.OutputGate(None, 512, 1e-5)), x, x, x,
+                                     None) == kda.KDA_ERR_INVALID_ARGUMENT

@@ -337,3 +337,60 @@ def test_prologue_negative_eigenvalues_beta():
                           f["alpha"], f["b"], f["A_log"], f["dt_bias"], negative_eigenvalues=True)
     np.testing.assert_allclose(W.from_device(out[4]), ref[4], rtol=1e-5, atol=1e-6)
     assert float(W.from_device(out[4]).max()) > 1.0   # the doubled range is in use
+
+
+# ------------------------------------------------------------------ output epilogue
+
+@pytest.mark.parametrize("io,d,lens", [("bf16", 128, [1, 70, 200]), ("bf16", 128, [64, 64]),
+                                       ("fp32", 64, [33, 90]), ("fp32", 128, [65])])
+def test_prefill_output_gate(io, d, lens):
+    """o <- rmsnorm(o) * w * sigmoid(gate) fused into the store: the bf16 state pass (its
+    gate-tile warp, fp32 staging) and the token kernel, against the oracle's epilogue."""
+    s = W.small("og", lens, H=3, d=d, io_dtype=io, seed=43, s0_std=0.02, varlen=len(set(lens)) > 1)
+    inp = W.make_inputs(s)
+    G = W.make_output_gate(s, s.total_tokens)
+    cu = _dev(inp["cu_seqlens"]) if s.varlen else None
+    o, fs, _ = kda.prefill(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["conv_w"]),
+                           _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]), _dev(inp["dt_bias"]),
+                           initial_state=_dev(inp["S0"]), cu_seqlens=cu, num_seqs=s.num_seqs,
+                           out_gate=_dev(G["gate"]), o_norm_weight=_dev(G["o_norm_weight"]),
+                           o_norm_eps=1e-5)
+    torch.cuda.synchronize()
+    f = f64_inputs(inp)
+    o_ref, s_ref, _, _ = oracle.forward(inp["cu_seqlens"], s.H, s.d, f["q"], f["k"], f["v"],
+                                        f["conv_w"], f["alpha"], f["b"], f["A_log"], f["dt_bias"],
+                                        state0=f["S0"], out_gate=W.as_f64(G["gate"]),
+                                        o_norm_weight=W.as_f64(G["o_norm_weight"]), o_norm_eps=1e-5)
+    tol = TOL[io]
+    eo = max_pair_err(W.from_device(o), o_ref, inp["cu_seqlens"], s.H)
+    assert eo <= tol, "gated o rel-L2 %.3g > %.0e" % (eo, tol)
+    assert max_state_err(W.from_device(fs), s_ref) <= tol
+
+
+@pytest.mark.parametrize("H,N", [(3, 5), (16, 40)])
+def test_decode_output_gate(H, N):
+    """The epilogue in both decode kernels (H=3: per item; H=16 x 40: the persistent ring)."""
+    d, T1, steps = 128, 20, 3
+    s = W.small("ogdec", [T1] * N, H=H, d=d, seed=44, s0_std=0.02)
+    inp = W.make_inputs(s)
+    o, st, cs = gpu_prefill(s, inp)
+    f = f64_inputs(inp)
+    _, s_ref, c_ref, _ = oracle_prefill(s, inp)
+    wgt = W.make_output_gate(s, N)["o_norm_weight"]
+    for step in range(steps):
+        x = _decode_inputs(s, step)
+        gate = W.make_output_gate(s, N, tag=step + 1)["gate"]
+        o_t = kda.decode_step(_dev(x["q"]), _dev(x["k"]), _dev(x["v"]), _dev(x["alpha"]),
+                              _dev(x["b"]), _dev(inp["conv_w"]), _dev(inp["A_log"]),
+                              _dev(inp["dt_bias"]), st, cs, out_gate=_dev(gate),
+                              o_norm_weight=_dev(wgt))
+        xf = {k: W.as_f64(v) for k, v in x.items()}
+        o_r, s_ref, c_ref = oracle.decode_step(H, d, s_ref, c_ref, xf["q"], xf["k"], xf["v"],
+                                               xf["alpha"], xf["b"], f["conv_w"], f["A_log"],
+                                               f["dt_bias"], out_gate=W.as_f64(gate),
+                                               o_norm_weight=W.as_f64(wgt))
+        torch.cuda.synchronize()
+        og = W.from_device(o_t)
+        worst = max(rel_l2(og[n, h], o_r[n, h]) for n in range(N) for h in range(H))
+        assert worst <= TOL["bf16"], (step, worst)
+    assert max_state_err(W.from_device(st), s_ref) <= TOL["bf16"]
