@@ -42,7 +42,7 @@ sys.path.insert(0, ROOT)
 # DRAM bytes (read + write) of one chunk_prep launch on 4x8192x32, from the ncu capture in
 # profiles/chunk_prep_prefill_1x8k.md scaled by the chunk-heads (x4); None when the kernel
 # has changed since that capture.
-CHUNK_PREP_TRAFFIC_BYTES = 4 * (269.198848e6 + 253.545728e6)
+CHUNK_PREP_TRAFFIC_BYTES = 4 * (269.172224e6 + 252.218368e6)
 
 HBM_FALLBACK_GBS = 6650.0
 BF16_FALLBACK_TFLOPS = 1590.0
@@ -220,6 +220,22 @@ def run_ours(args, rank, world, local_rank):
     de[64].record(stream)
     torch.cuda.synchronize(dev)
     dec_ms = [de[i].elapsed_time(de[i + 1]) for i in range(64)]
+    # the same steps with the output epilogue fused in
+    dG = W.make_output_gate(sd, sd.num_seqs)
+    d_gate, d_w = dup(dG["gate"]), dup(dG["o_norm_weight"])
+
+    def dstep_gated(x):
+        kda.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["b"], d_cw, d_A, d_dt, d_state,
+                        d_conv, out_gate=d_gate, o_norm_weight=d_w, out=d_out)
+
+    for i in range(3):
+        dstep_gated(dsteps[i])
+    de[0].record(stream)
+    for i in range(64):
+        dstep_gated(dsteps[i])
+    de[1].record(stream)
+    torch.cuda.synchronize(dev)
+    dec_gated_ms = de[0].elapsed_time(de[1]) / 64
     clock_info = clocks.stop()
 
     # ---- the other prefill workloads (reported beside the headline, not in `value`)
@@ -228,6 +244,10 @@ def run_ours(args, rank, world, local_rank):
         for wname in ("long_256k", "varlen_32"):
             extra[wname] = time_prefill_workload(W.spec(wname), dev, stream, args.warmup,
                                                  max(3, min(args.steps, 5)), peaks)
+        if args.batch == 4:   # the headline prefill with the output epilogue fused in
+            extra["prefill_4x8k_output_gate"] = time_prefill_workload(
+                W.spec("prefill_4x8k"), dev, stream, args.warmup, max(3, min(args.steps, 10)), peaks,
+                gated=True)
 
     # ---- e2e through the C ABI with host buffers
     pin = lambda t: t.detach().cpu().pin_memory()
@@ -319,7 +339,8 @@ def run_ours(args, rank, world, local_rank):
                    "ms_per_step": dec_step_ms, "algorithmic_bytes": dec_bytes, "GB_s": dec_gbs,
                    "frac_of_measured_hbm": dec_gbs / peaks["hbm_gbs"],
                    "frac_of_8000_datasheet": dec_gbs / 8000.0,
-                   "tokens_per_s": sd.num_seqs / (dec_step_ms * 1e-3)},
+                   "tokens_per_s": sd.num_seqs / (dec_step_ms * 1e-3),
+                   "output_gate_ms_per_step": dec_gated_ms},
         "e2e": None if args.no_e2e else {
             "value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -333,10 +354,10 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
-def time_prefill_workload(s, dev, stream, warmup, steps, peaks):
+def time_prefill_workload(s, dev, stream, warmup, steps, peaks, gated=False):
     """One kda_prefill over a whole workload (inputs resident in HBM), timed with CUDA
     events on the launching stream; chunk_prep / state-pass split from the library's
-    kernel timing."""
+    kernel timing.  gated: with the output epilogue (o_norm and sigmoid output gate)."""
     import torch
     from gated_delta_rule_70_b200 import kda
     from gated_delta_rule_70_b200 import workloads as W
@@ -365,11 +386,17 @@ def time_prefill_workload(s, dev, stream, warmup, steps, peaks):
     seq_len = T if s.varlen else s.seq_lens[0]
     ws = torch.empty(kda.prefill_workspace_size(kda.make_shape(N, seq_len, H, d, bf), s.varlen),
                      dtype=torch.uint8, device=dev)
+    gate = wgt = None
+    if gated:
+        G = W.make_output_gate(s, T)
+        gate, wgt = W.to_device(G["gate"], dev), W.to_device(G["o_norm_weight"], dev)
+        del G
 
     def step():
         kda.prefill(q, k, v, params["conv_w"], alpha, b, params["A_log"], params["dt_bias"],
                     initial_state=S0, cu_seqlens=cu, num_seqs=N, out=o, final_state=fs,
-                    final_conv_state=fc, workspace=ws, check=False)
+                    final_conv_state=fc, workspace=ws, out_gate=gate, o_norm_weight=wgt,
+                    check=False)
 
     for _ in range(warmup):
         step()
@@ -390,7 +417,9 @@ def time_prefill_workload(s, dev, stream, warmup, steps, peaks):
            "frac_of_measured_bf16": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
            "kernels_ms": {"chunk_prep": prep_ms, "state_pass": state_ms}, "steps": steps,
            "warmup": warmup}
-    del q, k, v, alpha, b, o, ws
+    if gated:
+        out["output_gate"] = "o <- o / sqrt(mean o^2 + 1e-5) * w * sigmoid(gate), fused into the state pass"
+    del q, k, v, alpha, b, o, ws, gate
     torch.cuda.empty_cache()
     return out
 
