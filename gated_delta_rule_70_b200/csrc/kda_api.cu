@@ -114,18 +114,37 @@ kda_status kda_prefill_gated(const kda_shape *shape, const void *q, const void *
                              const kda_output_gate *out_gate, void *o, float *final_state,
                              void *final_conv_state, void *workspace, size_t workspace_bytes,
                              void *stream_) {
+  kda_prefill_args a;
+  std::memset(&a, 0, sizeof a);
+  a.q = q; a.k = k; a.v = v; a.conv_w = conv_w; a.alpha = alpha; a.b = b;
+  a.A_log = A_log; a.dt_bias = dt_bias; a.initial_state = initial_state;
+  a.initial_conv_state = initial_conv_state; a.cu_seqlens = cu_seqlens;
+  a.o = o; a.final_state = final_state; a.final_conv_state = final_conv_state;
+  a.out_gate = out_gate;
+  a.snapshot_every = 1;
+  return kda_prefill_ex(shape, &a, workspace, workspace_bytes, stream_);
+}
+
+kda_status kda_prefill_ex(const kda_shape *shape, const kda_prefill_args *args, void *workspace,
+                          size_t workspace_bytes, void *stream_) {
   kda_status st = check_shape(shape);
   if (st != KDA_OK) return st;
+  if (args == nullptr) return KDA_ERR_INVALID_ARGUMENT;
   if (shape->num_seqs == 0) return KDA_OK;
+  const int32_t *cu_seqlens = args->cu_seqlens;
   const int64_t T = total_tokens(shape, cu_seqlens);
-  st = check_out_gate(out_gate, T);
+  st = check_out_gate(args->out_gate, T);
   if (st != KDA_OK) return st;
   if (T > 0) {
-    KDA_REQUIRE(q); KDA_REQUIRE(k); KDA_REQUIRE(v); KDA_REQUIRE(alpha); KDA_REQUIRE(b);
-    KDA_REQUIRE(o);
+    KDA_REQUIRE(args->q); KDA_REQUIRE(args->k); KDA_REQUIRE(args->v); KDA_REQUIRE(args->alpha);
+    KDA_REQUIRE(args->b); KDA_REQUIRE(args->o);
   }
-  KDA_REQUIRE(conv_w); KDA_REQUIRE(A_log); KDA_REQUIRE(dt_bias); KDA_REQUIRE(final_state);
-  KDA_OPTIONAL(initial_state); KDA_OPTIONAL(initial_conv_state); KDA_OPTIONAL(final_conv_state);
+  KDA_REQUIRE(args->conv_w); KDA_REQUIRE(args->A_log); KDA_REQUIRE(args->dt_bias);
+  KDA_REQUIRE(args->final_state);
+  KDA_OPTIONAL(args->initial_state); KDA_OPTIONAL(args->initial_conv_state);
+  KDA_OPTIONAL(args->final_conv_state); KDA_OPTIONAL(args->snapshots);
+  if (args->snapshots != nullptr && (args->snapshot_every < 1 || args->snapshot_capacity < 0))
+    return KDA_ERR_INVALID_ARGUMENT;
   if (cu_seqlens != nullptr && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)) return KDA_ERR_INVALID_ARGUMENT;
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)))
     return KDA_ERR_WORKSPACE;
@@ -141,16 +160,22 @@ kda_status kda_prefill_gated(const kda_shape *shape, const void *q, const void *
   cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), stream);
   if (e != cudaSuccess) return KDA_ERR_CUDA;
 
-  PrologueArgs pa = make_prologue_args(shape, T, q, k, v, conv_w, alpha, b, A_log, dt_bias,
-                                       initial_conv_state, cu_seqlens);
+  PrologueArgs pa = make_prologue_args(shape, T, args->q, args->k, args->v, args->conv_w,
+                                       args->alpha, args->b, args->A_log, args->dt_bias,
+                                       args->initial_conv_state, cu_seqlens);
   pa.err = err;
   RecurrenceArgs ra = make_recurrence_args(shape, T, nullptr, nullptr, nullptr, nullptr, nullptr,
-                                           initial_state, cu_seqlens, o, final_state);
+                                           args->initial_state, cu_seqlens, args->o,
+                                           args->final_state);
   ra.err = err;
-  if (out_gate != nullptr) {
-    ra.ogate = out_gate->gate; ra.onw = out_gate->weight; ra.oeps = out_gate->eps;
+  if (args->out_gate != nullptr) {
+    ra.ogate = args->out_gate->gate; ra.onw = args->out_gate->weight; ra.oeps = args->out_gate->eps;
   }
-  return cuda_status(run_prefill(pa, ra, final_conv_state, varlen, ws, L, stream));
+  if (args->snapshots != nullptr && args->snapshot_capacity > 0) {
+    ra.snap = args->snapshots; ra.snap_cap = args->snapshot_capacity;
+    ra.snap_every = (int64_t)args->snapshot_every * 64;
+  }
+  return cuda_status(run_prefill(pa, ra, args->final_conv_state, varlen, ws, L, stream));
 }
 
 kda_status kda_prefill_status(const void *workspace, void *stream_) {

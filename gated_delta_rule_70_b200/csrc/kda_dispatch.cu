@@ -72,6 +72,7 @@ cudaError_t run_chunk_path(PrepArgs pa, const RecurrenceArgs &ra, bool varlen, b
   sa.cu = ra.cu; sa.chunk_cu = chunk_cu; sa.records = ws + L.records; sa.max_slots = slots;
   sa.state0 = ra.state0; sa.scale = ra.scale; sa.o = ra.o; sa.state1 = ra.state1; sa.err = ra.err;
   if (ra.ogate != nullptr) { sa.onw = ra.onw; sa.oeps = ra.oeps; }
+  if (ra.snap != nullptr) { sa.snap = ra.snap; sa.snap_chunks = (int)(ra.snap_every / 64); sa.snap_cap = ra.snap_cap; }
   e = launch_state_pass(sa, ra.ogate, stream);
   clock_mark(timed, stream);
   return e;

@@ -47,6 +47,11 @@ struct RecurrenceArgs {
   const void *ogate;         // [T, H, D] io dtype
   const float *onw;          // [D]
   float oeps;
+  // state snapshots: snap[(n * snap_cap + j) * H + h] = state after (j + 1) * snap_every
+  // tokens of sequence n (snap_every a multiple of 64), j < snap_cap; nullptr: none
+  float *snap;
+  int64_t snap_every;
+  int snap_cap;
 };
 
 struct DecodeArgs {
@@ -107,6 +112,8 @@ struct StateArgs {
   int *err;
   const float *onw;          // output epilogue weight [128], with map_gate; nullptr: off
   float oeps;
+  float *snap;               // state snapshots, as in RecurrenceArgs (every snap_chunks chunks)
+  int snap_chunks, snap_cap;
   CUtensorMap map_gate;      // gate [T rows][H*128] bf16, 64-row boxes
 };
 

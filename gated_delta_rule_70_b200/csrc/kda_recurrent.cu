@@ -141,6 +141,16 @@ recurrence_kernel(RecurrenceArgs a) {
 #pragma unroll
         for (int c = 0; c < CPL; ++c) S[r][c] = fmaf(kk, dl[c], S[r][c]);
       }
+      if (a.snap != nullptr) {   // state snapshot after every snap_every tokens of the sequence
+        const int64_t done = tile0 + tt + 1 - s0;
+        if (done % a.snap_every == 0 && done / a.snap_every <= a.snap_cap) {
+          float *dst = a.snap + (((int64_t)n * a.snap_cap + done / a.snap_every - 1) * H + h) * D * D;
+#pragma unroll
+          for (int r = 0; r < 16; ++r)
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) __stcs(dst + (int64_t)(16 * w + r) * D + CPL * l + c, S[r][c]);
+        }
+      }
       buf ^= 1;
     }
   }

@@ -214,6 +214,13 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
     // garbage, but every address and every barrier stays the same), so the
     // warps never diverge around a barrier.  The flag is checked where all
     // epilogue threads have just passed the same named barrier.
+    // the snapshot slot that takes the state after chunk cc (a whole chunk), or nullptr
+    auto snap_after = [&](int cc) -> float * {
+      if (a.snap == nullptr || a.snap_chunks < 1 || (cc + 1) % a.snap_chunks != 0) return nullptr;
+      const int js = (cc + 1) / a.snap_chunks - 1;
+      if (js >= a.snap_cap) return nullptr;
+      return a.snap + (((int64_t)n * a.snap_cap + js) * H + h) * DK * DK;
+    };
     auto wait_one = [&](uint64_t *bb, uint32_t parity) {
       if (!umma::mbar_wait_bounded(bb, parity, WAIT_POLLS)) *(volatile int *)fail = 1;
       umma::fence_after_sync();
@@ -281,8 +288,9 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
         if (lane == 0) umma::mbar_arrive(&bar[B_EMIT]);   // gate slot cc % 2 is free again
       }
     };
-    // S^T columns *= e^{Gamma_C} of the record at rb; with s16: also write the bf16 copy there first
-    auto state_pass_over = [&](uint32_t rb, int s16) {
+    // S^T columns *= e^{Gamma_C} of the record at rb; with s16: also write the bf16 copy there first;
+    // with snap: store the state as it stands (before that decay) there, S[i][j] row-major
+    auto state_pass_over = [&](uint32_t rb, int s16, float *snap) {
       const float4 *egc = reinterpret_cast<const float4 *>(smem + rb + REC_EGC);
       uint32_t x[4][32];
 #pragma unroll
@@ -299,6 +307,10 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
           umma::tmem_st32(tmem + lane_base + TM_S16 + (uint32_t)s16 * 64 + q2 * 32, p);
         }
         handoff(&bar[B_S16]);   // the next D / O MMAs need only this copy
+      }
+      if (snap != nullptr) {   // lane j holds column j of S: each row store is 128 contiguous floats
+#pragma unroll
+        for (int i = 0; i < DK; ++i) __stcs(snap + (int64_t)i * DK + j, __uint_as_float(x[i >> 5][i & 31]));
       }
 #pragma unroll
       for (int e4 = 0; e4 < 32; ++e4) {
@@ -328,7 +340,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
     if (nchunks > 0) {   // chunk 0's decay
       wait_one(&bar[B_FULL0], 0);
       umma::tmem_wait_st();
-      state_pass_over(OFF_REC0, -1);
+      state_pass_over(OFF_REC0, -1, nullptr);
     }
     handoff(&bar[B_S16]);
 #pragma unroll 1
@@ -367,7 +379,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
       // the next chunk's bf16 state copy (handed off first), then its decay
       if (c + 1 < nchunks) {
         wait_one(&bar[B_FULL0 + (b ^ 1)], ((c + 1) >> 1) & 1);
-        state_pass_over(rec_off(c + 1), b ^ 1);
+        state_pass_over(rec_off(c + 1), b ^ 1, snap_after(c));
       }
       // the previous chunk's o, while the next chunk's first MMAs run (its barriers
       // make the fail flag uniform: stop here when a wait anywhere has given up)
@@ -383,15 +395,20 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
       emit_o(nchunks - 1, o_cols(nchunks - 1));
     }
     if (ok) {
-      // final state: S[i][j] = S^T[j][i]
+      // final state: S[i][j] = S^T[j][i] (and the last snapshot when the sequence ends on one)
       umma::tmem_wait_st();
+      float *last = nchunks > 0 && (s1 - s0) % ((int64_t)CH * (a.snap_chunks > 0 ? a.snap_chunks : 1)) == 0
+                        ? snap_after(nchunks - 1) : nullptr;
 #pragma unroll 1
       for (int cc = 0; cc < DK; cc += 32) {
         uint32_t x[32];
         umma::tmem_ld32(tmem + lane_base + TM_S32 + cc, x);
         umma::tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) a.state1[sg + (int64_t)(cc + e) * DK + j] = __uint_as_float(x[e]);
+        for (int e = 0; e < 32; ++e) {
+          a.state1[sg + (int64_t)(cc + e) * DK + j] = __uint_as_float(x[e]);
+          if (last != nullptr) last[(int64_t)(cc + e) * DK + j] = __uint_as_float(x[e]);
+        }
       }
     }
   }

@@ -28,7 +28,7 @@ KDA_BF16, KDA_FP32 = 0, 1
 EXPORTED = ["kda_prefill_workspace_size", "kda_prefill", "kda_prefill_status", "kda_prologue",
             "kda_recurrence", "kda_recurrence_workspace_size", "kda_decode_step",
             "kda_status_string", "kda_version", "kda_prefill_noalloc", "kda_kernel_timing",
-            "kda_kernel_times", "kda_prefill_gated", "kda_decode_step_gated"]
+            "kda_kernel_times", "kda_prefill_gated", "kda_decode_step_gated", "kda_prefill_ex"]
 
 
 class KdaLibraryError(RuntimeError):
@@ -54,6 +54,15 @@ KDA_FLAG_NEGATIVE_EIGENVALUES = 0x1
 class OutputGate(ctypes.Structure):
     """kda_output_gate: o <- o / sqrt(mean o^2 + eps) * weight * sigmoid(gate)."""
     _fields_ = [("gate", ctypes.c_void_p), ("weight", ctypes.c_void_p), ("eps", ctypes.c_float)]
+
+
+class PrefillArgs(ctypes.Structure):
+    """kda_prefill_args: every pointer of a kda_prefill_ex call."""
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("q", "k", "v", "conv_w", "alpha", "b", "A_log", "dt_bias", "initial_state",
+                 "initial_conv_state", "cu_seqlens", "o", "final_state", "final_conv_state",
+                 "out_gate", "snapshots")] + [("snapshot_every", ctypes.c_int32),
+                                              ("snapshot_capacity", ctypes.c_int32)]
 
 
 def library_path() -> str:
@@ -93,6 +102,8 @@ def load_library():
     lib.kda_prefill_gated.restype = i32
     lib.kda_decode_step_gated.argtypes = [SP] + [P] * 8 + [OG] + [P] * 3 + [P]
     lib.kda_decode_step_gated.restype = i32
+    lib.kda_prefill_ex.argtypes = [SP, ctypes.POINTER(PrefillArgs), P, sz, P]
+    lib.kda_prefill_ex.restype = i32
     lib.kda_status_string.argtypes = [i32]
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_version.argtypes = []
@@ -154,7 +165,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, conv_w: torch.Ten
             lower_bound: float = -5.0, l2norm_eps: float = 1e-6,
             scale: float = 1.0, negative_eigenvalues: bool = False,
             out_gate: Optional[torch.Tensor] = None, o_norm_weight: Optional[torch.Tensor] = None,
-            o_norm_eps: float = 1e-5,
+            o_norm_eps: float = 1e-5, snapshots: Optional[torch.Tensor] = None,
+            snapshot_every: int = 1,
             want_conv_state: bool = True, out: Optional[torch.Tensor] = None,
             final_state: Optional[torch.Tensor] = None,
             final_conv_state: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
@@ -163,8 +175,9 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, conv_w: torch.Ten
     b: [.., H].  Returns (o [T_total, H, d], final_state [N, H, d, d], final_conv_state
     [N, 3, 3*H*d] or None).  ``negative_eigenvalues``: beta = 2 sigmoid(b).  ``out_gate``
     [.., H, d] with ``o_norm_weight`` [d] fp32: the output epilogue o <- o / sqrt(mean o^2 +
-    o_norm_eps) * weight * sigmoid(out_gate).  ``check`` synchronises and raises on
-    device-side errors."""
+    o_norm_eps) * weight * sigmoid(out_gate).  ``snapshots`` [N, C, H, d, d] fp32: snapshot j
+    of sequence n (j < C) is the state after its first (j + 1) * 64 * snapshot_every tokens.
+    ``check`` synchronises and raises on device-side errors."""
     lib = load_library()
     H, d = alpha.shape[-2], alpha.shape[-1]
     if cu_seqlens is not None:
@@ -192,10 +205,15 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, conv_w: torch.Ten
     if ws is None or ws.numel() < ws_bytes:
         ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     og = _output_gate(out_gate, o_norm_weight, o_norm_eps)
-    st = lib.kda_prefill_gated(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(conv_w),
-                               _ptr(alpha), _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(initial_state),
-                               _ptr(initial_conv_state), _ptr(cu_seqlens), og, _ptr(o), _ptr(fs),
-                               _ptr(fc), _ptr(ws), ctypes.c_size_t(ws.numel()), _stream(dev))
+    og_struct = og._obj if og is not None else None
+    pa = PrefillArgs(*[_ptr(t) for t in (q, k, v, conv_w, alpha, b, A_log, dt_bias, initial_state,
+                                         initial_conv_state, cu_seqlens, o, fs, fc)],
+                     ctypes.cast(ctypes.pointer(og_struct), ctypes.c_void_p) if og_struct is not None
+                     else None,
+                     _ptr(snapshots), int(snapshot_every),
+                     int(snapshots.shape[1]) if snapshots is not None else 0)
+    st = lib.kda_prefill_ex(ctypes.byref(shape), ctypes.byref(pa), _ptr(ws),
+                            ctypes.c_size_t(ws.numel()), _stream(dev))
     _check(st, "kda_prefill")
     if check:
         _check(lib.kda_prefill_status(_ptr(ws), _stream(dev)), "kda_prefill (device)")

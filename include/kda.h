@@ -161,6 +161,42 @@ kda_status kda_prefill_gated(const kda_shape *shape,
                              void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * kda_prefill_ex -- kda_prefill with every optional output, through one
+ * argument block (NULL members: not wanted).  kda_prefill and
+ * kda_prefill_gated are this call with the extras off.
+ *
+ *   out_gate           the output epilogue (see kda_output_gate) or NULL
+ *   snapshots          [N, snapshot_capacity, H, d, d] fp32 or NULL: state
+ *                      snapshots aligned to the sequence start, for prefix
+ *                      caching (the "align" state-cache mode and chunked prefill
+ *                      the Ling-3.0-flash-VL page runs under vLLM): snapshot j
+ *                      of sequence n is the state after its first
+ *                      (j + 1) * 64 * snapshot_every tokens, S[i][j] as in
+ *                      final_state.  Only whole intervals are written, and at
+ *                      most snapshot_capacity per sequence; the rest of the
+ *                      buffer is left as it was.
+ *   snapshot_every     >= 1: 64-token chunks between snapshots
+ *   snapshot_capacity  >= 0: snapshots the buffer holds per sequence
+ */
+typedef struct {
+    const void *q, *k, *v, *conv_w, *alpha, *b;
+    const float *A_log, *dt_bias;
+    const float *initial_state;
+    const void *initial_conv_state;
+    const int32_t *cu_seqlens;
+    void *o;
+    float *final_state;
+    void *final_conv_state;
+    const kda_output_gate *out_gate;
+    float *snapshots;
+    int32_t snapshot_every;
+    int32_t snapshot_capacity;
+} kda_prefill_args;
+
+kda_status kda_prefill_ex(const kda_shape *shape, const kda_prefill_args *args,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * kda_prefill_status -- synchronises `stream` and reads the device error word
  * the last kda_prefill() on this workspace left: KDA_OK, KDA_ERR_INVALID_ARGUMENT
  * (bad cu_seqlens), KDA_ERR_TIMEOUT (a bounded wait gave up) or KDA_ERR_CUDA.

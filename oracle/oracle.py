@@ -164,6 +164,27 @@ def decode_step(H: int, D: int, state, conv_state, q, k, v, alpha, b, conv_w, A_
     return o, s1, c1
 
 
+def snapshots(cu_seqlens, H: int, D: int, every: int, cap: int, q, k, v, conv_w, alpha, b, A_log,
+              dt_bias, state0=None, conv0=None, **kw):
+    """State snapshots aligned to each sequence start: snap[n, j] (j < cap) is the final state
+    of the first (j + 1) * every tokens of sequence n, by definition; slots past the sequence
+    are NaN.  Composed from ``forward`` on those prefixes (no arithmetic of its own)."""
+    cu = _cu(cu_seqlens)
+    N = len(cu) - 1
+    q, k, v, alpha, b = map(_f, (q, k, v, alpha, b))
+    out = np.full((N, cap, H, D, D), np.nan)
+    for n in range(N):
+        a, z = int(cu[n]), int(cu[n + 1])
+        for j in range(min(cap, (z - a) // every)):
+            t = a + (j + 1) * every
+            s0 = None if state0 is None else np.ascontiguousarray(np.asarray(state0)[n:n + 1])
+            c0 = None if conv0 is None else np.ascontiguousarray(np.asarray(conv0)[n:n + 1])
+            _, s1, _, _ = forward([0, t - a], H, D, q[a:t], k[a:t], v[a:t], conv_w, alpha[a:t],
+                                  b[a:t], A_log, dt_bias, state0=s0, conv0=c0, **kw)
+            out[n, j] = s1[0]
+    return out
+
+
 def pair_inputs(f64: dict, H: int, D: int, cu, n: int, h: int, t_end: Optional[int] = None):
     """Slice packed fp64 inputs down to one (sequence n, head h) pair (H = 1), optionally
     keeping only the first t_end tokens of the sequence."""

@@ -394,3 +394,41 @@ def test_decode_output_gate(H, N):
         worst = max(rel_l2(og[n, h], o_r[n, h]) for n in range(N) for h in range(H))
         assert worst <= TOL["bf16"], (step, worst)
     assert max_state_err(W.from_device(st), s_ref) <= TOL["bf16"]
+
+
+# ------------------------------------------------------------------ state snapshots
+
+@pytest.mark.parametrize("io,d,lens,every,cap", [("bf16", 128, [64 * 5 + 7, 128, 300, 64, 0], 1, 6),
+                                                 ("bf16", 128, [64 * 6, 200], 2, 3),
+                                                 ("bf16", 128, [64 * 6], 2, 2),
+                                                 ("fp32", 64, [150, 64], 1, 3)])
+def test_prefill_state_snapshots(io, d, lens, every, cap):
+    """Snapshot j = the state after (j + 1) * 64 * every tokens of each sequence (the state
+    pass on the chunk path, the token kernel in fp32); slots past a sequence or past the
+    capacity stay untouched."""
+    s = W.small("snap", lens, H=2, d=d, io_dtype=io, seed=45, s0_std=0.02, varlen=len(set(lens)) > 1)
+    inp = W.make_inputs(s)
+    cu = _dev(inp["cu_seqlens"]) if s.varlen else None
+    snaps = torch.full((s.num_seqs, cap, s.H, d, d), float("nan"), dtype=torch.float32, device="cuda")
+    o, fs, _ = kda.prefill(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["conv_w"]),
+                           _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]), _dev(inp["dt_bias"]),
+                           initial_state=_dev(inp["S0"]), cu_seqlens=cu, num_seqs=s.num_seqs,
+                           snapshots=snaps, snapshot_every=every)
+    torch.cuda.synchronize()
+    f = f64_inputs(inp)
+    ref = oracle.snapshots(inp["cu_seqlens"], s.H, d, 64 * every, cap, f["q"], f["k"], f["v"],
+                           f["conv_w"], f["alpha"], f["b"], f["A_log"], f["dt_bias"], state0=f["S0"])
+    got = W.from_device(snaps)
+    tol = TOL[io]
+    for n in range(s.num_seqs):
+        for j in range(cap):
+            if np.isnan(ref[n, j]).all():
+                assert np.isnan(got[n, j]).all(), (n, j)   # not written
+            else:
+                for h in range(s.H):
+                    e = rel_l2(got[n, j, h], ref[n, j, h])
+                    assert e <= tol, (n, j, h, e)
+    # the plain outputs are unchanged by asking for snapshots
+    o_ref, s_ref, _, _ = oracle_prefill(s, inp)
+    assert max_pair_err(W.from_device(o), o_ref, inp["cu_seqlens"], s.H) <= tol
+    assert max_state_err(W.from_device(fs), s_ref) <= tol
