@@ -236,6 +236,26 @@ def run_ours(args, rank, world, local_rank):
     de[1].record(stream)
     torch.cuda.synchronize(dev)
     dec_gated_ms = de[0].elapsed_time(de[1]) / 64
+    # two tokens per sequence per call (a speculative token verified), with the state after
+    # each token kept: 32 calls over the same 64 tokens
+    mtp_x = [{kk: torch.stack([dsteps[2 * c][kk], dsteps[2 * c + 1][kk]], dim=1).contiguous()
+              for kk in dsteps[0]} for c in range(32)]
+    mtp_states = torch.empty((sd.num_seqs, 2, sd.H, sd.d, sd.d), dtype=torch.float32, device=dev)
+    mtp_out = torch.empty((sd.num_seqs, 2, sd.H, sd.d), dtype=bf, device=dev)
+
+    def dstep_mtp(x):
+        kda.decode_multi(x["q"], x["k"], x["v"], x["alpha"], x["b"], d_cw, d_A, d_dt, d_state,
+                         d_conv, step_states=mtp_states, out=mtp_out)
+
+    for c in range(3):
+        dstep_mtp(mtp_x[c])
+    de[0].record(stream)
+    for c in range(32):
+        dstep_mtp(mtp_x[c])
+    de[1].record(stream)
+    torch.cuda.synchronize(dev)
+    dec_mtp_ms = de[0].elapsed_time(de[1]) / 32
+    del mtp_x, mtp_states
     clock_info = clocks.stop()
 
     # ---- the other prefill workloads (reported beside the headline, not in `value`)
@@ -340,7 +360,10 @@ def run_ours(args, rank, world, local_rank):
                    "frac_of_measured_hbm": dec_gbs / peaks["hbm_gbs"],
                    "frac_of_8000_datasheet": dec_gbs / 8000.0,
                    "tokens_per_s": sd.num_seqs / (dec_step_ms * 1e-3),
-                   "output_gate_ms_per_step": dec_gated_ms},
+                   "output_gate_ms_per_step": dec_gated_ms,
+                   "two_tokens_with_step_states_ms_per_call": dec_mtp_ms,
+                   "two_tokens_algorithmic_bytes": decode_bytes(sd.num_seqs, sd.H, sd.d) +
+                   2 * sd.num_seqs * sd.H * sd.d * sd.d * 4 + 2 * sd.num_seqs * sd.H * sd.d * 2 * 5},
         "e2e": None if args.no_e2e else {
             "value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

@@ -259,14 +259,27 @@ kda_status kda_decode_step_gated(const kda_shape *shape, const void *q, const vo
                                  const void *conv_w, const float *A_log, const float *dt_bias,
                                  const kda_output_gate *out_gate, float *state, void *conv_state,
                                  void *o, void *stream_) {
+  if (shape == nullptr) return KDA_ERR_INVALID_ARGUMENT;
+  kda_shape one = *shape;
+  one.seq_len = 1;
+  return kda_decode_multi(&one, q, k, v, alpha, b, conv_w, A_log, dt_bias, out_gate, state,
+                          conv_state, o, nullptr, stream_);
+}
+
+kda_status kda_decode_multi(const kda_shape *shape, const void *q, const void *k, const void *v,
+                            const void *alpha, const void *b, const void *conv_w,
+                            const float *A_log, const float *dt_bias,
+                            const kda_output_gate *out_gate, float *state, void *conv_state,
+                            void *o, float *step_states, void *stream_) {
   kda_status st = check_shape(shape);
   if (st != KDA_OK) return st;
+  if (shape->seq_len < 1 || shape->seq_len > 16) return KDA_ERR_INVALID_ARGUMENT;
   if (shape->num_seqs == 0) return KDA_OK;
   st = check_out_gate(out_gate, shape->num_seqs);
   if (st != KDA_OK) return st;
   KDA_REQUIRE(q); KDA_REQUIRE(k); KDA_REQUIRE(v); KDA_REQUIRE(alpha); KDA_REQUIRE(b);
   KDA_REQUIRE(conv_w); KDA_REQUIRE(A_log); KDA_REQUIRE(dt_bias); KDA_REQUIRE(state);
-  KDA_REQUIRE(conv_state); KDA_REQUIRE(o);
+  KDA_REQUIRE(conv_state); KDA_REQUIRE(o); KDA_OPTIONAL(step_states);
   DecodeArgs a;
   std::memset(&a, 0, sizeof a);
   a.N = shape->num_seqs; a.H = shape->num_heads; a.D = shape->head_dim; a.io_dtype = shape->io_dtype;
@@ -277,6 +290,8 @@ kda_status kda_decode_step_gated(const kda_shape *shape, const void *q, const vo
   if (out_gate != nullptr) {
     a.ogate = out_gate->gate; a.onw = out_gate->weight; a.oeps = out_gate->eps;
   }
+  a.ntok = shape->seq_len;
+  a.step_states = step_states;
   a.state = state; a.conv_state = conv_state; a.o = o;
   return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream_)));
 }

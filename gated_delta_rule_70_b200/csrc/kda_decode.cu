@@ -55,120 +55,139 @@ decode_kernel(DecodeArgs a) {
     }
   }
 
-  // 2. prologue for this token and head.  Threads [0, D): q and k channel i;
-  //    threads [D, 2D): v channel i and the gate of key channel i.
+  // 2-4, once per token (a.ntok tokens of this sequence, in order; the state stays in
+  // registers and the conv history shifts in place between them)
   const T *__restrict__ cw = reinterpret_cast<const T *>(a.conv_w);
   T *__restrict__ cs = reinterpret_cast<T *>(a.conv_state) + (int64_t)n * 3 * 3 * HD;
   const int i = threadIdx.x % D;
   const bool first = threadIdx.x < D;
-  auto conv_channel = [&](int blk, const T *x) -> float {
-    const int64_t c = (int64_t)blk * HD + h * D + i;
-    const float x0 = to_f32(cs[0 * 3 * HD + c]), x1 = to_f32(cs[1 * 3 * HD + c]);
-    const float x2 = to_f32(cs[2 * 3 * HD + c]);
-    const T xn = x[(int64_t)n * HD + h * D + i];
-    float acc = to_f32(cw[c * KCONV + 0]) * x0;
-    acc = fmaf(to_f32(cw[c * KCONV + 1]), x1, acc);
-    acc = fmaf(to_f32(cw[c * KCONV + 2]), x2, acc);
-    acc = fmaf(to_f32(cw[c * KCONV + 3]), to_f32(xn), acc);
-    // shift the history in place: this thread is the only reader/writer of channel c
-    cs[0 * 3 * HD + c] = cs[1 * 3 * HD + c];
-    cs[1 * 3 * HD + c] = cs[2 * 3 * HD + c];
-    cs[2 * 3 * HD + c] = xn;
-    return silu_f(acc);
-  };
-  float qv = 0.f, kv = 0.f;
-  if (first) {
-    qv = conv_channel(0, reinterpret_cast<const T *>(a.q));
-    kv = conv_channel(1, reinterpret_cast<const T *>(a.k));
-    float sq = qv * qv, sk = kv * kv;
+  const int ntok = a.ntok > 0 ? a.ntok : 1;
+#pragma unroll 1
+  for (int tt = 0; tt < ntok; ++tt) {
+    const int64_t row = (int64_t)n * ntok + tt;   // token row in the [N, ntok, ...] inputs
+    // 2. prologue for this token and head.  Threads [0, D): q and k channel i;
+    //    threads [D, 2D): v channel i and the gate of key channel i.
+    auto conv_channel = [&](int blk, const T *x) -> float {
+      const int64_t c = (int64_t)blk * HD + h * D + i;
+      const float x0 = to_f32(cs[0 * 3 * HD + c]), x1 = to_f32(cs[1 * 3 * HD + c]);
+      const float x2 = to_f32(cs[2 * 3 * HD + c]);
+      const T xn = x[row * HD + h * D + i];
+      float acc = to_f32(cw[c * KCONV + 0]) * x0;
+      acc = fmaf(to_f32(cw[c * KCONV + 1]), x1, acc);
+      acc = fmaf(to_f32(cw[c * KCONV + 2]), x2, acc);
+      acc = fmaf(to_f32(cw[c * KCONV + 3]), to_f32(xn), acc);
+      // shift the history in place: this thread is the only reader/writer of channel c
+      cs[0 * 3 * HD + c] = cs[1 * 3 * HD + c];
+      cs[1 * 3 * HD + c] = cs[2 * 3 * HD + c];
+      cs[2 * 3 * HD + c] = xn;
+      return silu_f(acc);
+    };
+    float qv = 0.f, kv = 0.f;
+    if (first) {
+      qv = conv_channel(0, reinterpret_cast<const T *>(a.q));
+      kv = conv_channel(1, reinterpret_cast<const T *>(a.k));
+      float sq = qv * qv, sk = kv * kv;
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      sq += __shfl_xor_sync(0xffffffffu, sq, off);
-      sk += __shfl_xor_sync(0xffffffffu, sk, off);
+      for (int off = 16; off >= 1; off >>= 1) {
+        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        sk += __shfl_xor_sync(0xffffffffu, sk, off);
+      }
+      if (l == 0) { sm.norm_part[0][w] = sq; sm.norm_part[1][w] = sk; }
+    } else {
+      sm.v[i] = conv_channel(2, reinterpret_cast<const T *>(a.v));
+      const float al = to_f32(reinterpret_cast<const T *>(a.alpha)[(row * H + h) * D + i]);
+      const float g = gate_f(al + a.dt_bias[h * D + i], -expf(a.A_log[h]), a.lower_bound);
+      sm.eg[i] = expf(g);
+      if (i == 0) sm.beta = (a.beta2 ? 2.f : 1.f) * sigmoid_f(to_f32(reinterpret_cast<const T *>(a.b)[row * H + h]));
+      if (a.ogate) sm.gate[i] = to_f32(reinterpret_cast<const T *>(a.ogate)[(row * H + h) * D + i]);
     }
-    if (l == 0) { sm.norm_part[0][w] = sq; sm.norm_part[1][w] = sk; }
-  } else {
-    sm.v[i] = conv_channel(2, reinterpret_cast<const T *>(a.v));
-    const float al = to_f32(reinterpret_cast<const T *>(a.alpha)[((int64_t)n * H + h) * D + i]);
-    const float g = gate_f(al + a.dt_bias[h * D + i], -expf(a.A_log[h]), a.lower_bound);
-    sm.eg[i] = expf(g);
-    if (i == 0) sm.beta = (a.beta2 ? 2.f : 1.f) * sigmoid_f(to_f32(reinterpret_cast<const T *>(a.b)[(int64_t)n * H + h]));
-    if (a.ogate) sm.gate[i] = to_f32(reinterpret_cast<const T *>(a.ogate)[((int64_t)n * H + h) * D + i]);
-  }
-  __syncthreads();
-  if (first) {
-    float sq = 0.f, sk = 0.f;
+    __syncthreads();
+    if (first) {
+      float sq = 0.f, sk = 0.f;
 #pragma unroll
-    for (int ww = 0; ww < D / 32; ++ww) { sq += sm.norm_part[0][ww]; sk += sm.norm_part[1][ww]; }
-    sm.q[i] = qv * rsqrtf(sq + a.eps);
-    sm.k[i] = kv * rsqrtf(sk + a.eps);
-  }
-  __syncthreads();
+      for (int ww = 0; ww < D / 32; ++ww) { sq += sm.norm_part[0][ww]; sk += sm.norm_part[1][ww]; }
+      sm.q[i] = qv * rsqrtf(sq + a.eps);
+      sm.k[i] = kv * rsqrtf(sk + a.eps);
+    }
+    __syncthreads();
 
-  // 3. decay, then the column reductions p = S'^T k and r = S'^T q
-  float p[CPL], rr[CPL], qk = 0.f;
+    // 3. decay, then the column reductions p = S'^T k and r = S'^T q
+    float p[CPL], rr[CPL], qk = 0.f;
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) { p[c] = 0.f; rr[c] = 0.f; }
+    for (int c = 0; c < CPL; ++c) { p[c] = 0.f; rr[c] = 0.f; }
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      const int ii = 16 * w + r;
+      const float e = sm.eg[ii], kk = sm.k[ii], qq = sm.q[ii];
+      qk = fmaf(qq, kk, qk);
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        S[r][c] *= e;
+        p[c] = fmaf(kk, S[r][c], p[c]);
+        rr[c] = fmaf(qq, S[r][c], rr[c]);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) { sm.red_p[w][CPL * l + c] = p[c]; sm.red_r[w][CPL * l + c] = rr[c]; }
+    if (l == 0) sm.red_qk[w] = qk;
+    __syncthreads();
+    float P[CPL], R[CPL], QK = 0.f;
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) { P[c] = 0.f; R[c] = 0.f; }
+#pragma unroll
+    for (int ww = 0; ww < W; ++ww) {
+      QK += sm.red_qk[ww];
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) { P[c] += sm.red_p[ww][CPL * l + c]; R[c] += sm.red_r[ww][CPL * l + c]; }
+    }
+    const float bt = sm.beta;
+    float dl[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) dl[c] = bt * (sm.v[CPL * l + c] - P[c]);
+    if (w == 0) {
+      T *o = reinterpret_cast<T *>(a.o) + (row * H + h) * D + CPL * l;
+      float ov[CPL];
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) ov[c] = a.scale * fmaf(QK, dl[c], R[c]);
+      if (a.ogate) {   // output epilogue: o_norm over the row, then the sigmoid gate
+        float ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) ss = fmaf(ov[c], ov[c], ss);
+#pragma unroll
+        for (int sh = 16; sh >= 1; sh >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, sh);
+        const float rn = rsqrtf(ss * (1.f / D) + a.oeps);
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) ov[c] = ov[c] * rn * a.onw[CPL * l + c] * sigmoid_f(sm.gate[CPL * l + c]);
+      }
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) o[c] = from_f32<T>(ov[c]);
+    }
+
+    // 4. S = S' + k d^T (in registers); the state after this token when asked for
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      const float kk = sm.k[16 * w + r];
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) S[r][c] = fmaf(kk, dl[c], S[r][c]);
+    }
+    if (a.step_states != nullptr) {
+      float *dst = a.step_states + (row * H + h) * D * D;
+#pragma unroll
+      for (int r = 0; r < 16; ++r)
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) __stcs(dst + (int64_t)(16 * w + r) * D + CPL * l + c, S[r][c]);
+    }
+    __syncthreads();   // every read of this token's shared values is done
+  }
+
+  // 5. write the state back in place
 #pragma unroll
   for (int r = 0; r < 16; ++r) {
-    const int ii = 16 * w + r;
-    const float e = sm.eg[ii], kk = sm.k[ii], qq = sm.q[ii];
-    qk = fmaf(qq, kk, qk);
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      S[r][c] *= e;
-      p[c] = fmaf(kk, S[r][c], p[c]);
-      rr[c] = fmaf(qq, S[r][c], rr[c]);
-    }
-  }
-#pragma unroll
-  for (int c = 0; c < CPL; ++c) { sm.red_p[w][CPL * l + c] = p[c]; sm.red_r[w][CPL * l + c] = rr[c]; }
-  if (l == 0) sm.red_qk[w] = qk;
-  __syncthreads();
-  float P[CPL], R[CPL], QK = 0.f;
-#pragma unroll
-  for (int c = 0; c < CPL; ++c) { P[c] = 0.f; R[c] = 0.f; }
-#pragma unroll
-  for (int ww = 0; ww < W; ++ww) {
-    QK += sm.red_qk[ww];
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) { P[c] += sm.red_p[ww][CPL * l + c]; R[c] += sm.red_r[ww][CPL * l + c]; }
-  }
-  const float bt = sm.beta;
-  float dl[CPL];
-#pragma unroll
-  for (int c = 0; c < CPL; ++c) dl[c] = bt * (sm.v[CPL * l + c] - P[c]);
-  if (w == 0) {
-    T *o = reinterpret_cast<T *>(a.o) + ((int64_t)n * H + h) * D + CPL * l;
-    float ov[CPL];
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) ov[c] = a.scale * fmaf(QK, dl[c], R[c]);
-    if (a.ogate) {   // output epilogue: o_norm over the row, then the sigmoid gate
-      float ss = 0.f;
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) ss = fmaf(ov[c], ov[c], ss);
-#pragma unroll
-      for (int sh = 16; sh >= 1; sh >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, sh);
-      const float rn = rsqrtf(ss * (1.f / D) + a.oeps);
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) ov[c] = ov[c] * rn * a.onw[CPL * l + c] * sigmoid_f(sm.gate[CPL * l + c]);
-    }
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) o[c] = from_f32<T>(ov[c]);
-  }
-
-  // 4. write S = S' + k d^T back in place
-#pragma unroll
-  for (int r = 0; r < 16; ++r) {
-    const float kk = sm.k[16 * w + r];
     float *dst = Sg + (int64_t)(16 * w + r) * D + CPL * l;
     if constexpr (CPL == 4) {
-      __stcs(reinterpret_cast<float4 *>(dst),
-             make_float4(fmaf(kk, dl[0], S[r][0]), fmaf(kk, dl[1], S[r][1]),
-                         fmaf(kk, dl[2], S[r][2]), fmaf(kk, dl[3], S[r][3])));
+      __stcs(reinterpret_cast<float4 *>(dst), make_float4(S[r][0], S[r][1], S[r][2], S[r][3]));
     } else {
-      __stcs(reinterpret_cast<float2 *>(dst),
-             make_float2(fmaf(kk, dl[0], S[r][0]), fmaf(kk, dl[1], S[r][1])));
+      __stcs(reinterpret_cast<float2 *>(dst), make_float2(S[r][0], S[r][1]));
     }
   }
 }
@@ -452,7 +471,7 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_kernel(DecodeArgs a) {
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
   if ((int64_t)a.N * a.H == 0) return cudaSuccess;
-  if (a.io_dtype == KDA_BF16 && a.D == 128 && a.H % 8 == 0) {
+  if (a.io_dtype == KDA_BF16 && a.D == 128 && a.H % 8 == 0 && a.ntok <= 1 && a.step_states == nullptr) {
     cudaError_t e = cudaFuncSetAttribute(dec::decode_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)dec::SMEM_BYTES);
     if (e != cudaSuccess) return e;

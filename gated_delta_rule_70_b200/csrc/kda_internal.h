@@ -64,9 +64,11 @@ struct DecodeArgs {
   const float *A_log, *dt_bias;
   float lower_bound, eps, scale;
   int beta2;                 // beta = 2 sigmoid(b); 0: sigmoid(b)
-  const void *ogate;         // output epilogue [N, H, D] io dtype, or nullptr
+  const void *ogate;         // output epilogue [N, ntok, H, D] io dtype, or nullptr
   const float *onw;          // [D]
   float oeps;
+  int ntok;                  // tokens per sequence in this call (token inputs [N, ntok, ...]); 0 or 1: one
+  float *step_states;        // [N, ntok, H, D, D]: the state after each token, or nullptr
   float *state;              // [N, H, D, D] in place
   void *conv_state;          // [N, 3, 3*H*D] in place
   void *o;                   // [N, H, D]

@@ -28,7 +28,8 @@ KDA_BF16, KDA_FP32 = 0, 1
 EXPORTED = ["kda_prefill_workspace_size", "kda_prefill", "kda_prefill_status", "kda_prologue",
             "kda_recurrence", "kda_recurrence_workspace_size", "kda_decode_step",
             "kda_status_string", "kda_version", "kda_prefill_noalloc", "kda_kernel_timing",
-            "kda_kernel_times", "kda_prefill_gated", "kda_decode_step_gated", "kda_prefill_ex"]
+            "kda_kernel_times", "kda_prefill_gated", "kda_decode_step_gated", "kda_prefill_ex",
+            "kda_decode_multi"]
 
 
 class KdaLibraryError(RuntimeError):
@@ -104,6 +105,8 @@ def load_library():
     lib.kda_decode_step_gated.restype = i32
     lib.kda_prefill_ex.argtypes = [SP, ctypes.POINTER(PrefillArgs), P, sz, P]
     lib.kda_prefill_ex.restype = i32
+    lib.kda_decode_multi.argtypes = [SP] + [P] * 8 + [OG] + [P] * 4 + [P]
+    lib.kda_decode_multi.restype = i32
     lib.kda_status_string.argtypes = [i32]
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_version.argtypes = []
@@ -327,3 +330,25 @@ def kernel_times() -> Tuple[int, float, float]:
     if n < 0:
         raise KdaError(KDA_ERR_CUDA, "kda_kernel_times")
     return n, float(a.value), float(b.value)
+
+
+def decode_multi(q, k, v, alpha, b, conv_w, A_log, dt_bias, state: torch.Tensor,
+                 conv_state: torch.Tensor, *, lower_bound: float = -5.0, l2norm_eps: float = 1e-6,
+                 scale: float = 1.0, negative_eigenvalues: bool = False,
+                 out_gate: Optional[torch.Tensor] = None, o_norm_weight: Optional[torch.Tensor] = None,
+                 o_norm_eps: float = 1e-5, step_states: Optional[torch.Tensor] = None,
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """T new tokens per sequence (q, k, v [N, T, H*d]; alpha [N, T, H, d]; b [N, T, H]) in one
+    call; updates ``state`` and ``conv_state`` in place, fills ``step_states`` [N, T, H, d, d]
+    (the state after each token) when given, and returns o [N, T, H, d]."""
+    lib = load_library()
+    N, H, d = state.shape[0], state.shape[1], state.shape[2]
+    T = alpha.shape[1]
+    shape = make_shape(N, T, H, d, q.dtype, lower_bound, l2norm_eps, scale, negative_eigenvalues)
+    o = out if out is not None else torch.empty((N, T, H, d), dtype=q.dtype, device=q.device)
+    og = _output_gate(out_gate, o_norm_weight, o_norm_eps)
+    st = lib.kda_decode_multi(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b),
+                              _ptr(conv_w), _ptr(A_log), _ptr(dt_bias), og, _ptr(state),
+                              _ptr(conv_state), _ptr(o), _ptr(step_states), _stream(q.device))
+    _check(st, "kda_decode_multi")
+    return o

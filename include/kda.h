@@ -265,6 +265,33 @@ kda_status kda_decode_step(const kda_shape *shape,
                            const void *conv_w, const float *A_log, const float *dt_bias,
                            float *state, void *conv_state, void *o, void *stream);
 
+/*
+ * kda_decode_multi -- shape->seq_len (1 to 16) new tokens per sequence in one
+ * call, in order, for verifying speculative (MTP) tokens: the KDA layer's
+ * model predicts one extra token per step (AliceAI-Foundation KDA write-up,
+ * section "六": MTP with num_speculative_tokens 1 generates 2 tokens per forward).
+ *
+ *   q, k, v      [N, T, H*d]     io dtype, T = shape->seq_len
+ *   alpha        [N, T, H, d]    io dtype
+ *   b            [N, T, H]       io dtype
+ *   out_gate     NULL, or the output epilogue with gate [N, T, H, d]
+ *   state        [N, H, d, d]    fp32, in place: the state after all T tokens
+ *   conv_state   [N, 3, 3*H*d]   io dtype, shifted by T tokens in place
+ *   o            [N, T, H, d]    io dtype
+ *   step_states  [N, T, H, d, d] fp32 or NULL: the state after each token, so a
+ *                verifier that accepts t tokens resumes from step_states[:, t - 1]
+ *                (the conv state it needs is the last 3 raw tokens up to t)
+ *
+ * T = 1 without step_states is kda_decode_step_gated.  Needs no workspace.
+ */
+kda_status kda_decode_multi(const kda_shape *shape,
+                            const void *q, const void *k, const void *v,
+                            const void *alpha, const void *b,
+                            const void *conv_w, const float *A_log, const float *dt_bias,
+                            const kda_output_gate *out_gate,
+                            float *state, void *conv_state, void *o, float *step_states,
+                            void *stream);
+
 /* kda_decode_step with the output epilogue (gate [N, H, d]); out_gate NULL:
  * exactly kda_decode_step. */
 kda_status kda_decode_step_gated(const kda_shape *shape,

@@ -147,3 +147,16 @@ def test_output_gate_validation(lib):
     assert lib.kda_decode_step_gated(ctypes.byref(dsh), x, x, x, x, x, x, x, x,
                                      ctypes.byref(kda.OutputGate(None, 512, 1e-5)), x, x, x,
                                      None) == kda.KDA_ERR_INVALID_ARGUMENT
+
+
+def test_decode_multi_validation(lib):
+    import torch
+    P = ctypes.c_void_p
+    x = P(256)
+    for T, want in ((0, kda.KDA_ERR_INVALID_ARGUMENT), (17, kda.KDA_ERR_INVALID_ARGUMENT)):
+        sh = kda.make_shape(2, T, 2, 128, torch.bfloat16)
+        assert lib.kda_decode_multi(ctypes.byref(sh), x, x, x, x, x, x, x, x, None, x, x, x, None,
+                                    None) == want
+    sh = kda.make_shape(2, 4, 2, 128, torch.bfloat16)
+    assert lib.kda_decode_multi(ctypes.byref(sh), x, x, x, x, x, x, x, x, None, x, x, x, P(260),
+                                None) == kda.KDA_ERR_INVALID_ARGUMENT

@@ -432,3 +432,51 @@ def test_prefill_state_snapshots(io, d, lens, every, cap):
     o_ref, s_ref, _, _ = oracle_prefill(s, inp)
     assert max_pair_err(W.from_device(o), o_ref, inp["cu_seqlens"], s.H) <= tol
     assert max_state_err(W.from_device(fs), s_ref) <= tol
+
+
+# ------------------------------------------------------------------ multi-token decode
+
+@pytest.mark.parametrize("io,H,N,T,gated", [("bf16", 3, 5, 2, False), ("bf16", 16, 40, 4, False),
+                                            ("bf16", 8, 6, 3, True), ("fp32", 2, 3, 4, False)])
+def test_decode_multi(io, H, N, T, gated):
+    """T tokens per sequence in one call (speculative-token verification): o, the state and
+    conv state after the T tokens and the state after each token, against the oracle run
+    over those T tokens from the same state and conv history.  Two calls in a row."""
+    d = 128
+    s = W.small("dmulti", [24] * N, H=H, d=d, io_dtype=io, seed=46, s0_std=0.02)
+    inp = W.make_inputs(s)
+    o, st, cs = gpu_prefill(s, inp)
+    f = f64_inputs(inp)
+    _, s_ref, c_ref, _ = oracle_prefill(s, inp)
+    wgt = W.make_output_gate(s, N)["o_norm_weight"] if gated else None
+    for call in range(2):
+        xs = [_decode_inputs(s, call * T + t) for t in range(T)]
+        x = {k: np.ascontiguousarray(np.stack([xx[k] for xx in xs], axis=1)) for k in xs[0]}  # [N, T, ...]
+        gate = W.make_output_gate(s, N * T, tag=call + 1)["gate"].reshape(N, T, H, d) if gated else None
+        steps = torch.full((N, T, H, d, d), float("nan"), dtype=torch.float32, device="cuda")
+        o_t = kda.decode_multi(_dev(x["q"]), _dev(x["k"]), _dev(x["v"]), _dev(x["alpha"]),
+                               _dev(x["b"]), _dev(inp["conv_w"]), _dev(inp["A_log"]),
+                               _dev(inp["dt_bias"]), st, cs, step_states=steps,
+                               out_gate=_dev(gate) if gated else None,
+                               o_norm_weight=_dev(wgt) if gated else None)
+        torch.cuda.synchronize()
+        cu = np.arange(0, N * T + 1, T)
+        flat = lambda a, tail: W.as_f64(a).reshape((N * T,) + tail)
+        fx = dict(q=flat(x["q"], (H * d,)), k=flat(x["k"], (H * d,)), v=flat(x["v"], (H * d,)),
+                  alpha=flat(x["alpha"], (H, d)), b=flat(x["b"], (H,)))
+        kw = dict(out_gate=W.as_f64(gate).reshape(N * T, H, d), o_norm_weight=W.as_f64(wgt)) if gated else {}
+        o_r, s_new, c_new, _ = oracle.forward(cu, H, d, fx["q"], fx["k"], fx["v"], f["conv_w"],
+                                              fx["alpha"], fx["b"], f["A_log"], f["dt_bias"],
+                                              state0=s_ref, conv0=c_ref, **kw)
+        st_r = oracle.snapshots(cu, H, d, 1, T, fx["q"], fx["k"], fx["v"], f["conv_w"], fx["alpha"],
+                                fx["b"], f["A_log"], f["dt_bias"], state0=s_ref, conv0=c_ref)
+        tol = TOL[io]
+        og = W.from_device(o_t).reshape(N * T, H, d)
+        worst = max(rel_l2(og[i, h], o_r[i, h]) for i in range(N * T) for h in range(H))
+        assert worst <= tol, (call, worst)
+        gs = W.from_device(steps)
+        for t in range(T):
+            assert max_state_err(gs[:, t], st_r[:, t]) <= tol, (call, t)
+        s_ref, c_ref = s_new, c_new
+        assert max_state_err(W.from_device(st), s_ref) <= tol
+        np.testing.assert_array_equal(W.from_device(cs), c_ref)
