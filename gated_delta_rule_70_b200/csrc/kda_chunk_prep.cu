@@ -212,7 +212,13 @@ template <bool kFused>
 __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant__ PrepArgs a) {
   const int H = a.H;
   const int h = blockIdx.x % H;
-  const int64_t gchunk = blockIdx.x / H;
+  int64_t gchunk = blockIdx.x / H;
+  if (a.chunk_cu == nullptr && a.seg_len > 0) {   // a time segment of a dense batch
+    const int64_t per = (a.seq_len + CH - 1) / CH;
+    const int64_t cidx = a.seg_c0 + gchunk % a.seg_len;
+    if (cidx >= per) return;
+    gchunk = (gchunk / a.seg_len) * per + cidx;
+  }
   int n, nt;
   int64_t c0, cidx;
   if (!locate(a, gchunk, n, c0, nt, cidx)) return;
@@ -781,6 +787,7 @@ cudaError_t launch_chunk_prep(PrepArgs a, int64_t max_chunks, bool fused, const 
                               const void *k, const void *v, const void *alpha, cudaStream_t stream) {
   if (max_chunks == 0 || a.H == 0 || a.total_tokens == 0) return cudaSuccess;
   a.max_slots = max_chunks;
+  if (a.chunk_cu == nullptr && a.seg_len > 0) max_chunks = (int64_t)a.N * a.seg_len;   // grid of a segment
   if (!fused) return launch_prep_variant<false>(a, max_chunks, stream);
   const uint64_t rows = (uint64_t)a.total_tokens, cols = (uint64_t)a.H * chunkfmt::DK;
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;

@@ -6,6 +6,7 @@
 // on the raw inputs, so conv'd / normalised q, k, v and the gates never travel
 // through device memory.  Every other shape runs the prologue kernel and the
 // CUDA-core token kernel.
+#include <climits>
 #include <mutex>
 #include <vector>
 
@@ -45,6 +46,44 @@ bool clock_begin() {
   return g_clock.on && g_clock.ev.size() / 3 < kMaxTimedCalls;
 }
 
+// Time segments: when a dense batch has few (sequence, head) chains, the state pass
+// occupies few SMs for a long time while the rest idle.  The chunks are then split
+// into segments of kSegChunks: chunk_prep of segment s+1 runs on the caller's stream
+// while the state pass of segment s runs on a high-priority side stream (the state
+// passes carry the state from one segment to the next through final_state).  Only
+// stream order and events connect the two: no kernel waits on another.
+constexpr int kSegChunks = 64;
+
+struct SideStreams {
+  std::mutex mu;               // held while one call enqueues its segments
+  cudaStream_t stream[64] = {};
+  cudaEvent_t prep_done[64] = {}, pass_done[64] = {};
+  int sms[64] = {};
+};
+SideStreams g_side;
+
+// The side stream, its two events and the SM count of the current device (created once).
+cudaError_t side_resources(int &dev, cudaStream_t &side, cudaEvent_t &ev_prep, cudaEvent_t &ev_pass, int &sms) {
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (g_side.stream[dev] == nullptr) {
+    int lo = 0, hi = 0;
+    if ((e = cudaDeviceGetStreamPriorityRange(&lo, &hi)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&g_side.sms[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return e;
+    if ((e = cudaEventCreateWithFlags(&g_side.prep_done[dev], cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&g_side.pass_done[dev], cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithPriority(&g_side.stream[dev], cudaStreamNonBlocking, hi)) != cudaSuccess)
+      return e;
+  }
+  side = g_side.stream[dev];
+  ev_prep = g_side.prep_done[dev];
+  ev_pass = g_side.pass_done[dev];
+  sms = g_side.sms[dev];
+  return cudaSuccess;
+}
+
 cudaError_t run_chunk_path(PrepArgs pa, const RecurrenceArgs &ra, bool varlen, bool fused,
                            const PrologueArgs *raw, char *ws, const WsLayout &L,
                            cudaStream_t stream) {
@@ -58,24 +97,64 @@ cudaError_t run_chunk_path(PrepArgs pa, const RecurrenceArgs &ra, bool varlen, b
   pa.N = ra.N; pa.H = ra.H; pa.seq_len = ra.seq_len; pa.total_tokens = ra.total_tokens;
   pa.cu = ra.cu; pa.chunk_cu = chunk_cu;
   pa.records = ws + L.records; pa.err = ra.err;
-  const bool timed = clock_begin();
-  clock_mark(timed, stream);
-  cudaError_t e = launch_chunk_prep(pa, slots, fused, raw ? raw->q : nullptr, raw ? raw->k : nullptr,
-                                    raw ? raw->v : nullptr, raw ? raw->alpha : nullptr, stream);
-  clock_mark(timed, stream);
-  if (e != cudaSuccess) {
-    clock_mark(timed, stream);   // keep the events in triples
-    return e;
-  }
   StateArgs sa{};
   sa.N = ra.N; sa.H = ra.H; sa.seq_len = ra.seq_len; sa.total_tokens = ra.total_tokens;
   sa.cu = ra.cu; sa.chunk_cu = chunk_cu; sa.records = ws + L.records; sa.max_slots = slots;
   sa.state0 = ra.state0; sa.scale = ra.scale; sa.o = ra.o; sa.state1 = ra.state1; sa.err = ra.err;
+  sa.seg_c0 = 0; sa.seg_c1 = INT_MAX;
   if (ra.ogate != nullptr) { sa.onw = ra.onw; sa.oeps = ra.oeps; }
   if (ra.snap != nullptr) { sa.snap = ra.snap; sa.snap_chunks = (int)(ra.snap_every / 64); sa.snap_cap = ra.snap_cap; }
-  e = launch_state_pass(sa, ra.ogate, stream);
+  const void *rq = raw ? raw->q : nullptr, *rk = raw ? raw->k : nullptr;
+  const void *rv = raw ? raw->v : nullptr, *ralpha = raw ? raw->alpha : nullptr;
+
+  const int64_t per = varlen ? 0 : (ra.seq_len + 63) / 64;
+  int dev = 0, sms = 0;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_prep = nullptr, ev_pass = nullptr;
+  std::unique_lock<std::mutex> lock(g_side.mu, std::defer_lock);
+  bool segmented = !varlen && per >= 4 * kSegChunks && ra.state1 != nullptr && !ra.no_side_stream;
+  if (segmented) {
+    lock.lock();
+    segmented = side_resources(dev, side, ev_prep, ev_pass, sms) == cudaSuccess &&
+                2 * (int64_t)ra.N * ra.H <= sms;
+    if (!segmented) lock.unlock();
+  }
+
+  const bool timed = clock_begin();
   clock_mark(timed, stream);
-  return e;
+  cudaError_t e = cudaSuccess;
+  if (!segmented) {
+    e = launch_chunk_prep(pa, slots, fused, rq, rk, rv, ralpha, stream);
+    clock_mark(timed, stream);
+    if (e == cudaSuccess) e = launch_state_pass(sa, ra.ogate, stream);
+    else clock_mark(timed, stream);   // keep the events in triples
+    clock_mark(timed, stream);
+    return e;
+  }
+  // segment s: chunk_prep on `stream`, then (after it, on the side stream) the state pass,
+  // which starts from the state the previous segment's pass left in final_state
+  const int nseg = (int)((per + kSegChunks - 1) / kSegChunks);
+  for (int sg = 0; sg < nseg && e == cudaSuccess; ++sg) {
+    pa.seg_c0 = sg * kSegChunks;
+    pa.seg_len = kSegChunks;
+    e = launch_chunk_prep(pa, slots, fused, rq, rk, rv, ralpha, stream);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_prep, stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev_prep, 0);
+    if (e == cudaSuccess) {
+      StateArgs ss = sa;
+      ss.seg_c0 = sg * kSegChunks;
+      ss.seg_c1 = sg + 1 == nseg ? INT_MAX : (sg + 1) * kSegChunks;
+      if (sg > 0) ss.state0 = ra.state1;
+      e = launch_state_pass(ss, ra.ogate, side);
+    }
+  }
+  clock_mark(timed, stream);
+  // the caller's stream continues only after the last state pass (also on an error, so
+  // that nothing of this call is left running unordered)
+  cudaError_t e2 = cudaEventRecord(ev_pass, side);
+  if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(stream, ev_pass, 0);
+  clock_mark(timed, stream);
+  return e != cudaSuccess ? e : e2;
 }
 
 }  // namespace

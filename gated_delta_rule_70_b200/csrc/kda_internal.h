@@ -52,6 +52,9 @@ struct RecurrenceArgs {
   float *snap;
   int64_t snap_every;
   int snap_cap;
+  // 1: never use the side stream of the time-segmented schedule (its stream and events are
+  // created on first use); the entry point that must allocate nothing sets it
+  int no_side_stream;
 };
 
 struct DecodeArgs {
@@ -96,6 +99,8 @@ struct PrepArgs {
   const float *g, *beta;     // [T, H, 128], [T, H]
   void *records;             // [max_slots][H] records of chunkfmt::REC_STRIDE bytes
   int64_t max_slots;         // record slots (set by the launcher)
+  int seg_c0, seg_len;       // dense batches: chunks [seg_c0, seg_c0 + seg_len) of every sequence
+                             // (seg_len 0: all); varlen batches: unused
   int *err;
   // [T rows][H*128] bf16: q, k, v (67-row boxes: 3 history rows + 64) and alpha (64 rows)
   CUtensorMap map_q, map_k, map_v, map_alpha;
@@ -108,6 +113,7 @@ struct StateArgs {
   const void *records;
   int64_t max_slots;         // record slots in the workspace (chunks beyond are not read)
   const float *state0;       // [N, H, 128, 128] or nullptr
+  int seg_c0, seg_c1;        // chunks [seg_c0, seg_c1) of every sequence (0, INT_MAX: all)
   float scale;
   void *o;                   // [T, H, 128] bf16
   float *state1;

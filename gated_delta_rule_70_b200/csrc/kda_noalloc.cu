@@ -98,6 +98,7 @@ extern "C" kda_status kda_prefill_noalloc(
   ra.total_tokens = T; ra.io_dtype = s->io_dtype; ra.cu = cu_seqlens;
   ra.state0 = initial_state; ra.scale = s->scale; ra.o = o; ra.state1 = final_state;
   ra.lower_bound = s->lower_bound; ra.err = pa.err;
+  ra.no_side_stream = 1;   // (the segmented schedule would create a stream and events)
   if (run_prefill(pa, ra, final_conv_state, varlen, ws, L, stream) != cudaSuccess) return KDA_ERR_CUDA;
   return KDA_OK;
 }

@@ -95,8 +95,12 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
   const int n = blockIdx.x / H, h = blockIdx.x % H;
   int64_t s0, s1;
   seq_bounds(a.cu, n, a.seq_len, a.total_tokens, s0, s1);
-  int nchunks = (int)((s1 - s0 + CH - 1) / CH);
-  int64_t chunk0 = a.chunk_cu ? (int64_t)a.chunk_cu[n] : (int64_t)n * ((a.seq_len + CH - 1) / CH);
+  // this launch's chunks [k0, k1) of the sequence (a time segment, or all of it)
+  const int nall = (int)((s1 - s0 + CH - 1) / CH);
+  const int k0 = min(a.seg_c0, nall), k1 = min(a.seg_c1, nall);
+  int nchunks = k1 - k0;
+  const int64_t t0 = s0 + (int64_t)k0 * CH;   // first token of chunk 0 of this launch
+  int64_t chunk0 = (a.chunk_cu ? (int64_t)a.chunk_cu[n] : (int64_t)n * ((a.seq_len + CH - 1) / CH)) + k0;
   // only malformed cu_seqlens (overlapping clamped sequences) can exceed the record slots
   if (chunk0 < 0 || chunk0 > a.max_slots) chunk0 = a.max_slots;
   if (chunk0 + nchunks > a.max_slots) nchunks = (int)(a.max_slots - chunk0);
@@ -158,7 +162,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
         if (lane == 0) {
           umma::mbar_arrive_expect_tx(&bar[B_G0 + (c & 1)], GATE_BYTES);
           umma::tma_load_2d(smem + OFF_GATE + (c & 1) * GATE_BYTES, &a.map_gate, h * DK,
-                            (int)(s0 + (int64_t)c * CH), &bar[B_G0 + (c & 1)]);
+                            (int)(t0 + (int64_t)c * CH), &bar[B_G0 + (c & 1)]);
         }
         __syncwarp();
         issued = c + 1;
@@ -195,14 +199,20 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
       // This warp and the MMA warp meet at both named barriers once per chunk, every chunk,
       // whatever happens (after a failed wait the mbarrier waits return at once and the MMA
       // warp issues nothing), so neither can be left waiting at one.
+      // Chunk c+1's record and O^T buffer (normally long ready) are waited for while chunk
+      // c's state MMA and bf16 state copy run: even a completed wait costs a few hundred
+      // cycles, and only the bf16 state copy should stand before the D MMA.
+      auto pre = [&](int cc) {
+        (void)(wait_warp(&bar[B_FULL0 + (cc & 1)], (cc >> 1) & 1) &&
+               (cc < NOBUF || wait_warp(&bar[B_OE0 + (cc & (NOBUF - 1))], ((cc / NOBUF) - 1) & 1)));
+      };
+      if (nchunks > 0) pre(0);
       for (int c = 0; c < nchunks; ++c) {
-        const int b = c & 1, ob = c & (NOBUF - 1);
-        (void)(wait_warp(&bar[B_FULL0 + b], (c >> 1) & 1) &&
-               (c < NOBUF || wait_warp(&bar[B_OE0 + ob], ((c / NOBUF) - 1) & 1)) &&   // O^T of chunk c-4 left
-               wait_warp(&bar[B_S16], c & 1));
+        (void)wait_warp(&bar[B_S16], c & 1);
         umma::named_sync(BAR_GO_D, 64);
         (void)wait_warp(&bar[B_D16], c & 1);
         umma::named_sync(BAR_GO_S, 64);
+        if (c + 1 < nchunks) pre(c + 1);
       }
     } else if (warp == W_MMA) {
       // ---------------------------------------------------------- MMA issue
@@ -291,7 +301,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
       umma::fence_before_sync();
       __syncwarp();
       if (lane == 0) umma::mbar_arrive(&bar[B_OE0 + ob]);
-      const int64_t c0 = s0 + (int64_t)c * CH;
+      const int64_t c0 = t0 + (int64_t)c * CH;
       const int nvalid = (int)min((int64_t)CH, s1 - c0);
       if (!gated) {
 #pragma unroll
@@ -350,8 +360,9 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
     const int j = (warp & 3) * 32 + lane;               // TMEM lane = value channel
     const uint32_t lane_base = (uint32_t)(warp & 3) * 32u << 16;
     const int64_t sg = ((int64_t)n * H + h) * DK * DK;
-    // the snapshot slot that takes the state after chunk cc (a whole chunk), or nullptr
-    auto snap_after = [&](int cc) -> float * {
+    // the snapshot slot that takes the state after chunk cc of this launch (a whole chunk), or nullptr
+    auto snap_after = [&](int cl) -> float * {
+      const int cc = cl + k0;   // chunk index within the sequence
       if (a.snap == nullptr || a.snap_chunks < 1 || (cc + 1) % a.snap_chunks != 0) return nullptr;
       const int js = (cc + 1) / a.snap_chunks - 1;
       if (js >= a.snap_cap) return nullptr;
@@ -453,9 +464,11 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
       if (c + 1 < nchunks) state_pass_over(rec_off(c + 1), true, snap_after(c));
     }
     if (*(volatile int *)fail == 0) {
-      // final state: S[i][j] = S^T[j][i] (and the last snapshot when the sequence ends on one)
+      // final state: S[i][j] = S^T[j][i] (and the last snapshot when this launch ends on one)
       umma::tmem_wait_st();
-      float *last = nchunks > 0 && (s1 - s0) % ((int64_t)CH * (a.snap_chunks > 0 ? a.snap_chunks : 1)) == 0
+      // (a segment that ends inside the sequence ends on a whole chunk)
+      float *last = nchunks > 0 && (k1 < nall ||
+                                    (s1 - s0) % ((int64_t)CH * (a.snap_chunks > 0 ? a.snap_chunks : 1)) == 0)
                         ? snap_after(nchunks - 1) : nullptr;
 #pragma unroll 1
       for (int cc = 64 * hf; cc < 64 * hf + 64; cc += 32) {

@@ -480,3 +480,57 @@ def test_decode_multi(io, H, N, T, gated):
         s_ref, c_ref = s_new, c_new
         assert max_state_err(W.from_device(st), s_ref) <= tol
         np.testing.assert_array_equal(W.from_device(cs), c_ref)
+
+
+# ------------------------------------------------------------------ time-segmented schedule
+
+def test_prefill_time_segments_gated():
+    """Dense batches with few (sequence, head) chains and at least 256 chunks per sequence
+    run chunk_prep and the state pass in time segments of 64 chunks on two streams, the
+    state carried between segments through final_state.  Two sequences of 16428 tokens
+    (5 segments, the last one a ragged 44-token chunk), an initial state and the output
+    epilogue, against the oracle on everything."""
+    s = W.small("seg", [16428, 16428], H=2, d=128, seed=61, s0_std=0.02, varlen=False)
+    inp = W.make_inputs(s)
+    G = W.make_output_gate(s, s.total_tokens)
+    o, fs, fc = kda.prefill(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["conv_w"]),
+                            _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]), _dev(inp["dt_bias"]),
+                            initial_state=_dev(inp["S0"]), num_seqs=s.num_seqs,
+                            out_gate=_dev(G["gate"]), o_norm_weight=_dev(G["o_norm_weight"]),
+                            o_norm_eps=1e-5)
+    torch.cuda.synchronize()
+    f = f64_inputs(inp)
+    o_ref, s_ref, c_ref, _ = oracle.forward(inp["cu_seqlens"], s.H, s.d, f["q"], f["k"], f["v"],
+                                            f["conv_w"], f["alpha"], f["b"], f["A_log"], f["dt_bias"],
+                                            state0=f["S0"], out_gate=W.as_f64(G["gate"]),
+                                            o_norm_weight=W.as_f64(G["o_norm_weight"]), o_norm_eps=1e-5)
+    eo = max_pair_err(W.from_device(o), o_ref, inp["cu_seqlens"], s.H)
+    es = max_state_err(W.from_device(fs), s_ref)
+    assert eo <= TOL["bf16"], "o rel-L2 %.3g" % eo
+    assert es <= TOL["bf16"], "final_state rel-L2 %.3g" % es
+    np.testing.assert_array_equal(W.from_device(fc), c_ref)
+
+
+def test_prefill_time_segments_snapshots():
+    """Snapshots every 4096 tokens of a 16448-token sequence fall on the time-segment
+    boundaries of the two-stream schedule: each is stored as the final state of its
+    segment's state pass."""
+    every, cap = 64, 5
+    s = W.small("segsnap", [16448], H=2, d=128, seed=62, s0_std=0.02, varlen=False)
+    inp = W.make_inputs(s)
+    snaps = torch.full((1, cap, s.H, 128, 128), float("nan"), dtype=torch.float32, device="cuda")
+    o, fs, _ = kda.prefill(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["conv_w"]),
+                           _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]), _dev(inp["dt_bias"]),
+                           initial_state=_dev(inp["S0"]), num_seqs=1, snapshots=snaps, snapshot_every=every)
+    torch.cuda.synchronize()
+    f = f64_inputs(inp)
+    ref = oracle.snapshots(inp["cu_seqlens"], s.H, 128, 64 * every, cap, f["q"], f["k"], f["v"],
+                           f["conv_w"], f["alpha"], f["b"], f["A_log"], f["dt_bias"], state0=f["S0"])
+    got = W.from_device(snaps)
+    for j in range(cap):
+        if np.isnan(ref[0, j]).all():
+            assert np.isnan(got[0, j]).all(), j
+        else:
+            for h in range(s.H):
+                e = rel_l2(got[0, j, h], ref[0, j, h])
+                assert e <= TOL["bf16"], (j, h, e)
