@@ -486,10 +486,10 @@ def test_decode_multi(io, H, N, T, gated):
 
 def test_prefill_time_segments_gated():
     """Dense batches with few (sequence, head) chains and at least 256 chunks per sequence
-    run chunk_prep and the state pass in time segments of 64 chunks on two streams, the
+    run chunk_prep and the state pass in time segments of 128 chunks on two streams, the
     state carried between segments through final_state.  Two sequences of 16428 tokens
-    (5 segments, the last one a ragged 44-token chunk), an initial state and the output
-    epilogue, against the oracle on everything."""
+    (3 segments, the last one a single ragged 44-token chunk), an initial state and the
+    output epilogue, against the oracle on everything."""
     s = W.small("seg", [16428, 16428], H=2, d=128, seed=61, s0_std=0.02, varlen=False)
     inp = W.make_inputs(s)
     G = W.make_output_gate(s, s.total_tokens)
@@ -512,9 +512,9 @@ def test_prefill_time_segments_gated():
 
 
 def test_prefill_time_segments_snapshots():
-    """Snapshots every 4096 tokens of a 16448-token sequence fall on the time-segment
-    boundaries of the two-stream schedule: each is stored as the final state of its
-    segment's state pass."""
+    """Snapshots every 4096 tokens of a 16448-token sequence (257 chunks: time segments
+    [0, 128), [128, 256), [256, 257)): those after chunks 128 and 256 end a segment and
+    are stored as its final state, the others are stored between chunks."""
     every, cap = 64, 5
     s = W.small("segsnap", [16448], H=2, d=128, seed=62, s0_std=0.02, varlen=False)
     inp = W.make_inputs(s)
