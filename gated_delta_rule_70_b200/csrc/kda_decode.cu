@@ -8,10 +8,12 @@
 //
 // HBM-bound by construction: each state element is read once, decayed, reduced,
 // corrected and written back once; o = S'^T q + (q.k) d lets one barrier carry
-// all column reductions.  Two kernels:
+// all column reductions.  Three kernels:
 //   - dec::decode_tma_kernel (bf16, head_dim 128, heads a multiple of 8): one
 //     persistent CTA per SM, a producer warp streaming (sequence, head) items
 //     through a 3-slot shared-memory ring by bulk copy;
+//   - dec::decode_tma_multi_kernel: the same for several tokens per call (or the
+//     per-token states), two slots that hold every token's inputs;
 //   - decode_kernel (every other shape): one CTA per (sequence, head), which
 //     issues all loads of its state slice before the token's prologue so the
 //     prologue's latency hides under the state stream.
@@ -219,7 +221,8 @@ constexpr uint32_t S_GATE = S_B + 128;              // bf16 output gate [128] (e
 constexpr uint32_t SLOT = S_GATE + 256;             // 72,832 B per item
 constexpr int NSLOT = 3;
 constexpr uint32_t OFF_SCR = NSLOT * SLOT;
-struct Scratch {
+template <int NS>
+struct ScratchT {
   float q[D], k[D], eg[D], v[D];
   float red_p[NC / 32][D], red_r[NC / 32][D], red_qk[NC / 32];
   float norm_part[2][4];
@@ -227,9 +230,10 @@ struct Scratch {
   float onw[D];     // output epilogue weight
   float beta;
   int fail;
-  int req[NSLOT];   // requests issued per slot (for the error path)
-  uint64_t full[NSLOT], empty[NSLOT];
+  int req[NS];      // requests issued per slot (for the error path)
+  uint64_t full[NS], empty[NS];
 };
+using Scratch = ScratchT<NSLOT>;
 constexpr uint32_t SMEM_BYTES = OFF_SCR + sizeof(Scratch);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(SLOT % 16 == 0 && S_QKV % 16 == 0 && S_HIST % 16 == 0 && S_W % 16 == 0 && S_DTB % 16 == 0 &&
@@ -467,6 +471,278 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_kernel(DecodeArgs a) {
   __syncthreads();
 }
 
+// ---------------------------------------------------------------------------
+// Multi-token variant (2 to MT_MAX tokens per sequence in one call, optionally the
+// state after each token): the same producer / compute split, with two ring slots
+// that hold the state and every token's inputs.  The conv history and the call's
+// tokens sit in one raw-row array per tensor (rows 0-2 the history, row 3 + t token
+// t), so token t's conv reads rows t .. t+3 and the new history is rows T .. T+2.
+// The state stays in registers across the tokens; the per-token states leave from
+// registers as 16-byte row stores.
+constexpr int MT_MAX = 16;
+constexpr uint32_t M_STATE = 0;                            // fp32 [128][128]
+constexpr uint32_t M_RAWT = (3 + MT_MAX) * 256;            // bf16 raw rows of one tensor: [3 + MT_MAX][128]
+constexpr uint32_t M_RAW = 65536;                          // [tensor][row][128]
+constexpr uint32_t M_ALPHA = M_RAW + 3 * M_RAWT;           // bf16 [MT_MAX][128]
+constexpr uint32_t M_W = M_ALPHA + MT_MAX * 256;           // bf16 conv weights [tensor][128][4]
+constexpr uint32_t M_DTB = M_W + 3072;                     // fp32 dt_bias [128]
+constexpr uint32_t M_B = M_DTB + 512;                      // bf16 b of the sequence's rows [MT_MAX][H <= 64]
+constexpr uint32_t M_GATE = M_B + MT_MAX * 128;            // bf16 output gate [MT_MAX][128]
+constexpr uint32_t M_SLOT = M_GATE + MT_MAX * 256;         // 93,952 B per item
+constexpr int M_NSLOT = 2;
+constexpr uint32_t M_OFF_SCR = M_NSLOT * M_SLOT;
+using MScratch = ScratchT<M_NSLOT>;
+constexpr uint32_t M_SMEM_BYTES = M_OFF_SCR + sizeof(MScratch);
+static_assert(M_SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(M_SLOT % 16 == 0 && M_RAW % 16 == 0 && M_RAWT % 16 == 0 && M_ALPHA % 16 == 0 && M_W % 16 == 0 &&
+              M_DTB % 16 == 0 && M_B % 16 == 0 && M_GATE % 16 == 0 && M_OFF_SCR % 16 == 0, "bulk copy alignment");
+
+__global__ void __launch_bounds__(NT, 1) decode_tma_multi_kernel(DecodeArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  MScratch &sc = *reinterpret_cast<MScratch *>(smem + M_OFF_SCR);
+  const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+  const int H = a.H, T = a.ntok;
+  const int64_t HD = (int64_t)H * D;
+  const int items = a.N * H;
+  const int G = gridDim.x;
+  const __nv_bfloat16 *cw = reinterpret_cast<const __nv_bfloat16 *>(a.conv_w);
+  __nv_bfloat16 *cs = reinterpret_cast<__nv_bfloat16 *>(a.conv_state);
+
+  if (tid == 0) {
+    for (int i = 0; i < M_NSLOT; ++i) {
+      umma::mbar_init(&sc.full[i], 1);
+      umma::mbar_init(&sc.empty[i], NC);
+      sc.req[i] = 0;
+    }
+    umma::mbar_fence_init();
+    sc.fail = 0;
+  }
+  if (tid < H) sc.alog[tid] = a.A_log[tid];
+  const bool gated = a.ogate != nullptr;
+  if (gated && tid < D) sc.onw[tid] = a.onw[tid];
+  __syncthreads();
+
+  if (w == NC / 32) {
+    // ---------------- producer warp: everything item `it` reads, into ring slot `slot`
+    const int ncopy = 1 + 9 + 3 * T + T + 3 + 1 + 1 + (gated ? T : 0);
+    const uint32_t bytes = D * D * 4 + 9 * 256 + 4 * T * 256 + 3072 + 512 + 2 * T * H + (gated ? T * 256 : 0);
+    auto request = [&](int it, int slot) {
+      const int n = it / H, h = it % H;
+      uint8_t *base = smem + slot * M_SLOT;
+      uint64_t *bar = &sc.full[slot];
+      if (l == 0) {
+        umma::mbar_arrive_expect_tx(bar, bytes);
+        ++sc.req[slot];
+      }
+      __syncwarp();
+      for (int c = l; c < ncopy; c += 32) {
+        int k = c;
+        if (k == 0) {
+          umma::bulk_g2s(base + M_STATE, a.state + (int64_t)it * D * D, D * D * 4, bar);
+        } else if ((k -= 1) < 9) {   // conv history: slot m of tensor blk into raw row m
+          const int m = k / 3, blk = k % 3;
+          umma::bulk_g2s(base + M_RAW + blk * M_RAWT + m * 256, cs + ((int64_t)n * 3 + m) * 3 * HD + blk * HD + h * D,
+                         256, bar);
+        } else if ((k -= 9) < 3 * T) {   // token t of tensor blk into raw row 3 + t
+          const int blk = k / T, t = k % T;
+          const void *tok = blk == 0 ? a.q : (blk == 1 ? a.k : a.v);
+          umma::bulk_g2s(base + M_RAW + blk * M_RAWT + (3 + t) * 256,
+                         reinterpret_cast<const __nv_bfloat16 *>(tok) + ((int64_t)n * T + t) * HD + h * D, 256, bar);
+        } else if ((k -= 3 * T) < T) {
+          umma::bulk_g2s(base + M_ALPHA + k * 256,
+                         reinterpret_cast<const __nv_bfloat16 *>(a.alpha) + (((int64_t)n * T + k) * H + h) * D, 256, bar);
+        } else if ((k -= T) < 3) {
+          umma::bulk_g2s(base + M_W + k * 1024, cw + ((int64_t)k * HD + h * D) * KCONV, 1024, bar);
+        } else if ((k -= 3) == 0) {
+          umma::bulk_g2s(base + M_DTB, a.dt_bias + h * D, 512, bar);
+        } else if (k == 1) {   // the T rows of b of sequence n (16-byte aligned for H % 8 == 0)
+          umma::bulk_g2s(base + M_B, reinterpret_cast<const __nv_bfloat16 *>(a.b) + (int64_t)n * T * H, 2 * T * H, bar);
+        } else {
+          const int t = k - 2;
+          umma::bulk_g2s(base + M_GATE + t * 256,
+                         reinterpret_cast<const __nv_bfloat16 *>(a.ogate) + (((int64_t)n * T + t) * H + h) * D, 256, bar);
+        }
+      }
+      __syncwarp();
+    };
+    int it = blockIdx.x;
+    if (it < items) request(it, 0);
+    if (it + G < items) request(it + G, 1);
+#pragma unroll 1
+    for (int j = 0; it < items; ++j, it += G) {
+      const int slot = j & 1;
+      // item j's final state is in its slot: store it
+      int ok = l == 0 ? (int)umma::mbar_wait_bounded(&sc.empty[slot], (j >> 1) & 1, WAIT_POLLS) : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) { sc.fail = 1; break; }
+      if (l == 0) {
+        umma::bulk_s2g(a.state + (int64_t)it * D * D, smem + slot * M_SLOT + M_STATE, D * D * 4);
+        umma::bulk_commit();
+      }
+      // two items ahead, into this same slot once the store has read it
+      if (it + 2 * G < items) {
+        if (l == 0) umma::bulk_wait_read<0>();
+        __syncwarp();
+        request(it + 2 * G, slot);
+      }
+      if (*(volatile int *)&sc.fail) break;
+    }
+    if (l == 0) umma::bulk_wait<0>();
+    if (*(volatile int *)&sc.fail) {
+      if (l < M_NSLOT && sc.req[l] > 0) (void)umma::mbar_wait_bounded(&sc.full[l], (sc.req[l] - 1) & 1, WAIT_POLLS);
+    }
+  } else {
+    // ---------------- compute warps
+    const bool first = tid < D;
+    const int i = tid % D;   // q/k channel (first half) or v / gate channel (second half)
+#pragma unroll 1
+    for (int kk = 0, it = blockIdx.x; it < items; ++kk, it += G) {
+      const int slot = kk & 1;
+      const int n = it / H, h = it % H;
+      uint8_t *base = smem + slot * M_SLOT;
+      float *S_s = reinterpret_cast<float *>(base + M_STATE);
+      const bool landed = umma::mbar_wait_bounded(&sc.full[slot], (kk >> 1) & 1, WAIT_POLLS);
+      if (!umma::named_sync_and(BAR_COMPUTE, NC, landed && !*(volatile int *)&sc.fail)) {
+        if (tid == 0) sc.fail = 1;
+        break;
+      }
+      // the state, rows 16w..16w+15, columns 4l..4l+3, into registers for all T tokens
+      float S[16][4];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const float4 x = *reinterpret_cast<const float4 *>(S_s + (16 * w + r) * D + 4 * l);
+        S[r][0] = x.x; S[r][1] = x.y; S[r][2] = x.z; S[r][3] = x.w;
+      }
+      const __nv_bfloat16 *raw = reinterpret_cast<const __nv_bfloat16 *>(base + M_RAW);
+      const __nv_bfloat16 *wts = reinterpret_cast<const __nv_bfloat16 *>(base + M_W);
+#pragma unroll 1
+      for (int t = 0; t < T; ++t) {
+        const int64_t row = (int64_t)n * T + t;   // token row in the [N, T, ...] inputs
+        // 1. prologue of token t: conv4 + SiLU over raw rows t .. t+3 of the channel
+        auto conv_channel = [&](int blk) -> float {
+          const __nv_bfloat16 *wc = wts + (blk * D + i) * KCONV;
+          const __nv_bfloat16 *x = raw + (blk * (3 + MT_MAX) + t) * D + i;
+          float acc = __bfloat162float(wc[0]) * __bfloat162float(x[0]);
+          acc = fmaf(__bfloat162float(wc[1]), __bfloat162float(x[D]), acc);
+          acc = fmaf(__bfloat162float(wc[2]), __bfloat162float(x[2 * D]), acc);
+          acc = fmaf(__bfloat162float(wc[3]), __bfloat162float(x[3 * D]), acc);
+          return silu_f(acc);
+        };
+        float qv = 0.f, kv = 0.f;
+        if (first) {
+          qv = conv_channel(0);
+          kv = conv_channel(1);
+          float sq = qv * qv, sk = kv * kv;
+#pragma unroll
+          for (int off = 16; off >= 1; off >>= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+          }
+          if (l == 0) { sc.norm_part[0][w] = sq; sc.norm_part[1][w] = sk; }
+        } else {
+          sc.v[i] = conv_channel(2);
+          const float al = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base + M_ALPHA)[t * D + i]);
+          const float g = gate_f(al + reinterpret_cast<const float *>(base + M_DTB)[i], -expf(sc.alog[h]),
+                                 a.lower_bound);
+          sc.eg[i] = expf(g);
+          if (i == 0)
+            sc.beta = (a.beta2 ? 2.f : 1.f) *
+                      sigmoid_f(__bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(base + M_B)[t * H + h]));
+        }
+        umma::named_sync(BAR_COMPUTE, NC);
+        if (first) {
+          const float sq = sc.norm_part[0][0] + sc.norm_part[0][1] + sc.norm_part[0][2] + sc.norm_part[0][3];
+          const float sk = sc.norm_part[1][0] + sc.norm_part[1][1] + sc.norm_part[1][2] + sc.norm_part[1][3];
+          sc.q[i] = qv * rsqrtf(sq + a.eps);
+          sc.k[i] = kv * rsqrtf(sk + a.eps);
+        }
+        umma::named_sync(BAR_COMPUTE, NC);
+
+        // 2. decay, then the column reductions p = S'^T k and r = S'^T q
+        float p[4] = {0.f, 0.f, 0.f, 0.f}, rr[4] = {0.f, 0.f, 0.f, 0.f}, qk = 0.f;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          const int ii = 16 * w + r;
+          const float e = sc.eg[ii], k_ = sc.k[ii], q_ = sc.q[ii];
+          qk = fmaf(q_, k_, qk);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            S[r][c] *= e;
+            p[c] = fmaf(k_, S[r][c], p[c]);
+            rr[c] = fmaf(q_, S[r][c], rr[c]);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) { sc.red_p[w][4 * l + c] = p[c]; sc.red_r[w][4 * l + c] = rr[c]; }
+        if (l == 0) sc.red_qk[w] = qk;
+        umma::named_sync(BAR_COMPUTE, NC);
+        float P[4] = {0.f, 0.f, 0.f, 0.f}, R[4] = {0.f, 0.f, 0.f, 0.f}, QK = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < NC / 32; ++ww) {
+          QK += sc.red_qk[ww];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) { P[c] += sc.red_p[ww][4 * l + c]; R[c] += sc.red_r[ww][4 * l + c]; }
+        }
+        const float bt = sc.beta;
+        float dl[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) dl[c] = bt * (sc.v[4 * l + c] - P[c]);
+        if (w == 0) {
+          __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o) + (row * H + h) * D + 4 * l;
+          float ov[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) ov[c] = a.scale * fmaf(QK, dl[c], R[c]);
+          if (gated) {   // output epilogue: o_norm over the row, then the sigmoid gate
+            float ss = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) ss = fmaf(ov[c], ov[c], ss);
+#pragma unroll
+            for (int sh = 16; sh >= 1; sh >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, sh);
+            const float rn = rsqrtf(ss * (1.f / D) + a.oeps);
+            const __nv_bfloat16 *gr = reinterpret_cast<const __nv_bfloat16 *>(base + M_GATE) + t * D + 4 * l;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              ov[c] = ov[c] * rn * sc.onw[4 * l + c] * sigmoid_f(__bfloat162float(gr[c]));
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) o[c] = __float2bfloat16_rn(ov[c]);
+        }
+        // 3. S = S' + k d^T in registers; the state after this token when asked for
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          const float k_ = sc.k[16 * w + r];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) S[r][c] = fmaf(k_, dl[c], S[r][c]);
+        }
+        if (a.step_states != nullptr) {
+          float *dst = a.step_states + (row * H + h) * D * D;
+#pragma unroll
+          for (int r = 0; r < 16; ++r)
+            __stcs(reinterpret_cast<float4 *>(dst + (int64_t)(16 * w + r) * D + 4 * l),
+                   make_float4(S[r][0], S[r][1], S[r][2], S[r][3]));
+        }
+        umma::named_sync(BAR_COMPUTE, NC);   // every read of this token's shared values is done
+      }
+      // 4. the conv history after the call: raw rows T .. T+2 (channel i of q, k / of v)
+#pragma unroll
+      for (int bb = 0; bb < 2; ++bb) {
+        const int blk = first ? bb : 2;
+        if (bb == 1 && !first) break;
+#pragma unroll
+        for (int m = 0; m < 3; ++m)
+          cs[((int64_t)n * 3 + m) * 3 * HD + blk * HD + h * D + i] = raw[(blk * (3 + MT_MAX) + T + m) * D + i];
+      }
+      // 5. the final state back into the slot; the producer stores it
+#pragma unroll
+      for (int r = 0; r < 16; ++r)
+        *reinterpret_cast<float4 *>(S_s + (16 * w + r) * D + 4 * l) = make_float4(S[r][0], S[r][1], S[r][2], S[r][3]);
+      umma::fence_proxy_async_smem();
+      umma::mbar_arrive(&sc.empty[slot]);
+    }
+  }
+  __syncthreads();
+}
+
 }  // namespace dec
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
@@ -480,6 +756,18 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const int items = a.N * a.H;
     dec::decode_tma_kernel<<<items < sms ? items : sms, dec::NT, dec::SMEM_BYTES, stream>>>(a);
+    return cudaGetLastError();
+  }
+  if (a.io_dtype == KDA_BF16 && a.D == 128 && a.H % 8 == 0 && a.H <= 64 && a.ntok >= 1 &&
+      a.ntok <= dec::MT_MAX) {   // several tokens, or the per-token states
+    cudaError_t e = cudaFuncSetAttribute(dec::decode_tma_multi_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dec::M_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const int items = a.N * a.H;
+    dec::decode_tma_multi_kernel<<<items < sms ? items : sms, dec::NT, dec::M_SMEM_BYTES, stream>>>(a);
     return cudaGetLastError();
   }
   return launch_decode_simt(a, stream);
