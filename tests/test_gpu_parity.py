@@ -437,11 +437,14 @@ def test_prefill_state_snapshots(io, d, lens, every, cap):
 # ------------------------------------------------------------------ multi-token decode
 
 @pytest.mark.parametrize("io,H,N,T,gated", [("bf16", 3, 5, 2, False), ("bf16", 16, 40, 4, False),
-                                            ("bf16", 8, 6, 3, True), ("fp32", 2, 3, 4, False)])
+                                            ("bf16", 8, 6, 3, True), ("fp32", 2, 3, 4, False),
+                                            ("bf16", 64, 2, 16, True), ("bf16", 8, 3, 1, False)])
 def test_decode_multi(io, H, N, T, gated):
     """T tokens per sequence in one call (speculative-token verification): o, the state and
     conv state after the T tokens and the state after each token, against the oracle run
-    over those T tokens from the same state and conv history.  Two calls in a row."""
+    over those T tokens from the same state and conv history.  Two calls in a row.  bf16
+    with H a multiple of 8 runs the persistent multi-token kernel, here up to its limits
+    (16 tokens, 64 heads: 95 bulk copies per item; T = 1 with per-token states)."""
     d = 128
     s = W.small("dmulti", [24] * N, H=H, d=d, io_dtype=io, seed=46, s0_std=0.02)
     inp = W.make_inputs(s)
