@@ -607,15 +607,15 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
     if (p == 0) {
       if (!upper) {
         // gi 0: lo = diagonal (col 0), hi = R_1 (col 64); gi 1: hi = diagonal (col 16)
+        uint32_t vc[16];
         umma::tmem_ld16(tb + 0, va);
         umma::tmem_ld16(tb + 64, vb2);
+        umma::tmem_ld16(tb + 16, vc);
         umma::tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) v[e] = hh ? vb2[e] : va[e];
         emit(0, v, false, hh == 0);
-        umma::tmem_ld16(tb + 16, va);
-        umma::tmem_wait_ld();
-        emit(1, va, hh == 0, true);
+        emit(1, vc, hh == 0, true);
       } else if (is_q) {   // groups 2-3 of blocks 0-1: zero
 #pragma unroll
         for (int e = 0; e < 16; ++e) va[e] = 0u;
@@ -624,29 +624,29 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
       }
     } else if (!upper) {
       // gi 0: lo = R_2 (col 80), hi = R_3 (col 112); gi 1: 96 / 128
+      uint32_t vc[16], vd[16];
       umma::tmem_ld16(tb + 80, va);
       umma::tmem_ld16(tb + 112, vb2);
+      umma::tmem_ld16(tb + 96, vc);
+      umma::tmem_ld16(tb + 128, vd);
       umma::tmem_wait_ld();
 #pragma unroll
       for (int e = 0; e < 16; ++e) v[e] = hh ? vb2[e] : va[e];
       emit(0, v, false, false);
-      umma::tmem_ld16(tb + 96, va);
-      umma::tmem_ld16(tb + 128, vb2);
-      umma::tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) v[e] = hh ? vb2[e] : va[e];
+      for (int e = 0; e < 16; ++e) v[e] = hh ? vd[e] : vc[e];
       emit(1, v, false, false);
     } else {
       // gi 2: lo = diagonal (col 32), hi = R_3 (col 144); gi 3: hi = diagonal (col 48)
+      uint32_t vc[16];
       umma::tmem_ld16(tb + 32, va);
       umma::tmem_ld16(tb + 144, vb2);
+      umma::tmem_ld16(tb + 48, vc);
       umma::tmem_wait_ld();
 #pragma unroll
       for (int e = 0; e < 16; ++e) v[e] = hh ? vb2[e] : va[e];
       emit(2, v, false, hh == 0);
-      umma::tmem_ld16(tb + 48, va);
-      umma::tmem_wait_ld();
-      emit(3, va, hh == 0, true);
+      emit(3, vc, hh == 0, true);
     }
   }
   umma::fence_before_sync();
@@ -720,17 +720,18 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
     const int i = (warp & 3) * 32 + lane;   // TMEM lane: key channel (W^T) / value channel (U^T)
     const bool isW = warp < 4;
     uint8_t *dst = rec + (isW ? REC_WT : REC_U);
+    uint32_t rr[2][32];   // both column halves in flight before one wait
+    umma::tmem_ld32(tmem + lane_base + (isW ? TM_W : TM_U), rr[0]);
+    umma::tmem_ld32(tmem + lane_base + (isW ? TM_W : TM_U) + 32, rr[1]);
+    umma::tmem_wait_ld();
 #pragma unroll
     for (int c32 = 0; c32 < 2; ++c32) {
-      uint32_t rr[32];
-      umma::tmem_ld32(tmem + lane_base + (isW ? TM_W : TM_U) + c32 * 32, rr);
-      umma::tmem_wait_ld();
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t w4[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          w4[e] = pack_bf16(__uint_as_float(rr[q4 * 8 + 2 * e]), __uint_as_float(rr[q4 * 8 + 2 * e + 1]));
+          w4[e] = pack_bf16(__uint_as_float(rr[c32][q4 * 8 + 2 * e]), __uint_as_float(rr[c32][q4 * 8 + 2 * e + 1]));
         *reinterpret_cast<uint4 *>(dst + row64_off(i, c32 * 4 + q4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
     }
