@@ -76,6 +76,10 @@ constexpr uint32_t OFF_R = 32768;             // R_all: 160 rows x 128 ch: 40 KB
 constexpr uint32_t OFF_SB = 0;                // diag(beta) A_kk fp32 [64][TSS]
 constexpr uint32_t OFF_ST = 64 * TSS * 4;     // T fp32 [64][TSS]
 constexpr uint32_t OFF_TB = 35840;            // T_b [t][s] bf16, 8 KB
+// Record parts staged in their record image, then sent by one bulk store each
+// (a lane per 128-byte row would scatter 16-byte pieces over 32 rows per store):
+constexpr uint32_t OFF_AQS = 45056;           // A_qk, 8 KB (after the intra MMA, beside the solve)
+constexpr uint32_t OFF_WUS = 0;               // -W^T | U^T, 32 KB (after the W/U MMA)
 constexpr uint32_t OFF_KT = 73728;            // k e^{Gamma}: 16 KB
 constexpr uint32_t OFF_V = 90112;             // v: 16 KB (written as soon as v is known)
 // Per-channel constants of the chunk (after the prologue, which stages the conv
@@ -96,6 +100,8 @@ static_assert(OFF_ST + 64 * TSS * 4 <= OFF_TB && OFF_TB + 8192 <= OFF_KT && OFF_
               "solve scratch overlaps");
 static_assert(OFF_TB % 1024 == 0 && OFF_KT % 1024 == 0 && OFF_V % 1024 == 0 && OFF_R % 1024 == 0,
               "SW128 alignment");
+static_assert(OFF_TB + 8192 <= OFF_AQS && OFF_AQS + 8192 <= OFF_KT && OFF_WUS + 32768 <= OFF_TB &&
+              REC_U == REC_WT + 16384 && REC_WT == 0, "record staging");
 static_assert(OFF_DTB + 512 <= OFF_WTOT && C_M + 2560 <= OFF_WTOT, "constant area");
 static_assert(OFF_DTB % 16 == 0 && OFF_WCONV % 16 == 0, "bulk copy alignment");
 
@@ -588,8 +594,8 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
           const bool k0 = !zero && (!diag || s <= t), k1 = !zero && (!diag || s + 1 <= t);
           w8[e2] = pack_bf16(k0 ? __uint_as_float(v[2 * e2]) : 0.f, k1 ? __uint_as_float(v[2 * e2 + 1]) : 0.f);
         }
-        *reinterpret_cast<uint4 *>(rec + REC_AQ + tr_off(64, t, 2 * gi)) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-        *reinterpret_cast<uint4 *>(rec + REC_AQ + tr_off(64, t, 2 * gi + 1)) = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+        *reinterpret_cast<uint4 *>(smem + OFF_AQS + tr_off(64, t, 2 * gi)) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+        *reinterpret_cast<uint4 *>(smem + OFF_AQS + tr_off(64, t, 2 * gi + 1)) = make_uint4(w8[4], w8[5], w8[6], w8[7]);
       } else {      // beta_t A_kk row t, s < t, fp32 into the solve scratch
         float4 *dst = reinterpret_cast<float4 *>(sBm + t * TSS + 16 * gi);
 #pragma unroll
@@ -649,8 +655,13 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
       emit(3, vc, hh == 0, true);
     }
   }
+  umma::fence_proxy_async_smem();   // A_qk staged: visible to the bulk store
   umma::fence_before_sync();
   __syncthreads();
+  if (tid == 0) {
+    umma::bulk_s2g(rec + REC_AQ, smem + OFF_AQS, 8192);
+    umma::bulk_commit();
+  }
 
   // ---------------------------------------------------------------- T = (I + B)^{-1}
   if (warp < 4) {  // diagonal 16x16 blocks: warp = block, lane = column (lanes 16..31 mirror)
@@ -719,7 +730,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   if (ok) {
     const int i = (warp & 3) * 32 + lane;   // TMEM lane: key channel (W^T) / value channel (U^T)
     const bool isW = warp < 4;
-    uint8_t *dst = rec + (isW ? REC_WT : REC_U);
+    uint8_t *dst = smem + OFF_WUS + (isW ? REC_WT : REC_U);
     uint32_t rr[2][32];   // both column halves in flight before one wait
     umma::tmem_ld32(tmem + lane_base + (isW ? TM_W : TM_U), rr[0]);
     umma::tmem_ld32(tmem + lane_base + (isW ? TM_W : TM_U) + 32, rr[1]);
@@ -737,8 +748,14 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
     }
   }
   if (!ok && tid == 0 && a.err) atomicExch(a.err, ERR_TIMEOUT);
+  umma::fence_proxy_async_smem();   // -W^T | U^T staged: visible to the bulk store
   umma::fence_before_sync();
   __syncthreads();
+  if (tid == 0) {
+    umma::bulk_s2g(rec + REC_WT, smem + OFF_WUS, 32768);
+    umma::bulk_commit();
+    umma::bulk_wait_read<0>();   // shared memory must stay until both stores have read it
+  }
   if (warp == 0) {
     umma::fence_after_sync();
     umma::tmem_dealloc(tmem, 256);
