@@ -82,6 +82,10 @@ constexpr uint32_t OFF_AQS = 45056;           // A_qk, 8 KB (after the intra MMA
 constexpr uint32_t OFF_WUS = 0;               // -W^T | U^T, 32 KB (after the W/U MMA)
 constexpr uint32_t OFF_KT = 73728;            // k e^{Gamma}: 16 KB
 constexpr uint32_t OFF_V = 90112;             // v: 16 KB (written as soon as v is known)
+// The conv weights as the prologue reads them, [tensor][pair p][channel group cg][16 B]
+// (landed as [tensor][channel][4 taps]: a thread's 16-byte reads then fell 8-way on the
+// same banks); in the k e^{Gamma} area, which the operands fill only later.
+constexpr uint32_t OFF_WRL = OFF_KT;
 // Per-channel constants of the chunk (after the prologue, which stages the conv
 // weights and dt_bias of the head in the same bytes):
 constexpr uint32_t OFF_C = 106496;
@@ -100,6 +104,7 @@ static_assert(OFF_ST + 64 * TSS * 4 <= OFF_TB && OFF_TB + 8192 <= OFF_KT && OFF_
               "solve scratch overlaps");
 static_assert(OFF_TB % 1024 == 0 && OFF_KT % 1024 == 0 && OFF_V % 1024 == 0 && OFF_R % 1024 == 0,
               "SW128 alignment");
+static_assert(OFF_WRL + 3072 <= OFF_V, "re-laid conv weights");
 static_assert(OFF_TB + 8192 <= OFF_AQS && OFF_AQS + 8192 <= OFF_KT && OFF_WUS + 32768 <= OFF_TB &&
               REC_U == REC_WT + 16384 && REC_WT == 0, "record staging");
 static_assert(OFF_DTB + 512 <= OFF_WTOT && C_M + 2560 <= OFF_WTOT, "constant area");
@@ -311,6 +316,11 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
                              : make_uint4(0, 0, 0, 0);
     }
     ok = wait_vote(bar_tma, 0, ok);
+    if (tid < 192) {   // conv weights into the conflict-free layout (one 16-byte piece each)
+      const int blk = tid >> 6, cgw = (tid >> 2) & 15, pw = tid & 3;
+      *reinterpret_cast<uint4 *>(smem + OFF_WRL + blk * 1024 + pw * 256 + cgw * 16) =
+          *reinterpret_cast<const uint4 *>(smem + OFF_WCONV + blk * 1024 + cgw * 64 + pw * 16);
+    }
     if (hist) {
 #pragma unroll
       for (int blk = 0; blk < 3; ++blk)
@@ -319,6 +329,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
           *reinterpret_cast<uint4 *>(smem + (blk == 0 ? OFF_RAWQ : blk == 1 ? OFF_RAWK : OFF_RAWV) +
                                      m * RAW_ROW + cg * 16) = hraw[blk][m];
     }
+    __syncthreads();   // the re-laid conv weights
     // conv4 + SiLU (+ L2 norm over the head's 128 channels for q and k), two
     // channels at a time; v first, it goes straight into its operand tile
 #pragma unroll
@@ -332,7 +343,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         // taps of channels 2p and 2p+1: (t0 t1), (t2 t3) of each, 16 bytes
-        const uint4 wq = *reinterpret_cast<const uint4 *>(smem + OFF_WCONV + blk * 1024 + cg * 64 + p * 16);
+        const uint4 wq = *reinterpret_cast<const uint4 *>(smem + OFF_WRL + blk * 1024 + p * 256 + cg * 16);
         const float2 wa = bf2_f2(wq.x), wb = bf2_f2(wq.y), wc = bf2_f2(wq.z), wd = bf2_f2(wq.w);
         const float2 w0 = make_float2(wa.x, wc.x), w1 = make_float2(wa.y, wc.y);
         const float2 w2 = make_float2(wb.x, wd.x), w3 = make_float2(wb.y, wd.y);
