@@ -300,16 +300,14 @@ def run_ours(args, rank, world, local_rank):
     d2h = ho.numel() * ho.element_size() + hs.numel() * hs.element_size()
 
     # ---- max over ranks
-    stats = torch.tensor([elapsed_ms, 0.0 if args.no_e2e else e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(stats, op=torch.distributed.ReduceOp.MAX)
-    elapsed_ms, e2e_ms = float(stats[0]), float(stats[1])
-    if rank != 0:
+    from gated_delta_rule_70_b200 import dist as kdist
+    elapsed_ms, e2e_ms = kdist.max_over_ranks([elapsed_ms, 0.0 if args.no_e2e else e2e_ms], device=dev)
+    if not kdist.report_rank(rank):
         return None
 
     ms_per_step = elapsed_ms / args.steps
     tokens = T_total * world
-    value = tokens / (ms_per_step * 1e-3)
+    value = kdist.whole_job_rate(T_total, world, ms_per_step)
     flops = prefill_flops_per_token_head(d) * T_total * H
     tc_tflops = flops / (ms_per_step * 1e-3) / 1e12
     # algorithmic bytes per launch ("Rooflines"): chunk_prep reads the raw
@@ -544,9 +542,8 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from gated_delta_rule_70_b200 import dist as kdist
+    rank, world, local_rank = kdist.world_info(os.environ)
     if args.impl == "reference":
         line = run_reference(args, rank)
         if line is not None:
