@@ -27,7 +27,17 @@
  * Conventions shared by every entry point
  *   - Every pointer is a DEVICE pointer unless stated otherwise; the caller
  *     owns every buffer, including the workspace.  The library allocates no
- *     memory, keeps no global state and is thread-safe across streams.
+ *     device memory and is thread-safe across streams.  Its one piece of
+ *     global state: a dense prefill (kda_prefill, kda_prefill_gated,
+ *     kda_prefill_ex, kda_recurrence) with at least 256 chunks of 64 tokens per
+ *     sequence and at most (SMs / 2) (sequence, head) pairs runs in time
+ *     segments, chunk preparation on `stream` and the state pass of the
+ *     previous segment on a high-priority side stream created on first use per
+ *     device, with events ordering the two; `stream` waits for the last state
+ *     pass before the call's later work.  Such calls from several host threads
+ *     are serialised while they enqueue.  Under stream capture the fork to the
+ *     side stream and the join back are captured with the rest.
+ *     kda_prefill_noalloc never takes this path.
  *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
  *     legacy default stream).  Return codes report argument checks and launch
  *     errors; device-side conditions are reported by kda_prefill_status().
@@ -345,7 +355,9 @@ kda_status kda_prefill_noalloc(const kda_shape *shape,
  * kda_kernel_timing(1) makes every later kda_prefill / kda_prefill_noalloc /
  * kda_recurrence call that takes the chunk path record CUDA events on its
  * stream before chunk_prep, between chunk_prep and the state pass, and after
- * the state pass (up to 4096 calls are kept; later ones are not timed).
+ * the state pass (up to 4096 calls are kept; later ones are not timed).  In
+ * the time-segmented schedule the middle event follows the last segment's
+ * chunk_prep, so the two durations are the overlapped part and the tail.
  * kda_kernel_timing(0) stops recording and drops what was kept.
  * kda_kernel_times() waits for the recorded events, writes the mean duration
  * in milliseconds of chunk_prep to *prep_ms and of the state pass to *state_ms
