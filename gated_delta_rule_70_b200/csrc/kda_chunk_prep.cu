@@ -13,7 +13,9 @@
 //   D  = U - W S,   O = (q e^{Gamma}) S + A_qk D,   S' = diag(e^{Gamma_C}) S + (k e^{Gamma_C - Gamma})^T D.
 // This kernel writes -W^T, U^T, A_qk, q e^{Gamma}, k e^{Gamma_C - Gamma} and
 // e^{Gamma_C} of each (chunk, head) as one record, already in the
-// shared-memory image the state pass copies in.
+// shared-memory image the state pass copies in.  A_qk and -W^T | U^T are built in
+// that image in free shared memory and leave by one bulk store each; the two token-row
+// parts are stored directly (whole 256-byte rows per half-warp).
 //
 // Prologue (fused variant, the prefill entry points): the chunk's raw q, k, v
 // (with the 3 tokens before it for the causal conv) and alpha arrive by TMA;
