@@ -84,9 +84,11 @@ constexpr uint32_t OFF_AQS = 45056;           // A_qk, 8 KB (after the intra MMA
 constexpr uint32_t OFF_WUS = 0;               // -W^T | U^T, 32 KB (after the W/U MMA)
 constexpr uint32_t OFF_KT = 73728;            // k e^{Gamma}: 16 KB
 constexpr uint32_t OFF_V = 90112;             // v: 16 KB (written as soon as v is known)
-// The conv weights as the prologue reads them, [tensor][pair p][channel group cg][16 B]
-// (landed as [tensor][channel][4 taps]: a thread's 16-byte reads then fell 8-way on the
-// same banks); in the k e^{Gamma} area, which the operands fill only later.
+// The conv weights as the prologue uses them: fp32 tap pairs (w_t of channels 2p and 2p+1),
+// [tensor][pair p][taps 0-1 | taps 2-3][channel group cg][16 B], 2 KB per tensor.  They land
+// as bf16 [tensor][channel][4 taps] (read as they are, a thread's 16-byte reads fell 8-way on
+// the same banks and each pair took a dozen unpacking instructions); in the k e^{Gamma}
+// area, which the operands fill only later.
 constexpr uint32_t OFF_WRL = OFF_KT;
 // Per-channel constants of the chunk (after the prologue, which stages the conv
 // weights and dt_bias of the head in the same bytes):
@@ -106,7 +108,7 @@ static_assert(OFF_ST + 64 * TSS * 4 <= OFF_TB && OFF_TB + 8192 <= OFF_KT && OFF_
               "solve scratch overlaps");
 static_assert(OFF_TB % 1024 == 0 && OFF_KT % 1024 == 0 && OFF_V % 1024 == 0 && OFF_R % 1024 == 0,
               "SW128 alignment");
-static_assert(OFF_WRL + 3072 <= OFF_V, "re-laid conv weights");
+static_assert(OFF_WRL + 3 * 2048 <= OFF_V, "re-laid conv weights");
 static_assert(OFF_TB + 8192 <= OFF_AQS && OFF_AQS + 8192 <= OFF_KT && OFF_WUS + 32768 <= OFF_TB &&
               REC_U == REC_WT + 16384 && REC_WT == 0, "record staging");
 static_assert(OFF_DTB + 512 <= OFF_WTOT && C_M + 2560 <= OFF_WTOT, "constant area");
@@ -298,7 +300,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   float2 g2[4][4];             // gate in base 2, [token][channel pair]
   float btj = 0.f;             // beta of token tid (tid < 64)
   if constexpr (kFused) {
-    const float negA2 = -expf(a.A_log[h]) * LOG2E;   // the gate is kept in base 2
+    const float negA = -expf(a.A_log[h]);
     const float lb2 = a.lower_bound * LOG2E;
     if (tid < 64 && tid < nt)
       btj = (a.beta2 ? 2.f : 1.f) *
@@ -318,10 +320,13 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
                              : make_uint4(0, 0, 0, 0);
     }
     ok = wait_vote(bar_tma, 0, ok);
-    if (tid < 192) {   // conv weights into the conflict-free layout (one 16-byte piece each)
+    if (tid < 192) {   // conv weights into fp32 tap pairs (one channel pair each)
       const int blk = tid >> 6, cgw = (tid >> 2) & 15, pw = tid & 3;
-      *reinterpret_cast<uint4 *>(smem + OFF_WRL + blk * 1024 + pw * 256 + cgw * 16) =
-          *reinterpret_cast<const uint4 *>(smem + OFF_WCONV + blk * 1024 + cgw * 64 + pw * 16);
+      const uint4 wq = *reinterpret_cast<const uint4 *>(smem + OFF_WCONV + blk * 1024 + cgw * 64 + pw * 16);
+      const float2 wa = bf2_f2(wq.x), wb = bf2_f2(wq.y), wc = bf2_f2(wq.z), wd = bf2_f2(wq.w);
+      uint8_t *dw = smem + OFF_WRL + blk * 2048 + pw * 512 + cgw * 16;
+      *reinterpret_cast<float4 *>(dw) = make_float4(wa.x, wc.x, wa.y, wc.y);         // taps 0, 1
+      *reinterpret_cast<float4 *>(dw + 256) = make_float4(wb.x, wd.x, wb.y, wd.y);   // taps 2, 3
     }
     if (hist) {
 #pragma unroll
@@ -344,11 +349,11 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
       float2 y[4][4];
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
-        // taps of channels 2p and 2p+1: (t0 t1), (t2 t3) of each, 16 bytes
-        const uint4 wq = *reinterpret_cast<const uint4 *>(smem + OFF_WRL + blk * 1024 + p * 256 + cg * 16);
-        const float2 wa = bf2_f2(wq.x), wb = bf2_f2(wq.y), wc = bf2_f2(wq.z), wd = bf2_f2(wq.w);
-        const float2 w0 = make_float2(wa.x, wc.x), w1 = make_float2(wa.y, wc.y);
-        const float2 w2 = make_float2(wb.x, wd.x), w3 = make_float2(wb.y, wd.y);
+        // tap t of channels 2p and 2p+1 as one fp32 pair w_t
+        const float4 wl = *reinterpret_cast<const float4 *>(smem + OFF_WRL + blk * 2048 + p * 512 + cg * 16);
+        const float4 wh = *reinterpret_cast<const float4 *>(smem + OFF_WRL + blk * 2048 + p * 512 + 256 + cg * 16);
+        const float2 w0 = make_float2(wl.x, wl.y), w1 = make_float2(wl.z, wl.w);
+        const float2 w2 = make_float2(wh.x, wh.y), w3 = make_float2(wh.z, wh.w);
         float2 x[7];
 #pragma unroll
         for (int r = 0; r < 7; ++r) x[r] = bf2_f2(word(xr[r], p));
@@ -382,8 +387,9 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
         else *reinterpret_cast<uint4 *>(smem + OFF_V + tr_off(64, tg * 4 + j, cg)) = packed;
       }
     }
-    // gate g = max(-exp(A_log) softplus(alpha + dt_bias), lower_bound), in base 2;
-    // softplus(x) = max(x, 0) + ln 2 * log2(1 + 2^{-|x| log2 e})
+    // gate g = max(-exp(A_log) softplus(alpha + dt_bias), lower_bound), kept in base 2:
+    // g log2(e) = -exp(A_log) log2(1 + 2^{x log2 e}).  Where the exponential overflows the
+    // gate is -inf before the clamp, which then gives the lower bound, as it should.
     float2 bias[4];
     {
       const float4 b0 = *reinterpret_cast<const float4 *>(smem + OFF_DTB + cg * 32);
@@ -398,11 +404,8 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         const float2 x = add2(bf2_f2(word(ar, p)), bias[p]);
-        const float2 e = ex2_2(mul2(make_float2(fabsf(x.x), fabsf(x.y)), f2(-LOG2E)));
-        const float2 l = add2(e, f2(1.f));
-        const float2 lg = make_float2(lg2_approx(l.x), lg2_approx(l.y));
-        const float2 sp = fma2(lg, f2(kLn2), make_float2(fmaxf(x.x, 0.f), fmaxf(x.y, 0.f)));
-        const float2 g = mul2(sp, f2(negA2));
+        const float2 l = add2(ex2_2(mul2(x, f2(LOG2E))), f2(1.f));
+        const float2 g = mul2(make_float2(lg2_approx(l.x), lg2_approx(l.y)), f2(negA));
         g2[j][p] = valid ? make_float2(fmaxf(g.x, lb2), fmaxf(g.y, lb2)) : f2(0.f);
       }
     }
