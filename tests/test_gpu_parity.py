@@ -208,6 +208,14 @@ def test_prefill_bf16_saturated_gates(lower_bound):
     check_prefill(s)
 
 
+@pytest.mark.parametrize("alpha_mu", [100.0, -100.0])
+def test_prefill_bf16_extreme_gate_inputs(alpha_mu):
+    """alpha + dt_bias far beyond where exp overflows (every gate at the lower bound) or
+    underflows (no decay): the kernels' base-2 softplus must agree with the oracle's."""
+    s = W.small("xgate", [150], H=2, d=128, seed=31, alpha_mu=alpha_mu, s0_std=0.02)
+    check_prefill(s)
+
+
 def test_prefill_in_place_state():
     """final_state may be the same buffer as initial_state."""
     s = W.small("inplace", [100, 100], H=2, d=128, seed=18, s0_std=0.02)
