@@ -15,7 +15,9 @@ larger than L2, so no flush is needed between steps.  Per-kernel durations come
 from CUDA events the library records on the launching stream between its
 kernels (kda_kernel_timing) inside the timed region.  `e2e` repeats the step through the same
 C ABI with host (pinned) inputs: H2D copies, the prefill and the D2H read of
-o and the final state are all inside its timed region.
+o and the final state are all inside its timed region, pipelined over three
+streams with two device buffer sets (one step's H2D overlaps the previous
+step's prefill and D2H).
 
 Multi-GPU (torchrun, one process per GPU): the (sequence, head) units are
 independent, so every rank runs its own batch with no data-path collective
@@ -269,30 +271,58 @@ def run_ours(args, rank, world, local_rank):
                 W.spec("prefill_4x8k"), dev, stream, args.warmup, max(3, min(args.steps, 10)), peaks,
                 gated=True)
 
-    # ---- e2e through the C ABI with host buffers
+    # ---- e2e through the C ABI with host buffers.  Pipelined over three streams with two
+    # device buffer sets: step i+1's H2D (its own stream) overlaps step i's prefill (the
+    # caller's stream) and step i's D2H (a third stream); PCIe carries both directions at
+    # once.  Every step copies its inputs in and its o and final state out; the timed
+    # region runs from the first H2D to the last D2H.
     pin = lambda t: t.detach().cpu().pin_memory()
     hq, hk, hv, ha, hb = pin(q), pin(k), pin(v), pin(alpha), pin(b)
     ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     hs = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
-    e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, 5))
-
-    def e2e_step():
-        q.copy_(hq, non_blocking=True); k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True); alpha.copy_(ha, non_blocking=True)
-        b.copy_(hb, non_blocking=True)
-        kda.prefill(q, k, v, conv_w, alpha, b, A_log, dt_bias, initial_state=S0, num_seqs=N,
-                    out=o, final_state=fs, workspace=ws, want_conv_state=False, check=False)
-        ho.copy_(o, non_blocking=True)
-        hs.copy_(fs, non_blocking=True)
-
+    e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, 10))
+    slots = [(q, k, v, alpha, b, o, fs)]
     if e2e_steps:
-        e2e_step()
+        slots.append(tuple(torch.empty_like(t) for t in slots[0]))
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    in_ready, done, out_free = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    used = [False, False]
+
+    def e2e_step(i):
+        sl = i % 2
+        dq, dk, dv, da, db, do, dfs = slots[sl]
+        with torch.cuda.stream(s_in):
+            if used[sl]:
+                s_in.wait_event(done[sl])        # step i-2's prefill has read this slot
+            for dst, src in ((dq, hq), (dk, hk), (dv, hv), (da, ha), (db, hb)):
+                dst.copy_(src, non_blocking=True)
+            in_ready[sl].record(s_in)
+        stream.wait_event(in_ready[sl])
+        if used[sl]:
+            stream.wait_event(out_free[sl])      # step i-2's outputs have left this slot
+        kda.prefill(dq, dk, dv, conv_w, da, db, A_log, dt_bias, initial_state=S0, num_seqs=N,
+                    out=do, final_state=dfs, workspace=ws, want_conv_state=False, check=False)
+        done[sl].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done[sl])
+            ho.copy_(do, non_blocking=True)
+            hs.copy_(dfs, non_blocking=True)
+            out_free[sl].record(s_out)
+        used[sl] = True
+
+    for i in range(2 if e2e_steps else 0):
+        e2e_step(i)
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    stream.wait_stream(s_in)
+    stream.wait_stream(s_out)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps if e2e_steps else float("nan")
@@ -364,7 +394,8 @@ def run_ours(args, rank, world, local_rank):
                    2 * sd.num_seqs * sd.H * sd.d * sd.d * 4 + 2 * sd.num_seqs * sd.H * sd.d * 2 * 5},
         "e2e": None if args.no_e2e else {
             "value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps,
+            "schedule": "pipelined: H2D, prefill and D2H on three streams, two device buffer sets"},
         "other_workloads": extra,
         "gpu_launches": launches_per_step * args.steps + 64,
         "clocks": clock_info,
@@ -469,13 +500,13 @@ def cpu_baseline(seconds: float = 15.0, tokens: int = None):
     L = s.seq_lens[0]
     f_par = {kk: W.as_f64(vv) for kk, vv in params.items()}
 
-    def run_seq(n, t1):
+    def run_seq(n, t1, nthreads=0):
         tok = W.make_tokens(s, n * L, n * L + t1)
         f = {kk: W.as_f64(vv) for kk, vv in tok.items()}
         t0 = time.perf_counter()
         _, _, _, used = oracle.forward([0, t1], s.H, s.d, f["q"], f["k"], f["v"], f_par["conv_w"],
                                        f["alpha"], f["b"], f_par["A_log"], f_par["dt_bias"],
-                                       state0=S0_all[n:n + 1])
+                                       state0=S0_all[n:n + 1], nthreads=nthreads)
         return time.perf_counter() - t0, used
 
     if tokens is not None:
@@ -490,9 +521,14 @@ def cpu_baseline(seconds: float = 15.0, tokens: int = None):
         done += 1
         if total >= seconds:
             break
+    one_t = 512
+    one_dt, _ = run_seq(0, one_t, nthreads=1)
     return {"value": done * L / total, "unit": "tokens/s", "cores": int(used), "kind": "oracle",
             "sample": "%d of the 4 sequences of prefill B=4 T=8192 H=32 d=128 (%d tokens x 32 heads), "
-                      "fp64 C oracle, %d threads over heads, %.1f s" % (done, done * L, used, total)}
+                      "fp64 C oracle, %d threads over heads, %.1f s" % (done, done * L, used, total),
+            "one_core": {"value": one_t / one_dt, "unit": "tokens/s", "cores": 1,
+                         "sample": "first %d tokens of sequence 0, all 32 heads, 1 thread, %.1f s"
+                                   % (one_t, one_dt)}}
 
 
 def run_reference(args, rank):
