@@ -138,6 +138,27 @@ def test_prefill_bf16_varlen_edges():
     check_prefill(s)
 
 
+@pytest.mark.parametrize("varlen", [True, False])
+def test_prefill_all_sequences_empty(varlen):
+    """Zero tokens in the whole batch: no arithmetic, so the final state and the conv history
+    are the initial ones bit for bit (zeros when none is given)."""
+    s = W.small("empty", [0, 0, 0], H=2, d=128, seed=30, s0_std=0.02, varlen=varlen)
+    inp = W.make_inputs(s)
+    conv0 = W._store(np.random.default_rng(6).standard_normal((3, 3, 3 * 2 * 128)).astype(np.float32),
+                     "bf16")
+    o, fs, fc = gpu_prefill(s, inp, conv0)
+    o_ref, s_ref, c_ref, _ = oracle_prefill(s, inp, conv0)
+    assert o.numel() == 0 and o_ref.size == 0
+    np.testing.assert_array_equal(W.from_device(fs), s_ref)
+    np.testing.assert_array_equal(W.from_device(fc), c_ref)
+    cu = _dev(inp["cu_seqlens"]) if varlen else None
+    _, fs0, fc0 = kda.prefill(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["conv_w"]),
+                              _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]),
+                              _dev(inp["dt_bias"]), cu_seqlens=cu, num_seqs=3)
+    torch.cuda.synchronize()
+    assert not W.from_device(fs0).any() and not W.from_device(fc0).any()
+
+
 def test_prefill_bf16_slow_decay():
     """alpha ~ N(-2, 1): the slow-decay distribution of the long-context workload."""
     s = W.small("slow", [300], H=2, d=128, seed=16, alpha_mu=-2.0)
