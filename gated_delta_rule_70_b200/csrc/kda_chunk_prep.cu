@@ -186,12 +186,12 @@ __device__ __forceinline__ void solve_columns(const float *sB, float *sT, int co
         const float *xrow = sT + (16 * I + 4 * m4 + e) * TSS + col;
 #pragma unroll
         for (int c = 0; c < NP; ++c)
-          y[e & 1][c] = fma2(f2(tt[e]), *reinterpret_cast<const float2 *>(xrow + 2 * c), y[e & 1][c]);
+          y[e & 1][c] = fma2(f2(-tt[e]), *reinterpret_cast<const float2 *>(xrow + 2 * c), y[e & 1][c]);
       }
     }
     __syncwarp();
 #pragma unroll
-    for (int c = 0; c < NP; ++c) *reinterpret_cast<float2 *>(dst + 2 * c) = mul2(add2(y[0][c], y[1][c]), f2(-1.f));
+    for (int c = 0; c < NP; ++c) *reinterpret_cast<float2 *>(dst + 2 * c) = add2(y[0][c], y[1][c]);   // already negated
     __syncwarp();
   }
 }
@@ -396,6 +396,8 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
       const float4 b1 = *reinterpret_cast<const float4 *>(smem + OFF_DTB + cg * 32 + 16);
       bias[0] = make_float2(b0.x, b0.y); bias[1] = make_float2(b0.z, b0.w);
       bias[2] = make_float2(b1.x, b1.y); bias[3] = make_float2(b1.z, b1.w);
+#pragma unroll
+      for (int p = 0; p < 4; ++p) bias[p] = mul2(bias[p], f2(LOG2E));   // (alpha + dt_bias) log2 e by one fma
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -403,8 +405,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
       const bool valid = 4 * tg + j < nt;
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
-        const float2 x = add2(bf2_f2(word(ar, p)), bias[p]);
-        const float2 l = add2(ex2_2(mul2(x, f2(LOG2E))), f2(1.f));
+        const float2 l = add2(ex2_2(fma2(bf2_f2(word(ar, p)), f2(LOG2E), bias[p])), f2(1.f));
         const float2 g = mul2(make_float2(lg2_approx(l.x), lg2_approx(l.y)), f2(negA));
         g2[j][p] = valid ? make_float2(fmaxf(g.x, lb2), fmaxf(g.y, lb2)) : f2(0.f);
       }
@@ -549,7 +550,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         const float2 kd = mul2(bf2_f2(word(kb[j], p)),
-                               ex2_2(add2(m[p], mul2(g2[j][p], f2(-1.f)))));   // within 2^{+-8|g|max}
+                               ex2_2(fma2(g2[j][p], f2(-1.f), m[p])));   // within 2^{+-8|g|max}
         Rd[p] = f2_bf2(kd);
         Kh[p] = f2_bf2(mul2(kd, cK[p]));
         K1[p] = blkI < 3 ? f2_bf2(mul2(kd, c1[p])) : 0u;
