@@ -44,7 +44,7 @@ sys.path.insert(0, ROOT)
 # DRAM bytes (read + write) of one chunk_prep launch on 4x8192x32, from the ncu capture in
 # profiles/chunk_prep_prefill_1x8k.md scaled by the chunk-heads (x4); None when the kernel
 # has changed since that capture.
-CHUNK_PREP_TRAFFIC_BYTES = None
+CHUNK_PREP_TRAFFIC_BYTES = 4 * (269.164288e6 + 253.294592e6)
 
 HBM_FALLBACK_GBS = 6650.0
 BF16_FALLBACK_TFLOPS = 1590.0
