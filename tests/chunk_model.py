@@ -1,0 +1,107 @@
+"""A plain fp64 numpy model of the chunked form the tensor-core kernels compute.
+
+Test infrastructure, not the oracle: the oracle runs the per-token loop of the
+AliceAI-Foundation KDA write-up ("二、KDA 线性注意力"); this model re-associates that loop
+over 64-token chunks the way the prefill kernels do, so that a CPU test can hold the
+factorisation itself against the oracle, independently of any GPU.
+
+Per chunk (length <= 64, padded with zero tokens and zero gates), per key channel c:
+
+  Gamma_t      = sum_{s <= t} g_s                         (cumulative gate, kept in base 2)
+  m_I          = Gamma after token 16 I + 7                (reference of 16-token block I)
+  L_t          = x_t 2^{Gamma_t - m_I(t)}                  (x = q or k)
+  R^(I)_s      = k_s 2^{m_I - Gamma_s}, built for s in an earlier block J as
+                 (k_s 2^{m_J - Gamma_s}) 2^{m_I - m_J}
+  A_qk[t, s]   = L_q,t . R^(I(t))_s          (s <= t)
+  A_kk[t, s]   = beta_t L_k,t . R^(I(t))_s   (s < t)
+  T            = (I + A_kk)^{-1}
+  W            = T diag(beta) (K 2^Gamma),   U = T diag(beta) V
+
+and across chunks, with S the [d_k, d_v] state:
+
+  D = U - W S;   O = (Q 2^Gamma) S + A_qk D;   S <- diag(2^{Gamma_C}) S + (K 2^{Gamma_C - Gamma})^T D.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+CH = 64   # chunk length
+SB = 16   # sub-block length
+LOG2E = 1.4426950408889634
+
+
+def block_refs(G2: np.ndarray) -> np.ndarray:
+    """References m_I [4, d_k] of a padded 64-token chunk's base-2 cumulative gate G2 [64, d_k]."""
+    return np.stack([G2[SB * I + SB // 2 - 1] for I in range(CH // SB)])
+
+
+def chunk_factors(q, k, v, g, beta, mistake=None):
+    """One padded chunk (q, k, v [64, d], g [64, d_k] natural-log gates, beta [64]) ->
+    (A_qk, W, U, Q 2^Gamma, K 2^{Gamma_C - Gamma}, 2^{Gamma_C}, the log2 exponents of every
+    L and R factor taken).  ``mistake`` plants one plausible error, for the test that shows
+    the comparison with the oracle catches it."""
+    G2 = np.cumsum(g * LOG2E, axis=0)
+    m = block_refs(G2)
+    blk = np.arange(CH) // SB
+    L_exp = G2 - m[blk]                       # exponent of every L factor
+    Lq = q * np.exp2(L_exp)
+    Lk = k * np.exp2(L_exp)
+    Rd_exp = m[blk] - G2                      # the diagonal-block R factor
+    Rd = k * np.exp2(Rd_exp)
+    exps = [L_exp, Rd_exp]
+    A_qk = np.zeros((CH, CH))
+    A_kk = np.zeros((CH, CH))
+    for I in range(CH // SB):
+        rows = slice(SB * I, SB * (I + 1))
+        R = np.zeros((CH, k.shape[1]))
+        for J in range(I + 1):
+            cols = slice(SB * J, SB * (J + 1))
+            c_exp = m[I] - m[J]               # <= 0: the later block's constant
+            if mistake == "no_block_constant":
+                c_exp = np.zeros_like(c_exp)
+            exps.append(np.broadcast_to(c_exp, (1, k.shape[1])))
+            R[cols] = Rd[cols] * np.exp2(c_exp)
+        A_qk[rows] = Lq[rows] @ R.T
+        A_kk[rows] = beta[rows, None] * (Lk[rows] @ R.T)
+    t = np.arange(CH)
+    A_qk *= t[:, None] >= t[None, :]
+    A_kk *= (t[:, None] >= t[None, :]) if mistake == "kk_diagonal" else (t[:, None] > t[None, :])
+    T = np.linalg.inv(np.eye(CH) + A_kk)
+    Kt = k * np.exp2(G2)
+    if mistake == "beta_after_T":
+        W = beta[:, None] * (T @ Kt)
+        U = beta[:, None] * (T @ v)
+    else:
+        W = T @ (beta[:, None] * Kt)
+        U = T @ (beta[:, None] * v)
+    Qt = q * np.exp2(G2)
+    Kh = k * np.exp2(G2[-1] - G2)
+    return A_qk, W, U, Qt, Kh, np.exp2(G2[-1]), exps
+
+
+def chunked_forward(cu_seqlens, q, k, v, g, beta, state0=None, mistake=None):
+    """The chunked form over packed prepared inputs (q, k, v, g [T, H, d], beta [T, H]) ->
+    (o [T, H, d], final state [N, H, d, d]), the same contract as the oracle's recurrence."""
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    T, H, d = q.shape
+    N = len(cu) - 1
+    o = np.zeros((T, H, d))
+    s1 = np.zeros((N, H, d, d))
+    for n in range(N):
+        a, z = int(cu[n]), int(cu[n + 1])
+        for h in range(H):
+            S = np.zeros((d, d)) if state0 is None else np.array(state0[n, h], dtype=np.float64)
+            for c0 in range(a, z, CH):
+                c1 = min(c0 + CH, z)
+                L = c1 - c0
+                pad = lambda x: np.concatenate([x, np.zeros((CH - L,) + x.shape[1:])])
+                A_qk, W, U, Qt, Kh, eGC, _ = chunk_factors(
+                    pad(q[c0:c1, h]), pad(k[c0:c1, h]), pad(v[c0:c1, h]), pad(g[c0:c1, h]),
+                    pad(beta[c0:c1, h]), mistake)
+                D = U - W @ S
+                O = Qt @ S + A_qk @ D
+                o[c0:c1, h] = O[:L]
+                S = eGC[:, None] * S + Kh.T @ D
+            s1[n, h] = S
+    return o, s1

@@ -1,0 +1,83 @@
+"""The chunked form of the prefill kernels (tests/chunk_model.py), in fp64, against the
+oracle's token loop; and the exponent ranges its split decay factors stay in.
+
+CPU only.  The prepared inputs are drawn directly (unit-norm q and k, gates in
+[lower_bound, 0], beta in (0, 1)), since the factorisation starts after the prologue.
+"""
+
+import numpy as np
+import pytest
+
+from oracle import oracle
+from tests import chunk_model as CM
+
+
+def prepared(lens, H, d, lb, seed, gate_lo=None):
+    rng = np.random.default_rng(seed)
+    T = int(sum(lens))
+    unit = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)
+    q = unit(rng.standard_normal((T, H, d)))
+    k = unit(rng.standard_normal((T, H, d)))
+    v = rng.standard_normal((T, H, d))
+    lo = lb if gate_lo is None else gate_lo
+    g = rng.uniform(lo, 0.0, (T, H, d))
+    g[rng.random((T, H, d)) < 0.05] = lb    # some gates sit on the bound
+    beta = rng.uniform(0.05, 1.0, (T, H))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    S0 = 0.1 * rng.standard_normal((len(lens), H, d, d))
+    return cu, q, k, v, g, beta, S0
+
+
+def rel(x, ref):
+    return np.linalg.norm(x - ref) / max(np.linalg.norm(ref), 1e-300)
+
+
+@pytest.mark.parametrize("lens,lb,seed", [([150, 64, 1, 0, 70], -5.0, 0),
+                                          ([200], -10.0, 1),
+                                          ([65, 127], -0.5, 2)])
+def test_chunked_form_equals_token_loop(lens, lb, seed):
+    """Chunks, sub-block references, T = (I + A_kk)^-1, W, U and the inter-chunk update
+    reproduce the per-token recurrence (ragged tails, an empty and a one-token sequence)."""
+    cu, q, k, v, g, beta, S0 = prepared(lens, H=2, d=16, lb=lb, seed=seed)
+    o_ref, s_ref = oracle.recurrence(cu, q, k, v, g, beta, state0=S0)
+    o, s = CM.chunked_forward(cu, q, k, v, g, beta, state0=S0)
+    assert rel(o, o_ref) < 1e-10
+    assert rel(s, s_ref) < 1e-10
+
+
+@pytest.mark.parametrize("mistake", ["no_block_constant", "kk_diagonal", "beta_after_T"])
+def test_chunked_form_comparison_catches_a_planted_mistake(mistake):
+    """The comparison is not vacuous: an R row of an earlier block without its block constant,
+    A_kk with its diagonal, or beta applied after T each break the agreement.  (Any reference
+    m_I used consistently on both sides is exact: it only moves the exponent ranges.)"""
+    cu, q, k, v, g, beta, S0 = prepared([130], H=1, d=8, lb=-2.0, seed=3)
+    o_ref, _ = oracle.recurrence(cu, q, k, v, g, beta, state0=S0)
+    o, _ = CM.chunked_forward(cu, q, k, v, g, beta, state0=S0, mistake=mistake)
+    assert rel(o, o_ref) > 1e-3
+
+
+@pytest.mark.parametrize("lb", [-5.0, -5.5, -8.0, -10.0])
+def test_split_factors_stay_in_fp32_normal_range(lb):
+    """Every L and R factor the kernels exponentiate spans at most 8 gates: |log2| <=
+    8 |lb| log2 e (2^+-116 at the path's limit of -10), so none overflows fp32 or drops
+    below its normal range (2^-126), where the special-function exponential flushes to 0."""
+    rng = np.random.default_rng(4)
+    d = 8
+    g = np.full((CM.CH, d), lb)               # the worst case: every gate on the bound
+    g[:, ::2] = rng.uniform(lb, 0.0, (CM.CH, d // 2))
+    x = np.ones((CM.CH, d))
+    *_, exps = CM.chunk_factors(x, x, x, g, np.full(CM.CH, 0.5))
+    worst = max(np.max(e) for e in exps), min(np.min(e) for e in exps)
+    bound = 8 * abs(lb) * CM.LOG2E + 1e-9
+    assert worst[0] <= bound
+    L_exp, Rd_exp = exps[0], exps[1]
+    assert np.min(L_exp) >= -bound and np.min(Rd_exp) >= -bound
+    assert bound < 126.0 or lb < -10.0
+
+
+def test_block_start_reference_would_leave_the_normal_range():
+    """Why the reference sits mid-block: from the block's start a factor spans 16 gates,
+    and at gates of -5.5 the last token's factor falls below 2^-126."""
+    span_from_start = 16 * 5.5 * CM.LOG2E
+    span_mid = 8 * 5.5 * CM.LOG2E
+    assert span_from_start > 126.0 > span_mid
