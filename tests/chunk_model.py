@@ -31,19 +31,21 @@ SB = 16   # sub-block length
 LOG2E = 1.4426950408889634
 
 
-def block_refs(G2: np.ndarray) -> np.ndarray:
-    """References m_I [4, d_k] of a padded 64-token chunk's base-2 cumulative gate G2 [64, d_k]."""
-    return np.stack([G2[SB * I + SB // 2 - 1] for I in range(CH // SB)])
+def block_refs(G2: np.ndarray, sb: int = SB) -> np.ndarray:
+    """References m_I [64 / sb, d_k] of a padded 64-token chunk's base-2 cumulative gate
+    G2 [64, d_k]: Gamma after the middle token of each sb-token block."""
+    return np.stack([G2[sb * I + sb // 2 - 1] for I in range(CH // sb)])
 
 
-def chunk_factors(q, k, v, g, beta, mistake=None):
+def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB):
     """One padded chunk (q, k, v [64, d], g [64, d_k] natural-log gates, beta [64]) ->
     (A_qk, W, U, Q 2^Gamma, K 2^{Gamma_C - Gamma}, 2^{Gamma_C}, the log2 exponents of every
     L and R factor taken).  ``mistake`` plants one plausible error, for the test that shows
-    the comparison with the oracle catches it."""
+    the comparison with the oracle catches it.  ``sb`` is the sub-block length (16 in the
+    kernels)."""
     G2 = np.cumsum(g * LOG2E, axis=0)
-    m = block_refs(G2)
-    blk = np.arange(CH) // SB
+    m = block_refs(G2, sb)
+    blk = np.arange(CH) // sb
     L_exp = G2 - m[blk]                       # exponent of every L factor
     Lq = q * np.exp2(L_exp)
     Lk = k * np.exp2(L_exp)
@@ -52,11 +54,11 @@ def chunk_factors(q, k, v, g, beta, mistake=None):
     exps = [L_exp, Rd_exp]
     A_qk = np.zeros((CH, CH))
     A_kk = np.zeros((CH, CH))
-    for I in range(CH // SB):
-        rows = slice(SB * I, SB * (I + 1))
+    for I in range(CH // sb):
+        rows = slice(sb * I, sb * (I + 1))
         R = np.zeros((CH, k.shape[1]))
         for J in range(I + 1):
-            cols = slice(SB * J, SB * (J + 1))
+            cols = slice(sb * J, sb * (J + 1))
             c_exp = m[I] - m[J]               # <= 0: the later block's constant
             if mistake == "no_block_constant":
                 c_exp = np.zeros_like(c_exp)
@@ -80,7 +82,7 @@ def chunk_factors(q, k, v, g, beta, mistake=None):
     return A_qk, W, U, Qt, Kh, np.exp2(G2[-1]), exps
 
 
-def chunked_forward(cu_seqlens, q, k, v, g, beta, state0=None, mistake=None):
+def chunked_forward(cu_seqlens, q, k, v, g, beta, state0=None, mistake=None, sb: int = SB):
     """The chunked form over packed prepared inputs (q, k, v, g [T, H, d], beta [T, H]) ->
     (o [T, H, d], final state [N, H, d, d]), the same contract as the oracle's recurrence."""
     cu = np.asarray(cu_seqlens, dtype=np.int64)
@@ -98,7 +100,7 @@ def chunked_forward(cu_seqlens, q, k, v, g, beta, state0=None, mistake=None):
                 pad = lambda x: np.concatenate([x, np.zeros((CH - L,) + x.shape[1:])])
                 A_qk, W, U, Qt, Kh, eGC, _ = chunk_factors(
                     pad(q[c0:c1, h]), pad(k[c0:c1, h]), pad(v[c0:c1, h]), pad(g[c0:c1, h]),
-                    pad(beta[c0:c1, h]), mistake)
+                    pad(beta[c0:c1, h]), mistake, sb)
                 D = U - W @ S
                 O = Qt @ S + A_qk @ D
                 o[c0:c1, h] = O[:L]

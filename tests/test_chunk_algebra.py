@@ -81,3 +81,24 @@ def test_block_start_reference_would_leave_the_normal_range():
     span_from_start = 16 * 5.5 * CM.LOG2E
     span_mid = 8 * 5.5 * CM.LOG2E
     assert span_from_start > 126.0 > span_mid
+
+
+@pytest.mark.parametrize("sb", [8, 32, 64])
+def test_chunked_form_holds_for_other_sub_block_lengths(sb):
+    """The factorisation is exact for any sub-block length; only the exponent ranges move."""
+    cu, q, k, v, g, beta, S0 = prepared([150], H=1, d=8, lb=-5.0, seed=5)
+    o_ref, s_ref = oracle.recurrence(cu, q, k, v, g, beta, state0=S0)
+    o, s = CM.chunked_forward(cu, q, k, v, g, beta, state0=S0, sb=sb)
+    assert rel(o, o_ref) < 1e-10 and rel(s, s_ref) < 1e-10
+
+
+@pytest.mark.parametrize("lb,fits", [(-5.0, True), (-5.45, True), (-5.5, False)])
+def test_32_token_sub_blocks_fit_only_near_the_default_bound(lb, fits):
+    """With 32-token sub-blocks a factor spans up to 16 gates: inside fp32's normal range
+    (|log2| < 126) at the default bound of -5 and just above it, outside from -5.5."""
+    g = np.full((CM.CH, 4), lb)
+    x = np.ones((CM.CH, 4))
+    *_, exps = CM.chunk_factors(x, x, x, g, np.full(CM.CH, 0.5), sb=32)
+    span = max(np.max(np.abs(exps[0])), np.max(np.abs(exps[1])))
+    assert (span < 126.0) == fits
+
