@@ -340,9 +340,9 @@ def run_ours(args, rank, world, local_rank):
     value = kdist.whole_job_rate(T_total, world, ms_per_step)
     flops = prefill_flops_per_token_head(d) * T_total * H
     tc_tflops = flops / (ms_per_step * 1e-3) / 1e12
-    # algorithmic bytes per launch ("Rooflines"): chunk_prep reads the raw
-    # q, k, v, alpha, b of every token and writes one record per (chunk, head); the state
-    # pass reads the records and the initial state and writes o and the final state.
+    # algorithmic bytes per launch: chunk_prep reads the raw q, k, v, alpha (4 x d x 2 B)
+    # and b (2 B) of every token-head and writes one 74,240-byte record per (chunk, head);
+    # the state pass reads the records and the initial state and writes o and the final state.
     esz = 2
     chunks = N * ((s.seq_lens[0] + 63) // 64)
     rec_written = 74240
@@ -390,6 +390,7 @@ def run_ours(args, rank, world, local_rank):
                    "tokens_per_s": sd.num_seqs / (dec_step_ms * 1e-3),
                    "output_gate_ms_per_step": dec_gated_ms,
                    "two_tokens_with_step_states_ms_per_call": dec_mtp_ms,
+                   "gpu_launches": 64 + 64 + 32,   # one per decode call, in its own timed regions
                    "two_tokens_algorithmic_bytes": decode_bytes(sd.num_seqs, sd.H, sd.d) +
                    2 * sd.num_seqs * sd.H * sd.d * sd.d * 4 + 2 * sd.num_seqs * sd.H * sd.d * 2 * 5},
         "e2e": None if args.no_e2e else {
@@ -397,7 +398,7 @@ def run_ours(args, rank, world, local_rank):
             "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps,
             "schedule": "pipelined: H2D, prefill and D2H on three streams, two device buffer sets"},
         "other_workloads": extra,
-        "gpu_launches": launches_per_step * args.steps + 64,
+        "gpu_launches": launches_per_step * args.steps,   # the timed prefill steps
         "clocks": clock_info,
         "peaks": peaks,
     }
