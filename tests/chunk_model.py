@@ -26,6 +26,8 @@ from __future__ import annotations
 
 import numpy as np
 
+from gated_delta_rule_70_b200 import workloads as W
+
 CH = 64   # chunk length
 SB = 16   # sub-block length
 LOG2E = 1.4426950408889634
@@ -37,18 +39,39 @@ def block_refs(G2: np.ndarray, sb: int = SB) -> np.ndarray:
     return np.stack([G2[sb * I + sb // 2 - 1] for I in range(CH // sb)])
 
 
-def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB):
+# where the kernels hold bf16 values (each a separate rounding site of the emulation)
+SITES = ("qkv", "LR", "A_qk", "T_b", "W", "U", "Qt", "Kh", "S_copy", "D", "o")
+
+
+def _bf16(x):
+    """Round to bf16 (nearest even), back in fp64."""
+    return W.bf16_to_f32(W.bf16_bits(np.asarray(x, dtype=np.float32))).astype(np.float64)
+
+
+def _rounder(bf16):
+    """bf16: False (no rounding), True (every site) or a collection of SITES names ->
+    site -> rounding function."""
+    on = set(SITES) if bf16 is True else set(bf16 or ())
+    assert on <= set(SITES), on - set(SITES)
+    return lambda site: _bf16 if site in on else (lambda x: x)
+
+
+def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB, bf16=False):
     """One padded chunk (q, k, v [64, d], g [64, d_k] natural-log gates, beta [64]) ->
     (A_qk, W, U, Q 2^Gamma, K 2^{Gamma_C - Gamma}, 2^{Gamma_C}, the log2 exponents of every
     L and R factor taken).  ``mistake`` plants one plausible error, for the test that shows
     the comparison with the oracle catches it.  ``sb`` is the sub-block length (16 in the
-    kernels)."""
+    kernels).  ``bf16`` rounds where the kernels hold bf16: the MMA operands L and R, T diag(beta),
+    and the record's A_qk, W, U, Q 2^Gamma and K 2^{Gamma_C - Gamma}; A_kk, T, the gates and
+    2^{Gamma_C} stay wide (fp32 in the kernels, fp64 here).  A collection of SITES names
+    rounds at those sites only."""
+    rb = _rounder(bf16)
     G2 = np.cumsum(g * LOG2E, axis=0)
     m = block_refs(G2, sb)
     blk = np.arange(CH) // sb
     L_exp = G2 - m[blk]                       # exponent of every L factor
-    Lq = q * np.exp2(L_exp)
-    Lk = k * np.exp2(L_exp)
+    Lq = rb("LR")(q * np.exp2(L_exp))
+    Lk = rb("LR")(k * np.exp2(L_exp))
     Rd_exp = m[blk] - G2                      # the diagonal-block R factor
     Rd = k * np.exp2(Rd_exp)
     exps = [L_exp, Rd_exp]
@@ -63,28 +86,35 @@ def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB):
             if mistake == "no_block_constant":
                 c_exp = np.zeros_like(c_exp)
             exps.append(np.broadcast_to(c_exp, (1, k.shape[1])))
-            R[cols] = Rd[cols] * np.exp2(c_exp)
+            R[cols] = rb("LR")(Rd[cols] * np.exp2(c_exp))
         A_qk[rows] = Lq[rows] @ R.T
         A_kk[rows] = beta[rows, None] * (Lk[rows] @ R.T)
     t = np.arange(CH)
     A_qk *= t[:, None] >= t[None, :]
     A_kk *= (t[:, None] >= t[None, :]) if mistake == "kk_diagonal" else (t[:, None] > t[None, :])
+    A_qk = rb("A_qk")(A_qk)
     T = np.linalg.inv(np.eye(CH) + A_kk)
-    Kt = k * np.exp2(G2)
+    Kt = rb("LR")(k * np.exp2(G2))
     if mistake == "beta_after_T":
         W = beta[:, None] * (T @ Kt)
         U = beta[:, None] * (T @ v)
     else:
-        W = T @ (beta[:, None] * Kt)
-        U = T @ (beta[:, None] * v)
-    Qt = q * np.exp2(G2)
-    Kh = k * np.exp2(G2[-1] - G2)
+        Tb = rb("T_b")(T * beta[None, :])            # T diag(beta)
+        W = rb("W")(Tb @ Kt)
+        U = rb("U")(Tb @ v)
+    Qt = rb("Qt")(q * np.exp2(G2))
+    Kh = rb("Kh")(k * np.exp2(G2[-1] - G2))
     return A_qk, W, U, Qt, Kh, np.exp2(G2[-1]), exps
 
 
-def chunked_forward(cu_seqlens, q, k, v, g, beta, state0=None, mistake=None, sb: int = SB):
+def chunked_forward(cu_seqlens, q, k, v, g, beta, state0=None, mistake=None, sb: int = SB,
+                    bf16=False):
     """The chunked form over packed prepared inputs (q, k, v, g [T, H, d], beta [T, H]) ->
-    (o [T, H, d], final state [N, H, d, d]), the same contract as the oracle's recurrence."""
+    (o [T, H, d], final state [N, H, d, d]), the same contract as the oracle's recurrence.
+    ``bf16`` also rounds q, k, v, the state's copy that the MMAs read, D (after U is added)
+    and o, as the kernels do; the state itself stays wide."""
+    rb = _rounder(bf16)
+    q, k, v = rb("qkv")(q), rb("qkv")(k), rb("qkv")(v)
     cu = np.asarray(cu_seqlens, dtype=np.int64)
     T, H, d = q.shape
     N = len(cu) - 1
@@ -100,10 +130,11 @@ def chunked_forward(cu_seqlens, q, k, v, g, beta, state0=None, mistake=None, sb:
                 pad = lambda x: np.concatenate([x, np.zeros((CH - L,) + x.shape[1:])])
                 A_qk, W, U, Qt, Kh, eGC, _ = chunk_factors(
                     pad(q[c0:c1, h]), pad(k[c0:c1, h]), pad(v[c0:c1, h]), pad(g[c0:c1, h]),
-                    pad(beta[c0:c1, h]), mistake, sb)
-                D = U - W @ S
-                O = Qt @ S + A_qk @ D
-                o[c0:c1, h] = O[:L]
+                    pad(beta[c0:c1, h]), mistake, sb, bf16)
+                Sb = rb("S_copy")(S)
+                D = rb("D")(U - W @ Sb)
+                O = Qt @ Sb + A_qk @ D
+                o[c0:c1, h] = rb("o")(O[:L])
                 S = eGC[:, None] * S + Kh.T @ D
             s1[n, h] = S
     return o, s1

@@ -102,3 +102,53 @@ def test_32_token_sub_blocks_fit_only_near_the_default_bound(lb, fits):
     span = max(np.max(np.abs(exps[0])), np.max(np.abs(exps[1])))
     assert (span < 126.0) == fits
 
+
+
+def _emulated_errors(s, sites=True):
+    """Largest per-(sequence, head) rel-L2 error of o and of the final state when the chunked
+    form rounds to bf16 at ``sites`` (all of the kernels' bf16 points by default), against
+    the oracle, on a workload's own inputs."""
+    from gated_delta_rule_70_b200 import workloads as W
+    inp = W.make_inputs(s)
+    f = {k: W.as_f64(v) for k, v in inp.items() if k != "cu_seqlens"}
+    cu = inp["cu_seqlens"]
+    qn, kn, vc, g, beta = oracle.prologue(cu, s.H, s.d, f["q"], f["k"], f["v"], f["conv_w"],
+                                          f["alpha"], f["b"], f["A_log"], f["dt_bias"],
+                                          lower_bound=s.lower_bound)
+    o_ref, s_ref = oracle.recurrence(cu, qn, kn, vc, g, beta, state0=f["S0"])
+    o, st = CM.chunked_forward(cu, qn, kn, vc, g, beta, state0=f["S0"], bf16=sites)
+    eo = max(rel(o[cu[n]:cu[n + 1], h], o_ref[cu[n]:cu[n + 1], h])
+             for n in range(len(cu) - 1) for h in range(s.H) if cu[n + 1] > cu[n])
+    es = max(rel(st[n, h], s_ref[n, h]) for n in range(len(cu) - 1) for h in range(s.H))
+    return eo, es
+
+
+@pytest.mark.parametrize("lens,H,seed,alpha_mu,lb,varlen", [
+    ([150, 70], 2, 5, 0.0, -5.0, True),      # the smoke check's inputs
+    ([200, 200], 4, 11, 0.0, -5.0, False),
+    ([300], 2, 16, -2.0, -5.0, False),       # slow decay
+    ([200], 2, 27, 3.0, -10.0, False),       # gates at a lower bound of -10
+])
+def test_bf16_rounding_points_fit_the_tolerance(lens, H, seed, alpha_mu, lb, varlen):
+    """The precision design: rounding to bf16 wherever the kernels hold bf16 (q, k, v after
+    the prologue, the MMA operands, T diag(beta), the record, the state's MMA copy, D and o)
+    costs between 1e-3 and 6e-3 of the oracle's o and final state, inside the 1e-2 bar with
+    room for the fp32 accumulation and the special-function approximations on top."""
+    from gated_delta_rule_70_b200 import workloads as W
+    s = W.small("emu", lens, H=H, d=128, seed=seed, s0_std=0.02, alpha_mu=alpha_mu,
+                varlen=varlen)
+    s.lower_bound = lb
+    eo, es = _emulated_errors(s)
+    assert 1e-3 < eo < 6e-3, eo
+    assert 1e-3 < es < 6e-3, es
+
+
+def test_each_bf16_site_alone_costs_about_one_rounding():
+    """No single rounding site is amplified by the factorisation: each alone stays below
+    3e-3 (bf16's unit roundoff is 2^-9 = 2e-3), and every site changes something."""
+    from gated_delta_rule_70_b200 import workloads as W
+    s = W.small("emu1", [200, 200], H=2, d=128, seed=11, s0_std=0.02)
+    for site in CM.SITES:
+        eo, es = _emulated_errors(s, [site])
+        assert max(eo, es) < 3e-3, (site, eo, es)
+        assert max(eo, es) > 1e-6, (site, eo, es)
