@@ -104,7 +104,7 @@ def test_32_token_sub_blocks_fit_only_near_the_default_bound(lb, fits):
 
 
 
-def _emulated_errors(s, sites=True):
+def _emulated_errors(s, sites=True, sb=CM.SB):
     """Largest per-(sequence, head) rel-L2 error of o and of the final state when the chunked
     form rounds to bf16 at ``sites`` (all of the kernels' bf16 points by default), against
     the oracle, on a workload's own inputs."""
@@ -116,7 +116,7 @@ def _emulated_errors(s, sites=True):
                                           f["alpha"], f["b"], f["A_log"], f["dt_bias"],
                                           lower_bound=s.lower_bound)
     o_ref, s_ref = oracle.recurrence(cu, qn, kn, vc, g, beta, state0=f["S0"])
-    o, st = CM.chunked_forward(cu, qn, kn, vc, g, beta, state0=f["S0"], bf16=sites)
+    o, st = CM.chunked_forward(cu, qn, kn, vc, g, beta, state0=f["S0"], bf16=sites, sb=sb)
     eo = max(rel(o[cu[n]:cu[n + 1], h], o_ref[cu[n]:cu[n + 1], h])
              for n in range(len(cu) - 1) for h in range(s.H) if cu[n + 1] > cu[n])
     es = max(rel(st[n, h], s_ref[n, h]) for n in range(len(cu) - 1) for h in range(s.H))
@@ -152,3 +152,16 @@ def test_each_bf16_site_alone_costs_about_one_rounding():
         eo, es = _emulated_errors(s, [site])
         assert max(eo, es) < 3e-3, (site, eo, es)
         assert max(eo, es) > 1e-6, (site, eo, es)
+
+
+@pytest.mark.parametrize("alpha_mu", [0.0, 3.0])
+def test_32_token_sub_blocks_keep_the_precision_budget(alpha_mu):
+    """At the default bound, 32-token sub-blocks round at the same sites with the same
+    budget (alpha_mu = 3 puts most gates on the bound of -5)."""
+    from gated_delta_rule_70_b200 import workloads as W
+    s = W.small("emu32", [200, 70], H=2, d=128, seed=28, s0_std=0.02, alpha_mu=alpha_mu)
+    e16 = _emulated_errors(s)
+    e32 = _emulated_errors(s, sb=32)
+    assert max(e32) < 6e-3
+    assert max(e32) < 1.1 * max(e16)
+
