@@ -14,6 +14,7 @@ import tempfile
 import pytest
 
 from oracle import oracle
+from tests import test_golden as golden
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "kda_oracle.c")
@@ -42,6 +43,42 @@ MUTATIONS = {
     "ogate_channel_shift": ("J->ogate[(row * H + h) * D + j]", "J->ogate[(row * H + h) * D + (j + 1) % D]"),
 }
 
+
+def _order_mutations(ind: str, out_lhs: str, beta: str):
+    """The loop's order changed: the output read before the write, or the prediction taken
+    before the decay (``ind``: the loop body's indentation; the forward pass and the
+    recurrence entry spell the output store and beta differently)."""
+    decay = (ind + "for (int64_t i = 0; i < D; ++i) {\n" + ind + "    double e = exp(gt[i]);\n" + ind +
+             "    for (int64_t j = 0; j < D; ++j) S[i * D + j] *= e;\n" + ind + "}\n")
+    predict = (ind + "for (int64_t j = 0; j < D; ++j) {\n" + ind + "    double acc = 0.0;\n" + ind +
+               "    for (int64_t i = 0; i < D; ++i) acc += kt[i] * S[i * D + j];\n" + ind +
+               "    p[j] = acc;\n" + ind + "}\n")
+    write = (ind + "for (int64_t i = 0; i < D; ++i)\n" + ind +
+             "    for (int64_t j = 0; j < D; ++j) S[i * D + j] += kt[i] * dl[j];\n")
+    read = (ind + "for (int64_t j = 0; j < D; ++j) {\n" + ind + "    double acc = 0.0;\n" + ind +
+            "    for (int64_t i = 0; i < D; ++i) acc += qt[i] * S[i * D + j];\n" + ind +
+            "    " + out_lhs + "\n" + ind + "}\n")
+    correct = ind + "for (int64_t j = 0; j < D; ++j) dl[j] = (vt[j] - p[j]) * " + beta + ";\n"
+    return (decay + predict + correct, predict + decay + correct), (write + read, read + write)
+
+
+_fw = _order_mutations(" " * 8, "ot[j] = J->scale * acc;", "beta")
+_rc = _order_mutations(" " * 16, "o[(row * H + h) * D + j] = scale * acc;", "bt")
+MUTATIONS["predict_before_decay"] = _fw[0]   # (_fw[1] does not apply: see below)
+MUTATIONS["predict_before_decay_rec"] = _rc[0]
+MUTATIONS["read_before_write_rec"] = _rc[1]
+# in the forward pass the output pointer is declared between the write and the read
+_WRITE = ("        for (int64_t i = 0; i < D; ++i)\n"
+          "            for (int64_t j = 0; j < D; ++j) S[i * D + j] += kt[i] * dl[j];\n")
+_READ = ("        double *ot = J->o + (row * H + h) * D;\n"
+         "        for (int64_t j = 0; j < D; ++j) {\n"
+         "            double acc = 0.0;\n"
+         "            for (int64_t i = 0; i < D; ++i) acc += qt[i] * S[i * D + j];\n"
+         "            ot[j] = J->scale * acc;\n"
+         "        }\n")
+MUTATIONS["read_before_write"] = (_WRITE + _READ, _READ + _WRITE)
+
+
 PIN_TESTS = [
     lambda: [pins.test_recurrence_matches_unrolled_product(T, D, s)
              for T, D, s in [(1, 2, 0), (3, 3, 1), (8, 4, 2)]],
@@ -60,6 +97,8 @@ PIN_TESTS = [
     pins.test_output_gate_acts_channel_by_channel,
     pins.test_output_gate_weight_is_per_channel,
     pins.test_output_gate_eps_inside_the_mean_square,
+    golden.test_hand_worked_recurrence,
+    golden.test_gate_and_beta_closed_forms,
 ]
 
 
