@@ -48,6 +48,34 @@ def _bf16(x):
     return W.bf16_to_f32(W.bf16_bits(np.asarray(x, dtype=np.float32))).astype(np.float64)
 
 
+def _tf32(x):
+    """Round to tf32 (10 explicit mantissa bits, nearest with ties away from zero, as the
+    conversion to tf32 does), back in fp64."""
+    u = np.asarray(x, dtype=np.float32).copy().view(np.uint32)
+    u = (u + np.uint32(0x1000)) & np.uint32(0xFFFFE000)
+    return u.view(np.float32).astype(np.float64)
+
+
+def blocked_inverse(A, tf32: bool = False, bf16: bool = False):
+    """(I + A)^{-1} for a strictly lower-triangular 64 x 64 A, by blocks: the 16 x 16 diagonal
+    blocks' inverses D_i by substitution, then T_ij = -D_i (A_ij D_j) for the blocks next to the
+    diagonal, then the 32 x 32 halves T_21 = -T_2 (A_21 T_1).  Every product there is a small
+    dense matrix product (tensor-core shaped); ``tf32`` (or ``bf16``) rounds their operands to
+    that type and keeps the accumulation wide."""
+    r = _tf32 if tf32 else (_bf16 if bf16 else (lambda x: x))
+    n = A.shape[0]
+    T = np.zeros_like(A)
+    for i in range(0, n, 16):
+        T[i:i + 16, i:i + 16] = np.linalg.inv(np.eye(16) + A[i:i + 16, i:i + 16])
+    for j in (0, 32):
+        i = j + 16
+        X = r(A[i:i + 16, j:j + 16]) @ r(T[j:j + 16, j:j + 16])
+        T[i:i + 16, j:j + 16] = -(r(T[i:i + 16, i:i + 16]) @ r(X))
+    X = r(A[32:, :32]) @ r(T[:32, :32])
+    T[32:, :32] = -(r(T[32:, 32:]) @ r(X))
+    return T
+
+
 def _rounder(bf16):
     """bf16: False (no rounding), True (every site) or a collection of SITES names ->
     site -> rounding function."""
@@ -56,7 +84,7 @@ def _rounder(bf16):
     return lambda site: _bf16 if site in on else (lambda x: x)
 
 
-def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB, bf16=False):
+def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB, bf16=False, solve: str = "direct"):
     """One padded chunk (q, k, v [64, d], g [64, d_k] natural-log gates, beta [64]) ->
     (A_qk, W, U, Q 2^Gamma, K 2^{Gamma_C - Gamma}, 2^{Gamma_C}, the log2 exponents of every
     L and R factor taken).  ``mistake`` plants one plausible error, for the test that shows
@@ -64,7 +92,8 @@ def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB, bf16=False):
     kernels).  ``bf16`` rounds where the kernels hold bf16: the MMA operands L and R, T diag(beta),
     and the record's A_qk, W, U, Q 2^Gamma and K 2^{Gamma_C - Gamma}; A_kk, T, the gates and
     2^{Gamma_C} stay wide (fp32 in the kernels, fp64 here).  A collection of SITES names
-    rounds at those sites only."""
+    rounds at those sites only.  ``solve``: "direct" (a plain inverse), "blocked",
+    "blocked_tf32" or "blocked_bf16" (``blocked_inverse``)."""
     rb = _rounder(bf16)
     G2 = np.cumsum(g * LOG2E, axis=0)
     m = block_refs(G2, sb)
@@ -93,7 +122,10 @@ def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB, bf16=False):
     A_qk *= t[:, None] >= t[None, :]
     A_kk *= (t[:, None] >= t[None, :]) if mistake == "kk_diagonal" else (t[:, None] > t[None, :])
     A_qk = rb("A_qk")(A_qk)
-    T = np.linalg.inv(np.eye(CH) + A_kk)
+    if solve == "direct":
+        T = np.linalg.inv(np.eye(CH) + A_kk)
+    else:
+        T = blocked_inverse(A_kk, tf32=solve == "blocked_tf32", bf16=solve == "blocked_bf16")
     Kt = rb("LR")(k * np.exp2(G2))
     if mistake == "beta_after_T":
         W = beta[:, None] * (T @ Kt)
@@ -108,7 +140,7 @@ def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB, bf16=False):
 
 
 def chunked_forward(cu_seqlens, q, k, v, g, beta, state0=None, mistake=None, sb: int = SB,
-                    bf16=False):
+                    bf16=False, solve: str = "direct"):
     """The chunked form over packed prepared inputs (q, k, v, g [T, H, d], beta [T, H]) ->
     (o [T, H, d], final state [N, H, d, d]), the same contract as the oracle's recurrence.
     ``bf16`` also rounds q, k, v, the state's copy that the MMAs read, D (after U is added)
@@ -130,7 +162,7 @@ def chunked_forward(cu_seqlens, q, k, v, g, beta, state0=None, mistake=None, sb:
                 pad = lambda x: np.concatenate([x, np.zeros((CH - L,) + x.shape[1:])])
                 A_qk, W, U, Qt, Kh, eGC, _ = chunk_factors(
                     pad(q[c0:c1, h]), pad(k[c0:c1, h]), pad(v[c0:c1, h]), pad(g[c0:c1, h]),
-                    pad(beta[c0:c1, h]), mistake, sb, bf16)
+                    pad(beta[c0:c1, h]), mistake, sb, bf16, solve)
                 Sb = rb("S_copy")(S)
                 D = rb("D")(U - W @ Sb)
                 O = Qt @ Sb + A_qk @ D
