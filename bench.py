@@ -524,12 +524,41 @@ def cpu_baseline(seconds: float = 15.0, tokens: int = None):
             break
     one_t = 512
     one_dt, _ = run_seq(0, one_t, nthreads=1)
+    dec = cpu_decode_baseline()
     return {"value": done * L / total, "unit": "tokens/s", "cores": int(used), "kind": "oracle",
             "sample": "%d of the 4 sequences of prefill B=4 T=8192 H=32 d=128 (%d tokens x 32 heads), "
                       "fp64 C oracle, %d threads over heads, %.1f s" % (done, done * L, used, total),
             "one_core": {"value": one_t / one_dt, "unit": "tokens/s", "cores": 1,
                          "sample": "first %d tokens of sequence 0, all 32 heads, 1 thread, %.1f s"
-                                   % (one_t, one_dt)}}
+                                   % (one_t, one_dt)},
+            "decode": dec}
+
+
+def cpu_decode_baseline(seqs: int = 32, steps: int = 4):
+    """The fp64 oracle on a bounded sample of the decode workload (256 sequences x 32 heads,
+    d=128): its first ``seqs`` sequences, all heads, ``steps`` decode steps from an N(0, 0.02)
+    state and conv history (the cost does not depend on their values).  Tokens/s counts one
+    token per sequence per step, as the GPU decode figure does."""
+    from gated_delta_rule_70_b200 import workloads as W
+    from oracle import oracle
+
+    sd = W.spec("decode_256")
+    H, d = sd.H, sd.d
+    par = {kk: W.as_f64(vv) for kk, vv in W.make_params(sd).items()}
+    rng = np.random.default_rng(0)
+    state = 0.02 * rng.standard_normal((seqs, H, d, d))
+    conv = W.as_f64(W.bf16_bits(rng.standard_normal((seqs, 3, 3 * H * d)).astype(np.float32)))
+    total = 0.0
+    for i in range(steps):
+        x = {kk: W.as_f64(vv)[:seqs] for kk, vv in W.make_decode_step(sd, i).items()}
+        t0 = time.perf_counter()
+        _, state, conv = oracle.decode_step(H, d, state, conv, x["q"], x["k"], x["v"], x["alpha"],
+                                            x["b"], par["conv_w"], par["A_log"], par["dt_bias"])
+        total += time.perf_counter() - t0
+    return {"value": seqs * steps / total, "unit": "tokens/s", "cores": int(os.cpu_count() or 1),
+            "kind": "oracle",
+            "sample": "decode 256 seqs x 32 heads, d=128: first %d sequences, all heads, %d steps, "
+                      "fp64 C oracle, threads over heads, %.2f s" % (seqs, steps, total)}
 
 
 def run_reference(args, rank):
