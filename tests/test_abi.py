@@ -160,3 +160,17 @@ def test_decode_multi_validation(lib):
     sh = kda.make_shape(2, 4, 2, 128, torch.bfloat16)
     assert lib.kda_decode_multi(ctypes.byref(sh), x, x, x, x, x, x, x, x, None, x, x, x, P(260),
                                 None) == kda.KDA_ERR_INVALID_ARGUMENT
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """Without libkda.so every call raises: there is no host fallback to run instead."""
+    import torch
+    monkeypatch.setattr(kda, "_LIB_PATH", os.path.join(ROOT, "no_such_dir", "libkda.so"))
+    monkeypatch.setattr(kda, "_lib", None)
+    with pytest.raises(kda.KdaLibraryError):
+        kda.load_library()
+    x = torch.zeros((64, 256), dtype=torch.bfloat16)
+    with pytest.raises(kda.KdaLibraryError):
+        kda.prefill(x, x, x, torch.zeros((3, 256, 4), dtype=torch.bfloat16),
+                    torch.zeros((64, 2, 128), dtype=torch.bfloat16),
+                    torch.zeros((64, 2), dtype=torch.bfloat16), torch.zeros(2), torch.zeros((2, 128)))
