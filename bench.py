@@ -41,10 +41,10 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-# DRAM bytes (read + write) of one chunk_prep launch on 4x8192x32, from the ncu capture in
-# profiles/chunk_prep_prefill_1x8k.md scaled by the chunk-heads (x4); None when the kernel
-# has changed since that capture.
-CHUNK_PREP_TRAFFIC_BYTES = 4 * (269.164288e6 + 253.294592e6)
+# DRAM bytes (read + write) of one chunk_prep launch on 4x8192x32: an ncu capture of the
+# 1x8192x32 launch scaled by the chunk-heads (x4); None while the kernel has changed since
+# the capture.
+CHUNK_PREP_TRAFFIC_BYTES = None
 
 HBM_FALLBACK_GBS = 6650.0
 BF16_FALLBACK_TFLOPS = 1590.0
@@ -65,6 +65,19 @@ def measured_peaks():
 def prefill_flops_per_token_head(d: int, c: int = C) -> float:
     """Algorithmic flops of the chunked form per (token, head): C(3dk + 2dv) + 6 dk dv + C^2/3."""
     return c * (3 * d + 2 * d) + 6 * d * d + c * c / 3.0
+
+
+def prefill_algorithmic_bytes(tokens: int, seqs: int, H: int, d: int, esz: int = 2) -> int:
+    """The fused minimum a prefill must move: q, k, v and alpha in (4 H d), b in (H), o out
+    (H d), all in the io dtype (41,024 B per token at H = 32, d = 128 bf16), plus the fp32
+    initial and final states (2 N H d^2 x 4 B)."""
+    return tokens * (4 * H * d * esz + H * esz + H * d * esz) + 2 * seqs * H * d * d * 4
+
+
+def prologue_bytes_per_token_head(d: int, esz: int = 2) -> int:
+    """The standalone prologue: q, k, v, alpha (4 d) and b in; q, k, v out (3 d) in the io
+    dtype, g (d) and beta out in fp32: 2,310 B at d = 128 bf16."""
+    return 4 * d * esz + esz + 3 * d * esz + 4 * d + 4
 
 
 # ---------------------------------------------------------------- clocks
@@ -131,6 +144,13 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     peaks = measured_peaks()
 
+    if args.only == "decode":   # profiling run: the decode kernels on a random state
+        sd, dec_ms, dec_gated_ms, dec_mtp_ms = decode_figures(dev, torch.cuda.current_stream(dev),
+                                                              seeded=False)
+        return {"metric": "decode only (profiling run)", "ms_per_step": float(np.median(dec_ms)),
+                "output_gate_ms_per_step": dec_gated_ms,
+                "two_tokens_with_step_states_ms_per_call": dec_mtp_ms} if rank == 0 else None
+
     s = W.spec("prefill_4x8k")
     if args.batch != 4:   # profiling runs: the same distributions on fewer sequences
         s = W.Spec("prefill_%dx8k" % args.batch, "bf16", [8192] * args.batch, H=32, d=128, seed=1,
@@ -149,6 +169,13 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     ws = torch.empty(kda.prefill_workspace_size(kda.make_shape(N, s.seq_lens[0], H, d, bf), False),
                      dtype=torch.uint8, device=dev)
+
+    if args.only == "prologue":   # profiling run: the standalone prologue alone
+        pro_ms = time_prologue(q, k, v, conv_w, alpha, b, A_log, dt_bias, N, stream, args.warmup,
+                               args.steps)
+        gbs = prologue_bytes_per_token_head(d) * T_total * H / (pro_ms * 1e-3) / 1e9
+        return {"metric": "prologue only (profiling run)", "ms": pro_ms, "GB_s": gbs,
+                "frac_of_measured_hbm": gbs / peaks["hbm_gbs"]} if rank == 0 else None
 
     def step(ev=None):
         if ev is not None:
@@ -186,6 +213,11 @@ def run_ours(args, rank, world, local_rank):
     timed_calls, prep_ms, state_ms = kda.kernel_times()
     kda.kernel_timing(False)
 
+    # ---- the standalone prologue (conv4 + SiLU, L2 norm, gate, beta) on the same inputs
+    pro_ms = time_prologue(q, k, v, conv_w, alpha, b, A_log, dt_bias, N, stream, args.warmup,
+                           args.steps)
+    pro_bytes = prologue_bytes_per_token_head(d) * T_total * H
+
     if args.only == "prefill":
         clock_info = clocks.stop()
         line = {"metric": "prefill only (profiling run)", "ms_per_step": elapsed_ms / args.steps,
@@ -194,14 +226,231 @@ def run_ours(args, rank, world, local_rank):
         return line if rank == 0 else None
 
     # ---- decode workload (state from a T=1024 prefill), timed per step
+    sd, dec_ms, dec_gated_ms, dec_mtp_ms = decode_figures(dev, stream)
+    clock_info = clocks.stop()
+
+    # ---- the other prefill workloads (reported beside the headline, not in `value`)
+    extra = {}
+    if not args.no_extra:
+        for wname in ("long_256k", "varlen_32"):
+            extra[wname] = time_prefill_workload(W.spec(wname), dev, stream, args.warmup,
+                                                 max(3, min(args.steps, 5)), peaks)
+        if args.batch == 4:   # the headline prefill with the output epilogue fused in
+            extra["prefill_4x8k_output_gate"] = time_prefill_workload(
+                W.spec("prefill_4x8k"), dev, stream, args.warmup, max(3, min(args.steps, 10)), peaks,
+                gated=True)
+
+    # ---- e2e through the C ABI with host buffers.  Pipelined over three streams with two
+    # device buffer sets: step i+1's H2D (its own stream) overlaps step i's prefill (the
+    # caller's stream) and step i's D2H (a third stream); PCIe carries both directions at
+    # once.  Every step copies its inputs in and its o and final state out; the timed
+    # region runs from the first H2D to the last D2H.
+    pin = lambda t: t.detach().cpu().pin_memory()
+    hq, hk, hv, ha, hb, hS0 = pin(q), pin(k), pin(v), pin(alpha), pin(b), pin(S0)
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hs = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
+    e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, 10))
+    slots = [(q, k, v, alpha, b, S0, o, fs)]
+    if e2e_steps:
+        slots.append(tuple(torch.empty_like(t) for t in slots[0]))
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    in_ready, done, out_free = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    used = [False, False]
+
+    def e2e_step(i):
+        sl = i % 2
+        dq, dk, dv, da, db, dS0, do, dfs = slots[sl]
+        with torch.cuda.stream(s_in):
+            if used[sl]:
+                s_in.wait_event(done[sl])        # step i-2's prefill has read this slot
+            for dst, src in ((dq, hq), (dk, hk), (dv, hv), (da, ha), (db, hb), (dS0, hS0)):
+                dst.copy_(src, non_blocking=True)
+            in_ready[sl].record(s_in)
+        stream.wait_event(in_ready[sl])
+        if used[sl]:
+            stream.wait_event(out_free[sl])      # step i-2's outputs have left this slot
+        kda.prefill(dq, dk, dv, conv_w, da, db, A_log, dt_bias, initial_state=dS0, num_seqs=N,
+                    out=do, final_state=dfs, workspace=ws, want_conv_state=False, check=False)
+        done[sl].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(done[sl])
+            ho.copy_(do, non_blocking=True)
+            hs.copy_(dfs, non_blocking=True)
+            out_free[sl].record(s_out)
+        used[sl] = True
+
+    for i in range(2 if e2e_steps else 0):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    stream.wait_stream(s_in)
+    stream.wait_stream(s_out)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps if e2e_steps else float("nan")
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, ha, hb, hS0))
+    d2h = ho.numel() * ho.element_size() + hs.numel() * hs.element_size()
+
+    # ---- max over ranks
+    from gated_delta_rule_70_b200 import dist as kdist
+    elapsed_ms, e2e_ms = kdist.max_over_ranks([elapsed_ms, 0.0 if args.no_e2e else e2e_ms], device=dev)
+    if not kdist.report_rank(rank):
+        return None
+
+    ms_per_step = elapsed_ms / args.steps
+    tokens = T_total * world
+    value = kdist.whole_job_rate(T_total, world, ms_per_step)
+    flops = prefill_flops_per_token_head(d) * T_total * H
+    tc_tflops = flops / (ms_per_step * 1e-3) / 1e12
+    # Algorithmic bytes of the step (the fused minimum: inputs once, o and the states once),
+    # credited to the dominant kernel's time and to the whole step.  Beside them, each
+    # kernel's own bytes: chunk_prep reads the raw q, k, v, alpha and b and writes one
+    # 74,240-byte record per (chunk, head); the state pass reads the records and the initial
+    # state and writes o and the final state.  The records' round trip is traffic the
+    # two-kernel split adds, not algorithmic work.
+    esz = 2
+    alg_bytes = prefill_algorithmic_bytes(T_total, N, H, d, esz)
+    chunks = N * ((s.seq_lens[0] + 63) // 64)
+    rec_written = 74240
+    prep_bytes = T_total * H * (4 * d * esz + esz) + chunks * H * rec_written
+    state_bytes = chunks * H * rec_written + T_total * H * d * esz + 2 * N * H * d * d * 4
+    dominant = ("chunk_prep", prep_ms, prep_bytes) if prep_ms >= state_ms else \
+        ("state_pass", state_ms, state_bytes)
+    dom_gbs = alg_bytes / (dominant[1] * 1e-3) / 1e9 if dominant[1] > 0 else 0.0
+    dom_own_gbs = dominant[2] / (dominant[1] * 1e-3) / 1e9 if dominant[1] > 0 else 0.0
+    step_gbs = alg_bytes / (ms_per_step * 1e-3) / 1e9
+    dec_step_ms = float(np.median(dec_ms))
+    dec_bytes = decode_bytes(sd.num_seqs, sd.H, sd.d)
+    dec_gbs = dec_bytes / (dec_step_ms * 1e-3) / 1e9
+    # two tokens per call with the state after each kept: one state read, two states written
+    # (the per-token ones; the last is also the in-place state), the second token's inputs
+    mtp_bytes = decode_bytes(sd.num_seqs, sd.H, sd.d) + 2 * sd.num_seqs * sd.H * sd.d * sd.d * 4 + \
+        2 * sd.num_seqs * sd.H * sd.d * 2 * 5
+    line = {
+        "metric": "KDA prefill tokens/s and % bf16 TC peak; decode state GB/s vs HBM peak",
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "prefill B=%d T=8192 H=32 d=128 bf16 I/O fp32 state (S0~N(0,0.02))" % args.batch,
+                   "global_batch": args.batch * world, "seq_len": 8192, "heads": H, "head_dim": d,
+                   "parallelism": "dp%d (independent sequences per rank)" % world,
+                   "l2": "inputs 1.3 GB > 126 MB L2, no flush"},
+        "tc": {"algorithmic_tflops": tc_tflops, "flop_per_token_head": prefill_flops_per_token_head(d),
+               "frac_of_measured_bf16": tc_tflops / peaks["bf16_tflops"],
+               "frac_of_2250_datasheet": tc_tflops / 2250.0},
+        "kernels_ms": {"prefill_call": call_ms, "chunk_prep": prep_ms, "state_pass": state_ms,
+                       "timed_calls": timed_calls},
+        "roofline": {"kernel": dominant[0], "bound": "hbm", "achieved": dom_gbs,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dom_gbs / peaks["hbm_gbs"],
+                     "traffic": (CHUNK_PREP_TRAFFIC_BYTES * args.batch / 4
+                                 if dominant[0] == "chunk_prep" and CHUNK_PREP_TRAFFIC_BYTES else None),
+                     "algorithmic_bytes": alg_bytes,
+                     "algorithmic_bytes_rule": "41,024 B per token (q, k, v, alpha, b in; o out; "
+                                               "bf16) + 2 N H d^2 x 4 B of fp32 state",
+                     "kernel_ms": dominant[1],
+                     "step": {"ms": ms_per_step, "achieved": step_gbs,
+                              "frac": step_gbs / peaks["hbm_gbs"]},
+                     "kernel_bytes": dominant[2], "kernel_bytes_gbs": dom_own_gbs,
+                     "kernel_bytes_frac": dom_own_gbs / peaks["hbm_gbs"],
+                     "record_round_trip_bytes": 2 * chunks * H * rec_written,
+                     "peak_source": peaks["source"] + " (burst copy)"},
+        "prologue": {"kernel": "prologue_kernel (kda_prologue, standalone)", "ms": pro_ms,
+                     "algorithmic_bytes": pro_bytes,
+                     "bytes_rule": "2,310 B per token-head (q, k, v, alpha, b in; q, k, v, g, "
+                                   "beta out)",
+                     "GB_s": pro_bytes / (pro_ms * 1e-3) / 1e9,
+                     "frac_of_measured_hbm": pro_bytes / (pro_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "frac_of_8000_datasheet": pro_bytes / (pro_ms * 1e-3) / 1e9 / 8000.0},
+        "decode": {"workload": "256 seqs x 32 heads, d=128, fp32 state, 64 steps",
+                   "ms_per_step": dec_step_ms, "algorithmic_bytes": dec_bytes, "GB_s": dec_gbs,
+                   "frac_of_measured_hbm": dec_gbs / peaks["hbm_gbs"],
+                   "frac_of_8000_datasheet": dec_gbs / 8000.0,
+                   "tokens_per_s": sd.num_seqs / (dec_step_ms * 1e-3),
+                   "output_gate_ms_per_step": dec_gated_ms,
+                   "two_tokens_with_step_states_ms_per_call": dec_mtp_ms,
+                   "two_tokens_GB_s": mtp_bytes / (dec_mtp_ms * 1e-3) / 1e9,
+                   "two_tokens_frac_of_measured_hbm": mtp_bytes / (dec_mtp_ms * 1e-3) / 1e9 /
+                   peaks["hbm_gbs"],
+                   "gpu_launches": 64 + 64 + 32,   # one per decode call, in its own timed regions
+                   "two_tokens_algorithmic_bytes": mtp_bytes},
+        "e2e": None if args.no_e2e else {
+            "value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps,
+            "schedule": "pipelined: H2D, prefill and D2H on three streams, two device buffer sets"},
+        "other_workloads": extra,
+        "gpu_launches": launches_per_step * args.steps,   # the timed prefill steps
+        "clocks": clock_info,
+        "peaks": peaks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+    return line
+
+
+def time_prologue(q, k, v, conv_w, alpha, b, A_log, dt_bias, N, stream, warmup, steps):
+    """Mean ms of one kda_prologue call over the batch (outputs preallocated), CUDA events on
+    the launching stream."""
+    import torch
+    from gated_delta_rule_70_b200 import kda
+    T, H, d = alpha.shape
+    dev = q.device
+    out = tuple(torch.empty((T, H, d), dtype=q.dtype, device=dev) for _ in range(3)) + \
+        (torch.empty((T, H, d), dtype=torch.float32, device=dev),
+         torch.empty((T, H), dtype=torch.float32, device=dev), None)
+
+    def one():
+        kda.prologue(q, k, v, conv_w, alpha, b, A_log, dt_bias, num_seqs=N, out=out)
+
+    for _ in range(warmup):
+        one()
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    e[0].record(stream)
+    for _ in range(steps):
+        one()
+    e[1].record(stream)
+    torch.cuda.synchronize(dev)
+    return e[0].elapsed_time(e[1]) / steps
+
+
+def decode_figures(dev, stream, seeded=True):
+    """Decode timings on the 256 x 32 workload: 64 single-token steps (median per step), the
+    same steps with the output epilogue, and 32 two-token calls with per-token states.
+    seeded: the state comes from the workload's T=1024 prefill (else a random one, for
+    profiling runs that must hold little device memory)."""
+    import torch
+    from gated_delta_rule_70_b200 import kda
+    from gated_delta_rule_70_b200 import workloads as W
+    bf = torch.bfloat16
     sd = W.spec("decode_256")
-    dinp = W.make_inputs(sd)
     dup = lambda a: W.to_device(a, dev)
-    d_o, d_state, d_conv = kda.prefill(dup(dinp["q"]), dup(dinp["k"]), dup(dinp["v"]),
-                                       dup(dinp["conv_w"]), dup(dinp["alpha"]), dup(dinp["b"]),
-                                       dup(dinp["A_log"]), dup(dinp["dt_bias"]),
-                                       num_seqs=sd.num_seqs)
-    del dinp, d_o
+    if seeded:   # the workload's own state: a T=1024 prefill of every sequence
+        dinp = W.make_inputs(sd)
+        d_o, d_state, d_conv = kda.prefill(dup(dinp["q"]), dup(dinp["k"]), dup(dinp["v"]),
+                                           dup(dinp["conv_w"]), dup(dinp["alpha"]),
+                                           dup(dinp["b"]), dup(dinp["A_log"]),
+                                           dup(dinp["dt_bias"]), num_seqs=sd.num_seqs)
+        del dinp, d_o
+        torch.cuda.empty_cache()
+    else:        # profiling runs: an N(0, 0.02) state and conv history of the same shapes
+        rng = np.random.default_rng(0)
+        d_state = dup(0.02 * rng.standard_normal((sd.num_seqs, sd.H, sd.d, sd.d), dtype=np.float32))
+        d_conv = dup(W.bf16_bits(rng.standard_normal((sd.num_seqs, 3, 3 * sd.H * sd.d),
+                                                     dtype=np.float32)))
     dsteps = [W.make_decode_step(sd, i) for i in range(64)]
     dsteps = [{kk: dup(vv) for kk, vv in x.items()} for x in dsteps]
     d_cw, d_A, d_dt = dup(W.make_params(sd)["conv_w"]), dup(W.make_params(sd)["A_log"]), \
@@ -258,154 +507,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     dec_mtp_ms = de[0].elapsed_time(de[1]) / 32
     del mtp_x, mtp_states
-    clock_info = clocks.stop()
-
-    # ---- the other prefill workloads (reported beside the headline, not in `value`)
-    extra = {}
-    if not args.no_extra:
-        for wname in ("long_256k", "varlen_32"):
-            extra[wname] = time_prefill_workload(W.spec(wname), dev, stream, args.warmup,
-                                                 max(3, min(args.steps, 5)), peaks)
-        if args.batch == 4:   # the headline prefill with the output epilogue fused in
-            extra["prefill_4x8k_output_gate"] = time_prefill_workload(
-                W.spec("prefill_4x8k"), dev, stream, args.warmup, max(3, min(args.steps, 10)), peaks,
-                gated=True)
-
-    # ---- e2e through the C ABI with host buffers.  Pipelined over three streams with two
-    # device buffer sets: step i+1's H2D (its own stream) overlaps step i's prefill (the
-    # caller's stream) and step i's D2H (a third stream); PCIe carries both directions at
-    # once.  Every step copies its inputs in and its o and final state out; the timed
-    # region runs from the first H2D to the last D2H.
-    pin = lambda t: t.detach().cpu().pin_memory()
-    hq, hk, hv, ha, hb = pin(q), pin(k), pin(v), pin(alpha), pin(b)
-    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    hs = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
-    e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, 10))
-    slots = [(q, k, v, alpha, b, o, fs)]
-    if e2e_steps:
-        slots.append(tuple(torch.empty_like(t) for t in slots[0]))
-    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev = lambda: torch.cuda.Event()
-    in_ready, done, out_free = [ev(), ev()], [ev(), ev()], [ev(), ev()]
-    used = [False, False]
-
-    def e2e_step(i):
-        sl = i % 2
-        dq, dk, dv, da, db, do, dfs = slots[sl]
-        with torch.cuda.stream(s_in):
-            if used[sl]:
-                s_in.wait_event(done[sl])        # step i-2's prefill has read this slot
-            for dst, src in ((dq, hq), (dk, hk), (dv, hv), (da, ha), (db, hb)):
-                dst.copy_(src, non_blocking=True)
-            in_ready[sl].record(s_in)
-        stream.wait_event(in_ready[sl])
-        if used[sl]:
-            stream.wait_event(out_free[sl])      # step i-2's outputs have left this slot
-        kda.prefill(dq, dk, dv, conv_w, da, db, A_log, dt_bias, initial_state=S0, num_seqs=N,
-                    out=do, final_state=dfs, workspace=ws, want_conv_state=False, check=False)
-        done[sl].record(stream)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(done[sl])
-            ho.copy_(do, non_blocking=True)
-            hs.copy_(dfs, non_blocking=True)
-            out_free[sl].record(s_out)
-        used[sl] = True
-
-    for i in range(2 if e2e_steps else 0):
-        e2e_step(i)
-    torch.cuda.synchronize(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    s_in.wait_event(e0)
-    s_out.wait_event(e0)
-    for i in range(e2e_steps):
-        e2e_step(i)
-    stream.wait_stream(s_in)
-    stream.wait_stream(s_out)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps if e2e_steps else float("nan")
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, ha, hb))
-    d2h = ho.numel() * ho.element_size() + hs.numel() * hs.element_size()
-
-    # ---- max over ranks
-    from gated_delta_rule_70_b200 import dist as kdist
-    elapsed_ms, e2e_ms = kdist.max_over_ranks([elapsed_ms, 0.0 if args.no_e2e else e2e_ms], device=dev)
-    if not kdist.report_rank(rank):
-        return None
-
-    ms_per_step = elapsed_ms / args.steps
-    tokens = T_total * world
-    value = kdist.whole_job_rate(T_total, world, ms_per_step)
-    flops = prefill_flops_per_token_head(d) * T_total * H
-    tc_tflops = flops / (ms_per_step * 1e-3) / 1e12
-    # algorithmic bytes per launch: chunk_prep reads the raw q, k, v, alpha (4 x d x 2 B)
-    # and b (2 B) of every token-head and writes one 74,240-byte record per (chunk, head);
-    # the state pass reads the records and the initial state and writes o and the final state.
-    esz = 2
-    chunks = N * ((s.seq_lens[0] + 63) // 64)
-    rec_written = 74240
-    prep_bytes = T_total * H * (4 * d * esz + esz) + chunks * H * rec_written
-    state_bytes = chunks * H * rec_written + T_total * H * d * esz + 2 * N * H * d * d * 4
-    prep_gbs = prep_bytes / (prep_ms * 1e-3) / 1e9 if prep_ms > 0 else 0.0
-    state_gbs = state_bytes / (state_ms * 1e-3) / 1e9 if state_ms > 0 else 0.0
-    dominant = ("chunk_prep", prep_ms, prep_bytes, prep_gbs) if prep_ms >= state_ms else \
-        ("state_pass", state_ms, state_bytes, state_gbs)
-    dec_step_ms = float(np.median(dec_ms))
-    dec_bytes = decode_bytes(sd.num_seqs, sd.H, sd.d)
-    dec_gbs = dec_bytes / (dec_step_ms * 1e-3) / 1e9
-    line = {
-        "metric": "KDA prefill tokens/s and % bf16 TC peak; decode state GB/s vs HBM peak",
-        "value": value,
-        "unit": "tokens/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": ms_per_step,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": "prefill B=%d T=8192 H=32 d=128 bf16 I/O fp32 state (S0~N(0,0.02))" % args.batch,
-                   "global_batch": args.batch * world, "seq_len": 8192, "heads": H, "head_dim": d,
-                   "parallelism": "dp%d (independent sequences per rank)" % world,
-                   "l2": "inputs 1.3 GB > 126 MB L2, no flush"},
-        "tc": {"algorithmic_tflops": tc_tflops, "flop_per_token_head": prefill_flops_per_token_head(d),
-               "frac_of_measured_bf16": tc_tflops / peaks["bf16_tflops"],
-               "frac_of_2250_datasheet": tc_tflops / 2250.0},
-        "kernels_ms": {"prefill_call": call_ms, "chunk_prep": prep_ms, "state_pass": state_ms,
-                       "timed_calls": timed_calls},
-        "roofline": {"kernel": dominant[0], "bound": "hbm", "achieved": dominant[3],
-                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": dominant[3] / peaks["hbm_gbs"],
-                     "traffic": (CHUNK_PREP_TRAFFIC_BYTES * args.batch / 4
-                                 if dominant[0] == "chunk_prep" and CHUNK_PREP_TRAFFIC_BYTES else None),
-                     "algorithmic_bytes": dominant[2],
-                     "peak_source": peaks["source"] + " (burst copy)"},
-        "decode": {"workload": "256 seqs x 32 heads, d=128, fp32 state, 64 steps",
-                   "ms_per_step": dec_step_ms, "algorithmic_bytes": dec_bytes, "GB_s": dec_gbs,
-                   "frac_of_measured_hbm": dec_gbs / peaks["hbm_gbs"],
-                   "frac_of_8000_datasheet": dec_gbs / 8000.0,
-                   "tokens_per_s": sd.num_seqs / (dec_step_ms * 1e-3),
-                   "output_gate_ms_per_step": dec_gated_ms,
-                   "two_tokens_with_step_states_ms_per_call": dec_mtp_ms,
-                   "gpu_launches": 64 + 64 + 32,   # one per decode call, in its own timed regions
-                   "two_tokens_algorithmic_bytes": decode_bytes(sd.num_seqs, sd.H, sd.d) +
-                   2 * sd.num_seqs * sd.H * sd.d * sd.d * 4 + 2 * sd.num_seqs * sd.H * sd.d * 2 * 5},
-        "e2e": None if args.no_e2e else {
-            "value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps,
-            "schedule": "pipelined: H2D, prefill and D2H on three streams, two device buffer sets"},
-        "other_workloads": extra,
-        "gpu_launches": launches_per_step * args.steps,   # the timed prefill steps
-        "clocks": clock_info,
-        "peaks": peaks,
-    }
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
-    return line
-
+    return sd, dec_ms, dec_gated_ms, dec_mtp_ms
 
 def time_prefill_workload(s, dev, stream, warmup, steps, peaks, gated=False):
     """One kda_prefill over a whole workload (inputs resident in HBM), timed with CUDA
@@ -600,7 +702,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=4,
                     help="prefill sequences (the measured workload is 4; smaller only for profiling)")
-    ap.add_argument("--only", choices=["all", "prefill"], default="all")
+    ap.add_argument("--only", choices=["all", "prefill", "prologue", "decode"], default="all",
+                    help="profiling runs: one part alone (the JSON line is not a bench result)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the long (1x262144) and varlen (32 sequences) prefill workloads")

@@ -9,13 +9,7 @@
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
-namespace {
-
-using namespace kda;
-
-constexpr size_t kAlign = 256;
-
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+namespace kda {
 
 kda_status check_shape(const kda_shape *s) {
   if (s == nullptr) return KDA_ERR_INVALID_ARGUMENT;
@@ -30,6 +24,16 @@ kda_status check_shape(const kda_shape *s) {
   if (s->num_heads > 64) return KDA_ERR_UNSUPPORTED;
   return KDA_OK;
 }
+
+}  // namespace kda
+
+namespace {
+
+using namespace kda;
+
+constexpr size_t kAlign = 256;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Total packed tokens: dense N * seq_len, varlen seq_len.
 int64_t total_tokens(const kda_shape *s, const int32_t *cu) {
@@ -75,7 +79,16 @@ RecurrenceArgs make_recurrence_args(const kda_shape *s, int64_t T, const void *q
   ra.cu = cu; ra.qn = qn; ra.kn = kn; ra.vc = vc; ra.g = g; ra.beta = beta;
   ra.state0 = state0; ra.scale = s->scale; ra.o = o; ra.state1 = state1;
   ra.lower_bound = s->lower_bound;
+  ra.wait_polls = wait_polls_for(s->flags);
   return ra;
+}
+
+// The status a device status word maps to (bad cu_seqlens before a timeout).
+kda_status word_status(int word) {
+  if (word == ERR_NONE) return KDA_OK;
+  if (word & ERR_BAD_CU_SEQLENS) return KDA_ERR_INVALID_ARGUMENT;
+  if (word & (ERR_TIMEOUT_PREP | ERR_TIMEOUT_STATE | ERR_TIMEOUT_DECODE)) return KDA_ERR_TIMEOUT;
+  return KDA_ERR_CUDA;
 }
 
 }  // namespace
@@ -175,19 +188,22 @@ kda_status kda_prefill_ex(const kda_shape *shape, const kda_prefill_args *args, 
     ra.snap = args->snapshots; ra.snap_cap = args->snapshot_capacity;
     ra.snap_every = (int64_t)args->snapshot_every * 64;
   }
+  ra.side_stream = static_cast<cudaStream_t>(args->side_stream);
   return cuda_status(run_prefill(pa, ra, args->final_conv_state, varlen, ws, L, stream));
 }
 
-kda_status kda_prefill_status(const void *workspace, void *stream_) {
-  if (workspace == nullptr) return KDA_ERR_INVALID_ARGUMENT;
+kda_status kda_device_status(const int32_t *word_ptr, void *stream_) {
+  if (word_ptr == nullptr || (reinterpret_cast<uintptr_t>(word_ptr) & 3u)) return KDA_ERR_INVALID_ARGUMENT;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
   int word = 0;
-  if (cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+  if (cudaMemcpy(&word, word_ptr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
     return KDA_ERR_CUDA;
-  if (word == ERR_BAD_CU_SEQLENS) return KDA_ERR_INVALID_ARGUMENT;
-  if (word == ERR_TIMEOUT) return KDA_ERR_TIMEOUT;
-  return word == ERR_NONE ? KDA_OK : KDA_ERR_CUDA;
+  return word_status(word);
+}
+
+kda_status kda_prefill_status(const void *workspace, void *stream_) {
+  return kda_device_status(static_cast<const int32_t *>(workspace), stream_);
 }
 
 kda_status kda_prologue(const kda_shape *shape, const void *q, const void *k, const void *v,
@@ -271,29 +287,49 @@ kda_status kda_decode_multi(const kda_shape *shape, const void *q, const void *k
                             const float *A_log, const float *dt_bias,
                             const kda_output_gate *out_gate, float *state, void *conv_state,
                             void *o, float *step_states, void *stream_) {
+  kda_decode_args a;
+  std::memset(&a, 0, sizeof a);
+  a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.b = b; a.conv_w = conv_w;
+  a.A_log = A_log; a.dt_bias = dt_bias; a.out_gate = out_gate;
+  a.state = state; a.conv_state = conv_state; a.o = o; a.step_states = step_states;
+  return kda_decode_ex(shape, &a, stream_);
+}
+
+kda_status kda_decode_ex(const kda_shape *shape, const kda_decode_args *args, void *stream_) {
   kda_status st = check_shape(shape);
   if (st != KDA_OK) return st;
+  if (args == nullptr) return KDA_ERR_INVALID_ARGUMENT;
   if (shape->seq_len < 1 || shape->seq_len > 16) return KDA_ERR_INVALID_ARGUMENT;
-  if (shape->num_seqs == 0) return KDA_OK;
-  st = check_out_gate(out_gate, shape->num_seqs);
+  if (args->status != nullptr && (reinterpret_cast<uintptr_t>(args->status) & 3u))
+    return KDA_ERR_INVALID_ARGUMENT;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (shape->num_seqs == 0)
+    return args->status == nullptr ? KDA_OK
+                                   : cuda_status(cudaMemsetAsync(args->status, 0, sizeof(int32_t), stream));
+  st = check_out_gate(args->out_gate, shape->num_seqs);
   if (st != KDA_OK) return st;
-  KDA_REQUIRE(q); KDA_REQUIRE(k); KDA_REQUIRE(v); KDA_REQUIRE(alpha); KDA_REQUIRE(b);
-  KDA_REQUIRE(conv_w); KDA_REQUIRE(A_log); KDA_REQUIRE(dt_bias); KDA_REQUIRE(state);
-  KDA_REQUIRE(conv_state); KDA_REQUIRE(o); KDA_OPTIONAL(step_states);
+  KDA_REQUIRE(args->q); KDA_REQUIRE(args->k); KDA_REQUIRE(args->v); KDA_REQUIRE(args->alpha);
+  KDA_REQUIRE(args->b); KDA_REQUIRE(args->conv_w); KDA_REQUIRE(args->A_log);
+  KDA_REQUIRE(args->dt_bias); KDA_REQUIRE(args->state); KDA_REQUIRE(args->conv_state);
+  KDA_REQUIRE(args->o); KDA_OPTIONAL(args->step_states);
   DecodeArgs a;
   std::memset(&a, 0, sizeof a);
   a.N = shape->num_seqs; a.H = shape->num_heads; a.D = shape->head_dim; a.io_dtype = shape->io_dtype;
-  a.q = q; a.k = k; a.v = v; a.alpha = alpha; a.b = b; a.conv_w = conv_w;
-  a.A_log = A_log; a.dt_bias = dt_bias;
+  a.q = args->q; a.k = args->k; a.v = args->v; a.alpha = args->alpha; a.b = args->b;
+  a.conv_w = args->conv_w; a.A_log = args->A_log; a.dt_bias = args->dt_bias;
   a.lower_bound = shape->lower_bound; a.eps = shape->l2norm_eps; a.scale = shape->scale;
   a.beta2 = (shape->flags & KDA_FLAG_NEGATIVE_EIGENVALUES) != 0;
-  if (out_gate != nullptr) {
-    a.ogate = out_gate->gate; a.onw = out_gate->weight; a.oeps = out_gate->eps;
+  if (args->out_gate != nullptr) {
+    a.ogate = args->out_gate->gate; a.onw = args->out_gate->weight; a.oeps = args->out_gate->eps;
   }
   a.ntok = shape->seq_len;
-  a.step_states = step_states;
-  a.state = state; a.conv_state = conv_state; a.o = o;
-  return cuda_status(launch_decode(a, static_cast<cudaStream_t>(stream_)));
+  a.step_states = args->step_states;
+  a.state = args->state; a.conv_state = args->conv_state; a.o = args->o;
+  a.err = args->status;
+  a.wait_polls = wait_polls_for(shape->flags);
+  if (a.err != nullptr && cudaMemsetAsync(a.err, 0, sizeof(int32_t), stream) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  return cuda_status(launch_decode(a, stream));
 }
 
 const char *kda_status_string(kda_status status) {

@@ -98,7 +98,8 @@ constexpr uint32_t OFF_DTB = OFF_C + 3 * 1024;   // [128] fp32
 constexpr uint32_t C_M = OFF_C;               // m_0..m_3 (block references), Gamma_C  [5][128]
 constexpr uint32_t OFF_WTOT = OFF_C + 4096;   // per-warp gate sums [8][128], then their prefixes
 constexpr uint32_t OFF_BETA = OFF_C + 8192;   // beta[64]
-constexpr uint32_t OFF_BAR = OFF_BETA + 256;  // MMA barrier, TMA barrier, TMEM address
+constexpr uint32_t OFF_BAR = OFF_BETA + 256;  // MMA barrier, TMA barrier, TMEM address, OFF_PEND
+constexpr uint32_t OFF_PEND = OFF_BAR + 20;   // the phase a failed wait left outstanding
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 64;
 constexpr uint32_t TMA_BYTES = 3 * RAW_ROWS * RAW_ROW + CH * RAW_ROW + 3 * 1024 + 512;
 static_assert(OFF_RAWK >= RAW_ROWS * RAW_ROW && OFF_RAWV >= OFF_RAWK + RAW_ROWS * RAW_ROW &&
@@ -130,13 +131,32 @@ constexpr uint32_t TM_P = 0;
 constexpr uint32_t TM_W = 0;
 constexpr uint32_t TM_U = 64;
 
-constexpr uint32_t WAIT_POLLS = 1u << 22;
-
-__device__ __forceinline__ bool wait_vote(uint64_t *bar, uint32_t parity, bool ok) {
-  const bool mine = ok && umma::mbar_wait_bounded(bar, parity, WAIT_POLLS);
+// Bounded waits.  Each CTA has at most one asynchronous phase outstanding at a time
+// (the input copies, then each MMA commit, every one waited before the next is
+// issued).  When a wait gives up, the CTA issues nothing more, records that phase in
+// shared memory (barrier offset and parity) and, before it frees its tensor memory and
+// leaves, waits for it once more with the full limit, so no copy or MMA of this CTA can
+// still be writing when it is gone.
+// Only thread 0 issues MMAs and bulk stores and drains, and it wrote the record
+// itself; the other threads read it only after a later block barrier.
+__device__ __forceinline__ bool failed(const uint8_t *smem) {
+  return *reinterpret_cast<const volatile uint32_t *>(smem + OFF_PEND) != 0;
+}
+// CTA-wide: every thread waits (`polls` polls) and they vote; no wait once failed.
+// Returns whether this and every earlier wait succeeded.
+__device__ __forceinline__ bool vote(uint8_t *smem, uint32_t bar_off, uint32_t parity, uint32_t polls) {
+  const bool before = !failed(smem);
+  const bool mine = before && umma::mbar_wait_bounded(reinterpret_cast<uint64_t *>(smem + bar_off), parity, polls);
   const bool all = __syncthreads_and(mine) != 0;
   umma::fence_after_sync();
+  if (before && !all && threadIdx.x == 0)
+    *reinterpret_cast<volatile uint32_t *>(smem + OFF_PEND) = bar_off | parity;   // bar_off > 0
   return all;
+}
+// After a failure, thread 0 waits out the outstanding phase with the full limit.
+__device__ __forceinline__ void drain(uint8_t *smem) {
+  const uint32_t p = *reinterpret_cast<const volatile uint32_t *>(smem + OFF_PEND);
+  if (p != 0) (void)umma::mbar_wait_bounded(reinterpret_cast<uint64_t *>(smem + (p & ~7u)), p & 1u, kWaitPolls);
 }
 
 // Off-diagonal blocks of T in the columns [col, col + NC) of column block J:
@@ -240,7 +260,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
 
   extern __shared__ __align__(1024) uint8_t smem[];
   if (umma::smem_u32(smem) & 1023u) {   // the swizzled operands need a 1024-byte aligned base
-    if (threadIdx.x == 0 && a.err) atomicExch(a.err, ERR_TIMEOUT);
+    if (threadIdx.x == 0 && a.err) atomicOr(a.err, ERR_TIMEOUT_PREP);
     return;
   }
   uint8_t *rec = reinterpret_cast<uint8_t *>(a.records) + (gchunk * H + h) * (int64_t)REC_STRIDE;
@@ -263,6 +283,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
       umma::mbar_init(bar_mma, 1);
       umma::mbar_init(bar_tma, 1);
       umma::mbar_fence_init();
+      *reinterpret_cast<uint32_t *>(smem + OFF_PEND) = 0u;
     }
     __syncwarp();
     if constexpr (kFused) {
@@ -293,7 +314,6 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   __syncthreads();
   umma::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  bool ok = true;
 
   // ---------------------------------------------------------------- inputs
   uint4 qb[4], kb[4];          // bf16 q, k (normalised) of this thread's 4 tokens x 8 channels
@@ -319,7 +339,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
                                    c0p + (((int64_t)n * 3 + m) * 3 + blk) * H * DK + h * DK + cg * 8)
                              : make_uint4(0, 0, 0, 0);
     }
-    ok = wait_vote(bar_tma, 0, ok);
+    (void)vote(smem, OFF_BAR + 8, 0, a.wait_polls);   // bar_tma
     if (tid < 192) {   // conv weights into fp32 tap pairs (one channel pair each)
       const int blk = tid >> 6, cgw = (tid >> 2) & 15, pw = tid & 3;
       const uint4 wq = *reinterpret_cast<const uint4 *>(smem + OFF_WCONV + blk * 1024 + cgw * 64 + pw * 16);
@@ -575,7 +595,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
 
   // ---------------------------------------------------------------- intra MMA
   uint32_t phase = 0;
-  if (tid == 0) {
+  if (tid == 0 && !failed(smem)) {
     umma::fence_after_sync();
     const uint32_t idesc = umma::make_idesc_bf16(128, 160, 0, 0);
 #pragma unroll
@@ -584,7 +604,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
                    idesc, s > 0);
     umma::mma_commit(bar_mma);
   }
-  ok = wait_vote(bar_mma, phase, ok);
+  bool ok = vote(smem, OFF_BAR, phase, a.wait_polls);   // bar_mma
   phase ^= 1u;
 
   // ---------------------------------------------------------------- A_qk (bf16) and diag(beta) A_kk
@@ -675,7 +695,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   umma::fence_proxy_async_smem();   // A_qk staged: visible to the bulk store
   umma::fence_before_sync();
   __syncthreads();
-  if (tid == 0) {
+  if (tid == 0 && !failed(smem)) {
     umma::bulk_s2g(rec + REC_AQ, smem + OFF_AQS, 8192);
     umma::bulk_commit();
   }
@@ -730,7 +750,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   __syncthreads();
 
   // ---------------------------------------------------------------- W^T, U^T (P has been read)
-  if (tid == 0) {
+  if (tid == 0 && !failed(smem)) {
     umma::fence_after_sync();
     const uint32_t idesc_w = umma::make_idesc_bf16(128, 64, 1, 0, 1);   // -W^T: A negated
     const uint32_t idesc_u = umma::make_idesc_bf16(128, 64, 1, 0);
@@ -741,7 +761,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
     }
     umma::mma_commit(bar_mma);
   }
-  ok = wait_vote(bar_mma, phase, ok);
+  ok = vote(smem, OFF_BAR, phase, a.wait_polls);   // bar_mma
 
   // ---------------------------------------------------------------- -W^T (warps 0-3), U^T (4-7) rows
   if (ok) {
@@ -764,14 +784,18 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
       }
     }
   }
-  if (!ok && tid == 0 && a.err) atomicExch(a.err, ERR_TIMEOUT);
   umma::fence_proxy_async_smem();   // -W^T | U^T staged: visible to the bulk store
   umma::fence_before_sync();
   __syncthreads();
   if (tid == 0) {
-    umma::bulk_s2g(rec + REC_WT, smem + OFF_WUS, 32768);
-    umma::bulk_commit();
-    umma::bulk_wait_read<0>();   // shared memory must stay until both stores have read it
+    if (!failed(smem)) {
+      umma::bulk_s2g(rec + REC_WT, smem + OFF_WUS, 32768);
+      umma::bulk_commit();
+    } else {
+      drain(smem);
+      if (a.err) atomicOr(a.err, ERR_TIMEOUT_PREP);
+    }
+    umma::bulk_wait_read<0>();   // shared memory must stay until every store has read it
   }
   if (warp == 0) {
     umma::fence_after_sync();
@@ -793,7 +817,7 @@ __global__ void chunk_table_kernel(const int32_t *cu, int N, int64_t total, int3
     acc += (int32_t)((e - s + CH - 1) / CH);
   }
   chunk_cu[N] = acc;
-  if (!good && err != nullptr) atomicExch(err, ERR_BAD_CU_SEQLENS);
+  if (!good && err != nullptr) atomicOr(err, ERR_BAD_CU_SEQLENS);
 }
 
 }  // namespace prep

@@ -11,10 +11,14 @@ namespace kda {
 
 constexpr int KCONV = 4;  // causal conv kernel size; 3 history tokens
 
-// Device error word codes (kept in the first bytes of the prefill workspace).
+// Bits of the device status word (the first int32 of the prefill workspace, or a
+// decode call's status word), set with atomicOr.
 constexpr int ERR_NONE = 0;
-constexpr int ERR_BAD_CU_SEQLENS = 1;
-constexpr int ERR_TIMEOUT = 2;
+constexpr int ERR_BAD_CU_SEQLENS = KDA_STATUS_BAD_CU_SEQLENS;
+constexpr int ERR_TIMEOUT_PREP = KDA_STATUS_TIMEOUT_PREP;
+constexpr int ERR_TIMEOUT_STATE = KDA_STATUS_TIMEOUT_STATE;
+constexpr int ERR_TIMEOUT_DECODE = KDA_STATUS_TIMEOUT_DECODE;
+
 
 struct Bf16 {
   using T = __nv_bfloat16;

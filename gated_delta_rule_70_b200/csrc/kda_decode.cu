@@ -238,7 +238,6 @@ constexpr uint32_t SMEM_BYTES = OFF_SCR + sizeof(Scratch);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(SLOT % 16 == 0 && S_QKV % 16 == 0 && S_HIST % 16 == 0 && S_W % 16 == 0 && S_DTB % 16 == 0 &&
               S_B % 16 == 0 && S_GATE % 16 == 0, "bulk copy alignment");
-constexpr uint32_t WAIT_POLLS = 1u << 22;
 constexpr uint32_t BAR_COMPUTE = 1;                 // named barrier of the compute warps
 
 __global__ void __launch_bounds__(NT, 1) decode_tma_kernel(DecodeArgs a) {
@@ -312,7 +311,7 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_kernel(DecodeArgs a) {
     for (int j = 0; it < items; ++j, it += G) {
       const int slot = j % NSLOT;
       // item j's state is final in its slot: store it
-      int ok = l == 0 ? (int)umma::mbar_wait_bounded(&sc.empty[slot], (j / NSLOT) & 1, WAIT_POLLS) : 0;
+      int ok = l == 0 ? (int)umma::mbar_wait_bounded(&sc.empty[slot], (j / NSLOT) & 1, a.wait_polls) : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) { sc.fail = 1; break; }
       if (l == 0) {
@@ -332,7 +331,7 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_kernel(DecodeArgs a) {
     if (l == 0) umma::bulk_wait<0>();
     if (*(volatile int *)&sc.fail) {
       // copies requested into a slot may still be landing: wait (bounded) for each slot's last
-      if (l < NSLOT && sc.req[l] > 0) (void)umma::mbar_wait_bounded(&sc.full[l], (sc.req[l] - 1) & 1, WAIT_POLLS);
+      if (l < NSLOT && sc.req[l] > 0) (void)umma::mbar_wait_bounded(&sc.full[l], (sc.req[l] - 1) & 1, kWaitPolls);
     }
   } else {
     // ---------------- compute warps
@@ -346,7 +345,7 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_kernel(DecodeArgs a) {
       float *S_s = reinterpret_cast<float *>(base + S_STATE);
       // all compute threads agree to go on: the slot has landed and nobody failed.
       // The barrier also closes every read of the previous item's scratch values.
-      const bool landed = umma::mbar_wait_bounded(&sc.full[slot], (k / NSLOT) & 1, WAIT_POLLS);
+      const bool landed = umma::mbar_wait_bounded(&sc.full[slot], (k / NSLOT) & 1, a.wait_polls);
       if (!umma::named_sync_and(BAR_COMPUTE, NC, landed && !*(volatile int *)&sc.fail)) {
         if (tid == 0) sc.fail = 1;
         break;
@@ -469,6 +468,7 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_kernel(DecodeArgs a) {
     }
   }
   __syncthreads();
+  if (tid == 0 && *(volatile int *)&sc.fail && a.err) atomicOr(a.err, ERR_TIMEOUT_DECODE);
 }
 
 // ---------------------------------------------------------------------------
@@ -572,7 +572,7 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_multi_kernel(DecodeArgs a) {
     for (int j = 0; it < items; ++j, it += G) {
       const int slot = j & 1;
       // item j's final state is in its slot: store it
-      int ok = l == 0 ? (int)umma::mbar_wait_bounded(&sc.empty[slot], (j >> 1) & 1, WAIT_POLLS) : 0;
+      int ok = l == 0 ? (int)umma::mbar_wait_bounded(&sc.empty[slot], (j >> 1) & 1, a.wait_polls) : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) { sc.fail = 1; break; }
       if (l == 0) {
@@ -589,7 +589,7 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_multi_kernel(DecodeArgs a) {
     }
     if (l == 0) umma::bulk_wait<0>();
     if (*(volatile int *)&sc.fail) {
-      if (l < M_NSLOT && sc.req[l] > 0) (void)umma::mbar_wait_bounded(&sc.full[l], (sc.req[l] - 1) & 1, WAIT_POLLS);
+      if (l < M_NSLOT && sc.req[l] > 0) (void)umma::mbar_wait_bounded(&sc.full[l], (sc.req[l] - 1) & 1, kWaitPolls);
     }
   } else {
     // ---------------- compute warps
@@ -601,7 +601,7 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_multi_kernel(DecodeArgs a) {
       const int n = it / H, h = it % H;
       uint8_t *base = smem + slot * M_SLOT;
       float *S_s = reinterpret_cast<float *>(base + M_STATE);
-      const bool landed = umma::mbar_wait_bounded(&sc.full[slot], (kk >> 1) & 1, WAIT_POLLS);
+      const bool landed = umma::mbar_wait_bounded(&sc.full[slot], (kk >> 1) & 1, a.wait_polls);
       if (!umma::named_sync_and(BAR_COMPUTE, NC, landed && !*(volatile int *)&sc.fail)) {
         if (tid == 0) sc.fail = 1;
         break;
@@ -741,6 +741,7 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_multi_kernel(DecodeArgs a) {
     }
   }
   __syncthreads();
+  if (tid == 0 && *(volatile int *)&sc.fail && a.err) atomicOr(a.err, ERR_TIMEOUT_DECODE);
 }
 
 }  // namespace dec

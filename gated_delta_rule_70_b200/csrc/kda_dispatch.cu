@@ -47,44 +47,30 @@ bool clock_begin() {
 }
 
 // Time segments: when a dense batch has few (sequence, head) chains, the state pass
-// occupies few SMs for a long time while the rest idle.  The chunks are then split
-// into segments of kSegChunks: chunk_prep of segment s+1 runs on the caller's stream
-// while the state pass of segment s runs on a high-priority side stream (the state
-// passes carry the state from one segment to the next through final_state).  Only
-// stream order and events connect the two: no kernel waits on another.  (Measured on
-// the 1 x 262144 x 32 prefill: segments of 32, 64, 128, 256 and 512 chunks gave 12.3,
-// 10.9, 10.1, 10.2 and 10.6 ms.)
+// occupies few SMs for a long time while the rest idle.  Given a side stream by the
+// caller, the chunks are then split into segments of kSegChunks: chunk_prep of segment
+// s+1 runs on the caller's stream while the state pass of segment s runs on the side
+// stream (the state passes carry the state from one segment to the next through
+// final_state).  Only stream order and two events, created and released by the call,
+// connect the two: no kernel waits on another.  (Measured on the 1 x 262144 x 32
+// prefill: segments of 32, 64, 128, 256 and 512 chunks gave 12.3, 10.9, 10.1, 10.2 and
+// 10.6 ms.)
 constexpr int kSegChunks = 128;
 
-struct SideStreams {
-  std::mutex mu;               // held while one call enqueues its segments
-  cudaStream_t stream[64] = {};
-  cudaEvent_t prep_done[64] = {}, pass_done[64] = {};
-  int sms[64] = {};
-};
-SideStreams g_side;
-
-// The side stream, its two events and the SM count of the current device (created once).
-cudaError_t side_resources(int &dev, cudaStream_t &side, cudaEvent_t &ev_prep, cudaEvent_t &ev_pass, int &sms) {
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (g_side.stream[dev] == nullptr) {
-    int lo = 0, hi = 0;
-    if ((e = cudaDeviceGetStreamPriorityRange(&lo, &hi)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&g_side.sms[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-      return e;
-    if ((e = cudaEventCreateWithFlags(&g_side.prep_done[dev], cudaEventDisableTiming)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&g_side.pass_done[dev], cudaEventDisableTiming)) != cudaSuccess) return e;
-    if ((e = cudaStreamCreateWithPriority(&g_side.stream[dev], cudaStreamNonBlocking, hi)) != cudaSuccess)
-      return e;
+// The call's two events (prep of a segment done; the last state pass done).
+struct SegEvents {
+  cudaEvent_t prep = nullptr, pass = nullptr;
+  cudaError_t create() {
+    cudaError_t e = cudaEventCreateWithFlags(&prep, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&pass, cudaEventDisableTiming);
+    return e;
   }
-  side = g_side.stream[dev];
-  ev_prep = g_side.prep_done[dev];
-  ev_pass = g_side.pass_done[dev];
-  sms = g_side.sms[dev];
-  return cudaSuccess;
-}
+  // (an event may be destroyed while work that records or waits on it is pending)
+  ~SegEvents() {
+    if (prep) cudaEventDestroy(prep);
+    if (pass) cudaEventDestroy(pass);
+  }
+};
 
 cudaError_t run_chunk_path(PrepArgs pa, const RecurrenceArgs &ra, bool varlen, bool fused,
                            const PrologueArgs *raw, char *ws, const WsLayout &L,
@@ -98,11 +84,12 @@ cudaError_t run_chunk_path(PrepArgs pa, const RecurrenceArgs &ra, bool varlen, b
   const int64_t slots = max_chunk_slots(ra.N, ra.total_tokens, ra.seq_len, varlen);
   pa.N = ra.N; pa.H = ra.H; pa.seq_len = ra.seq_len; pa.total_tokens = ra.total_tokens;
   pa.cu = ra.cu; pa.chunk_cu = chunk_cu;
-  pa.records = ws + L.records; pa.err = ra.err;
+  pa.records = ws + L.records; pa.err = ra.err; pa.wait_polls = ra.wait_polls;
   StateArgs sa{};
   sa.N = ra.N; sa.H = ra.H; sa.seq_len = ra.seq_len; sa.total_tokens = ra.total_tokens;
   sa.cu = ra.cu; sa.chunk_cu = chunk_cu; sa.records = ws + L.records; sa.max_slots = slots;
   sa.state0 = ra.state0; sa.scale = ra.scale; sa.o = ra.o; sa.state1 = ra.state1; sa.err = ra.err;
+  sa.wait_polls = ra.wait_polls;
   sa.seg_c0 = 0; sa.seg_c1 = INT_MAX;
   if (ra.ogate != nullptr) { sa.onw = ra.onw; sa.oeps = ra.oeps; }
   if (ra.snap != nullptr) { sa.snap = ra.snap; sa.snap_chunks = (int)(ra.snap_every / 64); sa.snap_cap = ra.snap_cap; }
@@ -110,16 +97,16 @@ cudaError_t run_chunk_path(PrepArgs pa, const RecurrenceArgs &ra, bool varlen, b
   const void *rv = raw ? raw->v : nullptr, *ralpha = raw ? raw->alpha : nullptr;
 
   const int64_t per = varlen ? 0 : (ra.seq_len + 63) / 64;
-  int dev = 0, sms = 0;
-  cudaStream_t side = nullptr;
-  cudaEvent_t ev_prep = nullptr, ev_pass = nullptr;
-  std::unique_lock<std::mutex> lock(g_side.mu, std::defer_lock);
-  bool segmented = !varlen && per >= 2 * kSegChunks && ra.state1 != nullptr && !ra.no_side_stream;
+  cudaStream_t side = ra.side_stream;
+  SegEvents ev;
+  bool segmented = !varlen && per >= 2 * kSegChunks && ra.state1 != nullptr && side != nullptr;
   if (segmented) {
-    lock.lock();
-    segmented = side_resources(dev, side, ev_prep, ev_pass, sms) == cudaSuccess &&
-                2 * (int64_t)ra.N * ra.H <= sms;
-    if (!segmented) lock.unlock();
+    int dev = 0, sms = 0;
+    cudaError_t e0 = cudaGetDevice(&dev);
+    if (e0 == cudaSuccess) e0 = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e0 != cudaSuccess) return e0;
+    segmented = 2 * (int64_t)ra.N * ra.H <= sms;
+    if (segmented && (e0 = ev.create()) != cudaSuccess) return e0;
   }
 
   const bool timed = clock_begin();
@@ -140,8 +127,8 @@ cudaError_t run_chunk_path(PrepArgs pa, const RecurrenceArgs &ra, bool varlen, b
     pa.seg_c0 = sg * kSegChunks;
     pa.seg_len = kSegChunks;
     e = launch_chunk_prep(pa, slots, fused, rq, rk, rv, ralpha, stream);
-    if (e == cudaSuccess) e = cudaEventRecord(ev_prep, stream);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev_prep, 0);
+    if (e == cudaSuccess) e = cudaEventRecord(ev.prep, stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev.prep, 0);
     if (e == cudaSuccess) {
       StateArgs ss = sa;
       ss.seg_c0 = sg * kSegChunks;
@@ -153,8 +140,8 @@ cudaError_t run_chunk_path(PrepArgs pa, const RecurrenceArgs &ra, bool varlen, b
   clock_mark(timed, stream);
   // the caller's stream continues only after the last state pass (also on an error, so
   // that nothing of this call is left running unordered)
-  cudaError_t e2 = cudaEventRecord(ev_pass, side);
-  if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(stream, ev_pass, 0);
+  cudaError_t e2 = cudaEventRecord(ev.pass, side);
+  if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(stream, ev.pass, 0);
   clock_mark(timed, stream);
   return e != cudaSuccess ? e : e2;
 }

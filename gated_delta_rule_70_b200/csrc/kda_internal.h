@@ -52,9 +52,9 @@ struct RecurrenceArgs {
   float *snap;
   int64_t snap_every;
   int snap_cap;
-  // 1: never use the side stream of the time-segmented schedule (its stream and events are
-  // created on first use); the entry point that must allocate nothing sets it
-  int no_side_stream;
+  // the caller's side stream for the time-segmented schedule, or nullptr (no segments)
+  cudaStream_t side_stream;
+  uint32_t wait_polls;       // polls per ordinary bounded wait (kWaitPolls; 0 in the failure test)
 };
 
 struct DecodeArgs {
@@ -75,6 +75,8 @@ struct DecodeArgs {
   float *state;              // [N, H, D, D] in place
   void *conv_state;          // [N, 3, 3*H*D] in place
   void *o;                   // [N, H, D]
+  int *err;                  // device status word or nullptr
+  uint32_t wait_polls;       // polls per ordinary bounded wait
 };
 
 // Tensor-core chunk path (bf16, head_dim 128): chunk_prep writes one record
@@ -102,6 +104,7 @@ struct PrepArgs {
   int seg_c0, seg_len;       // dense batches: chunks [seg_c0, seg_c0 + seg_len) of every sequence
                              // (seg_len 0: all); varlen batches: unused
   int *err;
+  uint32_t wait_polls;       // polls per ordinary bounded wait
   // [T rows][H*128] bf16: q, k, v (67-row boxes: 3 history rows + 64) and alpha (64 rows)
   CUtensorMap map_q, map_k, map_v, map_alpha;
 };
@@ -118,6 +121,7 @@ struct StateArgs {
   void *o;                   // [T, H, 128] bf16
   float *state1;
   int *err;
+  uint32_t wait_polls;       // polls per ordinary bounded wait
   const float *onw;          // output epilogue weight [128], with map_gate; nullptr: off
   float oeps;
   float *snap;               // state snapshots, as in RecurrenceArgs (every snap_chunks chunks)
@@ -170,6 +174,18 @@ inline WsLayout workspace_layout(int N, int H, int D, int seq_len, int64_t T, in
   }
   L.total = off;
   return L;
+}
+
+// Shape checks shared by every entry point: KDA_OK, KDA_ERR_INVALID_ARGUMENT or
+// KDA_ERR_UNSUPPORTED.
+kda_status check_shape(const kda_shape *s);
+// Polls of one bounded mbarrier wait (each poll is an mbarrier.try_wait, which may
+// itself suspend for a while), and the limit every drain of in-flight copies and
+// tensor-core work uses after a wait has given up.  A call with
+// KDA_FLAG_TEST_EXPIRE_WAITS passes 0 for its ordinary waits, never for a drain.
+constexpr uint32_t kWaitPolls = 1u << 22;
+inline uint32_t wait_polls_for(uint32_t flags) {
+  return (flags & KDA_FLAG_TEST_EXPIRE_WAITS) ? 0u : kWaitPolls;
 }
 
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t stream);

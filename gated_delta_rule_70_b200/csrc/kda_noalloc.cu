@@ -28,6 +28,9 @@ static __device__ __align__(256) unsigned char g_prefill_scratch[KDA_NOALLOC_SCR
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mu;
+// Looked up once per device and kept for the life of the process; after a
+// cudaDeviceReset of a device its entry here would be stale, so the entry point
+// must not be used on a device that has been reset.
 void *g_scratch_addr[kMaxDevices] = {};
 
 // Device address of this device's copy of the scratch array (set up on first use).
@@ -56,11 +59,8 @@ extern "C" kda_status kda_prefill_noalloc(
     const void *alpha, const void *b, const float *A_log, const float *dt_bias,
     const float *initial_state, const void *initial_conv_state, const int32_t *cu_seqlens, void *o,
     float *final_state, void *final_conv_state, void *stream_) {
-  if (s == nullptr || s->num_seqs < 0 || s->seq_len < 0 || s->num_heads < 1 ||
-      (s->io_dtype != KDA_BF16 && s->io_dtype != KDA_FP32) || (s->flags & ~KDA_FLAGS_KNOWN))
-    return KDA_ERR_INVALID_ARGUMENT;
-  if (s->head_dim != 64 && s->head_dim != 128) return KDA_ERR_UNSUPPORTED;
-  if (s->num_heads > 64) return KDA_ERR_UNSUPPORTED;
+  const kda_status st = check_shape(s);   // the same shape rules as kda_prefill
+  if (st != KDA_OK) return st;
   if (s->num_seqs == 0) return KDA_OK;
   const int64_t T = cu_seqlens ? (int64_t)s->seq_len : (int64_t)s->num_seqs * s->seq_len;
   const bool varlen = cu_seqlens != nullptr;
@@ -98,7 +98,8 @@ extern "C" kda_status kda_prefill_noalloc(
   ra.total_tokens = T; ra.io_dtype = s->io_dtype; ra.cu = cu_seqlens;
   ra.state0 = initial_state; ra.scale = s->scale; ra.o = o; ra.state1 = final_state;
   ra.lower_bound = s->lower_bound; ra.err = pa.err;
-  ra.no_side_stream = 1;   // (the segmented schedule would create a stream and events)
+  ra.wait_polls = wait_polls_for(s->flags);
+  ra.side_stream = nullptr;   // one launch per kernel: the segmented schedule would create events
   if (run_prefill(pa, ra, final_conv_state, varlen, ws, L, stream) != cudaSuccess) return KDA_ERR_CUDA;
   return KDA_OK;
 }

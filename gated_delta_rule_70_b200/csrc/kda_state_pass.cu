@@ -79,7 +79,6 @@ __device__ __forceinline__ uint32_t o_cols(int c) { return TM_O + (uint32_t)(c &
 // bf16 D^T columns of MMA k-step s (tokens 16s .. 16s+15), packed where each warpgroup read them
 __device__ __forceinline__ uint32_t d16_col(int s) { return TM_D + (uint32_t)(32 * (s >> 1) + 8 * (s & 1)); }
 
-constexpr uint32_t WAIT_POLLS = 1u << 22;
 // B_OC / B_OE: one per O^T buffer (commit of chunk c's MMAs / its O^T has left TMEM)
 enum { B_FULL0 = 0, B_FULL1, B_D, B_S, B_D16, B_S16, B_REL0, B_REL1, B_OC0, B_OC1, B_OC2, B_OC3,
        B_OE0, B_OE1, B_OE2, B_OE3, B_G0, B_G1, B_GE0, B_GE1, B_COUNT };
@@ -135,7 +134,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
   // waits return at once, so every role runs out its loop without stalling and every
   // thread of a role keeps the same control flow (addresses never depend on data).
   auto wait_one = [&](uint64_t *bb, uint32_t parity) {
-    if (*(volatile int *)fail == 0 && !umma::mbar_wait_bounded(bb, parity, WAIT_POLLS))
+    if (*(volatile int *)fail == 0 && !umma::mbar_wait_bounded(bb, parity, a.wait_polls))
       *(volatile int *)fail = 1;
     umma::fence_after_sync();
   };
@@ -145,7 +144,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
   // costs several hundred cycles even on a completed barrier.  wait_warp makes the
   // outcome warp-uniform.
   auto wait_warp = [&](uint64_t *bb, uint32_t parity) -> bool {
-    bool ok = *(volatile int *)fail == 0 && umma::mbar_wait_bounded(bb, parity, WAIT_POLLS);
+    bool ok = *(volatile int *)fail == 0 && umma::mbar_wait_bounded(bb, parity, a.wait_polls);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok && lane == 0) *(volatile int *)fail = 1;
     umma::fence_after_sync();
@@ -169,7 +168,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
       }
       // copies still in flight into this CTA's shared memory: wait (bounded) for them
       for (int k = issued - 2 < 0 ? 0 : issued - 2; k < issued; ++k)
-        (void)umma::mbar_wait_bounded(&bar[B_G0 + (k & 1)], (k >> 1) & 1, WAIT_POLLS);
+        (void)umma::mbar_wait_bounded(&bar[B_G0 + (k & 1)], (k >> 1) & 1, kWaitPolls);
     } else if (warp == W_REC) {
       // ---------------------------------------------------------- record copies
       // chunk c+2 goes into chunk c's buffer once every MMA of chunk c is done (the
@@ -193,7 +192,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
         issued = c + 3;
       }
       for (int k = issued - 2 < 0 ? 0 : issued - 2; k < issued; ++k)
-        (void)umma::mbar_wait_bounded(&bar[B_FULL0 + (k & 1)], (k >> 1) & 1, WAIT_POLLS);
+        (void)umma::mbar_wait_bounded(&bar[B_FULL0 + (k & 1)], (k >> 1) & 1, kWaitPolls);
     } else if (warp == W_WAIT) {
       // ---------------------------------------------------------- waits for the MMA issue
       // This warp and the MMA warp meet at both named barriers once per chunk, every chunk,
@@ -270,7 +269,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
         }
       }
       // nothing of this CTA's may still run on the tensor cores when TMEM is freed
-      if (last != nullptr) (void)umma::mbar_wait_bounded(last, last_parity, WAIT_POLLS);
+      if (last != nullptr) (void)umma::mbar_wait_bounded(last, last_parity, kWaitPolls);
     }
   } else if (warp >= NCH / 32) {
     // ------------------------------------------------------------ output (warps 8-11)
@@ -485,7 +484,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
   }
   umma::fence_before_sync();
   __syncthreads();
-  if (tid == 0 && *(volatile int *)fail != 0 && a.err) atomicExch(a.err, ERR_TIMEOUT);
+  if (tid == 0 && *(volatile int *)fail != 0 && a.err) atomicOr(a.err, ERR_TIMEOUT_STATE);
   if (warp == 0) {
     umma::fence_after_sync();
     umma::tmem_dealloc(tmem, 512);

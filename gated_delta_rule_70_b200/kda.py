@@ -29,7 +29,7 @@ EXPORTED = ["kda_prefill_workspace_size", "kda_prefill", "kda_prefill_status", "
             "kda_recurrence", "kda_recurrence_workspace_size", "kda_decode_step",
             "kda_status_string", "kda_version", "kda_prefill_noalloc", "kda_kernel_timing",
             "kda_kernel_times", "kda_prefill_gated", "kda_decode_step_gated", "kda_prefill_ex",
-            "kda_decode_multi"]
+            "kda_decode_multi", "kda_decode_ex", "kda_device_status"]
 
 
 class KdaLibraryError(RuntimeError):
@@ -50,6 +50,9 @@ class Shape(ctypes.Structure):
 
 
 KDA_FLAG_NEGATIVE_EIGENVALUES = 0x1
+KDA_FLAG_TEST_EXPIRE_WAITS = 0x80000000   # failure-path tests only (include/kda.h)
+KDA_STATUS_BAD_CU_SEQLENS, KDA_STATUS_TIMEOUT_PREP = 0x1, 0x2
+KDA_STATUS_TIMEOUT_STATE, KDA_STATUS_TIMEOUT_DECODE = 0x4, 0x8
 
 
 class OutputGate(ctypes.Structure):
@@ -63,7 +66,15 @@ class PrefillArgs(ctypes.Structure):
                 ("q", "k", "v", "conv_w", "alpha", "b", "A_log", "dt_bias", "initial_state",
                  "initial_conv_state", "cu_seqlens", "o", "final_state", "final_conv_state",
                  "out_gate", "snapshots")] + [("snapshot_every", ctypes.c_int32),
-                                              ("snapshot_capacity", ctypes.c_int32)]
+                                              ("snapshot_capacity", ctypes.c_int32),
+                                              ("side_stream", ctypes.c_void_p)]
+
+
+class DecodeArgs(ctypes.Structure):
+    """kda_decode_args: every pointer of a kda_decode_ex call (status: device int32 or None)."""
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("q", "k", "v", "alpha", "b", "conv_w", "A_log", "dt_bias", "out_gate", "state",
+                 "conv_state", "o", "step_states", "status")]
 
 
 def library_path() -> str:
@@ -107,6 +118,10 @@ def load_library():
     lib.kda_prefill_ex.restype = i32
     lib.kda_decode_multi.argtypes = [SP] + [P] * 8 + [OG] + [P] * 4 + [P]
     lib.kda_decode_multi.restype = i32
+    lib.kda_decode_ex.argtypes = [SP, ctypes.POINTER(DecodeArgs), P]
+    lib.kda_decode_ex.restype = i32
+    lib.kda_device_status.argtypes = [P, P]
+    lib.kda_device_status.restype = i32
     lib.kda_status_string.argtypes = [i32]
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_version.argtypes = []
@@ -147,9 +162,29 @@ def _dtype_code(dt: torch.dtype) -> int:
 
 def make_shape(num_seqs: int, seq_len: int, num_heads: int, head_dim: int, io_dtype: torch.dtype,
                lower_bound: float = -5.0, l2norm_eps: float = 1e-6, scale: float = 1.0,
-               negative_eigenvalues: bool = False) -> Shape:
+               negative_eigenvalues: bool = False, flags: int = 0) -> Shape:
+    """A kda_shape; ``flags`` adds raw KDA_FLAG_* bits (e.g. the failure-path test flag)."""
     return Shape(num_seqs, seq_len, num_heads, head_dim, lower_bound, l2norm_eps, scale,
-                 _dtype_code(io_dtype), KDA_FLAG_NEGATIVE_EIGENVALUES if negative_eigenvalues else 0)
+                 _dtype_code(io_dtype),
+                 (KDA_FLAG_NEGATIVE_EIGENVALUES if negative_eigenvalues else 0) | int(flags))
+
+
+_side_streams = {}
+
+
+def side_stream(device: torch.device) -> torch.cuda.Stream:
+    """A high-priority stream per device, handed to kda_prefill_ex as its side stream
+    (the time-segmented schedule of few long sequences runs its state passes there)."""
+    key = torch.device(device).index if torch.device(device).index is not None else \
+        torch.cuda.current_device()
+    if key not in _side_streams:
+        _side_streams[key] = torch.cuda.Stream(device=torch.device("cuda", key), priority=-100)
+    return _side_streams[key]
+
+
+def device_status(word: torch.Tensor) -> int:
+    """Synchronise the current stream and read a device status word (kda_device_status)."""
+    return int(load_library().kda_device_status(_ptr(word), _stream(word.device)))
 
 
 def prefill_workspace_size(shape: Shape, varlen: bool) -> int:
@@ -173,21 +208,26 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, conv_w: torch.Ten
             want_conv_state: bool = True, out: Optional[torch.Tensor] = None,
             final_state: Optional[torch.Tensor] = None,
             final_conv_state: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-            check: bool = True) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
+            check: bool = False, segments: bool = True,
+            flags: int = 0) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor]]:
     """KDA prefill.  q, k, v: [T_total, H*d] (or [B, T, H*d] dense); alpha: [.., H, d];
     b: [.., H].  Returns (o [T_total, H, d], final_state [N, H, d, d], final_conv_state
     [N, 3, 3*H*d] or None).  ``negative_eigenvalues``: beta = 2 sigmoid(b).  ``out_gate``
     [.., H, d] with ``o_norm_weight`` [d] fp32: the output epilogue o <- o / sqrt(mean o^2 +
     o_norm_eps) * weight * sigmoid(out_gate).  ``snapshots`` [N, C, H, d, d] fp32: snapshot j
     of sequence n (j < C) is the state after its first (j + 1) * 64 * snapshot_every tokens.
-    ``check`` synchronises and raises on device-side errors."""
+    The call is asynchronous on the current stream.  ``check=True`` then synchronises that
+    stream and raises on a device-side error (bad cu_seqlens, a bounded wait that gave up);
+    leave it off on hot paths.  ``segments``: hand the library this device's high-priority
+    side stream, so few long sequences run in overlapped time segments.  ``flags``: raw
+    KDA_FLAG_* bits added to the shape."""
     lib = load_library()
     H, d = alpha.shape[-2], alpha.shape[-1]
     if cu_seqlens is not None:
         N = cu_seqlens.numel() - 1
         T_total = q.numel() // (H * d)
         shape = make_shape(N, T_total, H, d, q.dtype, lower_bound, l2norm_eps, scale,
-                           negative_eigenvalues)
+                           negative_eigenvalues, flags)
     else:
         if q.dim() == 3:
             N, T = q.shape[0], q.shape[1]
@@ -195,7 +235,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, conv_w: torch.Ten
             N = 1 if num_seqs is None else num_seqs
             T = q.numel() // (H * d) // N
         T_total = N * T
-        shape = make_shape(N, T, H, d, q.dtype, lower_bound, l2norm_eps, scale, negative_eigenvalues)
+        shape = make_shape(N, T, H, d, q.dtype, lower_bound, l2norm_eps, scale, negative_eigenvalues,
+                           flags)
     dev = q.device
     o = out if out is not None else torch.empty((T_total, H, d), dtype=q.dtype, device=dev)
     fs = final_state if final_state is not None else torch.empty((N, H, d, d), dtype=torch.float32,
@@ -214,7 +255,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, conv_w: torch.Ten
                      ctypes.cast(ctypes.pointer(og_struct), ctypes.c_void_p) if og_struct is not None
                      else None,
                      _ptr(snapshots), int(snapshot_every),
-                     int(snapshots.shape[1]) if snapshots is not None else 0)
+                     int(snapshots.shape[1]) if snapshots is not None else 0,
+                     ctypes.c_void_p(side_stream(dev).cuda_stream) if segments else None)
     st = lib.kda_prefill_ex(ctypes.byref(shape), ctypes.byref(pa), _ptr(ws),
                             ctypes.c_size_t(ws.numel()), _stream(dev))
     _check(st, "kda_prefill")
@@ -303,19 +345,39 @@ def decode_step(q, k, v, alpha, b, conv_w, A_log, dt_bias, state: torch.Tensor,
                 conv_state: torch.Tensor, *, lower_bound: float = -5.0, l2norm_eps: float = 1e-6,
                 scale: float = 1.0, negative_eigenvalues: bool = False,
                 out_gate: Optional[torch.Tensor] = None, o_norm_weight: Optional[torch.Tensor] = None,
-                o_norm_eps: float = 1e-5, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                o_norm_eps: float = 1e-5, out: Optional[torch.Tensor] = None,
+                status: Optional[torch.Tensor] = None, flags: int = 0) -> torch.Tensor:
     """One token per sequence; updates ``state`` [N,H,d,d] and ``conv_state`` [N,3,3*H*d] in
-    place and returns o [N, H, d]."""
+    place and returns o [N, H, d].  ``status``: a device int32 the call zeroes and sets on a
+    device-side failure (read it with ``device_status``)."""
     lib = load_library()
     N, H, d = state.shape[0], state.shape[1], state.shape[2]
-    shape = make_shape(N, 1, H, d, q.dtype, lower_bound, l2norm_eps, scale, negative_eigenvalues)
+    shape = make_shape(N, 1, H, d, q.dtype, lower_bound, l2norm_eps, scale, negative_eigenvalues,
+                       flags)
     o = out if out is not None else torch.empty((N, H, d), dtype=q.dtype, device=q.device)
-    og = _output_gate(out_gate, o_norm_weight, o_norm_eps)
-    st = lib.kda_decode_step_gated(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
-                                   _ptr(b), _ptr(conv_w), _ptr(A_log), _ptr(dt_bias), og,
-                                   _ptr(state), _ptr(conv_state), _ptr(o), _stream(q.device))
+    if status is None:
+        og = _output_gate(out_gate, o_norm_weight, o_norm_eps)
+        st = lib.kda_decode_step_gated(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                       _ptr(b), _ptr(conv_w), _ptr(A_log), _ptr(dt_bias), og,
+                                       _ptr(state), _ptr(conv_state), _ptr(o), _stream(q.device))
+    else:
+        st = _decode_ex(lib, shape, q, k, v, alpha, b, conv_w, A_log, dt_bias, out_gate,
+                        o_norm_weight, o_norm_eps, state, conv_state, o, None, status)
     _check(st, "kda_decode_step")
     return o
+
+
+def _decode_ex(lib, shape, q, k, v, alpha, b, conv_w, A_log, dt_bias, out_gate, o_norm_weight,
+               o_norm_eps, state, conv_state, o, step_states, status):
+    og = None
+    if out_gate is not None or o_norm_weight is not None:
+        if out_gate is None or o_norm_weight is None:
+            raise ValueError("out_gate and o_norm_weight go together")
+        og = OutputGate(_ptr(out_gate), _ptr(o_norm_weight), float(o_norm_eps))
+    da = DecodeArgs(*[_ptr(t) for t in (q, k, v, alpha, b, conv_w, A_log, dt_bias)],
+                    ctypes.cast(ctypes.pointer(og), ctypes.c_void_p) if og is not None else None,
+                    *[_ptr(t) for t in (state, conv_state, o, step_states, status)])
+    return lib.kda_decode_ex(ctypes.byref(shape), ctypes.byref(da), _stream(q.device))
 
 
 def kernel_timing(enable: bool) -> None:
@@ -337,18 +399,19 @@ def decode_multi(q, k, v, alpha, b, conv_w, A_log, dt_bias, state: torch.Tensor,
                  scale: float = 1.0, negative_eigenvalues: bool = False,
                  out_gate: Optional[torch.Tensor] = None, o_norm_weight: Optional[torch.Tensor] = None,
                  o_norm_eps: float = 1e-5, step_states: Optional[torch.Tensor] = None,
-                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                 out: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                 flags: int = 0) -> torch.Tensor:
     """T new tokens per sequence (q, k, v [N, T, H*d]; alpha [N, T, H, d]; b [N, T, H]) in one
     call; updates ``state`` and ``conv_state`` in place, fills ``step_states`` [N, T, H, d, d]
-    (the state after each token) when given, and returns o [N, T, H, d]."""
+    (the state after each token) when given, and returns o [N, T, H, d].  ``status`` as in
+    ``decode_step``."""
     lib = load_library()
     N, H, d = state.shape[0], state.shape[1], state.shape[2]
     T = alpha.shape[1]
-    shape = make_shape(N, T, H, d, q.dtype, lower_bound, l2norm_eps, scale, negative_eigenvalues)
+    shape = make_shape(N, T, H, d, q.dtype, lower_bound, l2norm_eps, scale, negative_eigenvalues,
+                       flags)
     o = out if out is not None else torch.empty((N, T, H, d), dtype=q.dtype, device=q.device)
-    og = _output_gate(out_gate, o_norm_weight, o_norm_eps)
-    st = lib.kda_decode_multi(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(b),
-                              _ptr(conv_w), _ptr(A_log), _ptr(dt_bias), og, _ptr(state),
-                              _ptr(conv_state), _ptr(o), _ptr(step_states), _stream(q.device))
+    st = _decode_ex(lib, shape, q, k, v, alpha, b, conv_w, A_log, dt_bias, out_gate,
+                    o_norm_weight, o_norm_eps, state, conv_state, o, step_states, status)
     _check(st, "kda_decode_multi")
     return o

@@ -27,17 +27,9 @@
  * Conventions shared by every entry point
  *   - Every pointer is a DEVICE pointer unless stated otherwise; the caller
  *     owns every buffer, including the workspace.  The library allocates no
- *     device memory and is thread-safe across streams.  Its one piece of
- *     global state: a dense prefill (kda_prefill, kda_prefill_gated,
- *     kda_prefill_ex, kda_recurrence) with at least 256 chunks of 64 tokens per
- *     sequence and at most (SMs / 2) (sequence, head) pairs runs in time
- *     segments, chunk preparation on `stream` and the state pass of the
- *     previous segment on a high-priority side stream created on first use per
- *     device, with events ordering the two; `stream` waits for the last state
- *     pass before the call's later work.  Such calls from several host threads
- *     are serialised while they enqueue.  Under stream capture the fork to the
- *     side stream and the join back are captured with the rest.
- *     kda_prefill_noalloc never takes this path.
+ *     device memory, creates no streams and is thread-safe across streams;
+ *     its only process-wide state is the opt-in benchmark timing of
+ *     kda_kernel_timing().
  *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
  *     legacy default stream).  Return codes report argument checks and launch
  *     errors; device-side conditions are reported by kda_prefill_status().
@@ -98,7 +90,23 @@ typedef struct {
  * kda_allow_negative_eigenvalues switch (AliceAI-Foundation KDA write-up, section
  * "二": with the switch off, beta is not doubled and stays in (0, 1)). */
 #define KDA_FLAG_NEGATIVE_EIGENVALUES 0x1u
-#define KDA_FLAGS_KNOWN 0x1u
+/* For tests of the failure path only; never set it in normal use.  Every
+ * bounded device-side wait of the call (the mbarrier waits of chunk
+ * preparation, the state pass and the bf16 decode kernels) gives up at its
+ * first check.  Each kernel then stops issuing work, waits (with the normal
+ * limit) for the copies and tensor-core operations it already started, frees
+ * its tensor memory and returns; the call's status word reports
+ * KDA_ERR_TIMEOUT and the outputs are unspecified.  The next call without the
+ * flag runs normally. */
+#define KDA_FLAG_TEST_EXPIRE_WAITS 0x80000000u
+#define KDA_FLAGS_KNOWN (KDA_FLAG_NEGATIVE_EIGENVALUES | KDA_FLAG_TEST_EXPIRE_WAITS)
+
+/* Bits of the device status word (the first int32 of a prefill workspace, or a
+ * decode call's `status`), as kda_device_status() reads them. */
+#define KDA_STATUS_BAD_CU_SEQLENS 0x1    /* cu_seqlens malformed (accesses stayed clamped) */
+#define KDA_STATUS_TIMEOUT_PREP 0x2      /* a wait of chunk preparation gave up */
+#define KDA_STATUS_TIMEOUT_STATE 0x4     /* a wait of the state pass gave up */
+#define KDA_STATUS_TIMEOUT_DECODE 0x8    /* a wait of a decode kernel gave up */
 
 /* Bytes of device workspace kda_prefill() needs for this shape (0 on a bad
  * shape).  is_varlen != 0: shape->seq_len is the packed token total (the call
@@ -187,6 +195,18 @@ kda_status kda_prefill_gated(const kda_shape *shape,
  *                      buffer is left as it was.
  *   snapshot_every     >= 1: 64-token chunks between snapshots
  *   snapshot_capacity  >= 0: snapshots the buffer holds per sequence
+ *   side_stream        a cudaStream_t of the caller's (a high-priority one is
+ *                      best) or NULL.  Given one, a dense batch with at least
+ *                      256 chunks of 64 tokens per sequence and at most
+ *                      (SMs / 2) (sequence, head) pairs runs in time segments:
+ *                      chunk preparation of segment s + 1 on `stream` while
+ *                      the state pass of segment s runs on `side_stream`,
+ *                      ordered by two events the call creates and releases;
+ *                      `stream` waits for the last state pass before the call
+ *                      returns control of it.  Under stream capture the fork
+ *                      and the join are captured with the rest.  NULL: one
+ *                      launch of each kernel on `stream` (few long sequences
+ *                      then leave most SMs idle during the state pass).
  */
 typedef struct {
     const void *q, *k, *v, *conv_w, *alpha, *b;
@@ -201,17 +221,21 @@ typedef struct {
     float *snapshots;
     int32_t snapshot_every;
     int32_t snapshot_capacity;
+    void *side_stream;
 } kda_prefill_args;
 
 kda_status kda_prefill_ex(const kda_shape *shape, const kda_prefill_args *args,
                           void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * kda_prefill_status -- synchronises `stream` and reads the device error word
- * the last kda_prefill() on this workspace left: KDA_OK, KDA_ERR_INVALID_ARGUMENT
- * (bad cu_seqlens), KDA_ERR_TIMEOUT (a bounded wait gave up) or KDA_ERR_CUDA.
+ * kda_prefill_status -- synchronises `stream` and reads the device status word
+ * the last kda_prefill() on this workspace left (its first int32): KDA_OK,
+ * KDA_ERR_INVALID_ARGUMENT (bad cu_seqlens), KDA_ERR_TIMEOUT (a bounded wait
+ * gave up) or KDA_ERR_CUDA.  kda_device_status() is the same call on any
+ * status word (a decode call's `status` included).
  */
 kda_status kda_prefill_status(const void *workspace, void *stream);
+kda_status kda_device_status(const int32_t *word, void *stream);
 
 /*
  * kda_prologue -- the prologue alone (conv4 + SiLU, L2 norm, gate, beta).
@@ -302,6 +326,26 @@ kda_status kda_decode_multi(const kda_shape *shape,
                             float *state, void *conv_state, void *o, float *step_states,
                             void *stream);
 
+/*
+ * kda_decode_ex -- kda_decode_multi through one argument block, with a device
+ * status word.  `status` (device int32, or NULL) is zeroed by the call and
+ * gets KDA_STATUS_TIMEOUT_DECODE when a bounded wait of the decode kernel gave
+ * up; read it with kda_device_status().  kda_decode_step, kda_decode_step_gated
+ * and kda_decode_multi are this call with status NULL.
+ */
+typedef struct {
+    const void *q, *k, *v, *alpha, *b, *conv_w;
+    const float *A_log, *dt_bias;
+    const kda_output_gate *out_gate;
+    float *state;
+    void *conv_state;
+    void *o;
+    float *step_states;
+    int32_t *status;
+} kda_decode_args;
+
+kda_status kda_decode_ex(const kda_shape *shape, const kda_decode_args *args, void *stream);
+
 /* kda_decode_step with the output epilogue (gate [N, H, d]); out_gate NULL:
  * exactly kda_decode_step. */
 kda_status kda_decode_step_gated(const kda_shape *shape,
@@ -330,8 +374,11 @@ kda_status kda_decode_step_gated(const kda_shape *shape,
  *     1.2 KiB per token per head, e.g. 896 tokens at 32 heads) returns
  *     KDA_ERR_WORKSPACE and launches nothing.
  *   - The first call on each device looks up that device's address of the
- *     array (cudaGetSymbolAddress, with the device current).  Make that first
- *     call before any stream capture.
+ *     array (cudaGetSymbolAddress, with the device current) and keeps it for
+ *     the life of the process.  Make that first call before any stream
+ *     capture, and do not call this entry point on a device after a
+ *     cudaDeviceReset() of it: the kept address would be stale.
+ *   - The shape rules are kda_prefill's (the same checks, the same codes).
  *   - All calls share the one array and it keeps the previous call's
  *     contents; calls that overlap on the GPU (other streams, other threads)
  *     race with each other.  Serialise them.

@@ -33,7 +33,7 @@ def gpu_prefill(s: W.Spec, inp: dict, conv0=None, want_conv=True, neg=False):
                             _dev(inp["dt_bias"]), initial_state=_dev(inp["S0"]), cu_seqlens=cu,
                             initial_conv_state=_dev(conv0), num_seqs=s.num_seqs,
                             lower_bound=s.lower_bound, l2norm_eps=s.eps, scale=s.scale,
-                            negative_eigenvalues=neg, want_conv_state=want_conv)
+                            negative_eigenvalues=neg, want_conv_state=want_conv, check=True)
     torch.cuda.synchronize()
     return o, fs, fc
 
@@ -154,7 +154,7 @@ def test_prefill_all_sequences_empty(varlen):
     cu = _dev(inp["cu_seqlens"]) if varlen else None
     _, fs0, fc0 = kda.prefill(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["conv_w"]),
                               _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]),
-                              _dev(inp["dt_bias"]), cu_seqlens=cu, num_seqs=3)
+                              _dev(inp["dt_bias"]), cu_seqlens=cu, num_seqs=3, check=True)
     torch.cuda.synchronize()
     assert not W.from_device(fs0).any() and not W.from_device(fc0).any()
 
@@ -193,7 +193,7 @@ def test_prefill_bf16_continuation():
     p2 = part(T1, T1 + T2)
     o2, st2, cs2 = kda.prefill(_dev(p2["q"]), _dev(p2["k"]), _dev(p2["v"]), _dev(p2["conv_w"]),
                                _dev(p2["alpha"]), _dev(p2["b"]), _dev(p2["A_log"]), _dev(p2["dt_bias"]),
-                               initial_state=st1, initial_conv_state=cs1, num_seqs=1)
+                               initial_state=st1, initial_conv_state=cs1, num_seqs=1, check=True)
     torch.cuda.synchronize()
     o_cat = np.concatenate([W.from_device(o1), W.from_device(o2)])
     o_ref, s_ref, c_ref, _ = oracle_prefill(s, inp)
@@ -244,7 +244,7 @@ def test_prefill_in_place_state():
     st = _dev(inp["S0"]).clone()
     o, fs, _ = kda.prefill(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["conv_w"]),
                            _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]),
-                           _dev(inp["dt_bias"]), initial_state=st, num_seqs=2, final_state=st)
+                           _dev(inp["dt_bias"]), initial_state=st, num_seqs=2, final_state=st, check=True)
     o_ref, s_ref, _, _ = oracle_prefill(s, inp)
     assert max_state_err(W.from_device(st), s_ref) <= TOL["bf16"]
     assert max_pair_err(W.from_device(o), o_ref, inp["cu_seqlens"], s.H) <= TOL["bf16"]
@@ -383,7 +383,7 @@ def test_prefill_output_gate(io, d, lens):
                            _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]), _dev(inp["dt_bias"]),
                            initial_state=_dev(inp["S0"]), cu_seqlens=cu, num_seqs=s.num_seqs,
                            out_gate=_dev(G["gate"]), o_norm_weight=_dev(G["o_norm_weight"]),
-                           o_norm_eps=1e-5)
+                           o_norm_eps=1e-5, check=True)
     torch.cuda.synchronize()
     f = f64_inputs(inp)
     o_ref, s_ref, _, _ = oracle.forward(inp["cu_seqlens"], s.H, s.d, f["q"], f["k"], f["v"],
@@ -442,7 +442,7 @@ def test_prefill_state_snapshots(io, d, lens, every, cap):
     o, fs, _ = kda.prefill(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["conv_w"]),
                            _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]), _dev(inp["dt_bias"]),
                            initial_state=_dev(inp["S0"]), cu_seqlens=cu, num_seqs=s.num_seqs,
-                           snapshots=snaps, snapshot_every=every)
+                           snapshots=snaps, snapshot_every=every, check=True)
     torch.cuda.synchronize()
     f = f64_inputs(inp)
     ref = oracle.snapshots(inp["cu_seqlens"], s.H, d, 64 * every, cap, f["q"], f["k"], f["v"],
@@ -529,7 +529,7 @@ def test_prefill_time_segments_gated():
                             _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]), _dev(inp["dt_bias"]),
                             initial_state=_dev(inp["S0"]), num_seqs=s.num_seqs,
                             out_gate=_dev(G["gate"]), o_norm_weight=_dev(G["o_norm_weight"]),
-                            o_norm_eps=1e-5)
+                            o_norm_eps=1e-5, check=True)
     torch.cuda.synchronize()
     f = f64_inputs(inp)
     o_ref, s_ref, c_ref, _ = oracle.forward(inp["cu_seqlens"], s.H, s.d, f["q"], f["k"], f["v"],
@@ -553,7 +553,7 @@ def test_prefill_time_segments_snapshots():
     snaps = torch.full((1, cap, s.H, 128, 128), float("nan"), dtype=torch.float32, device="cuda")
     o, fs, _ = kda.prefill(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["conv_w"]),
                            _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]), _dev(inp["dt_bias"]),
-                           initial_state=_dev(inp["S0"]), num_seqs=1, snapshots=snaps, snapshot_every=every)
+                           initial_state=_dev(inp["S0"]), num_seqs=1, snapshots=snaps, snapshot_every=every, check=True)
     torch.cuda.synchronize()
     f = f64_inputs(inp)
     ref = oracle.snapshots(inp["cu_seqlens"], s.H, 128, 64 * every, cap, f["q"], f["k"], f["v"],
