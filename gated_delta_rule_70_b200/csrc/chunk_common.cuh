@@ -77,16 +77,18 @@ __device__ __forceinline__ uint32_t word(const uint4 &u, int i) {
 __device__ __forceinline__ float2 ex2_2(float2 x) {
   return make_float2(umma::ex2(x.x), umma::ex2(x.y));
 }
-// SiLU(x) = x sigmoid(x) with sigmoid(x) = 1/2 + tanh(x/2)/2, the tanh taken two
-// lanes at a time in half precision on the special-function unit (absolute
-// error of the sigmoid about 2^-12, below the bf16 rounding of the result).
-__device__ __forceinline__ float2 silu2(float2 x) {
-  const float2 hx = mul2(x, f2(0.5f));
-  uint32_t h, t;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(hx.y), "f"(hx.x));
-  asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(h));
+// SiLU(x) = x sigmoid(x) from h = x/2: with sigmoid(x) = 1/2 + tanh(x/2)/2,
+// SiLU(x) = h + h tanh(h), one fma once the tanh is known.  The tanh is taken two
+// lanes at a time in half precision on the special-function unit (absolute error
+// of the sigmoid about 2^-12, below the bf16 rounding of the result); h itself stays
+// fp32, so large |x| (where the half-precision tanh saturates to +-1) still gives
+// x or 0.
+__device__ __forceinline__ float2 silu2_from_half(float2 h) {
+  uint32_t hh, t;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(hh) : "f"(h.y), "f"(h.x));
+  asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(hh));
   const float2 th = __half22float2(*reinterpret_cast<const __half2 *>(&t));
-  return mul2(x, fma2(th, f2(0.5f), f2(0.5f)));
+  return fma2(h, th, h);
 }
 
 // sigmoid(x) = 1/2 + tanh(x/2)/2 two lanes at a time, the tanh in half precision

@@ -80,6 +80,7 @@ RecurrenceArgs make_recurrence_args(const kda_shape *s, int64_t T, const void *q
   ra.state0 = state0; ra.scale = s->scale; ra.o = o; ra.state1 = state1;
   ra.lower_bound = s->lower_bound;
   ra.wait_polls = wait_polls_for(s->flags);
+  ra.token_loop = (s->flags & KDA_FLAG_TOKEN_RECURRENCE) != 0;
   return ra;
 }
 

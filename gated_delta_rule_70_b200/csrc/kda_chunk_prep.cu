@@ -29,20 +29,22 @@
 //
 // Numerics: Gamma reaches 64 * (-5) = -320 inside a chunk, so e^{-Gamma}
 // overflows fp32.  The pairwise factor e^{Gamma_t - Gamma_s} is only ever split
-// around a reference close to both tokens: the 16-token sub-block I of a token
-// has the reference m_I = Gamma after its 8th token.  A token's L-side factor
-// e^{Gamma_t - m_I} and R-side factor e^{m_I - Gamma_t} then stay within
-// e^{+-8 |g|max} (2^{+-116} at a gate bound of -10), so neither overflows nor
-// drops to a subnormal the exponential would flush.  A row in block I against an
-// earlier block J uses k_s e^{m_J - Gamma_s} times e^{m_I - m_J} <= 1.  Per
-// element only two exponentials are taken, e^{Gamma_t - m_I} and e^{m_I - Gamma_t};
-// every other factor is one of them times a per-channel constant of the chunk,
-// all in base 2 on the special-function unit.
+// around a reference close to both tokens: the sub-block I of a token (16 or 32
+// tokens, kSub) has the reference m_I = Gamma after its (kSub/2)-th token.  A
+// token's L-side factor e^{Gamma_t - m_I} and R-side factor e^{m_I - Gamma_t} then
+// stay within e^{+-(kSub/2) |g|max}: with 16-token blocks 2^{+-116} at a gate bound of
+// -10, with 32-token blocks 2^{+-116} at -5.02, so neither overflows nor drops to a
+// subnormal the exponential would flush.  The host takes 32-token blocks whenever
+// the bound allows it (the pages' -5 does).  A row in block I against an earlier
+// block J uses k_s e^{m_J - Gamma_s} times e^{m_I - m_J} <= 1.  Per element only two
+// exponentials are taken, e^{Gamma_t - m_I} and e^{m_I - Gamma_t}; every other
+// factor is one of them times a per-channel constant of the chunk, all in base 2 on
+// the special-function unit.
 //
 // Structure: one CTA of 8 warps per (chunk, head), two CTAs per SM so that one
 // item's memory and tensor-core waits overlap the other's arithmetic.
 // Tensor-core work (tcgen05, fp32 accumulation in TMEM):
-//   [Lq; Lk] x R_all^T (M=128, N=160, K=128) -> A_qk and A_kk blocks
+//   [Lq; Lk] x R_all^T (M=128, N=160 or 96, K=128) -> A_qk and A_kk blocks
 //   W^T = K~^T T_b^T and U^T = V^T T_b^T      (M=128, N=64, K=64)
 // The 64x64 unit-lower-triangular solve runs in shared memory: 16x16 diagonal
 // blocks by forward substitution, then each warp owns a set of columns and
@@ -73,7 +75,7 @@ constexpr uint32_t OFF_RAWV = 34816;
 constexpr uint32_t OFF_RAWA = 52224;          // alpha: 64 rows
 // Intra-chunk MMA operands:
 constexpr uint32_t OFF_L = 0;                 // [q rows 0..63 | k rows 64..127] x 128 ch: 32 KB
-constexpr uint32_t OFF_R = 32768;             // R_all: 160 rows x 128 ch: 40 KB
+constexpr uint32_t OFF_R = 32768;             // R_all: up to 160 rows x 128 ch: 40 KB
 // Once the intra-chunk MMA has completed:
 constexpr uint32_t OFF_SB = 0;                // diag(beta) A_kk fp32 [64][TSS]
 constexpr uint32_t OFF_ST = 64 * TSS * 4;     // T fp32 [64][TSS]
@@ -122,9 +124,13 @@ __device__ __forceinline__ int cpos(int ch) { return ((ch & 7) >> 2) * 64 + (ch 
 static_assert(2 * (SMEM_BYTES + 1024) <= 233472, "two CTAs per SM");
 
 // R_all rows: [0,64) diagonal-block rows (every token against its own block's
-// reference), then R_1 (16 rows), R_2 (32), R_3 (48): R_I holds the tokens of blocks
-// before I against block I's reference.
-__host__ __device__ constexpr int r_row0(int I) { return I == 1 ? 64 : (I == 2 ? 80 : 112); }
+// reference), then R_I for each later block I: the tokens of the blocks before I
+// against block I's reference.  16-token blocks: R_1 (16 rows), R_2 (32), R_3 (48),
+// 160 rows in all; 32-token blocks: R_1 (32 rows), 96 rows in all.
+template <int kSub> __host__ __device__ constexpr int r_rows() { return kSub == 32 ? 96 : 160; }
+template <int kSub> __host__ __device__ constexpr int r_row0(int I) {
+  return kSub == 32 ? 64 : (I == 1 ? 64 : (I == 2 ? 80 : 112));
+}
 
 // TMEM columns (256 allocated): intra products; after they are read, W^T and U^T
 constexpr uint32_t TM_P = 0;
@@ -243,8 +249,11 @@ __device__ __forceinline__ bool locate(const PrepArgs &a, int64_t gchunk, int &n
   return true;
 }
 
-template <bool kFused>
+template <bool kFused, int kSub>
 __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant__ PrepArgs a) {
+  static_assert(kSub == 16 || kSub == 32, "sub-block length");
+  constexpr int NB = CH / kSub;            // sub-blocks per chunk
+  constexpr int RR = r_rows<kSub>();       // rows of R_all
   const int H = a.H;
   const int h = blockIdx.x % H;
   int64_t gchunk = blockIdx.x / H;
@@ -265,7 +274,8 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   }
   uint8_t *rec = reinterpret_cast<uint8_t *>(a.records) + (gchunk * H + h) * (int64_t)REC_STRIDE;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int cg = tid & 15, tg = tid >> 4, blkI = warp >> 1;   // tokens 4tg..4tg+3, all in block warp/2
+  const int cg = tid & 15, tg = tid >> 4;   // tokens 4tg..4tg+3 (warp w: tokens 8w..8w+7)
+  const int blkI = warp / (kSub / 8);        // their sub-block
   float *beta_s = reinterpret_cast<float *>(smem + OFF_BETA);
   float *wtot = reinterpret_cast<float *>(smem + OFF_WTOT);
   float *sBm = reinterpret_cast<float *>(smem + OFF_SB);
@@ -340,10 +350,12 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
                              : make_uint4(0, 0, 0, 0);
     }
     (void)vote(smem, OFF_BAR + 8, 0, a.wait_polls);   // bar_tma
-    if (tid < 192) {   // conv weights into fp32 tap pairs (one channel pair each)
+    if (tid < 192) {   // conv weights / 2 into fp32 tap pairs (one channel pair each): the
+                       // conv then yields x/2, the argument SiLU's tanh form starts from
       const int blk = tid >> 6, cgw = (tid >> 2) & 15, pw = tid & 3;
       const uint4 wq = *reinterpret_cast<const uint4 *>(smem + OFF_WCONV + blk * 1024 + cgw * 64 + pw * 16);
-      const float2 wa = bf2_f2(wq.x), wb = bf2_f2(wq.y), wc = bf2_f2(wq.z), wd = bf2_f2(wq.w);
+      const float2 wa = mul2(bf2_f2(wq.x), f2(0.5f)), wb = mul2(bf2_f2(wq.y), f2(0.5f));
+      const float2 wc = mul2(bf2_f2(wq.z), f2(0.5f)), wd = mul2(bf2_f2(wq.w), f2(0.5f));
       uint8_t *dw = smem + OFF_WRL + blk * 2048 + pw * 512 + cgw * 16;
       *reinterpret_cast<float4 *>(dw) = make_float4(wa.x, wc.x, wa.y, wc.y);         // taps 0, 1
       *reinterpret_cast<float4 *>(dw + 256) = make_float4(wb.x, wd.x, wb.y, wd.y);   // taps 2, 3
@@ -379,11 +391,11 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
         for (int r = 0; r < 7; ++r) x[r] = bf2_f2(word(xr[r], p));
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          float2 acc = mul2(w0, x[j]);
+          float2 acc = mul2(w0, x[j]);   // x/2, exactly (the weights are halved)
           acc = fma2(w1, x[j + 1], acc);
           acc = fma2(w2, x[j + 2], acc);
           acc = fma2(w3, x[j + 3], acc);
-          y[j][p] = silu2(acc);
+          y[j][p] = silu2_from_half(acc);
         }
       }
 #pragma unroll
@@ -481,20 +493,21 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   if (tid < 64) beta_s[tid] = btj;
   __syncthreads();   // also: every read of the prologue staging is done
   // per channel: exclusive prefix of the warp sums (in place), the block references
-  // m_I (Gamma after token 16I+7, the end of warp 2I's tokens) and Gamma_C
+  // m_I (Gamma after token kSub I + kSub/2 - 1, the end of warp (kSub/8) I + kSub/16 - 1)
+  // and Gamma_C
   if (tid < 128) {
     const int pc = cpos(tid);   // this thread's channel, in the split-half layout
-    float acc = 0.f, m[4];
+    float acc = 0.f, m[NB];
 #pragma unroll
     for (int w2 = 0; w2 < 8; ++w2) {
       const float x = wtot[w2 * 128 + pc];
       wtot[w2 * 128 + pc] = acc;
       acc += x;
-      if ((w2 & 1) == 0) m[w2 >> 1] = acc;
+      if (w2 % (kSub / 8) == kSub / 16 - 1) m[w2 / (kSub / 8)] = acc;
     }
     float *cf = reinterpret_cast<float *>(smem);
 #pragma unroll
-    for (int I = 0; I < 4; ++I) cf[C_M / 4 + I * 128 + pc] = m[I];
+    for (int I = 0; I < NB; ++I) cf[C_M / 4 + I * 128 + pc] = m[I];
     cf[C_M / 4 + 4 * 128 + pc] = acc;
     reinterpret_cast<float *>(rec + REC_EGC)[tid] = umma::ex2(acc);   // e^{Gamma_C}
   }
@@ -554,15 +567,23 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
 #pragma unroll
       for (int p = 0; p < 4; ++p) cK[p] = ex2_2(add2(gc[p], mul2(m[p], f2(-1.f))));   // <= 1
     }
-    auto later = [&](int I2, float2 (&c)[4]) {   // 2^{m_I2 - m_I} <= 1
+    auto later = [&](int I2, float2 (&c)[4]) {   // 2^{m_I2 - m_I} <= 1 (32-token blocks: its root)
       float2 mi[4];
       lds_pairs(C_M + I2 * 512, mi);
 #pragma unroll
-      for (int p = 0; p < 4; ++p) c[p] = ex2_2(add2(mi[p], mul2(m[p], f2(-1.f))));
+      for (int p = 0; p < 4; ++p)
+        c[p] = ex2_2(mul2(add2(mi[p], mul2(m[p], f2(-1.f))), f2(kSub == 32 ? 0.5f : 1.f)));
     };
-    if (blkI < 3) later(blkI + 1, c1);
-    if (blkI < 2) later(blkI + 2, c2);
-    if (blkI < 1) later(3, c3);
+    // The row against the next block's reference is kd 2^{m_{I+1} - m_I}.  With 16-token
+    // blocks the constant spans 16 gates; with 32-token blocks it would span 32 (2^-231 at
+    // a bound of -5, flushed to zero) while kd and the L factor reach 2^+-115, so there the
+    // constant is c = 2^{(m_1 - m_0) / 2}, 16 gates, applied twice: kd c c flushes to zero
+    // only where the true product is below 2^-18 of q.k.
+    if (blkI < NB - 1) later(blkI + 1, c1);
+    if constexpr (NB > 2) {
+      if (blkI < NB - 2) later(blkI + 2, c2);
+      if (blkI < NB - 3) later(blkI + 3, c3);
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int t = tg * 4 + j;
@@ -573,21 +594,28 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
                                ex2_2(fma2(g2[j][p], f2(-1.f), m[p])));   // within 2^{+-8|g|max}
         Rd[p] = f2_bf2(kd);
         Kh[p] = f2_bf2(mul2(kd, cK[p]));
-        K1[p] = blkI < 3 ? f2_bf2(mul2(kd, c1[p])) : 0u;
-        K2[p] = blkI < 2 ? f2_bf2(mul2(kd, c2[p])) : 0u;
-        K3[p] = blkI < 1 ? f2_bf2(mul2(kd, c3[p])) : 0u;
+        if constexpr (kSub == 32)
+          K1[p] = blkI < NB - 1 ? f2_bf2(mul2(mul2(kd, c1[p]), c1[p])) : 0u;
+        else
+          K1[p] = blkI < NB - 1 ? f2_bf2(mul2(kd, c1[p])) : 0u;
+        if constexpr (NB > 2) {
+          K2[p] = blkI < NB - 2 ? f2_bf2(mul2(kd, c2[p])) : 0u;
+          K3[p] = blkI < NB - 3 ? f2_bf2(mul2(kd, c3[p])) : 0u;
+        }
       }
-      *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, t, cg)) = make_uint4(Rd[0], Rd[1], Rd[2], Rd[3]);
+      *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(RR, t, cg)) = make_uint4(Rd[0], Rd[1], Rd[2], Rd[3]);
       *reinterpret_cast<uint4 *>(rec + REC_KH + tr_off(64, t, cg)) = make_uint4(Kh[0], Kh[1], Kh[2], Kh[3]);
-      if (blkI < 3)
-        *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, r_row0(blkI + 1) + t, cg)) =
+      if (blkI < NB - 1)
+        *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(RR, r_row0<kSub>(blkI + 1) + t, cg)) =
             make_uint4(K1[0], K1[1], K1[2], K1[3]);
-      if (blkI < 2)
-        *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, r_row0(blkI + 2) + t, cg)) =
-            make_uint4(K2[0], K2[1], K2[2], K2[3]);
-      if (blkI < 1)
-        *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(160, r_row0(3) + t, cg)) =
-            make_uint4(K3[0], K3[1], K3[2], K3[3]);
+      if constexpr (NB > 2) {
+        if (blkI < NB - 2)
+          *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(RR, r_row0<kSub>(blkI + 2) + t, cg)) =
+              make_uint4(K2[0], K2[1], K2[2], K2[3]);
+        if (blkI < NB - 3)
+          *reinterpret_cast<uint4 *>(smem + OFF_R + tr_off(RR, r_row0<kSub>(3) + t, cg)) =
+              make_uint4(K3[0], K3[1], K3[2], K3[3]);
+      }
     }
   }
   umma::fence_proxy_async_smem();
@@ -597,10 +625,10 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   uint32_t phase = 0;
   if (tid == 0 && !failed(smem)) {
     umma::fence_after_sync();
-    const uint32_t idesc = umma::make_idesc_bf16(128, 160, 0, 0);
+    const uint32_t idesc = umma::make_idesc_bf16(128, RR, 0, 0);
 #pragma unroll
     for (int s = 0; s < DK / 16; ++s)
-      umma::mma_ss(tmem + TM_P, desc_k128(sbase + OFF_L, 128, s), desc_k128(sbase + OFF_R, 160, s),
+      umma::mma_ss(tmem + TM_P, desc_k128(sbase + OFF_L, 128, s), desc_k128(sbase + OFF_R, RR, s),
                    idesc, s > 0);
     umma::mma_commit(bar_mma);
   }
@@ -609,12 +637,13 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
 
   // ---------------------------------------------------------------- A_qk (bf16) and diag(beta) A_kk
   // Warp w reads TMEM lanes 32(w&3)..: q rows (w&3 = 0, 1) or k rows (2, 3) of
-  // tokens 32p..32p+31, p = w & 1; lane half hh gives the block I = 2p + hh.
-  // Column group gi (s = 16gi..16gi+15) of row t comes from the diagonal product
-  // (gi == I) or from R_I (gi < I); tcgen05.ld is warp-uniform, so both halves
-  // load both candidates and keep their own.  Warps 0-3 take column groups 0-1,
-  // warps 4-7 (the same lane quadrants) groups 2-3.  Blocks of diag(beta) A_kk
-  // right of the diagonal are never read, so only A_qk gets explicit zeros.
+  // tokens 32p..32p+31, p = w & 1.  Warps 0-3 take column groups 0-1 (s = 0..31),
+  // warps 4-7 (the same lane quadrants) groups 2-3.  A column group of row t comes
+  // from the diagonal product (t's own block, masked) or from R_I (an earlier block).
+  // 32-token blocks: a warp's lanes are exactly one block.  16-token blocks: lane half
+  // hh gives the block I = 2p + hh; tcgen05.ld is warp-uniform, so both halves load
+  // both candidates and keep their own.  Blocks of diag(beta) A_kk right of the
+  // diagonal are never read, so only A_qk gets explicit zeros.
   if (ok) {
     const int p = warp & 1, hh = lane >> 4;
     const int t = 32 * p + lane;
@@ -647,7 +676,36 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
       }
     };
     uint32_t va[16], vb2[16], v[16];
-    if (p == 0) {
+    if constexpr (kSub == 32) {
+      (void)vb2; (void)v; (void)hh;
+      uint32_t vc[16];
+      if (p == 0) {
+        if (!upper) {          // block 0, groups 0-1: the diagonal product, columns 0..31
+          umma::tmem_ld16(tb + 0, va);
+          umma::tmem_ld16(tb + 16, vc);
+          umma::tmem_wait_ld();
+          emit(0, va, false, true);
+          emit(1, vc, false, true);
+        } else if (is_q) {     // block 0 against block 1: zero
+#pragma unroll
+          for (int e = 0; e < 16; ++e) va[e] = 0u;
+          emit(2, va, true, false);
+          emit(3, va, true, false);
+        }
+      } else if (!upper) {     // block 1 against block 0: R_1, columns 64..95
+        umma::tmem_ld16(tb + 64, va);
+        umma::tmem_ld16(tb + 80, vc);
+        umma::tmem_wait_ld();
+        emit(0, va, false, false);
+        emit(1, vc, false, false);
+      } else {                 // block 1, groups 2-3: the diagonal product, columns 32..63
+        umma::tmem_ld16(tb + 32, va);
+        umma::tmem_ld16(tb + 48, vc);
+        umma::tmem_wait_ld();
+        emit(2, va, false, true);
+        emit(3, vc, false, true);
+      }
+    } else if (p == 0) {
       if (!upper) {
         // gi 0: lo = diagonal (col 0), hi = R_1 (col 64); gi 1: hi = diagonal (col 16)
         uint32_t vc[16];
@@ -831,14 +889,22 @@ cudaError_t launch_chunk_table(const int32_t *cu, int N, int64_t total, int32_t 
 }
 
 namespace {
-template <bool kFused>
-cudaError_t launch_prep_variant(const PrepArgs &a, int64_t max_chunks, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(prep::chunk_prep_kernel<kFused>,
+template <bool kFused, int kSub>
+cudaError_t launch_prep_sub(const PrepArgs &a, int64_t max_chunks, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(prep::chunk_prep_kernel<kFused, kSub>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prep::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  prep::chunk_prep_kernel<kFused><<<(unsigned)(max_chunks * a.H), prep::NT, prep::SMEM_BYTES, stream>>>(a);
+  prep::chunk_prep_kernel<kFused, kSub><<<(unsigned)(max_chunks * a.H), prep::NT, prep::SMEM_BYTES, stream>>>(a);
   return cudaGetLastError();
+}
+// 32-token sub-blocks split each decay factor over at most 16 gates: within 2^{+-116}
+// (the margin the 16-token blocks keep at a bound of -10) while |lower_bound| <= 5.02.
+constexpr float kSub32MinLowerBound = -5.02f;
+template <bool kFused>
+cudaError_t launch_prep_variant(const PrepArgs &a, int64_t max_chunks, cudaStream_t stream) {
+  return a.lower_bound >= kSub32MinLowerBound ? launch_prep_sub<kFused, 32>(a, max_chunks, stream)
+                                              : launch_prep_sub<kFused, 16>(a, max_chunks, stream);
 }
 }  // namespace
 

@@ -158,7 +158,7 @@ cudaError_t run_recurrence(const RecurrenceArgs &ra, bool varlen, char *ws, cons
     return run_chunk_path(pa, ra, varlen, false, nullptr, ws, L, stream);
   }
 #endif
-  return launch_recurrence(ra, stream);
+  return launch_cuda_core_recurrence(ra, stream);
 }
 
 cudaError_t run_prefill(PrologueArgs pa, RecurrenceArgs ra, void *final_conv_state, bool varlen,
@@ -178,7 +178,7 @@ cudaError_t run_prefill(PrologueArgs pa, RecurrenceArgs ra, void *final_conv_sta
     pa.beta = reinterpret_cast<float *>(ws + L.beta);
     if ((e = launch_prologue(pa, stream)) != cudaSuccess) return e;
     ra.qn = pa.qn; ra.kn = pa.kn; ra.vc = pa.vc; ra.g = pa.g; ra.beta = pa.beta;
-    e = launch_recurrence(ra, stream);
+    e = launch_cuda_core_recurrence(ra, stream);
   }
   if (e != cudaSuccess) return e;
   if (final_conv_state != nullptr) e = launch_conv_state_out(pa, final_conv_state, stream);

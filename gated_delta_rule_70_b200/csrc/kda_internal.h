@@ -55,6 +55,7 @@ struct RecurrenceArgs {
   // the caller's side stream for the time-segmented schedule, or nullptr (no segments)
   cudaStream_t side_stream;
   uint32_t wait_polls;       // polls per ordinary bounded wait (kWaitPolls; 0 in the failure test)
+  int token_loop;            // off the tensor-core path: the token kernel, not the fp32 chunk kernel
 };
 
 struct DecodeArgs {
@@ -200,6 +201,14 @@ cudaError_t launch_chunk_prep(PrepArgs a, int64_t max_chunks, bool fused, const 
 cudaError_t launch_state_pass(StateArgs a, const void *gate, cudaStream_t stream);
 cudaError_t launch_conv_state_out(const PrologueArgs &a, void *out, cudaStream_t stream);
 cudaError_t launch_recurrence(const RecurrenceArgs &a, cudaStream_t stream);
+// The chunkwise recurrence on CUDA cores in fp32 (prepared inputs, as launch_recurrence).
+cudaError_t launch_chunk_simt(const RecurrenceArgs &a, cudaStream_t stream);
+// Off the tensor-core path: the fp32 chunk kernel where its split factors fit fp32
+// (gate bound >= -10) unless the token loop was asked for, else the token kernel.
+inline cudaError_t launch_cuda_core_recurrence(const RecurrenceArgs &a, cudaStream_t stream) {
+  return !a.token_loop && a.lower_bound >= kTcMinLowerBound ? launch_chunk_simt(a, stream)
+                                                            : launch_recurrence(a, stream);
+}
 // The recurrence (a4-a8) for RecurrenceArgs `ra` with workspace `ws` laid out by
 // workspace_layout(): tensor-core chunk path for bf16 / head_dim 128, else the
 // CUDA-core token kernel.

@@ -99,6 +99,7 @@ extern "C" kda_status kda_prefill_noalloc(
   ra.state0 = initial_state; ra.scale = s->scale; ra.o = o; ra.state1 = final_state;
   ra.lower_bound = s->lower_bound; ra.err = pa.err;
   ra.wait_polls = wait_polls_for(s->flags);
+  ra.token_loop = (s->flags & KDA_FLAG_TOKEN_RECURRENCE) != 0;
   ra.side_stream = nullptr;   // one launch per kernel: the segmented schedule would create events
   if (run_prefill(pa, ra, final_conv_state, varlen, ws, L, stream) != cudaSuccess) return KDA_ERR_CUDA;
   return KDA_OK;

@@ -66,7 +66,7 @@ prologue_kernel(PrologueArgs a) {
   if (a.cu != nullptr && blockIdx.x == 0 && threadIdx.x == 0 && a.err != nullptr) {
     bool ok = a.cu[0] == 0 && (int64_t)a.cu[a.N] == total;
     for (int n = 0; n < a.N && ok; ++n) ok = a.cu[n + 1] >= a.cu[n];
-    if (!ok) atomicExch(a.err, ERR_BAD_CU_SEQLENS);
+    if (!ok) atomicOr(a.err, ERR_BAD_CU_SEQLENS);
   }
 
   const int n0 = seq_of_token(a.cu, a.N, a.seq_len, t0);

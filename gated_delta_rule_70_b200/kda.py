@@ -50,6 +50,7 @@ class Shape(ctypes.Structure):
 
 
 KDA_FLAG_NEGATIVE_EIGENVALUES = 0x1
+KDA_FLAG_TOKEN_RECURRENCE = 0x2           # off the tensor-core path: the token loop (include/kda.h)
 KDA_FLAG_TEST_EXPIRE_WAITS = 0x80000000   # failure-path tests only (include/kda.h)
 KDA_STATUS_BAD_CU_SEQLENS, KDA_STATUS_TIMEOUT_PREP = 0x1, 0x2
 KDA_STATUS_TIMEOUT_STATE, KDA_STATUS_TIMEOUT_DECODE = 0x4, 0x8

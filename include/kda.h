@@ -48,9 +48,11 @@
  * Supported shapes: head_dim 64 or 128; num_heads 1..64; any sequence
  * length >= 0.  bf16 with head_dim 128 and lower_bound >= -10 runs the
  * tensor-core chunk path (chunk_prep, with the prologue fused in, then the
- * state pass); other combinations run the prologue kernel and the CUDA-core
- * token kernel (fp32 test mode).  The bound keeps the chunk path's split decay
- * factors, which span up to 8 tokens of gate, inside fp32 and bf16 normal range.
+ * state pass).  Other combinations (fp32 I/O: the fp32 test mode; head_dim 64)
+ * run the prologue kernel and then, for lower_bound >= -10, the same chunkwise
+ * algebra on CUDA cores in fp32, or else (or with KDA_FLAG_TOKEN_RECURRENCE) the
+ * CUDA-core token loop.  The bound keeps the chunk algebra's split decay factors,
+ * which span up to 8 tokens of gate, inside fp32 and bf16 normal range.
  */
 #ifndef KDA_H
 #define KDA_H
@@ -90,6 +92,11 @@ typedef struct {
  * kda_allow_negative_eigenvalues switch (AliceAI-Foundation KDA write-up, section
  * "二": with the switch off, beta is not doubled and stays in (0, 1)). */
 #define KDA_FLAG_NEGATIVE_EIGENVALUES 0x1u
+/* Where the tensor-core chunk path does not apply (fp32 I/O, head_dim 64), run
+ * the recurrence token by token on CUDA cores, the loop exactly as the KDA
+ * write-up's section "二" states it, instead of the fp32 chunkwise kernel.  Both
+ * compute in fp32; gate bounds below -10 always take the token loop. */
+#define KDA_FLAG_TOKEN_RECURRENCE 0x2u
 /* For tests of the failure path only; never set it in normal use.  Every
  * bounded device-side wait of the call (the mbarrier waits of chunk
  * preparation, the state pass and the bf16 decode kernels) gives up at its
@@ -99,7 +106,8 @@ typedef struct {
  * KDA_ERR_TIMEOUT and the outputs are unspecified.  The next call without the
  * flag runs normally. */
 #define KDA_FLAG_TEST_EXPIRE_WAITS 0x80000000u
-#define KDA_FLAGS_KNOWN (KDA_FLAG_NEGATIVE_EIGENVALUES | KDA_FLAG_TEST_EXPIRE_WAITS)
+#define KDA_FLAGS_KNOWN \
+    (KDA_FLAG_NEGATIVE_EIGENVALUES | KDA_FLAG_TOKEN_RECURRENCE | KDA_FLAG_TEST_EXPIRE_WAITS)
 
 /* Bits of the device status word (the first int32 of a prefill workspace, or a
  * decode call's `status`), as kda_device_status() reads them. */

@@ -56,6 +56,13 @@ def _tf32(x):
     return u.view(np.float32).astype(np.float64)
 
 
+def _flush(x):
+    """fp32's flush to zero below its normal range (2^-126), which the special-function
+    exponential applies to its results."""
+    x = np.asarray(x, dtype=np.float64)
+    return np.where(np.abs(x) < 2.0 ** -126, 0.0, x)
+
+
 def blocked_inverse(A, tf32: bool = False, bf16: bool = False):
     """(I + A)^{-1} for a strictly lower-triangular 64 x 64 A, by blocks: the 16 x 16 diagonal
     blocks' inverses D_i by substitution, then T_ij = -D_i (A_ij D_j) for the blocks next to the
@@ -84,7 +91,8 @@ def _rounder(bf16):
     return lambda site: _bf16 if site in on else (lambda x: x)
 
 
-def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB, bf16=False, solve: str = "direct"):
+def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB, bf16=False, solve: str = "direct",
+                  flush: bool = False):
     """One padded chunk (q, k, v [64, d], g [64, d_k] natural-log gates, beta [64]) ->
     (A_qk, W, U, Q 2^Gamma, K 2^{Gamma_C - Gamma}, 2^{Gamma_C}, the log2 exponents of every
     L and R factor taken).  ``mistake`` plants one plausible error, for the test that shows
@@ -93,7 +101,11 @@ def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB, bf16=False, solv
     and the record's A_qk, W, U, Q 2^Gamma and K 2^{Gamma_C - Gamma}; A_kk, T, the gates and
     2^{Gamma_C} stay wide (fp32 in the kernels, fp64 here).  A collection of SITES names
     rounds at those sites only.  ``solve``: "direct" (a plain inverse), "blocked",
-    "blocked_tf32" or "blocked_bf16" (``blocked_inverse``)."""
+    "blocked_tf32" or "blocked_bf16" (``blocked_inverse``).  ``flush`` applies fp32's flush
+    to zero below 2^-126 to the exponentials and the R rows of earlier blocks, as the
+    kernels' arithmetic does; with 32-token blocks the earlier block's constant is then
+    taken as its root applied twice (the constant itself spans 32 gates, the root 16), as
+    the kernel does, unless ``mistake == "sb32_full_constant"``."""
     rb = _rounder(bf16)
     G2 = np.cumsum(g * LOG2E, axis=0)
     m = block_refs(G2, sb)
@@ -115,7 +127,13 @@ def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB, bf16=False, solv
             if mistake == "no_block_constant":
                 c_exp = np.zeros_like(c_exp)
             exps.append(np.broadcast_to(c_exp, (1, k.shape[1])))
-            R[cols] = rb("LR")(Rd[cols] * np.exp2(c_exp))
+            if not flush:
+                R[cols] = rb("LR")(Rd[cols] * np.exp2(c_exp))
+            elif sb == 32 and J < I and mistake != "sb32_full_constant":
+                ch = _flush(np.exp2(c_exp / 2))
+                R[cols] = rb("LR")(_flush(_flush(_flush(Rd[cols]) * ch) * ch))
+            else:
+                R[cols] = rb("LR")(_flush(_flush(Rd[cols]) * _flush(np.exp2(c_exp))))
         A_qk[rows] = Lq[rows] @ R.T
         A_kk[rows] = beta[rows, None] * (Lk[rows] @ R.T)
     t = np.arange(CH)
@@ -140,7 +158,7 @@ def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB, bf16=False, solv
 
 
 def chunked_forward(cu_seqlens, q, k, v, g, beta, state0=None, mistake=None, sb: int = SB,
-                    bf16=False, solve: str = "direct"):
+                    bf16=False, solve: str = "direct", flush: bool = False):
     """The chunked form over packed prepared inputs (q, k, v, g [T, H, d], beta [T, H]) ->
     (o [T, H, d], final state [N, H, d, d]), the same contract as the oracle's recurrence.
     ``bf16`` also rounds q, k, v, the state's copy that the MMAs read, D (after U is added)
@@ -162,7 +180,7 @@ def chunked_forward(cu_seqlens, q, k, v, g, beta, state0=None, mistake=None, sb:
                 pad = lambda x: np.concatenate([x, np.zeros((CH - L,) + x.shape[1:])])
                 A_qk, W, U, Qt, Kh, eGC, _ = chunk_factors(
                     pad(q[c0:c1, h]), pad(k[c0:c1, h]), pad(v[c0:c1, h]), pad(g[c0:c1, h]),
-                    pad(beta[c0:c1, h]), mistake, sb, bf16, solve)
+                    pad(beta[c0:c1, h]), mistake, sb, bf16, solve, flush)
                 Sb = rb("S_copy")(S)
                 D = rb("D")(U - W @ Sb)
                 O = Qt @ Sb + A_qk @ D

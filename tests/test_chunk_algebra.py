@@ -218,3 +218,21 @@ def test_collinear_keys_amplify_every_rounding_site():
     for site in ("T_b", "D", "qkv"):
         without = max(_errs(*x_col, bf16=[s for s in CM.SITES if s != site]))
         assert without > 0.75 * e_col, (site, without, e_col)
+
+
+@pytest.mark.parametrize("sb,mistake,ok", [(16, None, True), (32, None, True),
+                                           (32, "sb32_full_constant", False)])
+def test_earlier_block_rows_survive_fp32_flush_at_saturated_gates(sb, mistake, ok):
+    """With every gate on the bound (-5) the constant between the two 32-token blocks'
+    references spans 32 gates, 2^-231, and flushes to zero in fp32, while the factors it
+    multiplies reach 2^+-115: a row of block 1 against block 0 would lose entries worth
+    e^-5 q.k.  Taken as its root (16 gates) applied twice it survives; with 16-token blocks
+    the constant spans 16 gates and needs no split."""
+    cu, q, k, v, g, beta, S0 = prepared([128], H=1, d=8, lb=-5.0, seed=9, gate_lo=-5.0)
+    o_ref, s_ref = oracle.recurrence(cu, q, k, v, g, beta, state0=S0)
+    o, s = CM.chunked_forward(cu, q, k, v, g, beta, state0=S0, sb=sb, flush=True, mistake=mistake)
+    err = max(rel(o, o_ref), rel(s, s_ref))
+    if ok:
+        assert err < 1e-10
+    else:
+        assert err > 1e-3

@@ -26,14 +26,15 @@ def _dev(arr):
     return W.to_device(arr)
 
 
-def gpu_prefill(s: W.Spec, inp: dict, conv0=None, want_conv=True, neg=False):
+def gpu_prefill(s: W.Spec, inp: dict, conv0=None, want_conv=True, neg=False, flags=0):
     cu = _dev(inp["cu_seqlens"]) if s.varlen else None
     o, fs, fc = kda.prefill(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(inp["conv_w"]),
                             _dev(inp["alpha"]), _dev(inp["b"]), _dev(inp["A_log"]),
                             _dev(inp["dt_bias"]), initial_state=_dev(inp["S0"]), cu_seqlens=cu,
                             initial_conv_state=_dev(conv0), num_seqs=s.num_seqs,
                             lower_bound=s.lower_bound, l2norm_eps=s.eps, scale=s.scale,
-                            negative_eigenvalues=neg, want_conv_state=want_conv, check=True)
+                            negative_eigenvalues=neg, want_conv_state=want_conv, check=True,
+                            flags=flags)
     torch.cuda.synchronize()
     return o, fs, fc
 
@@ -74,9 +75,9 @@ def max_state_err(s_gpu, s_ref):
     return max(rel_l2(s_gpu[n, h], s_ref[n, h]) for n in range(N) for h in range(H))
 
 
-def check_prefill(s: W.Spec, conv0=None, neg=False):
+def check_prefill(s: W.Spec, conv0=None, neg=False, flags=0):
     inp = W.make_inputs(s)
-    o, fs, fc = gpu_prefill(s, inp, conv0, neg=neg)
+    o, fs, fc = gpu_prefill(s, inp, conv0, neg=neg, flags=flags)
     o_ref, s_ref, c_ref, _ = oracle_prefill(s, inp, conv0, neg=neg)
     tol = TOL[s.io_dtype]
     eo = max_pair_err(W.from_device(o), o_ref, inp["cu_seqlens"], s.H)
