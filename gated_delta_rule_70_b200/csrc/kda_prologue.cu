@@ -7,11 +7,15 @@
 // use_qk_l2norm_in_kernel; the gate formula), and the Ling-3.0-flash-VL config
 // table (kda_lower_bound = -5.0).
 //
-// Streaming design: a group of d/8 threads owns one (head, 16-token tile); each
+// Streaming design: a group of d/8 threads owns one (head, 8-token tile); each
 // thread owns 8 consecutive channels and walks the tile's tokens in order,
 // keeping the 3-token conv history in registers.  All global traffic is 16-byte
 // vector loads/stores; a warp touches 512 contiguous bytes per row (two heads
-// of d = 128).  The L2 norm is a shuffle reduction inside the group.
+// of d = 128).  The L2 norm is a shuffle reduction inside the group.  A thread
+// works through four phases (q, k, v, then alpha); with bf16 inputs the rows of a
+// phase are staged two phases ahead into the thread's own shared-memory slots by
+// asynchronous copies, so a thread's loads stay in flight while it computes (the
+// registers hold only the phase it works on).
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -19,6 +23,20 @@ namespace kda {
 
 constexpr int PRO_TPT = 8;       // tokens per thread (one tile)
 constexpr int PRO_THREADS = 256;
+constexpr int PRO_STAGES = 2;    // phases staged ahead (bf16)
+constexpr int PRO_ROWS = PRO_TPT + 3;   // a phase's rows: the 3 history tokens, then the tile
+constexpr uint32_t PRO_STAGE_BYTES = PRO_STAGES * PRO_ROWS * PRO_THREADS * 16;   // 88 KB
+
+// 16 bytes global -> shared, asynchronously; src_bytes 0 fills the slot with zeros
+// (the source address is then not read, but stays a valid one).
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+               :: "r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory");
+}
 
 // 8 consecutive elements held undecoded, so a tile's loads can all be issued
 // before any arithmetic (one round trip to HBM per tile, not one per token).
@@ -72,9 +90,52 @@ prologue_kernel(PrologueArgs a) {
   const int n0 = seq_of_token(a.cu, a.N, a.seq_len, t0);
   // the G lanes of this row group (all take the same trip counts)
   const unsigned group_mask = (G == 32 ? 0xffffffffu : ((1u << G) - 1u) << ((threadIdx.x % 32) & ~(G - 1)));
+  // whole tile inside one sequence: the conv phases take the staged rows; hist_in: its
+  // three history tokens belong to the same sequence too (else they come from the conv
+  // state or are zeros, loaded as the phase starts)
+  bool whole, hist_in;
+  {
+    int64_t s0, e0;
+    seq_bounds(a.cu, n0, a.seq_len, total, s0, e0);
+    whole = t0 + PRO_TPT <= e0 && t1 - t0 == PRO_TPT;
+    hist_in = t0 - 3 >= s0 && t0 >= 3;
+  }
+
+  // bf16: phase p's rows (p = 0, 1, 2: q, k, v at this thread's channels, history tokens
+  // t0-3..t0-1 in rows 0-2 and the tile in rows 3..; p = 3: alpha in rows 3..) in slot
+  // stage[p % 2][row][thread]; a commit group per phase (empty ones keep the count)
+  constexpr bool kStage = sizeof(T) == 2;
+  extern __shared__ __align__(16) uint4 pro_stage[];
+  auto slot = [&](int p, int r) { return pro_stage + ((p & 1) * PRO_ROWS + r) * PRO_THREADS + threadIdx.x; };
+  auto stage_phase = [&](int p) {
+    if constexpr (kStage) {
+      if (p < 3 && whole) {
+        const T *x = reinterpret_cast<const T *>(p == 0 ? a.q : (p == 1 ? a.k : a.v));
+        if (hist_in) {
+#pragma unroll
+          for (int m = 0; m < 3; ++m) cp_async16(slot(p, m), x + (t0 - 3 + m) * HD + c0, 16);
+        }
+#pragma unroll
+        for (int j = 0; j < PRO_TPT; ++j) cp_async16(slot(p, 3 + j), x + (t0 + j) * HD + c0, 16);
+      } else if (p == 3) {
+        const T *al = reinterpret_cast<const T *>(a.alpha) + h * D + lane_in_group * 8;
+#pragma unroll
+        for (int j = 0; j < PRO_TPT; ++j)
+          cp_async16(slot(p, 3 + j), al + (t0 + j < t1 ? t0 + j : t0) * HD, t0 + j < t1 ? 16u : 0u);
+      }
+      cp_async_commit();
+    }
+  };
+  stage_phase(0);
+  stage_phase(1);
+  // b of token t0 + lane (lanes 0..7 of the group; G >= 8), early: each of those lanes
+  // writes its token's beta at the end
+  const bool has_b = lane_in_group < PRO_TPT && t0 + lane_in_group < t1;
+  const float bme = has_b ? to_f32(reinterpret_cast<const T *>(a.b)[(t0 + lane_in_group) * H + h]) : 0.f;
 
 #pragma unroll 1
   for (int blk = 0; blk < 3; ++blk) {
+    if constexpr (kStage) cp_async_wait<1>();   // phase blk's rows have landed
     const T *__restrict__ x = reinterpret_cast<const T *>(blk == 0 ? a.q : (blk == 1 ? a.k : a.v));
     T *__restrict__ y = reinterpret_cast<T *>(blk == 0 ? a.qn : (blk == 1 ? a.kn : a.vc));
     const T *__restrict__ w = reinterpret_cast<const T *>(a.conv_w) + ((int64_t)blk * HD + c0) * KCONV;
@@ -106,7 +167,19 @@ prologue_kernel(PrologueArgs a) {
         }
       }
     };
-    load_history(t0);
+    bool staged_hist = false;
+    if constexpr (kStage) {
+      if (whole && hist_in) {
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+          Raw8<T> r;
+          r.u = *slot(blk, m);
+          r.get(hist[m]);
+        }
+        staged_hist = true;
+      }
+    }
+    if (!staged_hist) load_history(t0);
     // conv + SiLU (+ L2 norm for q, k) of one token whose raw input is xt
     auto emit = [&](int64_t t, const float (&xt)[8]) {
       float yt[8];
@@ -133,11 +206,14 @@ prologue_kernel(PrologueArgs a) {
       }
       store8(y + (t * H + h) * D + lane_in_group * 8, yt);
     };
-    if (t0 + PRO_TPT <= e && t1 - t0 == PRO_TPT) {
-      // whole tile inside one sequence: issue every load, then compute
+    if (whole) {
+      // whole tile inside one sequence: every load issued (or staged), then compute
       Raw8<T> raw[PRO_TPT];
 #pragma unroll
-      for (int j = 0; j < PRO_TPT; ++j) raw[j].load(x + (t0 + j) * HD + c0);
+      for (int j = 0; j < PRO_TPT; ++j) {
+        if constexpr (kStage) raw[j].u = *slot(blk, 3 + j);
+        else raw[j].load(x + (t0 + j) * HD + c0);
+      }
 #pragma unroll
       for (int j = 0; j < PRO_TPT; ++j) {
         float xt[8];
@@ -157,6 +233,7 @@ prologue_kernel(PrologueArgs a) {
         emit(t, xt);
       }
     }
+    stage_phase(blk + 2);   // into the slots this phase has finished with
   }
 
   // gate and beta
@@ -164,18 +241,13 @@ prologue_kernel(PrologueArgs a) {
   float bias[8];
   load8(a.dt_bias + h * D + lane_in_group * 8, bias);
   const T *__restrict__ alpha = reinterpret_cast<const T *>(a.alpha);
-  const T *__restrict__ bb = reinterpret_cast<const T *>(a.b);
   Raw8<T> araw[PRO_TPT];
-  float bvals[PRO_TPT];
+  if constexpr (kStage) cp_async_wait<0>();   // alpha's rows (zeros past the tile)
 #pragma unroll
   for (int j = 0; j < PRO_TPT; ++j) {
-    if (t0 + j < t1) {
-      araw[j].load(alpha + ((t0 + j) * H + h) * D + lane_in_group * 8);
-      bvals[j] = lane_in_group == 0 ? to_f32(bb[(t0 + j) * H + h]) : 0.f;
-    } else {
-      araw[j].zero();
-      bvals[j] = 0.f;
-    }
+    if constexpr (kStage) araw[j].u = *slot(3, 3 + j);
+    else if (t0 + j < t1) araw[j].load(alpha + ((t0 + j) * H + h) * D + lane_in_group * 8);
+    else araw[j].zero();
   }
 #pragma unroll
   for (int j = 0; j < PRO_TPT; ++j) {
@@ -186,8 +258,8 @@ prologue_kernel(PrologueArgs a) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) gt[i] = gate_f(al[i] + bias[i], negA, a.lower_bound);
     store8(a.g + (t * H + h) * D + lane_in_group * 8, gt);
-    if (lane_in_group == 0) a.beta[t * H + h] = (a.beta2 ? 2.f : 1.f) * sigmoid_f(bvals[j]);
   }
+  if (has_b) a.beta[(t0 + lane_in_group) * H + h] = (a.beta2 ? 2.f : 1.f) * sigmoid_f(bme);
 }
 
 // final_conv_state[n][m][c] = raw input of token (end_n - 3 + m), or the
@@ -224,8 +296,11 @@ cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t stream) {
   const int64_t threads = tiles * a.H * G;
   const int64_t blocks = (threads + PRO_THREADS - 1) / PRO_THREADS;
   if (a.io_dtype == KDA_BF16) {
-    if (a.D == 128) prologue_kernel<__nv_bfloat16, 128><<<(unsigned)blocks, PRO_THREADS, 0, stream>>>(a);
-    else prologue_kernel<__nv_bfloat16, 64><<<(unsigned)blocks, PRO_THREADS, 0, stream>>>(a);
+    auto kern = a.D == 128 ? prologue_kernel<__nv_bfloat16, 128> : prologue_kernel<__nv_bfloat16, 64>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)PRO_STAGE_BYTES);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)blocks, PRO_THREADS, PRO_STAGE_BYTES, stream>>>(a);
   } else {
     if (a.D == 128) prologue_kernel<float, 128><<<(unsigned)blocks, PRO_THREADS, 0, stream>>>(a);
     else prologue_kernel<float, 64><<<(unsigned)blocks, PRO_THREADS, 0, stream>>>(a);
