@@ -878,9 +878,39 @@ __global__ void chunk_table_kernel(const int32_t *cu, int N, int64_t total, int3
   if (!good && err != nullptr) atomicOr(err, ERR_BAD_CU_SEQLENS);
 }
 
+// order[r] = the sequence with the r-th most chunks (ties: lower index first); one CTA:
+// the chunk counts go to shared memory, then each thread ranks its sequences against all.
+constexpr int kOrderMaxSeqs = 2048;
+__global__ void __launch_bounds__(1024) seq_order_kernel(const int32_t *cu, int N, int64_t total,
+                                                         int32_t *order) {
+  __shared__ int32_t nch[kOrderMaxSeqs];
+  if (N > kOrderMaxSeqs) {   // many short sequences: the tail matters little, keep the order
+    for (int n = threadIdx.x; n < N; n += blockDim.x) order[n] = n;
+    return;
+  }
+  for (int n = threadIdx.x; n < N; n += blockDim.x) {
+    int64_t s, e;
+    seq_bounds(cu, n, 0, total, s, e);
+    nch[n] = (int32_t)((e - s + CH - 1) / CH);
+  }
+  __syncthreads();
+  for (int n = threadIdx.x; n < N; n += blockDim.x) {
+    const int32_t c = nch[n];
+    int rank = 0;
+    for (int m = 0; m < N; ++m) rank += (nch[m] > c) | (nch[m] == c && m < n);
+    order[rank] = n;
+  }
+}
+
 }  // namespace prep
 
 static_assert(kChunkRecordBytes == chunkfmt::REC_STRIDE, "record size");
+
+cudaError_t launch_seq_order(const int32_t *cu, int N, int64_t total, int32_t *order, cudaStream_t stream) {
+  if (N <= 0) return cudaSuccess;
+  prep::seq_order_kernel<<<1, 1024, 0, stream>>>(cu, N, total, order);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_chunk_table(const int32_t *cu, int N, int64_t total, int32_t *chunk_cu, int *err,
                                cudaStream_t stream) {

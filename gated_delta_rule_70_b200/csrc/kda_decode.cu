@@ -577,6 +577,11 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_multi_kernel(DecodeArgs a) {
       if (!ok) { sc.fail = 1; break; }
       if (l == 0) {
         umma::bulk_s2g(a.state + (int64_t)it * D * D, smem + slot * M_SLOT + M_STATE, D * D * 4);
+        if (a.step_states != nullptr) {   // the state after the last token is the final state
+          const int n = it / H, h = it % H;
+          umma::bulk_s2g(a.step_states + (((int64_t)n * T + T - 1) * H + h) * D * D,
+                         smem + slot * M_SLOT + M_STATE, D * D * 4);
+        }
         umma::bulk_commit();
       }
       // two items ahead, into this same slot once the store has read it
@@ -714,7 +719,7 @@ __global__ void __launch_bounds__(NT, 1) decode_tma_multi_kernel(DecodeArgs a) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) S[r][c] = fmaf(k_, dl[c], S[r][c]);
         }
-        if (a.step_states != nullptr) {
+        if (a.step_states != nullptr && t + 1 < T) {   // (the last one leaves with the slot)
           float *dst = a.step_states + (row * H + h) * D * D;
 #pragma unroll
           for (int r = 0; r < 16; ++r)

@@ -75,10 +75,12 @@ struct SegEvents {
 cudaError_t run_chunk_path(PrepArgs pa, const RecurrenceArgs &ra, bool varlen, bool fused,
                            const PrologueArgs *raw, char *ws, const WsLayout &L,
                            cudaStream_t stream) {
-  int32_t *chunk_cu = nullptr;
+  int32_t *chunk_cu = nullptr, *order = nullptr;
   if (varlen) {
     chunk_cu = reinterpret_cast<int32_t *>(ws + L.chunk_cu);
+    order = reinterpret_cast<int32_t *>(ws + L.order);
     cudaError_t e = launch_chunk_table(ra.cu, ra.N, ra.total_tokens, chunk_cu, ra.err, stream);
+    if (e == cudaSuccess) e = launch_seq_order(ra.cu, ra.N, ra.total_tokens, order, stream);
     if (e != cudaSuccess) return e;
   }
   const int64_t slots = max_chunk_slots(ra.N, ra.total_tokens, ra.seq_len, varlen);
@@ -87,7 +89,7 @@ cudaError_t run_chunk_path(PrepArgs pa, const RecurrenceArgs &ra, bool varlen, b
   pa.records = ws + L.records; pa.err = ra.err; pa.wait_polls = ra.wait_polls;
   StateArgs sa{};
   sa.N = ra.N; sa.H = ra.H; sa.seq_len = ra.seq_len; sa.total_tokens = ra.total_tokens;
-  sa.cu = ra.cu; sa.chunk_cu = chunk_cu; sa.records = ws + L.records; sa.max_slots = slots;
+  sa.cu = ra.cu; sa.chunk_cu = chunk_cu; sa.order = order; sa.records = ws + L.records; sa.max_slots = slots;
   sa.state0 = ra.state0; sa.scale = ra.scale; sa.o = ra.o; sa.state1 = ra.state1; sa.err = ra.err;
   sa.wait_polls = ra.wait_polls;
   sa.seg_c0 = 0; sa.seg_c1 = INT_MAX;

@@ -114,6 +114,7 @@ struct StateArgs {
   int N, H, seq_len;
   int64_t total_tokens;
   const int32_t *cu, *chunk_cu;
+  const int32_t *order;      // varlen: CTA slot -> sequence, longest first; nullptr: identity
   const void *records;
   int64_t max_slots;         // record slots in the workspace (chunks beyond are not read)
   const float *state0;       // [N, H, 128, 128] or nullptr
@@ -138,9 +139,10 @@ inline int64_t max_chunk_slots(int N, int64_t total_tokens, int seq_len, bool va
 
 // Workspace layout (byte offsets, 256-aligned):
 //   error word | qn | kn | vc | g | beta   (prologue outputs; token-kernel prefill only)
-//   | chunk table (N+1 int32) | chunk records    (tensor-core path only)
+//   | chunk table (N+1 int32) | sequence order (N int32, varlen) | chunk records
+//                                                           (tensor-core path only)
 struct WsLayout {
-  size_t err, qn, kn, vc, g, beta, chunk_cu, records, total;
+  size_t err, qn, kn, vc, g, beta, chunk_cu, order, records, total;
   bool tc;   // bf16 with head_dim 128: the tensor-core chunk path
 };
 // The tensor-core path splits e^{Gamma_t - Gamma_s} around a reference in the middle
@@ -169,6 +171,7 @@ inline WsLayout workspace_layout(int N, int H, int D, int seq_len, int64_t T, in
   }
   if (L.tc) {
     L.chunk_cu = off; off = up(off + (size_t)(N + 1) * 4);
+    if (varlen) { L.order = off; off = up(off + (size_t)N * 4); }
     off = (off + 1023) / 1024 * 1024;
     L.records = off;
     off += (size_t)max_chunk_slots(N, T, seq_len, varlen) * H * kChunkRecordBytes;
@@ -194,6 +197,9 @@ cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t stream);
 // (starts at 0, non-decreasing, ends at total) and flags ERR_BAD_CU_SEQLENS in *err.
 cudaError_t launch_chunk_table(const int32_t *cu, int N, int64_t total, int32_t *chunk_cu, int *err,
                                cudaStream_t stream);
+// order[r] = the sequence with the r-th most 64-token chunks (ties: lower index first), so
+// the state pass starts its longest chains first; identity for more than 2048 sequences.
+cudaError_t launch_seq_order(const int32_t *cu, int N, int64_t total, int32_t *order, cudaStream_t stream);
 // fused: run the prologue on the raw inputs in a.{conv_w, b, A_log, dt_bias, conv0}
 // and q, k, v, alpha (tensor maps built here); else read a.{qn, kn, vc, g, beta}.
 cudaError_t launch_chunk_prep(PrepArgs a, int64_t max_chunks, bool fused, const void *q,

@@ -91,7 +91,8 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
                                               ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H;
-  const int n = blockIdx.x / H, h = blockIdx.x % H;
+  const int n = a.order != nullptr ? a.order[blockIdx.x / H] : (int)(blockIdx.x / H);
+  const int h = blockIdx.x % H;
   int64_t s0, s1;
   seq_bounds(a.cu, n, a.seq_len, a.total_tokens, s0, s1);
   // this launch's chunks [k0, k1) of the sequence (a time segment, or all of it)
