@@ -47,8 +47,10 @@
 //   [Lq; Lk] x R_all^T (M=128, N=160 or 96, K=128) -> A_qk and A_kk blocks
 //   W^T = K~^T T_b^T and U^T = V^T T_b^T      (M=128, N=64, K=64)
 // The 64x64 unit-lower-triangular solve runs in shared memory: 16x16 diagonal
-// blocks by forward substitution, then each warp owns a set of columns and
-// runs block forward substitution down them with no block-wide barrier.
+// blocks by forward substitution, then the off-diagonal blocks as products of
+// 16x16 blocks on the warp-level tensor-core path (mma.sync, tf32 operands,
+// fp32 accumulation): first the blocks next to the diagonal, then the lower-left
+// 32x32 half from the two 32x32 diagonal halves.
 #include <algorithm>
 
 #include "chunk_common.cuh"
@@ -62,7 +64,9 @@ namespace prep {
 using namespace chunkfmt;
 
 constexpr int NT = 256;
-constexpr int TSS = 68;      // fp32 row stride of the solve scratch
+constexpr int TSS = 68;      // fp32 row stride of diag(beta) A_kk (ldmatrix rows in distinct banks)
+constexpr int TST = 72;      // fp32 row stride of T (a B fragment's rows c, c+4 and columns g: distinct banks)
+constexpr int TSX = 40;      // fp32 row stride of the 32 x 32 intermediate of the solve (likewise)
 constexpr float LOG2E = 1.4426950408889634f;
 
 // Shared memory (byte offsets from a 1024-aligned base); two CTAs fit on one SM.
@@ -78,8 +82,8 @@ constexpr uint32_t OFF_L = 0;                 // [q rows 0..63 | k rows 64..127]
 constexpr uint32_t OFF_R = 32768;             // R_all: up to 160 rows x 128 ch: 40 KB
 // Once the intra-chunk MMA has completed:
 constexpr uint32_t OFF_SB = 0;                // diag(beta) A_kk fp32 [64][TSS]
-constexpr uint32_t OFF_ST = 64 * TSS * 4;     // T fp32 [64][TSS]
-constexpr uint32_t OFF_TB = 35840;            // T_b [t][s] bf16, 8 KB
+constexpr uint32_t OFF_ST = 64 * TSS * 4;     // T fp32 [64][TST]
+constexpr uint32_t OFF_TB = 35840;            // T_b [t][s] bf16, 8 KB (before it: the solve's X [32][TSX])
 // Record parts staged in their record image, then sent by one bulk store each
 // (a lane per 128-byte row would scatter 16-byte pieces over 32 rows per store):
 constexpr uint32_t OFF_AQS = 45056;           // A_qk, 8 KB (after the intra MMA, beside the solve)
@@ -107,7 +111,8 @@ constexpr uint32_t TMA_BYTES = 3 * RAW_ROWS * RAW_ROW + CH * RAW_ROW + 3 * 1024 
 static_assert(OFF_RAWK >= RAW_ROWS * RAW_ROW && OFF_RAWV >= OFF_RAWK + RAW_ROWS * RAW_ROW &&
               OFF_RAWA >= OFF_RAWV + RAW_ROWS * RAW_ROW && OFF_RAWA + CH * RAW_ROW <= OFF_KT,
               "prologue staging overlaps");
-static_assert(OFF_ST + 64 * TSS * 4 <= OFF_TB && OFF_TB + 8192 <= OFF_KT && OFF_V + 16384 <= OFF_C,
+static_assert(OFF_ST + 64 * TST * 4 <= OFF_TB && OFF_TB + 8192 <= OFF_KT && OFF_V + 16384 <= OFF_C &&
+                  32 * TSX * 4 <= 8192 && OFF_ST % 16 == 0,
               "solve scratch overlaps");
 static_assert(OFF_TB % 1024 == 0 && OFF_KT % 1024 == 0 && OFF_V % 1024 == 0 && OFF_R % 1024 == 0,
               "SW128 alignment");
@@ -165,61 +170,26 @@ __device__ __forceinline__ void drain(uint8_t *smem) {
   if (p != 0) (void)umma::mbar_wait_bounded(reinterpret_cast<uint64_t *>(smem + (p & ~7u)), p & 1u, kWaitPolls);
 }
 
-// Off-diagonal blocks of T in the columns [col, col + NC) of column block J:
-// for I = J+1..3,  X = sum_{K=J}^{I-1} B_IK T_KJ,  T_IJ = -T_II X  (one warp;
-// lane = row r of the block and a group of NC columns).  X is parked where T_IJ
-// goes; no other warp touches these columns.
-template <int J, int NC>
-__device__ __forceinline__ void solve_columns(const float *sB, float *sT, int col, int r) {
-  constexpr int NP = NC / 2;   // column pairs; two accumulators each (even / odd terms) for ILP
+// 16 x 8 x 16 tiles of the solve on the warp-level tensor-core path (tf32 operands, fp32
+// accumulation), over row-major fp32 matrices in shared memory.
+// d += A[ra..ra+16)[ca..ca+16) * B[rb..rb+16)[cb..cb+8)   (A at shared address abase, row stride lda)
+__device__ __forceinline__ void tile_mma(float (&d)[4], uint32_t abase, int lda, int ra, int ca,
+                                         const float *bm, int ldb, int rb, int cb, int lane) {
+  const int mi = lane >> 3, g = lane >> 2, c = lane & 3;
 #pragma unroll
-  for (int I = J + 1; I < 4; ++I) {
-    float2 x[2][NP];
-#pragma unroll
-    for (int c = 0; c < NP; ++c) x[0][c] = x[1][c] = f2(0.f);
-#pragma unroll
-    for (int K = J; K < I; ++K) {
-#pragma unroll
-      for (int m4 = 0; m4 < 4; ++m4) {
-        const float4 bv = *reinterpret_cast<const float4 *>(sB + (16 * I + r) * TSS + 16 * K + 4 * m4);
-        const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float *trow = sT + (16 * K + 4 * m4 + e) * TSS + col;
-          if constexpr (NC == 2) {
-            x[e & 1][0] = fma2(f2(bb[e]), *reinterpret_cast<const float2 *>(trow), x[e & 1][0]);
-          } else {
-            const float4 tv = *reinterpret_cast<const float4 *>(trow);
-            x[e & 1][0] = fma2(f2(bb[e]), make_float2(tv.x, tv.y), x[e & 1][0]);
-            x[e & 1][1] = fma2(f2(bb[e]), make_float2(tv.z, tv.w), x[e & 1][1]);
-          }
-        }
-      }
-    }
-    float *dst = sT + (16 * I + r) * TSS + col;
-#pragma unroll
-    for (int c = 0; c < NP; ++c) *reinterpret_cast<float2 *>(dst + 2 * c) = add2(x[0][c], x[1][c]);
-    __syncwarp();
-    float2 y[2][NP];
-#pragma unroll
-    for (int c = 0; c < NP; ++c) y[0][c] = y[1][c] = f2(0.f);
-#pragma unroll
-    for (int m4 = 0; m4 < 4; ++m4) {
-      const float4 tv = *reinterpret_cast<const float4 *>(sT + (16 * I + r) * TSS + 16 * I + 4 * m4);
-      const float tt[4] = {tv.x, tv.y, tv.z, tv.w};   // row r of T_II (zero right of the diagonal)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float *xrow = sT + (16 * I + 4 * m4 + e) * TSS + col;
-#pragma unroll
-        for (int c = 0; c < NP; ++c)
-          y[e & 1][c] = fma2(f2(-tt[e]), *reinterpret_cast<const float2 *>(xrow + 2 * c), y[e & 1][c]);
-      }
-    }
-    __syncwarp();
-#pragma unroll
-    for (int c = 0; c < NP; ++c) *reinterpret_cast<float2 *>(dst + 2 * c) = add2(y[0][c], y[1][c]);   // already negated
-    __syncwarp();
+  for (int kk = 0; kk < 2; ++kk) {
+    uint32_t a[4];
+    umma::ldsm_x4(abase + (uint32_t)(((ra + (lane & 7) + (mi & 1) * 8) * lda + ca + 8 * kk + (mi >> 1) * 4) * 4), a);
+    const uint32_t b0 = __float_as_uint(bm[(rb + 8 * kk + c) * ldb + cb + g]);
+    const uint32_t b1 = __float_as_uint(bm[(rb + 8 * kk + c + 4) * ldb + cb + g]);
+    umma::mma_tf32(d, a, b0, b1);
   }
+}
+// m[r0..r0+16)[c0..c0+8) = sgn * d
+__device__ __forceinline__ void tile_store(float *m, int ld, int r0, int c0, int lane, const float (&d)[4], float sgn) {
+  const int g = lane >> 2, c = lane & 3;
+  *reinterpret_cast<float2 *>(m + (r0 + g) * ld + c0 + 2 * c) = make_float2(sgn * d[0], sgn * d[1]);
+  *reinterpret_cast<float2 *>(m + (r0 + g + 8) * ld + c0 + 2 * c) = make_float2(sgn * d[2], sgn * d[3]);
 }
 
 // The (sequence, chunk) of chunk slot `gchunk`: dense batches by division, varlen
@@ -759,7 +729,12 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   }
 
   // ---------------------------------------------------------------- T = (I + B)^{-1}
-  if (warp < 4) {  // diagonal 16x16 blocks: warp = block, lane = column (lanes 16..31 mirror)
+  // The 16 x 16 diagonal blocks D_I by forward substitution; then products of 16 x 16 blocks,
+  // each warp a 16 x 8 tile (columns 8 nh .. 8 nh + 7 of a block) on the warp-level tensor-core
+  // path:  T_10 = -D_1 (B_10 D_0),  T_32 = -D_3 (B_32 D_2);  then the lower-left 32 x 32 half
+  //   X = B_[10] T_[00]:  X_a0 = B_a0 D_0 + B_a1 T_10,  X_a1 = B_a1 D_1   (a = 2, 3)
+  //   T_[10] = -T_[11] X:  T_2b = -D_2 X_2b,  T_3b = -(T_32 X_2b + D_3 X_3b).
+  if (warp < 4) {  // diagonal blocks: warp = block, lane = column (lanes 16..31 mirror)
     const int o16 = warp * 16, cidx2 = lane & 15;
     float x[16];
 #pragma unroll
@@ -771,23 +746,50 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
     }
     if (lane < 16) {
 #pragma unroll
-      for (int r = 0; r < 16; ++r) sTm[(o16 + r) * TSS + o16 + cidx2] = x[r];
+      for (int r = 0; r < 16; ++r) sTm[(o16 + r) * TST + o16 + cidx2] = x[r];
     }
   }
   __syncthreads();
-  {  // off-diagonal blocks, column by column (column block 3 has none)
-    const int r = lane & 15, hh = lane >> 4;
-    if (warp < 4) solve_columns<0, 2>(sBm, sTm, 4 * warp + 2 * hh, r);
-    else if (warp < 6) solve_columns<1, 4>(sBm, sTm, 16 + 8 * (warp - 4) + 4 * hh, r);
-    else solve_columns<2, 4>(sBm, sTm, 32 + 8 * (warp - 6) + 4 * hh, r);
+  {
+    const uint32_t aB = sbase + OFF_SB, aT = sbase + OFF_ST;
+    float *sX = reinterpret_cast<float *>(smem + OFF_TB);
+    const int nh = warp & 1;
+    float xa[4] = {0.f, 0.f, 0.f, 0.f}, xb[4] = {0.f, 0.f, 0.f, 0.f};
+    const int ia = 16 * (2 + ((warp - 4) >> 1));   // warps 4-7: row block a of X
+    if (warp < 4) {   // T_10 (warps 0, 1) and T_32 (warps 2, 3)
+      const int i = 16 * ((warp >> 1) * 2 + 1), j = i - 16;
+      tile_mma(xa, aB, TSS, i, j, sTm, TST, j, j + 8 * nh, lane);    // B_ij D_j, parked where T_ij goes
+      tile_store(sTm, TST, i, j + 8 * nh, lane, xa, 1.f);
+      __syncwarp();
+      tile_mma(xb, aT, TST, i, i, sTm, TST, i, j + 8 * nh, lane);    // D_i (B_ij D_j)
+      __syncwarp();
+      tile_store(sTm, TST, i, j + 8 * nh, lane, xb, -1.f);
+    } else {          // B_a0 D_0 and X_a1 = B_a1 D_1 (need no T_10)
+      tile_mma(xa, aB, TSS, ia, 0, sTm, TST, 0, 8 * nh, lane);
+      tile_mma(xb, aB, TSS, ia, 16, sTm, TST, 16, 16 + 8 * nh, lane);
+    }
+    __syncthreads();
+    if (warp >= 4) {  // X_a0 = B_a0 D_0 + B_a1 T_10
+      tile_mma(xa, aB, TSS, ia, 16, sTm, TST, 16, 8 * nh, lane);
+      tile_store(sX, TSX, ia - 32, 8 * nh, lane, xa, 1.f);
+      tile_store(sX, TSX, ia - 32, 16 + 8 * nh, lane, xb, 1.f);
+    }
+    __syncthreads();
+    {                 // T_ab, a = 2 + warp / 4, b = (warp / 2) % 2
+      const int a = 2 + (warp >> 2), b = (warp >> 1) & 1;
+      float y[4] = {0.f, 0.f, 0.f, 0.f};
+      tile_mma(y, aT, TST, 16 * a, 32, sX, TSX, 0, 16 * b + 8 * nh, lane);       // T_a2 X_2b
+      if (a == 3) tile_mma(y, aT, TST, 48, 48, sX, TSX, 16, 16 * b + 8 * nh, lane);   // D_3 X_3b
+      tile_store(sTm, TST, 16 * a, 16 * b + 8 * nh, lane, y, -1.f);
+    }
   }
   __syncthreads();
 #pragma unroll
   for (int it = 0; it < 2; ++it) {  // T_b rows as bf16, K-major [t][s]
     const int e = tid + it * NT;
     const int t = e >> 3, c8 = e & 7;
-    const float4 t0 = *reinterpret_cast<const float4 *>(sTm + t * TSS + c8 * 8);
-    const float4 t1 = *reinterpret_cast<const float4 *>(sTm + t * TSS + c8 * 8 + 4);
+    const float4 t0 = *reinterpret_cast<const float4 *>(sTm + t * TST + c8 * 8);
+    const float4 t1 = *reinterpret_cast<const float4 *>(sTm + t * TST + c8 * 8 + 4);
     const float4 b0 = *reinterpret_cast<const float4 *>(beta_s + c8 * 8);
     const float4 b1 = *reinterpret_cast<const float4 *>(beta_s + c8 * 8 + 4);
     const float2 p0 = mul2(make_float2(t0.x, t0.y), make_float2(b0.x, b0.y));

@@ -105,6 +105,26 @@ __device__ __forceinline__ void mma_commit(uint64_t *mbar) {
                :: "r"(smem_u32(mbar)) : "memory");
 }
 
+// ---------------------------------------------------------------- warp-level MMA (mma.sync)
+
+// Four 8 x 8 matrices of 16-bit elements (8 rows of 16 bytes each); lanes 8i..8i+7 give the
+// row addresses of matrix i, and lane l receives word l % 4 of row l / 4 of matrix i in r[i].
+// For fp32 data a matrix is 8 rows x 4 floats, so one call loads a 16 x 8 tf32 A fragment.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr) : "memory");
+}
+// d += A B for one 16 x 8 x 8 tile with tf32 operands and fp32 accumulation.  Fragments (g = lane / 4,
+// c = lane % 4): a = A[g][c], A[g+8][c], A[g][c+4], A[g+8][c+4]; b = B[c][g], B[c+4][g];
+// d = D[g][2c], D[g][2c+1], D[g+8][2c], D[g+8][2c+1].  The operands are fp32 bit patterns, of
+// which the tf32 unit reads the sign, the exponent and the top 10 mantissa bits.
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 // ---------------------------------------------------------------- TMEM <-> registers
 
 // Each thread of the warp reads its lane (taddr lane base + laneid), 16 consecutive columns.

@@ -56,6 +56,13 @@ def _tf32(x):
     return u.view(np.float32).astype(np.float64)
 
 
+def _tf32_trunc(x):
+    """tf32 as the warp-level tensor-core path reads an fp32 operand: the low 13 mantissa bits
+    dropped (toward zero), back in fp64."""
+    u = np.asarray(x, dtype=np.float32).copy().view(np.uint32) & np.uint32(0xFFFFE000)
+    return u.view(np.float32).astype(np.float64)
+
+
 def _flush(x):
     """fp32's flush to zero below its normal range (2^-126), which the special-function
     exponential applies to its results."""
@@ -63,13 +70,13 @@ def _flush(x):
     return np.where(np.abs(x) < 2.0 ** -126, 0.0, x)
 
 
-def blocked_inverse(A, tf32: bool = False, bf16: bool = False):
+def blocked_inverse(A, tf32: bool = False, bf16: bool = False, tf32_trunc: bool = False):
     """(I + A)^{-1} for a strictly lower-triangular 64 x 64 A, by blocks: the 16 x 16 diagonal
     blocks' inverses D_i by substitution, then T_ij = -D_i (A_ij D_j) for the blocks next to the
     diagonal, then the 32 x 32 halves T_21 = -T_2 (A_21 T_1).  Every product there is a small
     dense matrix product (tensor-core shaped); ``tf32`` (or ``bf16``) rounds their operands to
     that type and keeps the accumulation wide."""
-    r = _tf32 if tf32 else (_bf16 if bf16 else (lambda x: x))
+    r = _tf32 if tf32 else (_bf16 if bf16 else (_tf32_trunc if tf32_trunc else (lambda x: x)))
     n = A.shape[0]
     T = np.zeros_like(A)
     for i in range(0, n, 16):
@@ -96,12 +103,13 @@ def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB, bf16=False, solv
     """One padded chunk (q, k, v [64, d], g [64, d_k] natural-log gates, beta [64]) ->
     (A_qk, W, U, Q 2^Gamma, K 2^{Gamma_C - Gamma}, 2^{Gamma_C}, the log2 exponents of every
     L and R factor taken).  ``mistake`` plants one plausible error, for the test that shows
-    the comparison with the oracle catches it.  ``sb`` is the sub-block length (16 in the
-    kernels).  ``bf16`` rounds where the kernels hold bf16: the MMA operands L and R, T diag(beta),
+    the comparison with the oracle catches it.  ``sb`` is the sub-block length (32 in the
+    kernels at gate bounds >= -5.02, else 16).  ``bf16`` rounds where the kernels hold bf16: the MMA operands L and R, T diag(beta),
     and the record's A_qk, W, U, Q 2^Gamma and K 2^{Gamma_C - Gamma}; A_kk, T, the gates and
     2^{Gamma_C} stay wide (fp32 in the kernels, fp64 here).  A collection of SITES names
     rounds at those sites only.  ``solve``: "direct" (a plain inverse), "blocked",
-    "blocked_tf32" or "blocked_bf16" (``blocked_inverse``).  ``flush`` applies fp32's flush
+    "blocked_tf32", "blocked_tf32_trunc" (the kernels' form) or "blocked_bf16"
+    (``blocked_inverse``).  ``flush`` applies fp32's flush
     to zero below 2^-126 to the exponentials and the R rows of earlier blocks, as the
     kernels' arithmetic does; with 32-token blocks the earlier block's constant is then
     taken as its root applied twice (the constant itself spans 32 gates, the root 16), as
@@ -143,7 +151,8 @@ def chunk_factors(q, k, v, g, beta, mistake=None, sb: int = SB, bf16=False, solv
     if solve == "direct":
         T = np.linalg.inv(np.eye(CH) + A_kk)
     else:
-        T = blocked_inverse(A_kk, tf32=solve == "blocked_tf32", bf16=solve == "blocked_bf16")
+        T = blocked_inverse(A_kk, tf32=solve == "blocked_tf32", bf16=solve == "blocked_bf16",
+                            tf32_trunc=solve == "blocked_tf32_trunc")
     Kt = rb("LR")(k * np.exp2(G2))
     if mistake == "beta_after_T":
         W = beta[:, None] * (T @ Kt)

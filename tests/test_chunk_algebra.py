@@ -195,10 +195,11 @@ def _errs(cu, q, k, v, g, beta, S0, **kw):
     return rel(o, o_ref), rel(s, s_ref)
 
 
-@pytest.mark.parametrize("solve", ["blocked_tf32", "blocked_bf16"])
+@pytest.mark.parametrize("solve", ["blocked_tf32", "blocked_tf32_trunc", "blocked_bf16"])
 @pytest.mark.parametrize("rho", [10.0, 0.5])
 def test_blocked_solve_on_tensor_cores_keeps_the_budget(solve, rho):
-    """The solve's products with tf32 or even bf16 operands (wide accumulation) add next to
+    """The solve's products with tf32 operands (rounded, or truncated as chunk_prep's warp-level
+    tensor-core products read fp32 data) or even bf16 ones, with wide accumulation, add next to
     nothing to the bf16 design's error, for independent keys and for strongly correlated ones."""
     x = _collinear_keys(rho)
     base = _errs(*x, bf16=True)
