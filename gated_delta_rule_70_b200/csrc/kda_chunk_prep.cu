@@ -192,25 +192,26 @@ __device__ __forceinline__ void tile_store(float *m, int ld, int r0, int c0, int
   *reinterpret_cast<float2 *>(m + (r0 + g + 8) * ld + c0 + 2 * c) = make_float2(sgn * d[2], sgn * d[3]);
 }
 
-// The (sequence, chunk) of chunk slot `gchunk`: dense batches by division, varlen
-// by the chunk table.  False for slots past the last chunk.
+// The (sequence, chunk) of chunk slot `gchunk`: dense batches by a 32-bit division,
+// varlen by one load from the slot table (every CTA pays for this before its first copy).
+// False for slots past the last chunk.
 __device__ __forceinline__ bool locate(const PrepArgs &a, int64_t gchunk, int &n, int64_t &c0, int &nt,
                                        int64_t &cidx) {
-  if (a.chunk_cu == nullptr) {
-    const int64_t per = (a.seq_len + CH - 1) / CH;
-    if (per == 0 || gchunk >= per * a.N) return false;
-    n = (int)(gchunk / per);
-    cidx = gchunk % per;
-  } else {
-    if (gchunk >= a.chunk_cu[a.N] || gchunk >= a.max_slots) return false;
-    int lo = 0, hi = a.N - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if ((int64_t)a.chunk_cu[mid] <= gchunk) lo = mid; else hi = mid - 1;
-    }
-    n = lo;
-    cidx = gchunk - a.chunk_cu[n];
+  if (a.slot_info != nullptr) {
+    if (gchunk >= a.max_slots) return false;
+    const int4 si = a.slot_info[gchunk];
+    if (si.x < 0) return false;
+    n = si.x;
+    cidx = si.y;
+    c0 = si.z;
+    nt = si.w;
+    return true;
   }
+  const uint32_t per = ((uint32_t)a.seq_len + CH - 1) / CH;
+  if (per == 0 || gchunk >= (int64_t)per * a.N) return false;
+  const uint32_t g32 = (uint32_t)gchunk, n32 = g32 / per;   // gchunk < the grid < 2^31
+  n = (int)n32;
+  cidx = g32 - n32 * per;
   int64_t s0, s1;
   seq_bounds(a.cu, n, a.seq_len, a.total_tokens, s0, s1);
   c0 = s0 + cidx * CH;
@@ -225,13 +226,15 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
   constexpr int NB = CH / kSub;            // sub-blocks per chunk
   constexpr int RR = r_rows<kSub>();       // rows of R_all
   const int H = a.H;
-  const int h = blockIdx.x % H;
-  int64_t gchunk = blockIdx.x / H;
+  const uint32_t gq = blockIdx.x / (uint32_t)H;
+  const int h = (int)(blockIdx.x - gq * (uint32_t)H);
+  int64_t gchunk = gq;
   if (a.chunk_cu == nullptr && a.seg_len > 0) {   // a time segment of a dense batch
-    const int64_t per = (a.seq_len + CH - 1) / CH;
-    const int64_t cidx = a.seg_c0 + gchunk % a.seg_len;
+    const uint32_t per = ((uint32_t)a.seq_len + CH - 1) / CH;
+    const uint32_t sq = gq / (uint32_t)a.seg_len;
+    const uint32_t cidx = (uint32_t)a.seg_c0 + (gq - sq * (uint32_t)a.seg_len);
     if (cidx >= per) return;
-    gchunk = (gchunk / a.seg_len) * per + cidx;
+    gchunk = (int64_t)sq * per + cidx;
   }
   int n, nt;
   int64_t c0, cidx;
@@ -880,6 +883,29 @@ __global__ void chunk_table_kernel(const int32_t *cu, int N, int64_t total, int3
   if (!good && err != nullptr) atomicOr(err, ERR_BAD_CU_SEQLENS);
 }
 
+// Per chunk slot of a varlen batch: its sequence, chunk index, first token and token count,
+// so that a chunk_prep CTA needs one load, not a binary search over chunk_cu.
+__global__ void slot_table_kernel(const int32_t *cu, const int32_t *chunk_cu, int N, int64_t total,
+                                  int64_t slots, int4 *info) {
+  const int64_t nchunks = chunk_cu[N];
+  for (int64_t s = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; s < slots;
+       s += (int64_t)gridDim.x * blockDim.x) {
+    int4 r = make_int4(-1, 0, 0, 0);
+    if (s < nchunks) {
+      int lo = 0, hi = N - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((int64_t)chunk_cu[mid] <= s) lo = mid; else hi = mid - 1;
+      }
+      int64_t s0, s1;
+      seq_bounds(cu, lo, 0, total, s0, s1);
+      const int64_t cidx = s - chunk_cu[lo], c0 = s0 + cidx * CH;
+      if (c0 < s1) r = make_int4(lo, (int)cidx, (int)c0, (int)(s1 - c0 < CH ? s1 - c0 : CH));
+    }
+    info[s] = r;
+  }
+}
+
 // order[r] = the sequence with the r-th most chunks (ties: lower index first); one CTA:
 // the chunk counts go to shared memory, then each thread ranks its sequences against all.
 constexpr int kOrderMaxSeqs = 2048;
@@ -911,6 +937,15 @@ static_assert(kChunkRecordBytes == chunkfmt::REC_STRIDE, "record size");
 cudaError_t launch_seq_order(const int32_t *cu, int N, int64_t total, int32_t *order, cudaStream_t stream) {
   if (N <= 0) return cudaSuccess;
   prep::seq_order_kernel<<<1, 1024, 0, stream>>>(cu, N, total, order);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_slot_table(const int32_t *cu, const int32_t *chunk_cu, int N, int64_t total,
+                              int64_t slots, int4 *info, cudaStream_t stream) {
+  if (slots <= 0) return cudaSuccess;
+  const int64_t blocks = (slots + 255) / 256;
+  prep::slot_table_kernel<<<(unsigned)(blocks < 1024 ? blocks : 1024), 256, 0, stream>>>(cu, chunk_cu, N, total,
+                                                                                       slots, info);
   return cudaGetLastError();
 }
 

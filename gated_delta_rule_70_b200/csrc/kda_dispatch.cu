@@ -76,16 +76,19 @@ cudaError_t run_chunk_path(PrepArgs pa, const RecurrenceArgs &ra, bool varlen, b
                            const PrologueArgs *raw, char *ws, const WsLayout &L,
                            cudaStream_t stream) {
   int32_t *chunk_cu = nullptr, *order = nullptr;
+  int4 *slot_info = nullptr;
+  const int64_t slots = max_chunk_slots(ra.N, ra.total_tokens, ra.seq_len, varlen);
   if (varlen) {
     chunk_cu = reinterpret_cast<int32_t *>(ws + L.chunk_cu);
     order = reinterpret_cast<int32_t *>(ws + L.order);
+    slot_info = reinterpret_cast<int4 *>(ws + L.slots);
     cudaError_t e = launch_chunk_table(ra.cu, ra.N, ra.total_tokens, chunk_cu, ra.err, stream);
+    if (e == cudaSuccess) e = launch_slot_table(ra.cu, chunk_cu, ra.N, ra.total_tokens, slots, slot_info, stream);
     if (e == cudaSuccess) e = launch_seq_order(ra.cu, ra.N, ra.total_tokens, order, stream);
     if (e != cudaSuccess) return e;
   }
-  const int64_t slots = max_chunk_slots(ra.N, ra.total_tokens, ra.seq_len, varlen);
   pa.N = ra.N; pa.H = ra.H; pa.seq_len = ra.seq_len; pa.total_tokens = ra.total_tokens;
-  pa.cu = ra.cu; pa.chunk_cu = chunk_cu;
+  pa.cu = ra.cu; pa.chunk_cu = chunk_cu; pa.slot_info = slot_info;
   pa.records = ws + L.records; pa.err = ra.err; pa.wait_polls = ra.wait_polls;
   StateArgs sa{};
   sa.N = ra.N; sa.H = ra.H; sa.seq_len = ra.seq_len; sa.total_tokens = ra.total_tokens;

@@ -89,6 +89,8 @@ struct PrepArgs {
   int64_t total_tokens;
   const int32_t *cu;         // [N + 1] or nullptr (dense)
   const int32_t *chunk_cu;   // [N + 1] chunk prefix (varlen) or nullptr (dense)
+  const int4 *slot_info;     // varlen: per chunk slot {sequence, chunk index, first token, tokens}
+                             // ({-1, ..} past the last chunk); nullptr (dense)
   float lower_bound, eps;
   int beta2;                 // fused: beta = 2 sigmoid(b); 0: sigmoid(b)
   // fused prologue: raw inputs (q, k, v, alpha read through the tensor maps)
@@ -139,10 +141,10 @@ inline int64_t max_chunk_slots(int N, int64_t total_tokens, int seq_len, bool va
 
 // Workspace layout (byte offsets, 256-aligned):
 //   error word | qn | kn | vc | g | beta   (prologue outputs; token-kernel prefill only)
-//   | chunk table (N+1 int32) | sequence order (N int32, varlen) | chunk records
-//                                                           (tensor-core path only)
+//   | chunk table (N+1 int32) | sequence order (N int32, varlen)
+//   | slot table (one int4 per chunk slot, varlen) | chunk records   (tensor-core path only)
 struct WsLayout {
-  size_t err, qn, kn, vc, g, beta, chunk_cu, order, records, total;
+  size_t err, qn, kn, vc, g, beta, chunk_cu, order, slots, records, total;
   bool tc;   // bf16 with head_dim 128: the tensor-core chunk path
 };
 // The tensor-core path splits e^{Gamma_t - Gamma_s} around a reference in the middle
@@ -171,7 +173,10 @@ inline WsLayout workspace_layout(int N, int H, int D, int seq_len, int64_t T, in
   }
   if (L.tc) {
     L.chunk_cu = off; off = up(off + (size_t)(N + 1) * 4);
-    if (varlen) { L.order = off; off = up(off + (size_t)N * 4); }
+    if (varlen) {
+      L.order = off; off = up(off + (size_t)N * 4);
+      L.slots = off; off = up(off + (size_t)max_chunk_slots(N, T, seq_len, varlen) * 16);
+    }
     off = (off + 1023) / 1024 * 1024;
     L.records = off;
     off += (size_t)max_chunk_slots(N, T, seq_len, varlen) * H * kChunkRecordBytes;
@@ -200,6 +205,10 @@ cudaError_t launch_chunk_table(const int32_t *cu, int N, int64_t total, int32_t 
 // order[r] = the sequence with the r-th most 64-token chunks (ties: lower index first), so
 // the state pass starts its longest chains first; identity for more than 2048 sequences.
 cudaError_t launch_seq_order(const int32_t *cu, int N, int64_t total, int32_t *order, cudaStream_t stream);
+// info[s] = {sequence, chunk index, first token, tokens} of chunk slot s < slots, {-1, 0, 0, 0}
+// past the last chunk (after launch_chunk_table has written chunk_cu).
+cudaError_t launch_slot_table(const int32_t *cu, const int32_t *chunk_cu, int N, int64_t total,
+                              int64_t slots, int4 *info, cudaStream_t stream);
 // fused: run the prologue on the raw inputs in a.{conv_w, b, A_log, dt_bias, conv0}
 // and q, k, v, alpha (tensor maps built here); else read a.{qn, kn, vc, g, beta}.
 cudaError_t launch_chunk_prep(PrepArgs a, int64_t max_chunks, bool fused, const void *q,
