@@ -384,9 +384,7 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
 #pragma unroll
           for (int p = 0; p < 4; ++p) y[j][p] = mul2(y[j][p], rn);
         }
-        const bool valid = 4 * tg + j < nt;
-        const uint4 packed = valid ? make_uint4(f2_bf2(y[j][0]), f2_bf2(y[j][1]), f2_bf2(y[j][2]), f2_bf2(y[j][3]))
-                                   : make_uint4(0, 0, 0, 0);
+        const uint4 packed = make_uint4(f2_bf2(y[j][0]), f2_bf2(y[j][1]), f2_bf2(y[j][2]), f2_bf2(y[j][3]));
         if (blk == 0) qb[j] = packed;
         else if (blk == 1) kb[j] = packed;
         else *reinterpret_cast<uint4 *>(smem + OFF_V + tr_off(64, tg * 4 + j, cg)) = packed;
@@ -407,12 +405,22 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const uint4 ar = *reinterpret_cast<const uint4 *>(smem + OFF_RAWA + (4 * tg + j) * RAW_ROW + cg * 16);
-      const bool valid = 4 * tg + j < nt;
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         const float2 l = add2(ex2_2(fma2(bf2_f2(word(ar, p)), f2(LOG2E), bias[p])), f2(1.f));
         const float2 g = mul2(make_float2(lg2_approx(l.x), lg2_approx(l.y)), f2(negA));
-        g2[j][p] = valid ? make_float2(fmaxf(g.x, lb2), fmaxf(g.y, lb2)) : f2(0.f);
+        g2[j][p] = make_float2(fmaxf(g.x, lb2), fmaxf(g.y, lb2));
+      }
+    }
+    if (nt < CH) {   // a sequence's last chunk: tokens past its end take no part (q, k, v, gate 0)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (4 * tg + j >= nt) {
+          qb[j] = kb[j] = make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4 *>(smem + OFF_V + tr_off(64, tg * 4 + j, cg)) = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+          for (int p = 0; p < 4; ++p) g2[j][p] = f2(0.f);
+        }
       }
     }
   } else {
