@@ -15,7 +15,9 @@
 // works through four phases (q, k, v, then alpha); with bf16 inputs the rows of a
 // phase are staged two phases ahead into the thread's own shared-memory slots by
 // asynchronous copies, so a thread's loads stay in flight while it computes (the
-// registers hold only the phase it works on).
+// registers hold only the phase it works on); a phase's conv weights are requested
+// before its rows are waited for.  With bf16 outputs the SiLU takes one special-function
+// operation (SiLU(x) = h + h tanh(h), h = x/2): the kernel is close to bound by that unit.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
@@ -135,18 +137,18 @@ prologue_kernel(PrologueArgs a) {
 
 #pragma unroll 1
   for (int blk = 0; blk < 3; ++blk) {
-    if constexpr (kStage) cp_async_wait<1>();   // phase blk's rows have landed
     const T *__restrict__ x = reinterpret_cast<const T *>(blk == 0 ? a.q : (blk == 1 ? a.k : a.v));
     T *__restrict__ y = reinterpret_cast<T *>(blk == 0 ? a.qn : (blk == 1 ? a.kn : a.vc));
     const T *__restrict__ w = reinterpret_cast<const T *>(a.conv_w) + ((int64_t)blk * HD + c0) * KCONV;
     float wr[8][KCONV];  // 8 channels x 4 taps = 32 contiguous elements, 2 channels per load
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) {
+    for (int i = 0; i < 8; i += 2) {   // issued before the wait for the rows: the two latencies overlap
       float t8[8];
       load8(w + i * KCONV, t8);
 #pragma unroll
       for (int j = 0; j < KCONV; ++j) { wr[i][j] = t8[j]; wr[i + 1][j] = t8[KCONV + j]; }
     }
+    if constexpr (kStage) cp_async_wait<1>();   // phase blk's rows have landed
     // history hist[m][i]: raw input at token (t - 3 + m), m = 0..2
     float hist[3][8];
     int n = n0;
@@ -189,7 +191,17 @@ prologue_kernel(PrologueArgs a) {
         acc = fmaf(wr[i][1], hist[1][i], acc);
         acc = fmaf(wr[i][2], hist[2][i], acc);
         acc = fmaf(wr[i][3], xt[i], acc);
-        yt[i] = silu_f(acc);
+        if constexpr (sizeof(T) == 2) {
+          // bf16 outputs: SiLU(x) = h + h tanh(h), h = x/2, with the special-function unit's
+          // fp32 tanh (one operation, relative error about 2^-11, under the bf16 rounding
+          // that follows); fp32 outputs keep the division form
+          const float hx = 0.5f * acc;
+          float th;
+          asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(hx));
+          yt[i] = fmaf(hx, th, hx);
+        } else {
+          yt[i] = silu_f(acc);
+        }
         hist[0][i] = hist[1][i];
         hist[1][i] = hist[2][i];
         hist[2][i] = xt[i];
