@@ -116,6 +116,32 @@ def test_prologue_parity(io, d, lens, varlen):
     np.testing.assert_allclose(W.from_device(beta), ref[4], rtol=2e-6, atol=1e-7)
 
 
+def test_prologue_parity_large_activations():
+    """q, k, v scaled by 40: most conv outputs sit where the SiLU's tanh has saturated (x/2 well
+    past 9), on both signs; outputs still match the oracle elementwise at one bf16 rounding, and
+    the fused prologue of the prefill (its own SiLU) matches through the whole recurrence."""
+    s = W.small("pro_big", [70, 33], H=2, d=128, seed=8, varlen=True)
+    inp = W.make_inputs(s)
+    for name in ("q", "k", "v"):
+        inp[name] = W._store(W.bf16_to_f32(inp[name]) * np.float32(40.0), "bf16")
+    qn, kn, vc, g, beta, _ = kda.prologue(_dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]),
+                                       _dev(inp["conv_w"]), _dev(inp["alpha"]), _dev(inp["b"]),
+                                       _dev(inp["A_log"]), _dev(inp["dt_bias"]),
+                                       cu_seqlens=_dev(inp["cu_seqlens"]), num_seqs=s.num_seqs)
+    torch.cuda.synchronize()
+    f = f64_inputs(inp)
+    ref = oracle.prologue(inp["cu_seqlens"], s.H, s.d, f["q"], f["k"], f["v"], f["conv_w"],
+                          f["alpha"], f["b"], f["A_log"], f["dt_bias"])
+    rt = 2.0 ** -8
+    for got, want in zip((qn, kn, vc), ref[:3]):
+        np.testing.assert_allclose(W.from_device(got), want, rtol=rt, atol=rt * 0.05 * 40)
+    # the prefill's fused prologue on the same inputs, against the oracle's whole recurrence
+    o, st, _ = gpu_prefill(s, inp)
+    o_ref, s_ref, _, _ = oracle_prefill(s, inp)
+    assert max_pair_err(W.from_device(o), o_ref, s.cu_seqlens, s.H) <= TOL["bf16"]
+    assert max_state_err(W.from_device(st), s_ref) <= TOL["bf16"]
+
+
 # ------------------------------------------------------------------ prefill, small
 
 def test_prefill_tiny_fp32_workload():
