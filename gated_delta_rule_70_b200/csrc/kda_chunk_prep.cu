@@ -23,9 +23,9 @@
 // so those intermediates never travel through device memory.  The other
 // variant reads them prepared (the recurrence entry point).  Elementwise work
 // runs two fp32 lanes per instruction; the SiLU's sigmoid is 1/2 + tanh(x/2)/2
-// with the tanh in half precision on the special-function unit (absolute
-// error about 2^-12, under the bf16 rounding of q, k, v); the gate and every
-// decay factor stay in fp32.
+// with the tanh on the special-function unit: fp32 for v, half precision for q and
+// k, two lanes at a time (absolute error about 2^-12 either way, under the bf16
+// rounding of q, k, v); the gate and every decay factor stay in fp32.
 //
 // Numerics: Gamma reaches 64 * (-5) = -320 inside a chunk, so e^{-Gamma}
 // overflows fp32.  The pairwise factor e^{Gamma_t - Gamma_s} is only ever split
@@ -368,7 +368,14 @@ __global__ void __launch_bounds__(NT, 2) chunk_prep_kernel(const __grid_constant
           acc = fma2(w1, x[j + 1], acc);
           acc = fma2(w2, x[j + 2], acc);
           acc = fma2(w3, x[j + 3], acc);
-          y[j][p] = silu2_from_half(acc);
+          if (blk == 2) {   // v: the fp32 tanh, one special-function operation per lane
+            float t0, t1;
+            asm("tanh.approx.f32 %0, %1;" : "=f"(t0) : "f"(acc.x));
+            asm("tanh.approx.f32 %0, %1;" : "=f"(t1) : "f"(acc.y));
+            y[j][p] = fma2(acc, make_float2(t0, t1), acc);
+          } else {
+            y[j][p] = silu2_from_half(acc);
+          }
         }
       }
 #pragma unroll
