@@ -148,9 +148,9 @@ struct WsLayout {
   bool tc;   // bf16 with head_dim 128: the tensor-core chunk path
 };
 // The tensor-core path splits e^{Gamma_t - Gamma_s} around a reference in the middle
-// of each 16-token block, so each factor spans at most 8 gates: for gates >= -10 that is
-// within 2^{+-116}, inside fp32 / bf16 normal range; shapes with a lower gate bound run
-// the token kernel.
+// of each sub-block (32 tokens for gate bounds >= -5.02, else 16), so each factor spans
+// at most 16 or 8 gates: within 2^{+-116}, inside fp32 / bf16 normal range, for gates
+// >= -5.02 or >= -10; shapes with a lower gate bound run the CUDA-core kernels.
 constexpr float kTcMinLowerBound = -10.0f;
 inline bool use_tensor_core_path(int io_dtype, int D, float lower_bound) {
   return io_dtype == KDA_BF16 && D == 128 && lower_bound >= kTcMinLowerBound;
