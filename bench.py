@@ -44,7 +44,7 @@ sys.path.insert(0, ROOT)
 # DRAM bytes (read + write) of one chunk_prep launch on 4x8192x32: an ncu capture of the
 # 1x8192x32 launch scaled by the chunk-heads (x4); None while the kernel has changed since
 # the capture.
-CHUNK_PREP_TRAFFIC_BYTES = 4 * (269.148672e6 + 255.733248e6)
+CHUNK_PREP_TRAFFIC_BYTES = 4 * (269.281536e6 + 254.379008e6)
 
 HBM_FALLBACK_GBS = 6650.0
 BF16_FALLBACK_TFLOPS = 1590.0
