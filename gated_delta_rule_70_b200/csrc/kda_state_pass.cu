@@ -25,14 +25,15 @@
 //   warps 8-11  the output: each chunk's O^T leaves TMEM, transposed through
 //               shared memory into 16-byte row stores, off the chain;
 //   warp 12     MMA issue; warp 13 record copies; warp 14 output-gate copies;
-//   warp 15     waits on the mbarriers the MMA issue depends on and releases the
-//               MMA warp through named barriers (a thread that issues tcgen05
-//               MMAs sees even a completed mbarrier phase several hundred cycles
-//               late; a named barrier hands over in a few tens).
-// Hand-offs are mbarriers: the MMA commits, "D in bf16 is ready", "the next
-// bf16 state copy is ready", "chunk c's MMAs are done" (its record buffer is
-// free; its O^T can leave) and "O^T of chunk c has left" (its TMEM buffer is
-// free).  O^T has four TMEM buffers (chunk index mod 4).
+//   warp 15     waits on the mbarriers the D MMA also depends on (the chunk's record
+//               has landed, its O^T buffer is free), so the MMA-issuing thread
+//               waits on none (a thread that issues tcgen05 MMAs sees even a
+//               completed mbarrier phase several hundred cycles late).
+// The chain hands its bf16 copies to the MMA warp at named barriers ("the bf16
+// state copy is ready", with warp 15; "D in bf16 is ready"), a few tens of cycles
+// each.  The other hand-offs are mbarriers: the MMA commits, "chunk c's MMAs are
+// done" (its record buffer is free; its O^T can leave) and "O^T of chunk c has
+// left" (its TMEM buffer is free).  O^T has four TMEM buffers (chunk index mod 4).
 //
 // Optional output epilogue (the layer's o_norm and sigmoid output gate, same
 // write-up sections "二" and "三"): o <- o / sqrt(mean o^2 + eps) * w * sigmoid(gate)
@@ -54,8 +55,13 @@ constexpr int NO = 128;          // output threads (warps 8-11)
 constexpr int W_MMA = 12, W_REC = 13, W_GATE = 14, W_WAIT = 15;
 constexpr int NT = 512;
 constexpr uint32_t BAR_OUT = 1;   // named barrier of the output warps
-constexpr uint32_t BAR_GO_D = 2;  // waiter -> MMA warp: chunk c's D / O MMAs may go
-constexpr uint32_t BAR_GO_S = 3;  // waiter -> MMA warp: chunk c's state / O MMAs may go
+constexpr uint32_t BAR_GO_D = 2;  // chain + waiter -> MMA warp: chunk c's D / O MMAs may go
+constexpr uint32_t BAR_GO_S = 3;  // chain -> MMA warp: chunk c's state / O MMAs may go
+// Every thread of the chain, the waiter and the MMA warp meets at BAR_GO_D once per chunk,
+// and the chain and the MMA warp at BAR_GO_S, whatever happens (no role leaves its loop
+// early), so no role can run a barrier generation ahead of another.
+constexpr uint32_t N_GO_D = NCH + 64;
+constexpr uint32_t N_GO_S = NCH + 32;
 constexpr uint32_t OFF_REC0 = 0;
 constexpr uint32_t OFF_REC1 = REC_STRIDE;
 constexpr uint32_t OFF_OST = 2 * REC_STRIDE;   // o of one chunk, [64 t][128 j]: bf16, or fp32 when gated
@@ -80,7 +86,7 @@ __device__ __forceinline__ uint32_t o_cols(int c) { return TM_O + (uint32_t)(c &
 __device__ __forceinline__ uint32_t d16_col(int s) { return TM_D + (uint32_t)(32 * (s >> 1) + 8 * (s & 1)); }
 
 // B_OC / B_OE: one per O^T buffer (commit of chunk c's MMAs / its O^T has left TMEM)
-enum { B_FULL0 = 0, B_FULL1, B_D, B_S, B_D16, B_S16, B_REL0, B_REL1, B_OC0, B_OC1, B_OC2, B_OC3,
+enum { B_FULL0 = 0, B_FULL1, B_D, B_S, B_REL0, B_REL1, B_OC0, B_OC1, B_OC2, B_OC3,
        B_OE0, B_OE1, B_OE2, B_OE3, B_G0, B_G1, B_GE0, B_GE1, B_COUNT };
 constexpr uint32_t BAR_AREA = 256;
 static_assert(8 * B_COUNT + 16 <= BAR_AREA, "barrier area");
@@ -119,9 +125,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
   }
   if (tid == 32) {
     for (int i = 0; i < B_COUNT; ++i)
-      umma::mbar_init(&bar[i], (i == B_D16 || i == B_S16)                               ? NCH / 32
-                               : ((i >= B_OE0 && i <= B_OE3) || i == B_GE0 || i == B_GE1) ? NO / 32
-                                                                                        : 1);
+      umma::mbar_init(&bar[i], ((i >= B_OE0 && i <= B_OE3) || i == B_GE0 || i == B_GE1) ? NO / 32 : 1);
     umma::mbar_fence_init();
     *fail = 0;
   }
@@ -196,9 +200,9 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
         (void)umma::mbar_wait_bounded(&bar[B_FULL0 + (k & 1)], (k >> 1) & 1, kWaitPolls);
     } else if (warp == W_WAIT) {
       // ---------------------------------------------------------- waits for the MMA issue
-      // This warp and the MMA warp meet at both named barriers once per chunk, every chunk,
+      // This warp meets the chain and the MMA warp at BAR_GO_D once per chunk, every chunk,
       // whatever happens (after a failed wait the mbarrier waits return at once and the MMA
-      // warp issues nothing), so neither can be left waiting at one.
+      // warp issues nothing), so no role can be left waiting at it.
       // Chunk c+1's record and O^T buffer (normally long ready) are waited for while chunk
       // c's state MMA and bf16 state copy run: even a completed wait costs a few hundred
       // cycles, and only the bf16 state copy should stand before the D MMA.
@@ -208,10 +212,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
       };
       if (nchunks > 0) pre(0);
       for (int c = 0; c < nchunks; ++c) {
-        (void)wait_warp(&bar[B_S16], c & 1);
-        umma::named_sync(BAR_GO_D, 64);
-        (void)wait_warp(&bar[B_D16], c & 1);
-        umma::named_sync(BAR_GO_S, 64);
+        umma::named_sync(BAR_GO_D, N_GO_D);   // with the chain's bf16 state copy of chunk c
         if (c + 1 < nchunks) pre(c + 1);
       }
     } else if (warp == W_MMA) {
@@ -221,10 +222,10 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
       const uint32_t id_s = umma::make_idesc_bf16(128, 128, 0, 1);
       uint64_t *last = nullptr;   // the barrier of the last commit and the phase it completes
       uint32_t last_parity = 0;
-      // released by the waiter warp (the same named-barrier steps for every chunk); after a
-      // failed wait anywhere nothing more is issued (warp-uniform)
-      auto go = [&](uint32_t id) -> bool {
-        umma::named_sync(id, 64);
+      // released by the chain and the waiter warp (the same named-barrier steps for every
+      // chunk); after a failed wait anywhere nothing more is issued (warp-uniform)
+      auto go = [&](uint32_t id, uint32_t count) -> bool {
+        umma::named_sync(id, count);
         umma::fence_after_sync();
         return !__any_sync(0xffffffffu, *(volatile int *)fail != 0);
       };
@@ -234,7 +235,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
         const uint32_t rb = sbase + rec_off(c);
         const int ob = c & (NOBUF - 1);
         const uint32_t ocol = tmem + o_cols(c);
-        issuing = go(BAR_GO_D) && issuing;
+        issuing = go(BAR_GO_D, N_GO_D) && issuing;
         if (issuing && lane == 0) {
           // D^T = S^T (-W^T) (the chain: committed alone), then O^T = S^T Q~^T
 #pragma unroll
@@ -250,7 +251,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
           last = &bar[B_D];
           last_parity = c & 1;
         }
-        issuing = go(BAR_GO_S) && issuing;
+        issuing = go(BAR_GO_S, N_GO_S) && issuing;
         if (issuing && lane == 0) {
           // S^T += D^T K^ (the chain), then O^T += D^T A_qk^T
 #pragma unroll
@@ -368,11 +369,12 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
       if (js >= a.snap_cap) return nullptr;
       return a.snap + (((int64_t)n * a.snap_cap + js) * H + h) * DK * DK;
     };
-    auto handoff = [&](uint64_t *bb) {   // this warp's TMEM stores are done: tell the issuer
+    // this warp's TMEM stores are done: meet the MMA warp at named barrier `id` (the
+    // canonical hand-off of tcgen05 stores to a tcgen05.mma issued by another thread)
+    auto handoff_go = [&](uint32_t id, uint32_t count) {
       umma::tmem_wait_st();
       umma::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) umma::mbar_arrive(bb);
+      umma::named_sync(id, count);
     };
     // This warpgroup's 64 S^T columns (key channels 64hf ..) *= e^{Gamma_C} of the record at rb;
     // with s16: also write their bf16 copy first; with snap: store the state as it stands
@@ -390,7 +392,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
         for (int e = 0; e < 32; ++e)
           p[e] = pack_bf16(__uint_as_float(x[e >> 4][(e & 15) * 2]), __uint_as_float(x[e >> 4][(e & 15) * 2 + 1]));
         umma::tmem_st32(tmem + lane_base + TM_S16 + 32 * hf, p);
-        handoff(&bar[B_S16]);   // the next D / O MMAs need only this copy
+        handoff_go(BAR_GO_D, N_GO_D);   // the next D / O MMAs need only this copy
       }
       if (snap != nullptr) {   // lane j holds column j of S: each row store is 128 contiguous floats
 #pragma unroll
@@ -427,7 +429,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
       umma::tmem_wait_st();
       state_pass_over(OFF_REC0, false, nullptr);
     }
-    handoff(&bar[B_S16]);
+    if (nchunks > 0) handoff_go(BAR_GO_D, N_GO_D);
 #pragma unroll 1
     for (int c = 0; c < nchunks; ++c) {
       const uint32_t rb = rec_off(c);
@@ -457,7 +459,7 @@ __global__ void __launch_bounds__(NT, 1) state_pass_kernel(const __grid_constant
         }
         umma::tmem_st16(tmem + lane_base + TM_D + 32 * hf, p);
       }
-      handoff(&bar[B_D16]);
+      handoff_go(BAR_GO_S, N_GO_S);
       if (c + 1 < nchunks) wait_one(&bar[B_FULL0 + ((c + 1) & 1)], ((c + 1) >> 1) & 1);   // its e^{Gamma_C}
       wait_one(&bar[B_S], c & 1);
       // the next chunk's bf16 state copy (handed off first), then its decay
