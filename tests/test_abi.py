@@ -57,13 +57,18 @@ def test_workspace_size_rules(lib):
     assert dense >= 4 * (8192 // 64) * 32 * record
     assert dense < 4 * (8192 // 64) * 32 * record + (1 << 20)
     assert varlen < dense  # 8192 packed tokens: ceil(8192/64) + 4 chunk slots
+    # varlen: those slots' records, plus one 16-byte slot-table entry per slot and the
+    # chunk table / sequence order
+    slots = 8192 // 64 + 4
+    assert varlen >= slots * 32 * record + slots * 16 + (4 + 1) * 4 + 4 * 4
+    assert varlen < slots * 32 * record + (1 << 20)
     assert kda.recurrence_workspace_size(sh, False) == dense
     # a gate bound the chunk factorisation cannot hold takes the token kernel:
     # the prologue's intermediates, no records
     low = kda.make_shape(4, 8192, 32, 128, torch.bfloat16, lower_bound=-12.0)
     assert kda.prefill_workspace_size(low, False) >= T * 32 * 128 * (3 * 2 + 4) + T * 32 * 4
     assert kda.recurrence_workspace_size(low, False) < 4096
-    # fp32 runs the token kernel
+    # fp32 runs the standalone prologue, then a CUDA-core kernel: the prologue's intermediates
     f32 = kda.make_shape(1, 256, 2, 64, torch.float32)
     assert kda.prefill_workspace_size(f32, False) >= 256 * 2 * 64 * (3 * 4 + 4) + 256 * 2 * 4
     bad = kda.make_shape(4, 8192, 32, 96, torch.bfloat16)
