@@ -99,6 +99,7 @@ extern "C" {
 size_t kda_prefill_workspace_size(const kda_shape *shape, int is_varlen) {
   if (check_shape(shape) != KDA_OK) return 0;
   const int64_t T = is_varlen ? (int64_t)shape->seq_len : (int64_t)shape->num_seqs * shape->seq_len;
+  if (check_tokens(T) != KDA_OK) return 0;
   return workspace_layout(shape->num_seqs, shape->num_heads, shape->head_dim, shape->seq_len, T,
                           shape->io_dtype, shape->lower_bound, is_varlen != 0, true).total;
 }
@@ -106,6 +107,7 @@ size_t kda_prefill_workspace_size(const kda_shape *shape, int is_varlen) {
 size_t kda_recurrence_workspace_size(const kda_shape *shape, int is_varlen) {
   if (check_shape(shape) != KDA_OK) return 0;
   const int64_t T = is_varlen ? (int64_t)shape->seq_len : (int64_t)shape->num_seqs * shape->seq_len;
+  if (check_tokens(T) != KDA_OK) return 0;
   return workspace_layout(shape->num_seqs, shape->num_heads, shape->head_dim, shape->seq_len, T,
                           shape->io_dtype, shape->lower_bound, is_varlen != 0, false).total;
 }
@@ -147,6 +149,7 @@ kda_status kda_prefill_ex(const kda_shape *shape, const kda_prefill_args *args, 
   if (shape->num_seqs == 0) return KDA_OK;
   const int32_t *cu_seqlens = args->cu_seqlens;
   const int64_t T = total_tokens(shape, cu_seqlens);
+  if (check_tokens(T) != KDA_OK) return KDA_ERR_UNSUPPORTED;
   st = check_out_gate(args->out_gate, T);
   if (st != KDA_OK) return st;
   if (T > 0) {
@@ -215,6 +218,7 @@ kda_status kda_prologue(const kda_shape *shape, const void *q, const void *k, co
   kda_status st = check_shape(shape);
   if (st != KDA_OK) return st;
   const int64_t T = total_tokens(shape, cu_seqlens);
+  if (check_tokens(T) != KDA_OK) return KDA_ERR_UNSUPPORTED;
   if (shape->num_seqs == 0) return KDA_OK;
   if (T > 0) {
     KDA_REQUIRE(q); KDA_REQUIRE(k); KDA_REQUIRE(v); KDA_REQUIRE(alpha); KDA_REQUIRE(b);
@@ -241,6 +245,7 @@ kda_status kda_recurrence(const kda_shape *shape, const void *qn, const void *kn
   if (st != KDA_OK) return st;
   if (shape->num_seqs == 0) return KDA_OK;
   const int64_t T = total_tokens(shape, cu_seqlens);
+  if (check_tokens(T) != KDA_OK) return KDA_ERR_UNSUPPORTED;
   if (T > 0) {
     KDA_REQUIRE(qn); KDA_REQUIRE(kn); KDA_REQUIRE(vc); KDA_REQUIRE(g); KDA_REQUIRE(beta);
     KDA_REQUIRE(o);

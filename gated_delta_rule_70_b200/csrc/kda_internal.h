@@ -188,6 +188,10 @@ inline WsLayout workspace_layout(int N, int H, int D, int seq_len, int64_t T, in
 // Shape checks shared by every entry point: KDA_OK, KDA_ERR_INVALID_ARGUMENT or
 // KDA_ERR_UNSUPPORTED.
 kda_status check_shape(const kda_shape *s);
+// A call's packed token total T: the kernels keep token rows and chunk coordinates in 32 bits.
+inline kda_status check_tokens(int64_t T) {
+  return T > (int64_t)INT32_MAX - 64 ? KDA_ERR_UNSUPPORTED : KDA_OK;
+}
 // Polls of one bounded mbarrier wait (each poll is an mbarrier.try_wait, which may
 // itself suspend for a while), and the limit every drain of in-flight copies and
 // tensor-core work uses after a wait has given up.  A call with

@@ -63,6 +63,7 @@ extern "C" kda_status kda_prefill_noalloc(
   if (st != KDA_OK) return st;
   if (s->num_seqs == 0) return KDA_OK;
   const int64_t T = cu_seqlens ? (int64_t)s->seq_len : (int64_t)s->num_seqs * s->seq_len;
+  if (check_tokens(T) != KDA_OK) return KDA_ERR_UNSUPPORTED;
   const bool varlen = cu_seqlens != nullptr;
   const WsLayout L = workspace_layout(s->num_seqs, s->num_heads, s->head_dim, s->seq_len, T,
                                       s->io_dtype, s->lower_bound, varlen, true);

@@ -98,6 +98,11 @@ def test_host_validation_codes(lib):
     assert _call_prefill(lib, bad_flags) == kda.KDA_ERR_INVALID_ARGUMENT
     nan_lb = kda.make_shape(1, 16, 2, 64, torch.float32, lower_bound=float("nan"))
     assert _call_prefill(lib, nan_lb) == kda.KDA_ERR_INVALID_ARGUMENT
+    # a dense batch of more than 2^31 - 65 tokens: refused before any launch, no workspace size
+    huge = kda.make_shape(65536, 65536, 2, 64, torch.float32)
+    assert _call_prefill(lib, huge) == kda.KDA_ERR_UNSUPPORTED
+    assert kda.prefill_workspace_size(huge, False) == 0
+    assert kda.prefill_workspace_size(huge, True) > 0   # varlen: seq_len is the packed total
     # misaligned tensor pointer
     assert _call_prefill(lib, ok, ptrs=ctypes.c_void_p(258)) == kda.KDA_ERR_INVALID_ARGUMENT
     # missing / small / misaligned workspace
